@@ -1,0 +1,152 @@
+/*
+ * quoka.h - C ABI of libquoka.so, the sm_100a (NVIDIA B200) implementation of
+ * the QUOKA query-oriented KV-selection step for chunked prefill.
+ *
+ * Source of the method: the QUOKA technical write-up "QUOKA: how it reshapes
+ * LLM prefill efficiency" (bqwf.cn, news item 915859), cited as [QUOKA §x]:
+ *   §2.1 Algorithm 1  query subselection: MQ = mean(Q over the chunk's
+ *                     tokens), SQ = -cos(Q, MQ), keep the top-NQ queries
+ *   §2.2              cosine score S_ij = Q_i.K_j / (|Q_i| |K_j|)
+ *   §2.3              GQA-aware aggregation: L2-normalise the chosen queries
+ *                     and the keys, mean the queries over each KV head's
+ *                     query-head group, S = Q_group K_norm^T (b,nkv,NQ,T),
+ *                     S_agg = max over the NQ queries (b,nkv,T),
+ *                     indices = topk(S_agg, BSA)
+ *   §4.2 problem 3    the selected KV is the attention's input KV, with the
+ *                     causal mask off for it
+ *
+ * Shapes and notation: b batch, nq query heads, nkv KV heads, G = nq / nkv,
+ * d head dim (64 or 128), BCP chunk length, T prior keys, NQ chosen queries
+ * (1 <= NQ <= BCP), BSA key budget, BSA_eff = min(BSA, T). Query head h reads
+ * KV head floor(h / G).
+ *
+ * Conventions shared by every call:
+ *   - All tensor data pointers are DEVICE pointers on the current CUDA device;
+ *     the caller owns all memory. The library never allocates or frees
+ *     device memory; scratch space is the caller's workspace `ws`
+ *     (device pointer, at least quoka_workspace_size() bytes, 256-byte
+ *     aligned).
+ *   - `stream` is a cudaStream_t passed as void* (NULL = legacy default
+ *     stream). Every call only enqueues work on it and returns; nothing
+ *     synchronises with the host.
+ *   - Arguments are validated on the host before anything is enqueued; on an
+ *     error return nothing has been enqueued.
+ *   - Faults that only the device can see (a key index outside [0, T), a
+ *     bounded wait that gave up) are latched into a status word at the start
+ *     of `ws` and read back with quoka_get_device_status(). Every call that
+ *     takes `ws` first clears that word (an asynchronous 4-byte memset on
+ *     `stream`), so the word reports the faults of the latest call.
+ *   - Calls on different streams with different workspaces may run
+ *     concurrently. Two calls sharing one workspace must be ordered.
+ */
+#ifndef QUOKA_H
+#define QUOKA_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+  QUOKA_OK = 0,
+  QUOKA_ERR_INVALID_ARG = 1, /* bad shape, stride, pointer or parameter */
+  QUOKA_ERR_UNSUPPORTED = 2, /* valid but not implemented (e.g. d not 64/128) */
+  QUOKA_ERR_WORKSPACE = 3,   /* ws is NULL, misaligned or too small */
+  QUOKA_ERR_CUDA = 4,        /* a CUDA runtime call or launch failed */
+  QUOKA_ERR_TIMEOUT = 5,     /* device: a bounded wait gave up */
+  QUOKA_ERR_BOUNDS = 6       /* device: an index was out of range (access skipped) */
+} quoka_status;
+
+typedef enum { QUOKA_F32 = 0, QUOKA_BF16 = 1 } quoka_dtype;
+
+/* A strided 4-D view of device memory. Strides are in ELEMENTS; stride[3]
+ * must be 1, every other stride must keep each row 16-byte aligned
+ * (stride * element size a multiple of 16), and `data` must be 16-byte
+ * aligned. Dimensions of extent 0 are allowed where stated. */
+typedef struct {
+  const void* data;
+  quoka_dtype dtype;
+  int64_t shape[4];
+  int64_t stride[4];
+} quoka_tensor;
+
+/* Bytes of workspace any call below needs for these sizes (the maximum over
+ * the calls, so one workspace serves all of them). Returns 0 only for
+ * invalid sizes. */
+size_t quoka_workspace_size(int b, int nq, int nkv, int d, int64_t T, int BCP,
+                            int NQ, int BSA, quoka_dtype dtype);
+
+/* Steps (a)-(e), [QUOKA §2.1 Algorithm 1, §2.2, §2.3]:
+ *   Q (b, nq, BCP, d), K (b, nkv, T, d), same dtype.
+ *   kv_idx   out (b, nkv, BSA_eff) int32, contiguous: for each (batch, KV
+ *            head) the BSA_eff keys with the largest S_agg, ties to the lower
+ *            key index, in ASCENDING key order. This sorted format is the one
+ *            quoka_gather_kv and quoka_sparse_gqa_attn read.
+ *   kv_count out (b, nkv) int32: number of valid entries per row (BSA_eff).
+ *   q_idx    out (b, nq, NQ) int32 or NULL: chosen chunk positions per query
+ *            head in rank order (descending SQ, ties to the lower position).
+ *   s_agg    out (b, nkv, T) float or NULL: the aggregated key scores.
+ * T may be 0 (nothing is selected). */
+quoka_status quoka_select(const quoka_tensor* Q, const quoka_tensor* K, int NQ,
+                          int BSA, int32_t* kv_idx, int32_t* kv_count,
+                          int32_t* q_idx, float* s_agg, void* ws,
+                          size_t ws_bytes, void* stream);
+
+/* Step (f), [QUOKA §4.2 problem 3]: Ksel[b, j, n] = K[b, j, kv_idx[b, j, n]]
+ * and the same for V, for n < kv_count[b, j] (rows past the count are left
+ * untouched).
+ *   K, V (b, nkv, T, d); kv_idx (b, nkv, BSA_eff) int32; kv_count (b, nkv).
+ *   Ksel, Vsel out (b, nkv, BSA_eff, d), contiguous, dtype of K.
+ * An index outside [0, T) is skipped and latched as QUOKA_ERR_BOUNDS in
+ * `ws` (which may be NULL, in which case it is only skipped). */
+quoka_status quoka_gather_kv(const quoka_tensor* K, const quoka_tensor* V,
+                             const int32_t* kv_idx, const int32_t* kv_count,
+                             int BSA_eff, void* Ksel, void* Vsel, void* ws,
+                             size_t ws_bytes, void* stream);
+
+/* Steps (f)+(g), [QUOKA §4.2 problem 3]: for every query head h, token t,
+ *   O[b,h,t] = sum_k softmax_k(scale * Q[b,h,t].k) v
+ * over the selected prior keys k = K[b, j, kv_idx[b, j, n]] (n < kv_count,
+ * no mask) and the chunk's own keys Kc[b, j, s] with s <= t (causal),
+ * j = floor(h / G). The selected rows are read in place (fused gather).
+ *   Q (b, nq, BCP, d); K, V (b, nkv, T, d); Kc, Vc (b, nkv, BCP, d).
+ *   O   out (b, nq, BCP, d), contiguous, dtype of Q.
+ *   lse out (b, nq, BCP) float or NULL: natural-log partition function
+ *       log sum_k exp(scale * q.k).
+ * bf16 inputs run on the tcgen05 tensor cores (fp32 accumulation and
+ * softmax); fp32 inputs run in fp32 on the CUDA cores. */
+quoka_status quoka_sparse_gqa_attn(const quoka_tensor* Q, const quoka_tensor* K,
+                                   const quoka_tensor* V, const int32_t* kv_idx,
+                                   const int32_t* kv_count, int BSA_eff,
+                                   const quoka_tensor* Kc, const quoka_tensor* Vc,
+                                   float scale, void* O, float* lse, void* ws,
+                                   size_t ws_bytes, void* stream);
+
+/* The whole step (a)-(g): quoka_select followed by quoka_sparse_gqa_attn on
+ * one stream, with no host synchronisation in between.
+ *   kv_idx_out (b, nkv, BSA_eff) int32 or NULL: the selected set (else kept
+ *   in ws). lse may be NULL. */
+quoka_status quoka_prefill_chunk(const quoka_tensor* Q, const quoka_tensor* K,
+                                 const quoka_tensor* V, const quoka_tensor* Kc,
+                                 const quoka_tensor* Vc, int NQ, int BSA,
+                                 float scale, void* O, float* lse,
+                                 int32_t* kv_idx_out, void* ws, size_t ws_bytes,
+                                 void* stream);
+
+/* Synchronises `stream`, then reads the device status word of `ws` into
+ * *device_status (a quoka_status value; QUOKA_OK if the latest call that
+ * used ws latched no device fault). Returns QUOKA_ERR_CUDA if the copy or
+ * the synchronisation failed, QUOKA_ERR_INVALID_ARG for NULL pointers. */
+quoka_status quoka_get_device_status(const void* ws, void* stream,
+                                     int32_t* device_status);
+
+/* A static, human-readable name of a status code. */
+const char* quoka_status_string(quoka_status status);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* QUOKA_H */

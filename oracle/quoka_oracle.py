@@ -55,6 +55,7 @@ __all__ = [
     "select_keys",
     "gather_kv",
     "sparse_attention",
+    "sparse_attention_rows",
     "select",
     "prefill_chunk",
 ]
@@ -267,3 +268,27 @@ def prefill_chunk(Q, K, V, Kc, Vc, NQ: int, BSA: int, scale: Optional[float] = N
     O, LSE = sparse_attention(Q, K, V, sel, Kc, Vc, scale)
     r.update(O=O, LSE=LSE, sel_used=sel)
     return r
+
+
+def sparse_attention_rows(Q, K, V, sel, Kc, Vc, rows, scale: Optional[float] = None):
+    """Step (g) for a list of (b, h, t) rows only, computed one by one:
+    returns (O_rows (n, d), LSE_rows (n,)). Same definition as
+    sparse_attention; used to check large workloads on a sample of rows."""
+    d = Q.shape[-1]
+    nq, nkv = Q.shape[1], Kc.shape[1]
+    G = nq // nkv
+    if scale is None:
+        scale = 1.0 / np.sqrt(d)
+    out = np.empty((len(rows), d))
+    lse = np.empty(len(rows))
+    for n, (bi, h, t) in enumerate(rows):
+        j = h // G
+        idx = np.asarray(sel[bi, j], dtype=np.int64)
+        keys = np.concatenate([_f64(K[bi, j][idx]), _f64(Kc[bi, j, :t + 1])], axis=0)
+        vals = np.concatenate([_f64(V[bi, j][idx]), _f64(Vc[bi, j, :t + 1])], axis=0)
+        logits = scale * (keys @ _f64(Q[bi, h, t]))
+        m = logits.max()
+        p = np.exp(logits - m)
+        out[n] = (p @ vals) / p.sum()
+        lse[n] = m + np.log(p.sum())
+    return out, lse

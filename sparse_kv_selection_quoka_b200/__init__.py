@@ -1,0 +1,28 @@
+"""QUOKA query-oriented KV selection + sparse GQA attention for NVIDIA B200.
+
+The compute path is libquoka.so (hand-written sm_100a CUDA kernels behind a
+C ABI, declared in include/quoka.h); this package holds that library's
+sources, its build script, a thin ctypes binding with the same entry-point
+names, and the seeded synthetic input generators.
+
+The binding is imported lazily so that the input generators can be used
+without the built library.
+"""
+
+__all__ = [
+    "quoka_workspace_size",
+    "quoka_select",
+    "quoka_gather_kv",
+    "quoka_sparse_gqa_attn",
+    "quoka_prefill_chunk",
+    "quoka_get_device_status",
+    "quoka_status_string",
+    "QuokaError",
+]
+
+
+def __getattr__(name):
+    if name in __all__ or name in ("load", "workspace_for", "tensor_view"):
+        from . import _lib
+        return getattr(_lib, name)
+    raise AttributeError(name)

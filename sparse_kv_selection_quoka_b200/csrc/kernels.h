@@ -1,0 +1,71 @@
+// Host-side launchers of the QUOKA kernels (internal to libquoka.so).
+// Every launcher only enqueues work on `stream` and returns the launch
+// error (cudaSuccess when the launch was accepted).
+#pragma once
+
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+namespace quoka {
+
+// Element-stride description of a (b, heads, rows, d) tensor.
+struct Strided {
+  const void* data;
+  int64_t sb, sh, st;  // strides of batch, head and row, in elements
+};
+
+// Step (a)+(b)+(c, first half): one CTA per (batch, query head). Writes the
+// chosen chunk positions in rank order and the L2-normalised chosen queries
+// Qhat (b, nq, NQ, d) fp32.
+cudaError_t launch_qsel(bool bf16, int d, Strided Q, int b, int nq, int BCP, int NQ,
+                        float* Qhat, int32_t* q_idx, cudaStream_t stream);
+
+// Step (c, second half): Q_group (b, nkv, NQ, d) fp32 = mean over the G
+// heads of each group of Qhat at the same rank; optionally also the bf16
+// hi/lo split (b, nkv, 2*NQ, d): rows [0, NQ) hi, rows [NQ, 2NQ) lo.
+cudaError_t launch_qgroup(int d, const float* Qhat, int b, int nq, int nkv, int NQ,
+                          float* Qg, uint16_t* Qg_hilo, cudaStream_t stream);
+
+// Step (d) on the CUDA cores (fp32 arithmetic; any input dtype).
+cudaError_t launch_score_simt(bool bf16, int d, Strided K, int b, int nkv, int64_t T,
+                              const float* Qg, int NQ, float* S_agg, cudaStream_t stream);
+
+// Step (d) on the tcgen05 tensor cores (bf16 K, Q_group as bf16 hi + lo).
+// Returns cudaErrorNotSupported when the shape has no tensor-core variant.
+cudaError_t launch_score_tc(int d, Strided K, int b, int nkv, int64_t T,
+                            const uint16_t* Qg_hilo, int NQ, float* S_agg, int* status,
+                            cudaStream_t stream);
+
+// Step (e): per (batch, KV head) cluster radix select of the BSA_eff
+// largest scores, ties to the lower index, written in ascending key order.
+// Requires 1 <= bsa <= T and T <= topk_max_T().
+int64_t topk_max_T();
+cudaError_t launch_topk(const float* S_agg, int b, int nkv, int64_t T, int bsa,
+                        int32_t* kv_idx, int32_t* kv_count, cudaStream_t stream);
+
+// Step (f): standalone gather of the selected K and V rows.
+cudaError_t launch_gather(bool bf16, int d, Strided K, Strided V, int b, int nkv, int64_t T,
+                          const int32_t* kv_idx, const int32_t* kv_count, int bsa,
+                          void* Ksel, void* Vsel, int* status, cudaStream_t stream);
+
+struct AttnArgs {
+  Strided Q, K, V, Kc, Vc;
+  int b, nq, nkv, d, BCP;
+  int64_t T;
+  const int32_t* kv_idx;    // (b, nkv, bsa)
+  const int32_t* kv_count;  // (b, nkv)
+  int bsa;
+  float scale;
+  void* O;                  // (b, nq, BCP, d) contiguous, dtype of Q
+  float* lse;               // (b, nq, BCP) or null
+  int* status;
+};
+
+// Steps (f)+(g) in fp32 on the CUDA cores (any input dtype).
+cudaError_t launch_attn_simt(bool bf16, const AttnArgs& a, cudaStream_t stream);
+
+// Steps (f)+(g) on the tcgen05 tensor cores (bf16 only).
+// Returns cudaErrorNotSupported when the shape has no tensor-core variant.
+cudaError_t launch_attn_tc(const AttnArgs& a, cudaStream_t stream);
+
+}  // namespace quoka

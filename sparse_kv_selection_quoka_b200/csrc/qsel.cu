@@ -1,0 +1,168 @@
+// Query subselection and GQA group mean.
+//
+// [QUOKA §2.1, Algorithm 1] MQ = mean of the chunk's queries over its tokens;
+// SQ = -cos(Q, MQ); the NQ queries with the largest SQ are kept, in rank
+// order. [QUOKA §2.3] the kept queries are L2-normalised and averaged over
+// the G query heads of each KV head, rank by rank.
+//
+// (QUOKA = the technical write-up "QUOKA: how it reshapes LLM prefill
+// efficiency", bqwf.cn news item 915859; § numbers are the write-up's.)
+#include "common.cuh"
+#include "kernels.h"
+
+namespace quoka {
+
+constexpr int QSEL_THREADS = 256;
+constexpr int QSEL_WARPS = QSEL_THREADS / 32;
+
+// One CTA per (query head, batch). Dynamic shared memory: SQ[BCP] floats
+// followed by the rank -> position table sel[NQ].
+template <typename T, int D>
+__global__ void __launch_bounds__(QSEL_THREADS)
+qsel_kernel(const T* __restrict__ Q, int64_t sQb, int64_t sQh, int64_t sQt, int BCP, int NQ,
+            float* __restrict__ Qhat, int32_t* __restrict__ q_idx) {
+  extern __shared__ float smem[];
+  float* SQ = smem;
+  int* sel = reinterpret_cast<int*>(smem + BCP);
+  __shared__ float part[QSEL_THREADS];
+  __shared__ float mq[D];
+  __shared__ float mq_norm;
+
+  const int h = blockIdx.x, bi = blockIdx.y, nq = gridDim.x;
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  const T* Qh = Q + bi * sQb + h * sQh;
+
+  // (a) mean over the chunk's tokens: column c = tid % D, token groups of
+  // QSEL_THREADS / D rows; partial sums combined in a fixed order.
+  constexpr int NGRP = QSEL_THREADS / D;
+  {
+    const int c = tid % D, grp = tid / D;
+    float acc = 0.f;
+    for (int t = grp; t < BCP; t += NGRP) acc += to_f32(Qh[(int64_t)t * sQt + c]);
+    part[tid] = acc;
+  }
+  for (int i = tid; i < NQ; i += QSEL_THREADS) sel[i] = 0;
+  __syncthreads();
+  if (tid < D) {
+    float s = 0.f;
+#pragma unroll
+    for (int g = 0; g < NGRP; ++g) s += part[g * D + tid];
+    mq[tid] = s / (float)BCP;
+  }
+  __syncthreads();
+  if (warp == 0) {
+    float s = 0.f;
+    for (int k = lane; k < D; k += 32) s += mq[k] * mq[k];
+    s = warp_sum(s);
+    if (lane == 0) mq_norm = sqrtf(s);
+  }
+  __syncthreads();
+
+  // (a) SQ[t] = -(q_t . MQ) / max(|q_t| |MQ|, 1e-8), one warp per token.
+  for (int t = warp; t < BCP; t += QSEL_WARPS) {
+    const T* q = Qh + (int64_t)t * sQt;
+    float dot = 0.f, qq = 0.f;
+#pragma unroll
+    for (int k = lane; k < D; k += 32) {
+      float v = to_f32(q[k]);
+      dot += v * mq[k];
+      qq += v * v;
+    }
+    dot = warp_sum(dot);
+    qq = warp_sum(qq);
+    if (lane == 0) SQ[t] = -dot / fmaxf(sqrtf(qq) * mq_norm, 1e-8f);
+  }
+  __syncthreads();
+
+  // (b) rank of token t = number of tokens that beat it (larger SQ, or equal
+  // SQ at a lower position); ranks below NQ are kept.
+  for (int t = tid; t < BCP; t += QSEL_THREADS) {
+    const float v = SQ[t];
+    int r = 0;
+    for (int u = 0; u < BCP; ++u) {
+      const float w = SQ[u];
+      r += (w > v) | ((w == v) & (u < t));
+    }
+    if (r < NQ) sel[r] = t;
+  }
+  __syncthreads();
+
+  // (c) L2-normalise the kept queries: one warp per rank.
+  for (int i = warp; i < NQ; i += QSEL_WARPS) {
+    const int t = sel[i];
+    const T* q = Qh + (int64_t)t * sQt;
+    float v[D / 32];
+    float qq = 0.f;
+#pragma unroll
+    for (int k = 0; k < D / 32; ++k) {
+      v[k] = to_f32(q[lane + 32 * k]);
+      qq += v[k] * v[k];
+    }
+    qq = warp_sum(qq);
+    const float nrm = fmaxf(sqrtf(qq), 1e-12f);
+    float* dst = Qhat + (((int64_t)bi * nq + h) * NQ + i) * D;
+#pragma unroll
+    for (int k = 0; k < D / 32; ++k) dst[lane + 32 * k] = v[k] / nrm;
+    if (lane == 0 && q_idx != nullptr) q_idx[((int64_t)bi * nq + h) * NQ + i] = t;
+  }
+}
+
+// Q_group[b, j, i, :] = (1/G) sum_{g<G} Qhat[b, jG+g, i, :], summed in head
+// order; optionally split into bf16 hi = rn(x) and lo = rn(x - hi).
+template <int D>
+__global__ void __launch_bounds__(D)
+qgroup_kernel(const float* __restrict__ Qhat, int nq, int NQ, float* __restrict__ Qg,
+              bf16* __restrict__ Qg_hilo) {
+  const int i = blockIdx.x, j = blockIdx.y, bi = blockIdx.z, nkv = gridDim.y;
+  const int G = nq / nkv;
+  const int k = threadIdx.x;
+  float acc = 0.f;
+  for (int g = 0; g < G; ++g) acc += Qhat[(((int64_t)bi * nq + j * G + g) * NQ + i) * D + k];
+  const float v = acc / (float)G;
+  const int64_t row = (int64_t)bi * nkv + j;
+  Qg[(row * NQ + i) * D + k] = v;
+  if (Qg_hilo != nullptr) {
+    const bf16 hi = __float2bfloat16_rn(v);
+    const bf16 lo = __float2bfloat16_rn(v - __bfloat162float(hi));
+    Qg_hilo[(row * 2 * NQ + i) * D + k] = hi;
+    Qg_hilo[(row * 2 * NQ + NQ + i) * D + k] = lo;
+  }
+}
+
+template <typename T, int D>
+static cudaError_t qsel_typed(Strided Q, int b, int nq, int BCP, int NQ, float* Qhat,
+                              int32_t* q_idx, cudaStream_t stream) {
+  const size_t smem = (size_t)BCP * sizeof(float) + (size_t)NQ * sizeof(int);
+  auto kern = qsel_kernel<T, D>;
+  if (smem > 48 * 1024) {
+    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    if (e != cudaSuccess) return e;
+  }
+  kern<<<dim3(nq, b), QSEL_THREADS, smem, stream>>>(static_cast<const T*>(Q.data), Q.sb, Q.sh, Q.st,
+                                                    BCP, NQ, Qhat, q_idx);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_qsel(bool is_bf16, int d, Strided Q, int b, int nq, int BCP, int NQ,
+                        float* Qhat, int32_t* q_idx, cudaStream_t stream) {
+  if (is_bf16) {
+    if (d == 128) return qsel_typed<bf16, 128>(Q, b, nq, BCP, NQ, Qhat, q_idx, stream);
+    if (d == 64) return qsel_typed<bf16, 64>(Q, b, nq, BCP, NQ, Qhat, q_idx, stream);
+  } else {
+    if (d == 128) return qsel_typed<float, 128>(Q, b, nq, BCP, NQ, Qhat, q_idx, stream);
+    if (d == 64) return qsel_typed<float, 64>(Q, b, nq, BCP, NQ, Qhat, q_idx, stream);
+  }
+  return cudaErrorNotSupported;
+}
+
+cudaError_t launch_qgroup(int d, const float* Qhat, int b, int nq, int nkv, int NQ, float* Qg,
+                          uint16_t* Qg_hilo, cudaStream_t stream) {
+  dim3 grid(NQ, nkv, b);
+  bf16* hl = reinterpret_cast<bf16*>(Qg_hilo);
+  if (d == 128) qgroup_kernel<128><<<grid, 128, 0, stream>>>(Qhat, nq, NQ, Qg, hl);
+  else if (d == 64) qgroup_kernel<64><<<grid, 64, 0, stream>>>(Qhat, nq, NQ, Qg, hl);
+  else return cudaErrorNotSupported;
+  return cudaGetLastError();
+}
+
+}  // namespace quoka

@@ -1,0 +1,356 @@
+// C ABI of libquoka.so: argument validation, workspace carving and the launch
+// sequence of the QUOKA step. See include/quoka.h for the contract of every
+// entry point.
+#include <cuda_runtime.h>
+#include <stdint.h>
+#include <string.h>
+
+#include <algorithm>
+
+#include "kernels.h"
+#include "quoka.h"
+
+namespace {
+
+using quoka::Strided;
+
+constexpr size_t kAlign = 256;
+
+size_t align_up(size_t x) { return (x + kAlign - 1) / kAlign * kAlign; }
+
+// Workspace layout. Every region starts on a 256-byte boundary.
+struct WsLayout {
+  size_t status = 0;    // int32 device status word
+  size_t qhat = 0;      // (b, nq, NQ, d) fp32: normalised chosen queries
+  size_t qgroup = 0;    // (b, nkv, NQ, d) fp32: group means
+  size_t qhilo = 0;     // (b, nkv, 2*NQ, d) bf16: hi / lo split of the group means
+  size_t qidx = 0;      // (b, nq, NQ) int32
+  size_t sagg = 0;      // (b, nkv, T) fp32
+  size_t kvidx = 0;     // (b, nkv, BSA_eff) int32
+  size_t kvcount = 0;   // (b, nkv) int32
+  size_t total = 0;
+};
+
+WsLayout ws_layout(int64_t b, int64_t nq, int64_t nkv, int64_t d, int64_t T, int64_t NQ,
+                   int64_t bsa_eff) {
+  WsLayout L;
+  size_t off = 0;
+  auto take = [&](size_t bytes) {
+    const size_t at = off;
+    off += align_up(bytes);
+    return at;
+  };
+  L.status = take(kAlign);
+  L.qhat = take((size_t)(b * nq * NQ * d) * 4);
+  L.qgroup = take((size_t)(b * nkv * NQ * d) * 4);
+  L.qhilo = take((size_t)(b * nkv * 2 * NQ * d) * 2);
+  L.qidx = take((size_t)(b * nq * NQ) * 4);
+  L.sagg = take((size_t)(b * nkv * T) * 4);
+  L.kvidx = take((size_t)(b * nkv * bsa_eff) * 4);
+  L.kvcount = take((size_t)(b * nkv) * 4);
+  L.total = off;
+  return L;
+}
+
+size_t elt_size(quoka_dtype t) { return t == QUOKA_BF16 ? 2 : 4; }
+
+bool aligned16(const void* p) { return ((uintptr_t)p & 15u) == 0; }
+
+// Checks a tensor's dtype, shape and strides. Extents equal to -1 in `want`
+// are free and returned through `want`.
+bool check_tensor(const quoka_tensor* t, quoka_dtype dtype, int64_t want[4]) {
+  if (t == nullptr) return false;
+  if (t->dtype != dtype) return false;
+  for (int i = 0; i < 4; ++i) {
+    if (t->shape[i] < 0) return false;
+    if (want[i] >= 0 && t->shape[i] != want[i]) return false;
+    want[i] = t->shape[i];
+  }
+  if (t->stride[3] != 1) return false;
+  const int64_t es = (int64_t)elt_size(dtype);
+  for (int i = 0; i < 3; ++i) {
+    if (t->stride[i] < 0) return false;
+    if ((t->stride[i] * es) % 16 != 0) return false;
+  }
+  int64_t n = 1;
+  for (int i = 0; i < 4; ++i) n *= t->shape[i];
+  if (n > 0 && (t->data == nullptr || !aligned16(t->data))) return false;
+  return true;
+}
+
+Strided strided(const quoka_tensor* t) {
+  return Strided{t->data, t->stride[0], t->stride[1], t->stride[2]};
+}
+
+bool supported_d(int64_t d) { return d == 64 || d == 128; }
+
+constexpr int64_t kMaxBCP = 16384;
+constexpr int64_t kMaxHeads = 65535;
+
+quoka_status cuda_status(cudaError_t e) {
+  if (e == cudaSuccess) return QUOKA_OK;
+  if (e == cudaErrorNotSupported) return QUOKA_ERR_UNSUPPORTED;
+  return QUOKA_ERR_CUDA;
+}
+
+struct SelectShapes {
+  int64_t b, nq, nkv, d, T, BCP;
+};
+
+quoka_status validate_select(const quoka_tensor* Q, const quoka_tensor* K, int NQ, int BSA,
+                             SelectShapes* s) {
+  if (Q == nullptr || K == nullptr) return QUOKA_ERR_INVALID_ARG;
+  int64_t qs[4] = {-1, -1, -1, -1};
+  if (!check_tensor(Q, Q->dtype, qs)) return QUOKA_ERR_INVALID_ARG;
+  if (Q->dtype != QUOKA_F32 && Q->dtype != QUOKA_BF16) return QUOKA_ERR_INVALID_ARG;
+  int64_t ks[4] = {qs[0], -1, -1, qs[3]};
+  if (!check_tensor(K, Q->dtype, ks)) return QUOKA_ERR_INVALID_ARG;
+  s->b = qs[0];
+  s->nq = qs[1];
+  s->BCP = qs[2];
+  s->d = qs[3];
+  s->nkv = ks[1];
+  s->T = ks[2];
+  if (s->b < 1 || s->nq < 1 || s->nkv < 1 || s->BCP < 1) return QUOKA_ERR_INVALID_ARG;
+  if (s->nq % s->nkv != 0) return QUOKA_ERR_INVALID_ARG;
+  if (NQ < 1 || NQ > s->BCP || BSA < 0) return QUOKA_ERR_INVALID_ARG;
+  if (!supported_d(s->d)) return QUOKA_ERR_UNSUPPORTED;
+  if (s->BCP > kMaxBCP || s->nq > kMaxHeads || s->nkv > kMaxHeads || s->b > kMaxHeads)
+    return QUOKA_ERR_UNSUPPORTED;
+  if (s->T > quoka::topk_max_T()) return QUOKA_ERR_UNSUPPORTED;
+  return QUOKA_OK;
+}
+
+quoka_status check_ws(void* ws, size_t ws_bytes, const WsLayout& L) {
+  if (ws == nullptr || ((uintptr_t)ws % kAlign) != 0 || ws_bytes < L.total) return QUOKA_ERR_WORKSPACE;
+  return QUOKA_OK;
+}
+
+template <typename P>
+P* at(void* ws, size_t off) {
+  return reinterpret_cast<P*>(static_cast<char*>(ws) + off);
+}
+
+// Steps (a)-(e) after validation. kv_idx / kv_count / q_idx / s_agg are the
+// final destinations (workspace regions when the caller passed none).
+quoka_status run_select(const quoka_tensor* Q, const quoka_tensor* K, const SelectShapes& s, int NQ,
+                        int bsa_eff, int32_t* kv_idx, int32_t* kv_count, int32_t* q_idx,
+                        float* s_agg, void* ws, const WsLayout& L, cudaStream_t stream) {
+  const bool bf = Q->dtype == QUOKA_BF16;
+  const int b = (int)s.b, nq = (int)s.nq, nkv = (int)s.nkv, d = (int)s.d, BCP = (int)s.BCP;
+  float* qhat = at<float>(ws, L.qhat);
+  float* qg = at<float>(ws, L.qgroup);
+  uint16_t* qhilo = at<uint16_t>(ws, L.qhilo);
+  int32_t* qidx = q_idx != nullptr ? q_idx : at<int32_t>(ws, L.qidx);
+  float* sagg = s_agg != nullptr ? s_agg : at<float>(ws, L.sagg);
+  int* status = at<int>(ws, L.status);
+
+  cudaError_t e = quoka::launch_qsel(bf, d, strided(Q), b, nq, BCP, NQ, qhat, qidx, stream);
+  if (e != cudaSuccess) return cuda_status(e);
+  e = quoka::launch_qgroup(d, qhat, b, nq, nkv, NQ, qg, bf ? qhilo : nullptr, stream);
+  if (e != cudaSuccess) return cuda_status(e);
+  if (s.T > 0) {
+    e = cudaErrorNotSupported;
+    if (bf) e = quoka::launch_score_tc(d, strided(K), b, nkv, s.T, qhilo, NQ, sagg, status, stream);
+    if (e == cudaErrorNotSupported)
+      e = quoka::launch_score_simt(bf, d, strided(K), b, nkv, s.T, qg, NQ, sagg, stream);
+    if (e != cudaSuccess) return cuda_status(e);
+  }
+  if (bsa_eff > 0) {
+    e = quoka::launch_topk(sagg, b, nkv, s.T, bsa_eff, kv_idx, kv_count, stream);
+    if (e != cudaSuccess) return cuda_status(e);
+  } else {
+    e = cudaMemsetAsync(kv_count, 0, sizeof(int32_t) * b * nkv, stream);
+    if (e != cudaSuccess) return QUOKA_ERR_CUDA;
+  }
+  return QUOKA_OK;
+}
+
+struct AttnShapes {
+  int64_t b, nq, nkv, d, T, BCP;
+};
+
+quoka_status validate_attn(const quoka_tensor* Q, const quoka_tensor* K, const quoka_tensor* V,
+                           const quoka_tensor* Kc, const quoka_tensor* Vc, AttnShapes* s) {
+  if (Q == nullptr || K == nullptr || V == nullptr || Kc == nullptr || Vc == nullptr)
+    return QUOKA_ERR_INVALID_ARG;
+  int64_t qs[4] = {-1, -1, -1, -1};
+  if (!check_tensor(Q, Q->dtype, qs)) return QUOKA_ERR_INVALID_ARG;
+  if (Q->dtype != QUOKA_F32 && Q->dtype != QUOKA_BF16) return QUOKA_ERR_INVALID_ARG;
+  int64_t ks[4] = {qs[0], -1, -1, qs[3]};
+  if (!check_tensor(K, Q->dtype, ks)) return QUOKA_ERR_INVALID_ARG;
+  int64_t vs[4] = {ks[0], ks[1], ks[2], ks[3]};
+  if (!check_tensor(V, Q->dtype, vs)) return QUOKA_ERR_INVALID_ARG;
+  int64_t kcs[4] = {qs[0], ks[1], qs[2], qs[3]};
+  if (!check_tensor(Kc, Q->dtype, kcs)) return QUOKA_ERR_INVALID_ARG;
+  int64_t vcs[4] = {qs[0], ks[1], qs[2], qs[3]};
+  if (!check_tensor(Vc, Q->dtype, vcs)) return QUOKA_ERR_INVALID_ARG;
+  s->b = qs[0];
+  s->nq = qs[1];
+  s->BCP = qs[2];
+  s->d = qs[3];
+  s->nkv = ks[1];
+  s->T = ks[2];
+  if (s->b < 1 || s->nq < 1 || s->nkv < 1 || s->BCP < 1) return QUOKA_ERR_INVALID_ARG;
+  if (s->nq % s->nkv != 0) return QUOKA_ERR_INVALID_ARG;
+  if (!supported_d(s->d)) return QUOKA_ERR_UNSUPPORTED;
+  if (s->BCP > kMaxBCP || s->nq > kMaxHeads || s->nkv > kMaxHeads || s->b > kMaxHeads)
+    return QUOKA_ERR_UNSUPPORTED;
+  if (s->T > (int64_t)INT32_MAX) return QUOKA_ERR_UNSUPPORTED;
+  return QUOKA_OK;
+}
+
+quoka_status run_attn(const quoka_tensor* Q, const quoka_tensor* K, const quoka_tensor* V,
+                      const quoka_tensor* Kc, const quoka_tensor* Vc, const AttnShapes& s,
+                      const int32_t* kv_idx, const int32_t* kv_count, int bsa_eff, float scale,
+                      void* O, float* lse, int* status, cudaStream_t stream) {
+  quoka::AttnArgs a;
+  a.Q = strided(Q);
+  a.K = strided(K);
+  a.V = strided(V);
+  a.Kc = strided(Kc);
+  a.Vc = strided(Vc);
+  a.b = (int)s.b;
+  a.nq = (int)s.nq;
+  a.nkv = (int)s.nkv;
+  a.d = (int)s.d;
+  a.BCP = (int)s.BCP;
+  a.T = s.T;
+  a.kv_idx = kv_idx;
+  a.kv_count = kv_count;
+  a.bsa = bsa_eff;
+  a.scale = scale;
+  a.O = O;
+  a.lse = lse;
+  a.status = status;
+  cudaError_t e = cudaErrorNotSupported;
+  if (Q->dtype == QUOKA_BF16) e = quoka::launch_attn_tc(a, stream);
+  if (e == cudaErrorNotSupported) e = quoka::launch_attn_simt(Q->dtype == QUOKA_BF16, a, stream);
+  return cuda_status(e);
+}
+
+}  // namespace
+
+extern "C" {
+
+size_t quoka_workspace_size(int b, int nq, int nkv, int d, int64_t T, int BCP, int NQ, int BSA,
+                            quoka_dtype dtype) {
+  if (b < 1 || nq < 1 || nkv < 1 || d < 1 || T < 0 || BCP < 1 || NQ < 1 || BSA < 0) return 0;
+  if (nq % nkv != 0 || (dtype != QUOKA_F32 && dtype != QUOKA_BF16)) return 0;
+  const int64_t bsa_eff = std::min<int64_t>(BSA, T);
+  return ws_layout(b, nq, nkv, d, T, NQ, bsa_eff).total;
+}
+
+quoka_status quoka_select(const quoka_tensor* Q, const quoka_tensor* K, int NQ, int BSA,
+                          int32_t* kv_idx, int32_t* kv_count, int32_t* q_idx, float* s_agg,
+                          void* ws, size_t ws_bytes, void* stream) {
+  SelectShapes s;
+  quoka_status st = validate_select(Q, K, NQ, BSA, &s);
+  if (st != QUOKA_OK) return st;
+  const int64_t bsa_eff = std::min<int64_t>(BSA, s.T);
+  if (kv_count == nullptr || (bsa_eff > 0 && kv_idx == nullptr)) return QUOKA_ERR_INVALID_ARG;
+  const WsLayout L = ws_layout(s.b, s.nq, s.nkv, s.d, s.T, NQ, bsa_eff);
+  st = check_ws(ws, ws_bytes, L);
+  if (st != QUOKA_OK) return st;
+  cudaStream_t cs = static_cast<cudaStream_t>(stream);
+  if (cudaMemsetAsync(at<int>(ws, L.status), 0, sizeof(int), cs) != cudaSuccess) return QUOKA_ERR_CUDA;
+  return run_select(Q, K, s, NQ, (int)bsa_eff, kv_idx, kv_count, q_idx, s_agg, ws, L, cs);
+}
+
+quoka_status quoka_gather_kv(const quoka_tensor* K, const quoka_tensor* V, const int32_t* kv_idx,
+                             const int32_t* kv_count, int BSA_eff, void* Ksel, void* Vsel,
+                             void* ws, size_t ws_bytes, void* stream) {
+  if (K == nullptr || V == nullptr || kv_count == nullptr || BSA_eff < 0) return QUOKA_ERR_INVALID_ARG;
+  int64_t ks[4] = {-1, -1, -1, -1};
+  if (!check_tensor(K, K->dtype, ks)) return QUOKA_ERR_INVALID_ARG;
+  if (K->dtype != QUOKA_F32 && K->dtype != QUOKA_BF16) return QUOKA_ERR_INVALID_ARG;
+  int64_t vs[4] = {ks[0], ks[1], ks[2], ks[3]};
+  if (!check_tensor(V, K->dtype, vs)) return QUOKA_ERR_INVALID_ARG;
+  if (!supported_d(ks[3])) return QUOKA_ERR_UNSUPPORTED;
+  if (ks[0] < 1 || ks[1] < 1 || ks[0] > kMaxHeads || ks[1] > kMaxHeads) return QUOKA_ERR_INVALID_ARG;
+  if (BSA_eff > 0 && (kv_idx == nullptr || Ksel == nullptr || Vsel == nullptr || !aligned16(Ksel) ||
+                      !aligned16(Vsel)))
+    return QUOKA_ERR_INVALID_ARG;
+  cudaStream_t cs = static_cast<cudaStream_t>(stream);
+  int* status = nullptr;
+  if (ws != nullptr) {
+    if (((uintptr_t)ws % kAlign) != 0 || ws_bytes < sizeof(int)) return QUOKA_ERR_WORKSPACE;
+    status = static_cast<int*>(ws);
+    if (cudaMemsetAsync(status, 0, sizeof(int), cs) != cudaSuccess) return QUOKA_ERR_CUDA;
+  }
+  cudaError_t e = quoka::launch_gather(K->dtype == QUOKA_BF16, (int)ks[3], strided(K), strided(V),
+                                       (int)ks[0], (int)ks[1], ks[2], kv_idx, kv_count, BSA_eff, Ksel,
+                                       Vsel, status, cs);
+  return cuda_status(e);
+}
+
+quoka_status quoka_sparse_gqa_attn(const quoka_tensor* Q, const quoka_tensor* K,
+                                   const quoka_tensor* V, const int32_t* kv_idx,
+                                   const int32_t* kv_count, int BSA_eff, const quoka_tensor* Kc,
+                                   const quoka_tensor* Vc, float scale, void* O, float* lse,
+                                   void* ws, size_t ws_bytes, void* stream) {
+  AttnShapes s;
+  quoka_status st = validate_attn(Q, K, V, Kc, Vc, &s);
+  if (st != QUOKA_OK) return st;
+  if (BSA_eff < 0 || kv_count == nullptr || (BSA_eff > 0 && kv_idx == nullptr)) return QUOKA_ERR_INVALID_ARG;
+  if (O == nullptr || !aligned16(O)) return QUOKA_ERR_INVALID_ARG;
+  if (!(scale > 0.f) || scale != scale) return QUOKA_ERR_INVALID_ARG;
+  if (ws == nullptr || ((uintptr_t)ws % kAlign) != 0 || ws_bytes < kAlign) return QUOKA_ERR_WORKSPACE;
+  cudaStream_t cs = static_cast<cudaStream_t>(stream);
+  int* status = static_cast<int*>(ws);
+  if (cudaMemsetAsync(status, 0, sizeof(int), cs) != cudaSuccess) return QUOKA_ERR_CUDA;
+  return run_attn(Q, K, V, Kc, Vc, s, kv_idx, kv_count, BSA_eff, scale, O, lse, status, cs);
+}
+
+quoka_status quoka_prefill_chunk(const quoka_tensor* Q, const quoka_tensor* K,
+                                 const quoka_tensor* V, const quoka_tensor* Kc,
+                                 const quoka_tensor* Vc, int NQ, int BSA, float scale, void* O,
+                                 float* lse, int32_t* kv_idx_out, void* ws, size_t ws_bytes,
+                                 void* stream) {
+  AttnShapes as;
+  quoka_status st = validate_attn(Q, K, V, Kc, Vc, &as);
+  if (st != QUOKA_OK) return st;
+  SelectShapes s;
+  st = validate_select(Q, K, NQ, BSA, &s);
+  if (st != QUOKA_OK) return st;
+  if (O == nullptr || !aligned16(O)) return QUOKA_ERR_INVALID_ARG;
+  if (!(scale > 0.f) || scale != scale) return QUOKA_ERR_INVALID_ARG;
+  const int64_t bsa_eff = std::min<int64_t>(BSA, s.T);
+  const WsLayout L = ws_layout(s.b, s.nq, s.nkv, s.d, s.T, NQ, bsa_eff);
+  st = check_ws(ws, ws_bytes, L);
+  if (st != QUOKA_OK) return st;
+  cudaStream_t cs = static_cast<cudaStream_t>(stream);
+  int* status = at<int>(ws, L.status);
+  if (cudaMemsetAsync(status, 0, sizeof(int), cs) != cudaSuccess) return QUOKA_ERR_CUDA;
+  int32_t* kv_idx = kv_idx_out != nullptr ? kv_idx_out : at<int32_t>(ws, L.kvidx);
+  int32_t* kv_count = at<int32_t>(ws, L.kvcount);
+  st = run_select(Q, K, s, NQ, (int)bsa_eff, kv_idx, kv_count, nullptr, nullptr, ws, L, cs);
+  if (st != QUOKA_OK) return st;
+  return run_attn(Q, K, V, Kc, Vc, as, kv_idx, kv_count, (int)bsa_eff, scale, O, lse, status, cs);
+}
+
+quoka_status quoka_get_device_status(const void* ws, void* stream, int32_t* device_status) {
+  if (ws == nullptr || device_status == nullptr) return QUOKA_ERR_INVALID_ARG;
+  cudaStream_t cs = static_cast<cudaStream_t>(stream);
+  int32_t v = 0;
+  if (cudaMemcpyAsync(&v, ws, sizeof(int32_t), cudaMemcpyDeviceToHost, cs) != cudaSuccess)
+    return QUOKA_ERR_CUDA;
+  if (cudaStreamSynchronize(cs) != cudaSuccess) return QUOKA_ERR_CUDA;
+  *device_status = v;
+  return QUOKA_OK;
+}
+
+const char* quoka_status_string(quoka_status status) {
+  switch (status) {
+    case QUOKA_OK: return "QUOKA_OK";
+    case QUOKA_ERR_INVALID_ARG: return "QUOKA_ERR_INVALID_ARG";
+    case QUOKA_ERR_UNSUPPORTED: return "QUOKA_ERR_UNSUPPORTED";
+    case QUOKA_ERR_WORKSPACE: return "QUOKA_ERR_WORKSPACE";
+    case QUOKA_ERR_CUDA: return "QUOKA_ERR_CUDA";
+    case QUOKA_ERR_TIMEOUT: return "QUOKA_ERR_TIMEOUT";
+    case QUOKA_ERR_BOUNDS: return "QUOKA_ERR_BOUNDS";
+  }
+  return "QUOKA_ERR_UNKNOWN";
+}
+
+}  // extern "C"

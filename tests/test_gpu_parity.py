@@ -1,0 +1,249 @@
+"""CUDA path vs the CPU oracle, element by element, on seeded inputs.
+
+Every call goes through the C ABI of libquoka.so (via the ctypes binding).
+Small shapes span several tiles and ragged tails and cover the degenerate
+cases (T = 0, BSA = 0, BSA >= T, NQ = 1, NQ = BCP, G = 1, d = 64, batch > 1);
+the full-size workloads are checked in the launch configuration the
+benchmark times, on every output the oracle can afford and on sampled rows
+otherwise.
+"""
+import numpy as np
+import pytest
+import torch
+
+from oracle import quoka_oracle as orc
+from sparse_kv_selection_quoka_b200 import inputs
+from tests import parity as P
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.fixture(scope="module", autouse=True)
+def _lib():
+    if not torch.cuda.is_available():
+        pytest.skip("no CUDA device")
+    import sparse_kv_selection_quoka_b200 as q
+    q.load()
+    return q
+
+
+def q():
+    import sparse_kv_selection_quoka_b200 as m
+    return m
+
+
+def run_select_and_check(x: inputs.ChunkInputs, dev=None):
+    """quoka_select vs the oracle; returns (oracle result on the GPU's query
+    choice, GPU kv_idx, GPU kv_count). `dev` optionally supplies the device
+    tensors (Q, K, V, Kc, Vc), e.g. strided views into one cache."""
+    dt = x.dtype
+    Q, K = (P.to_dev(x.Q, dt), P.to_dev(x.K, dt)) if dev is None else (dev[0], dev[1])
+    kv_idx, kv_count, q_idx, s_agg = q().quoka_select(Q, K, x.NQ, x.BSA, want_q_idx=True,
+                                                      want_s_agg=True)
+    ws = q().workspace_for(Q, K, x.NQ, x.BSA)
+    q().quoka_select(Q, K, x.NQ, x.BSA, ws=ws)
+    assert q().quoka_get_device_status(ws) == 0
+    torch.cuda.synchronize()
+    ref = orc.select(x.Q, x.K, x.NQ, x.BSA)
+    gq = q_idx.cpu().numpy().astype(np.int64)
+    if not P.check_q_idx(gq, ref["SQ"], ref["q_idx"]):
+        ref = orc.select(x.Q, x.K, x.NQ, x.BSA, override_q_idx=gq)
+    T = x.K.shape[2]
+    if T > 0:
+        err = np.abs(s_agg.cpu().numpy().astype(np.float64) - ref["S_agg"]).max()
+        assert err <= P.S_TOL, f"S_agg max-abs error {err:.3e}"
+    bsa_eff = min(x.BSA, T)
+    gi = kv_idx.cpu().numpy().astype(np.int64)
+    gc = kv_count.cpu().numpy()
+    assert gi.shape == (x.K.shape[0], x.K.shape[1], bsa_eff)
+    P.check_kv_sets(gi, gc, ref["S_agg"], bsa_eff, ref["sel"])
+    return ref, gi, gc
+
+
+def run_prefill_and_check(x: inputs.ChunkInputs, ref, gi, rows=None, dev=None):
+    dt = x.dtype
+    if dev is None:
+        dev = [P.to_dev(a, dt) for a in (x.Q, x.K, x.V, x.Kc, x.Vc)]
+    Q, K, V, Kc, Vc = dev
+    O, lse, kv_idx = q().quoka_prefill_chunk(Q, K, V, Kc, Vc, x.NQ, x.BSA, want_lse=True,
+                                             want_kv_idx=True)
+    torch.cuda.synchronize()
+    # the whole step selects the same set as quoka_select (deterministic)
+    np.testing.assert_array_equal(kv_idx.cpu().numpy(), gi)
+    Og = O.float().cpu().numpy().astype(np.float64)
+    Lg = lse.cpu().numpy().astype(np.float64)
+    tol = P.o_tol(dt)
+    if rows is None:
+        O_ref, L_ref = orc.sparse_attention(x.Q, x.K, x.V, gi, x.Kc, x.Vc)
+        err = np.abs(Og - O_ref).max()
+        lerr = np.abs(Lg - L_ref).max()
+    else:
+        O_ref, L_ref = orc.sparse_attention_rows(x.Q, x.K, x.V, gi, x.Kc, x.Vc, rows)
+        Os = np.stack([Og[r] for r in rows])
+        Ls = np.array([Lg[r] for r in rows])
+        err = np.abs(Os - O_ref).max()
+        lerr = np.abs(Ls - L_ref).max()
+    assert err <= tol, f"O max-abs error {err:.3e} > {tol}"
+    assert lerr <= max(P.LSE_TOL, tol), f"LSE max-abs error {lerr:.3e}"
+    return O
+
+
+SMALL = [
+    # b, nq, nkv, d, T, BCP, NQ, BSA, dtype, structure
+    (2, 6, 2, 128, 1000, 100, 7, 300, "bf16", "llama"),
+    (1, 8, 8, 64, 333, 37, 37, 50, "bf16", "iid"),
+    (1, 3, 1, 128, 0, 64, 4, 16, "bf16", "iid"),
+    (1, 4, 1, 128, 200, 64, 1, 500, "f32", "iid"),
+    (2, 16, 2, 128, 4096, 256, 16, 1024, "bf16", "qwen"),
+    (1, 4, 2, 128, 5000, 16, 16, 0, "bf16", "iid"),
+    (1, 2, 2, 64, 40000, 48, 3, 4000, "bf16", "iid"),
+    (1, 6, 3, 64, 777, 130, 9, 129, "f32", "llama"),
+    (3, 4, 4, 128, 129, 1, 1, 128, "bf16", "iid"),
+]
+
+
+@pytest.mark.parametrize("k", range(len(SMALL)), ids=[f"b{c[0]}_nq{c[1]}_nkv{c[2]}_d{c[3]}_T{c[4]}_L{c[5]}_NQ{c[6]}_BSA{c[7]}_{c[8]}" for c in SMALL])
+def test_small_shapes(k):
+    b, nq, nkv, d, T, BCP, NQ, BSA, dt, st = SMALL[k]
+    x = inputs.make_chunk(b, nq, nkv, d, T, BCP, NQ, BSA, dtype=dt, structure=st, seed=500 + k)
+    ref, gi, _ = run_select_and_check(x)
+    run_prefill_and_check(x, ref, gi)
+
+
+def test_tiny_fp32_workload():
+    x = inputs.make_workload(0)
+    ref, gi, _ = run_select_and_check(x)
+    run_prefill_and_check(x, ref, gi)
+
+
+def test_llama_workload():
+    x = inputs.make_workload(1)
+    ref, gi, _ = run_select_and_check(x)
+    run_prefill_and_check(x, ref, gi)
+
+
+def test_qwen_workload_T32k():
+    x = inputs.make_workload(2)
+    ref, gi, _ = run_select_and_check(x)
+    run_prefill_and_check(x, ref, gi)
+
+
+def test_long_workload_T128k():
+    x = inputs.make_workload(4)
+    ref, gi, _ = run_select_and_check(x)
+    r = np.random.default_rng(0)
+    nq, L = x.Q.shape[1], x.Q.shape[2]
+    rows = [(0, int(h), int(t)) for h, t in zip(r.integers(0, nq, 48), r.integers(0, L, 48))]
+    rows += [(0, 0, 0), (0, nq - 1, L - 1), (0, 5, 127), (0, 63, 128)]
+    run_prefill_and_check(x, ref, gi, rows=rows)
+
+
+@pytest.fixture(scope="module")
+def sweep():
+    s = inputs.make_sweep()
+    dev = [P.to_dev(a, s.dtype) for a in (s.Qs, s.Ks, s.Vs)]
+    return s, dev
+
+
+@pytest.mark.parametrize("c", [0, 1, 7, 40, 63])
+def test_sweep_chunks(c, sweep):
+    """Chunk c of the chunked-prefill sweep, called on strided views into one
+    (b, nkv, 16384, d) cache as the benchmark does."""
+    s, (Qs, Ks, Vs) = sweep
+    x = s.chunk(c)
+    L, T = s.BCP, c * s.BCP
+    dev = [Qs[:, :, T:T + L], Ks[:, :, :T], Vs[:, :, :T], Ks[:, :, T:T + L], Vs[:, :, T:T + L]]
+    ref, gi, _ = run_select_and_check(x, dev=dev)
+    r = np.random.default_rng(c)
+    b, nq = x.Q.shape[:2]
+    rows = [(int(bi), int(h), int(t)) for bi, h, t in zip(r.integers(0, b, 24), r.integers(0, nq, 24),
+                                                           r.integers(0, L, 24))]
+    run_prefill_and_check(x, ref, gi, rows=rows, dev=dev)
+
+
+def test_attention_on_given_selection_and_gather():
+    """quoka_sparse_gqa_attn and quoka_gather_kv on an externally given
+    sorted index set (the oracle's), independent of the selection kernels."""
+    x = inputs.make_chunk(2, 8, 2, 128, 3000, 200, 8, 700, dtype="bf16", structure="qwen", seed=5)
+    ref = orc.select(x.Q, x.K, x.NQ, x.BSA)
+    sel = ref["sel"]
+    dt = x.dtype
+    Q, K, V, Kc, Vc = (P.to_dev(a, dt) for a in (x.Q, x.K, x.V, x.Kc, x.Vc))
+    kv_idx = torch.from_numpy(sel.astype(np.int32)).cuda()
+    kv_count = torch.full((2, 2), sel.shape[2], dtype=torch.int32, device="cuda")
+    O, lse = q().quoka_sparse_gqa_attn(Q, K, V, kv_idx, kv_count, Kc, Vc, want_lse=True)
+    Ks, Vs = q().quoka_gather_kv(K, V, kv_idx, kv_count)
+    torch.cuda.synchronize()
+    O_ref, L_ref = orc.sparse_attention(x.Q, x.K, x.V, sel, x.Kc, x.Vc)
+    assert np.abs(O.float().cpu().numpy() - O_ref).max() <= P.O_TOL_BF16
+    assert np.abs(lse.cpu().numpy() - L_ref).max() <= P.O_TOL_BF16
+    Ks_ref, Vs_ref = orc.gather_kv(x.K, x.V, sel)
+    np.testing.assert_array_equal(Ks.float().cpu().numpy(), Ks_ref)
+    np.testing.assert_array_equal(Vs.float().cpu().numpy(), Vs_ref)
+
+
+def test_partial_count_uses_prefix_of_index_rows():
+    """kv_count below the row length: only the first kv_count indices of a
+    row take part (the rest may hold anything)."""
+    x = inputs.make_chunk(1, 4, 2, 64, 500, 40, 4, 100, dtype="f32", structure="iid", seed=6)
+    sel = np.stack([[np.sort(np.random.default_rng(k).choice(500, 100, replace=False)) for k in range(2)]])
+    counts = np.array([[60, 100]], dtype=np.int32)
+    idx = sel.copy()
+    idx[0, 0, 60:] = 10 ** 6  # never read
+    Q, K, V, Kc, Vc = (P.to_dev(a, "f32") for a in (x.Q, x.K, x.V, x.Kc, x.Vc))
+    ws = torch.zeros(256, dtype=torch.uint8, device="cuda")
+    O, _ = q().quoka_sparse_gqa_attn(Q, K, V, torch.from_numpy(idx.astype(np.int32)).cuda(),
+                                     torch.from_numpy(counts).cuda(), Kc, Vc, ws=ws)
+    assert q().quoka_get_device_status(ws) == 0
+    for j, n in enumerate([60, 100]):
+        rows = [(0, h, t) for h in range(2 * j, 2 * j + 2) for t in range(40)]
+        sub = np.zeros((1, 2, n), dtype=np.int64)
+        sub[0, j] = sel[0, j, :n]
+        O_ref, _ = orc.sparse_attention_rows(x.Q, x.K, x.V, sub, x.Kc, x.Vc, rows)
+        Og = O.cpu().numpy()
+        got = np.stack([Og[r] for r in rows])
+        assert np.abs(got - O_ref).max() <= P.O_TOL_F32
+
+
+def test_planted_exact_ties_go_to_lower_index():
+    """Identical key rows get bit-identical scores; at the budget boundary the
+    lower key indices must win, deterministically."""
+    x = inputs.make_chunk(1, 4, 2, 128, 2048, 64, 4, 300, dtype="bf16", structure="iid", seed=7)
+    ref0 = orc.select(x.Q, x.K, x.NQ, x.BSA)
+    for j in range(2):
+        s = ref0["S_agg"][0, j]
+        order = np.argsort(-s, kind="stable")
+        boundary = order[x.BSA - 1]
+        # make 40 other keys identical copies of the boundary key, straddling it
+        others = order[x.BSA - 20:x.BSA + 21]
+        for t in others:
+            x.K[0, j, t] = x.K[0, j, boundary]
+    ref, gi, _ = run_select_and_check(x)
+    for j in range(2):
+        np.testing.assert_array_equal(gi[0, j], ref["sel"][0, j])
+    # deterministic across runs
+    _, gi2, _ = run_select_and_check(x)
+    np.testing.assert_array_equal(gi, gi2)
+
+
+def test_dense_reduction_on_gpu():
+    """NQ = BCP and BSA = T: the CUDA step equals dense causal attention."""
+    x = inputs.make_chunk(1, 8, 2, 128, 700, 96, 96, 700, dtype="bf16", structure="llama", seed=8)
+    ref, gi, _ = run_select_and_check(x)
+    assert np.array_equal(gi[0, 0], np.arange(700))
+    run_prefill_and_check(x, ref, gi)
+
+
+def test_out_of_range_index_is_latched_not_read():
+    x = inputs.make_chunk(1, 2, 1, 64, 100, 8, 2, 10, dtype="f32", structure="iid", seed=9)
+    Q, K, V, Kc, Vc = (P.to_dev(a, "f32") for a in (x.Q, x.K, x.V, x.Kc, x.Vc))
+    idx = torch.tensor([[[1, 5, 99, 100, 2000]]], dtype=torch.int32, device="cuda")
+    cnt = torch.tensor([[5]], dtype=torch.int32, device="cuda")
+    ws = torch.zeros(256, dtype=torch.uint8, device="cuda")
+    q().quoka_sparse_gqa_attn(Q, K, V, idx, cnt, Kc, Vc, ws=ws)
+    assert q().quoka_get_device_status(ws) == 6
+    Ks, Vs = q().quoka_gather_kv(K, V, idx, cnt, ws=ws)
+    assert q().quoka_get_device_status(ws) == 6
+    torch.cuda.synchronize()
+    # the in-range rows were still gathered
+    np.testing.assert_array_equal(Ks[0, 0, :3].cpu().numpy(), x.K[0, 0, [1, 5, 99]])

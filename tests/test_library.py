@@ -1,0 +1,120 @@
+"""Host-side checks of libquoka.so that need no GPU: the library builds and
+loads, exports every entry point include/quoka.h declares, and rejects bad
+arguments on the host before anything is enqueued."""
+import ctypes
+import os
+import re
+import subprocess
+
+import pytest
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "quoka.h")
+
+
+@pytest.fixture(scope="module")
+def lib():
+    from sparse_kv_selection_quoka_b200 import build, _lib
+    build.build()
+    return _lib.load()
+
+
+def declared_functions():
+    src = open(HEADER).read()
+    src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
+    return sorted(set(re.findall(r"\b(quoka_[a-z_0-9]+)\s*\(", src)))
+
+
+def test_header_declares_the_boundary():
+    names = declared_functions()
+    for n in ("quoka_select", "quoka_gather_kv", "quoka_sparse_gqa_attn", "quoka_prefill_chunk",
+              "quoka_workspace_size", "quoka_get_device_status", "quoka_status_string"):
+        assert n in names
+
+
+def test_every_declared_symbol_is_exported(lib):
+    from sparse_kv_selection_quoka_b200 import _lib
+    out = subprocess.run(["nm", "-D", "--defined-only", _lib.LIB_PATH], capture_output=True,
+                         text=True, check=True).stdout
+    exported = set(re.findall(r"\bT (quoka_\w+)", out))
+    for n in declared_functions():
+        assert n in exported, f"{n} declared in quoka.h but not exported"
+        assert getattr(lib, n) is not None
+    assert set(_lib.EXPORTS) <= exported
+
+
+def test_status_strings(lib):
+    from sparse_kv_selection_quoka_b200 import _lib
+    for code, name in _lib.STATUS_NAMES.items():
+        assert lib.quoka_status_string(code).decode() == name
+
+
+def test_workspace_size_host_only(lib):
+    n = lib.quoka_workspace_size(1, 32, 8, 128, 32768, 512, 32, 4096, 1)
+    # at least S_agg (b*nkv*T fp32) and the selected indices
+    assert n >= 8 * 32768 * 4 + 8 * 4096 * 4
+    assert lib.quoka_workspace_size(1, 32, 8, 128, 32768, 512, 32, 4096, 1) % 256 == 0
+    assert lib.quoka_workspace_size(1, 30, 8, 128, 100, 64, 4, 10, 1) == 0    # nq % nkv
+    assert lib.quoka_workspace_size(1, 32, 8, 128, -1, 64, 4, 10, 1) == 0     # T < 0
+    assert lib.quoka_workspace_size(1, 32, 8, 128, 100, 64, 4, 10, 7) == 0    # dtype
+
+
+def _view(shape, dtype=1, data=0x10000, stride=None):
+    from sparse_kv_selection_quoka_b200._lib import quoka_tensor
+    v = quoka_tensor()
+    v.data = data
+    v.dtype = dtype
+    if stride is None:
+        stride = [shape[1] * shape[2] * shape[3], shape[2] * shape[3], shape[3], 1]
+    for i in range(4):
+        v.shape[i] = shape[i]
+        v.stride[i] = stride[i]
+    return v
+
+
+def test_select_rejects_bad_arguments_on_host(lib):
+    Q = _view((1, 8, 64, 128))
+    K = _view((1, 2, 500, 128))
+    ws = ctypes.c_void_p(0x100000)
+    buf = ctypes.c_void_p(0x200000)
+    call = lambda q, k, NQ, BSA, wsb=1 << 30: lib.quoka_select(ctypes.byref(q), ctypes.byref(k), NQ, BSA,
+                                                               buf, buf, None, None, ws, wsb, None)
+    assert call(Q, K, 0, 10) == 1                      # NQ < 1
+    assert call(Q, K, 65, 10) == 1                     # NQ > BCP
+    assert call(Q, K, 4, -1) == 1                      # BSA < 0
+    assert call(Q, _view((1, 3, 500, 128)), 4, 10) == 1           # nq % nkv
+    assert call(Q, _view((1, 2, 500, 128), dtype=0), 4, 10) == 1  # dtype mismatch
+    assert call(_view((1, 8, 64, 96)), _view((1, 2, 500, 96)), 4, 10) == 2  # d unsupported
+    assert call(_view((1, 8, 64, 128), data=0x10004), K, 4, 10) == 1        # misaligned data
+    assert call(_view((1, 8, 64, 128), stride=[8 * 64 * 128, 64 * 128, 129, 1]), K, 4, 10) == 1
+    assert call(_view((1, 8, 64, 128), stride=[8 * 64 * 128, 64 * 128, 128, 2]), K, 4, 10) == 1
+    assert call(Q, K, 4, 10, wsb=64) == 3              # workspace too small
+    assert lib.quoka_select(ctypes.byref(Q), ctypes.byref(K), 4, 10, buf, buf, None, None,
+                            ctypes.c_void_p(0x100010), 1 << 30, None) == 3  # misaligned ws
+    assert lib.quoka_select(None, ctypes.byref(K), 4, 10, buf, buf, None, None, ws, 1 << 30, None) == 1
+
+
+def test_attention_rejects_bad_arguments_on_host(lib):
+    Q = _view((1, 8, 64, 128))
+    K = _view((1, 2, 500, 128))
+    Kc = _view((1, 2, 64, 128))
+    buf = ctypes.c_void_p(0x200000)
+    ws = ctypes.c_void_p(0x100000)
+    f = lib.quoka_sparse_gqa_attn
+    B = ctypes.byref
+    assert f(B(Q), B(K), B(K), buf, buf, 10, B(_view((1, 2, 63, 128))), B(Kc), 0.1, buf, None, ws, 256, None) == 1
+    assert f(B(Q), B(K), B(K), buf, buf, 10, B(Kc), B(Kc), -1.0, buf, None, ws, 256, None) == 1
+    assert f(B(Q), B(K), B(K), buf, buf, -1, B(Kc), B(Kc), 0.1, buf, None, ws, 256, None) == 1
+    assert f(B(Q), B(K), B(K), buf, buf, 10, B(Kc), B(Kc), 0.1, None, None, ws, 256, None) == 1
+    assert f(B(Q), B(K), B(K), buf, buf, 10, B(Kc), B(Kc), 0.1, buf, None, None, 256, None) == 3
+    g = lib.quoka_prefill_chunk
+    assert g(B(Q), B(K), B(K), B(Kc), B(Kc), 4, 10, 0.1, buf, None, None, ws, 16, None) == 3
+    assert g(B(Q), B(K), B(K), B(Kc), B(Kc), 0, 10, 0.1, buf, None, None, ws, 1 << 30, None) == 1
+
+
+def test_binding_fails_loudly_without_library(tmp_path, monkeypatch):
+    from sparse_kv_selection_quoka_b200 import _lib
+    monkeypatch.setattr(_lib, "LIB_PATH", str(tmp_path / "missing.so"))
+    monkeypatch.setattr(_lib, "_lib", None)
+    with pytest.raises(ImportError):
+        _lib.load()

@@ -404,3 +404,22 @@ def test_planted_heavy_keys_are_selected_llama_shape():
     for j in range(x.K.shape[1]):
         kept = np.isin(x.meta["heavy_pos"][0, j], res["sel"][0, j]).mean()
         assert kept >= 0.75
+
+
+def test_attention_rows_match_sdpa_dense():
+    """The row-by-row attention used on large workloads, pinned to torch's
+    library attention in the dense reduction (everything selected)."""
+    r = rng(16)
+    b, nq, nkv, d, T, L = 2, 4, 2, 8, 11, 6
+    Q = r.standard_normal((b, nq, L, d))
+    K = r.standard_normal((b, nkv, T, d))
+    V = r.standard_normal((b, nkv, T, d))
+    Kc = r.standard_normal((b, nkv, L, d))
+    Vc = r.standard_normal((b, nkv, L, d))
+    sel = np.broadcast_to(np.arange(T), (b, nkv, T))
+    O_ref, lse_ref = _sdpa_dense_reference(Q, K, V, Kc, Vc, 1.0 / math.sqrt(d))
+    rows = [(bi, h, t) for bi in range(b) for h in range(nq) for t in range(L)]
+    O_rows, lse_rows = orc.sparse_attention_rows(Q, K, V, sel, Kc, Vc, rows)
+    for n, (bi, h, t) in enumerate(rows):
+        np.testing.assert_allclose(O_rows[n], O_ref[bi, h, t], atol=1e-12)
+        assert abs(lse_rows[n] - lse_ref[bi, h, t]) < 1e-12
