@@ -64,7 +64,8 @@ typedef enum { QUOKA_F32 = 0, QUOKA_BF16 = 1 } quoka_dtype;
 /* A strided 4-D view of device memory. Strides are in ELEMENTS; stride[3]
  * must be 1, every other stride must keep each row 16-byte aligned
  * (stride * element size a multiple of 16), and `data` must be 16-byte
- * aligned. Dimensions of extent 0 are allowed where stated. */
+ * aligned. Dimensions of extent 0 are allowed where stated; a view with no
+ * elements is never read, so its pointer and strides are not checked. */
 typedef struct {
   const void* data;
   quoka_dtype dtype;

@@ -66,15 +66,16 @@ bool check_tensor(const quoka_tensor* t, quoka_dtype dtype, int64_t want[4]) {
     if (want[i] >= 0 && t->shape[i] != want[i]) return false;
     want[i] = t->shape[i];
   }
+  int64_t n = 1;
+  for (int i = 0; i < 4; ++i) n *= t->shape[i];
+  if (n == 0) return true;  // nothing is read: pointer and strides are irrelevant
   if (t->stride[3] != 1) return false;
   const int64_t es = (int64_t)elt_size(dtype);
   for (int i = 0; i < 3; ++i) {
     if (t->stride[i] < 0) return false;
     if ((t->stride[i] * es) % 16 != 0) return false;
   }
-  int64_t n = 1;
-  for (int i = 0; i < 4; ++i) n *= t->shape[i];
-  if (n > 0 && (t->data == nullptr || !aligned16(t->data))) return false;
+  if (t->data == nullptr || !aligned16(t->data)) return false;
   return true;
 }
 
