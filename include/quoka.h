@@ -95,6 +95,35 @@ quoka_status quoka_select(const quoka_tensor* Q, const quoka_tensor* K, int NQ,
                           int32_t* q_idx, float* s_agg, void* ws,
                           size_t ws_bytes, void* stream);
 
+/* Size of the fixed device scratch array behind quoka_select_static. */
+#define QUOKA_STATIC_SCRATCH_BYTES (8u << 20)
+
+/* quoka_select without a workspace argument, for callers that cannot
+ * allocate device memory: for example a plugin hosted by a framework whose
+ * own allocator owns all device memory and forbids raw cudaMalloc, or code on
+ * a latency-critical path where cudaMalloc (which may synchronise the device)
+ * is not acceptable. The QUOKA write-up has no counterpart of this call; it
+ * only changes where the scratch lives.
+ *   Arguments, outputs and results are those of quoka_select, minus ws.
+ *   Scratch comes from a file-scope device array of
+ *   QUOKA_STATIC_SCRATCH_BYTES per device, held by every GPU that loads the
+ *   library until the process exits. Shapes whose quoka_workspace_size()
+ *   exceeds it are rejected with QUOKA_ERR_WORKSPACE before anything is
+ *   enqueued. Nothing is allocated (no cudaMalloc or cudaFree, no allocating
+ *   library call).
+ *   The first call on each device looks up the array's device address (with
+ *   that device current) and caches it; make that first call before any
+ *   stream capture begins.
+ *   All calls on a device share the array and it keeps the last call's
+ *   contents (each call clears its status word first; everything else is
+ *   rewritten before it is read). Calls that overlap on the GPU race on the
+ *   array: order them (one stream, or events between streams).
+ *   quoka_get_device_status() cannot reach this array; device faults of
+ *   these calls are not reported. */
+quoka_status quoka_select_static(const quoka_tensor* Q, const quoka_tensor* K, int NQ,
+                                 int BSA, int32_t* kv_idx, int32_t* kv_count,
+                                 int32_t* q_idx, float* s_agg, void* stream);
+
 /* Step (f), [QUOKA §4.2 problem 3]: Ksel[b, j, n] = K[b, j, kv_idx[b, j, n]]
  * and the same for V, for n < kv_count[b, j] (rows past the count are left
  * untouched).

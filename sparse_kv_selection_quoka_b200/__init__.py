@@ -18,6 +18,7 @@ __all__ = [
     "quoka_get_device_status",
     "quoka_status_string",
     "QuokaError",
+    "quoka_select_static",
 ]
 
 

@@ -43,6 +43,7 @@ EXPORTS = (
     "quoka_prefill_chunk",
     "quoka_get_device_status",
     "quoka_status_string",
+    "quoka_select_static",
 )
 
 
@@ -97,6 +98,8 @@ def load() -> ctypes.CDLL:
         lib.quoka_get_device_status.argtypes = [_P, _P, ctypes.POINTER(ctypes.c_int32)]
         lib.quoka_status_string.restype = ctypes.c_char_p
         lib.quoka_status_string.argtypes = [_I]
+        lib.quoka_select_static.restype = _I
+        lib.quoka_select_static.argtypes = [_T, _T, _I, _I, _P, _P, _P, _P, _P]
         _lib = lib
         return lib
 
@@ -256,3 +259,35 @@ def quoka_get_device_status(ws, stream=None) -> int:
 
 def quoka_status_string(status: int) -> str:
     return load().quoka_status_string(status).decode()
+
+
+STATIC_SCRATCH_BYTES = 8 << 20
+
+
+def quoka_select_static(Q, K, NQ: int, BSA: int, *, kv_idx=None, kv_count=None, q_idx=None,
+                        s_agg=None, want_q_idx=False, want_s_agg=False, stream=None):
+    """quoka_select for callers that cannot allocate device scratch: the
+    library uses its own fixed per-device scratch array (8 MiB) instead of a
+    workspace. Outputs the caller does not pass are allocated here with torch
+    (the C entry point itself allocates nothing). Calls sharing a device must
+    not overlap on the GPU."""
+    lib = load()
+    b, nq, BCP, d = Q.shape
+    nkv, T = K.shape[1], K.shape[2]
+    bsa_eff = min(BSA, T)
+    dev = Q.device
+    if kv_idx is None:
+        kv_idx = torch.empty((b, nkv, bsa_eff), dtype=torch.int32, device=dev)
+    if kv_count is None:
+        kv_count = torch.empty((b, nkv), dtype=torch.int32, device=dev)
+    if q_idx is None and want_q_idx:
+        q_idx = torch.empty((b, nq, NQ), dtype=torch.int32, device=dev)
+    if s_agg is None and want_s_agg:
+        s_agg = torch.empty((b, nkv, T), dtype=torch.float32, device=dev)
+    qv, kv = tensor_view(Q), tensor_view(K)
+    st = lib.quoka_select_static(ctypes.byref(qv), ctypes.byref(kv), NQ, BSA,
+                                 _ptr(kv_idx) if kv_idx.numel() else None, _ptr(kv_count),
+                                 _ptr(q_idx), _ptr(s_agg) if s_agg is not None and s_agg.numel() else None,
+                                 _stream(stream))
+    _check(st, "quoka_select_static")
+    return kv_idx, kv_count, q_idx, s_agg
