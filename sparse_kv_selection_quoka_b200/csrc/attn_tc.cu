@@ -8,23 +8,35 @@
 // (QUOKA = the technical write-up "QUOKA: how it reshapes LLM prefill
 // efficiency", bqwf.cn news item 915859.)
 //
-// One CTA per 128 query rows of one head. The key list is the selected prior
-// rows (read in place through the sorted index list: a fused gather) followed
-// by the chunk's keys, in tiles of 128 keys. Warp roles:
-//   warps 0-3  softmax: thread r owns query row r (= TMEM lane r); reads its
-//              S row from TMEM, applies the causal mask, online softmax in
-//              fp32 (exp2 on the MUFU), rescales the O accumulator in TMEM
-//              when the running max moves, writes P (bf16) to shared memory;
-//              final normalisation and store.
-//   warp 4     TMEM allocation and the single-thread MMA issue:
-//              S = Q K^T (M=128, N=128, K=128) into a double-buffered TMEM S,
-//              O += P V (M=128, N=128, K=128) into the TMEM O accumulator.
-//   warps 5-8  loaders: cp.async 16-byte row chunks (gathered by index) into
-//              a 2-stage K/V ring laid out in the 128-byte-swizzled UMMA
-//              layout; zero-fill past the end of the key list. Warps 5-6
-//              load the even tiles (and Q), warps 7-8 the odd tiles.
+// Work split. The query rows of one KV head j are cut into 128-row tiles
+// (one query head, 128 consecutive chunk positions each); a CTA takes two
+// such tiles (Q0, Q1) of the same KV head, so every K/V tile it brings in
+// feeds two 128x128x128 QK^T and two PV products. The key list of a CTA is
+// the selected prior rows (read in place through the sorted index list: the
+// gather is fused into the loads) followed by the chunk's keys, in tiles of
+// 128 keys. When the grid would fill less than half of the GPU, the key
+// tiles are split between the two CTAs of a cluster, and the partial results
+// are combined through distributed shared memory.
+//
+// Warp roles (384 threads):
+//   warps 0-3   softmax of Q0, warps 4-7 softmax of Q1: thread r owns query
+//               row r = TMEM lane r. Two passes over its S row in TMEM (row
+//               max, then exp2 on the MUFU); P is written back as bf16 over
+//               the S columns it has consumed, and is the A operand of PV
+//               straight from TMEM. The running max is only moved (and the O
+//               accumulator rescaled in TMEM) when it grows by more than 2^8,
+//               so rescales are rare. Final normalisation, combine and store.
+//   warp 8      TMEM allocation and the single-thread MMA issue, ordered
+//               QK0(i), PV1(i-1), QK1(i), PV0(i): while one softmax group
+//               works, the tensor core runs the other group's products.
+//   warps 9-11  loaders: cp.async 16-byte row chunks into a 2-stage K/V ring
+//               in the 128-byte-swizzled UMMA layout (zero-fill past the end
+//               of the key list); gather indices are prefetched a tile ahead;
+//               each thread's arrival on the stage barrier fires when its
+//               copies land.
+// TMEM: S0 | S1 | O0 | O1, 128 columns each (512).
 // Every wait is bounded: a wait that gives up records QUOKA_ERR_TIMEOUT and
-// the CTA unwinds (waits for its in-flight copies and MMAs, frees TMEM).
+// the CTA unwinds (waits for in-flight copies and MMAs, frees TMEM).
 #include "common.cuh"
 #include "kernels.h"
 #include "sm100.cuh"
@@ -35,67 +47,113 @@ using namespace sm100;
 
 namespace {
 
-constexpr int AT_M = 128;      // query rows per CTA
-constexpr int AT_N = 128;      // keys per tile
-constexpr int AT_D = 128;      // head dim
-constexpr int AT_STAGES = 2;   // K/V ring depth
-constexpr int AT_SM_WARPS = 4;
-constexpr int AT_MMA_WARP = 4;
-constexpr int AT_LD_WARPS = 4;
-constexpr int AT_LD_THREADS = AT_LD_WARPS * 32 / AT_STAGES;  // threads of one loader group
-constexpr int AT_THREADS = (AT_SM_WARPS + 1 + AT_LD_WARPS) * 32;
+constexpr int AT_D = 128;        // head dim
+constexpr int AT_N = 128;        // keys per tile
+constexpr int AT_STAGES = 2;     // K/V ring depth
+constexpr int AT_THREADS = 384;
+constexpr int AT_MMA_WARP = 8;
+constexpr int AT_LD_WARP0 = 9;
+constexpr int AT_LD_THREADS = 96;
+constexpr int AT_SM_THREADS = 256;
 constexpr int TILE_BYTES = 128 * AT_D * 2;  // 128 rows x 256 B
 constexpr int ATOM_BYTES = 128 * 128;       // one 64-column swizzle atom of a 128-row tile
 constexpr uint32_t TMEM_COLS = 512;
-constexpr uint32_t TM_S0 = 0, TM_S1 = 128, TM_O = 256;
+constexpr float RESCALE_THRESHOLD = 8.f;    // log2 units
 
-constexpr uint32_t IDESC_QK = idesc_bf16_f32(AT_M, AT_N, 0, 0);  // A=Q K-major, B=K K-major
-constexpr uint32_t IDESC_PV = idesc_bf16_f32(AT_M, AT_D, 0, 1);  // A=P K-major, B=V MN-major
+constexpr uint32_t IDESC_QK = idesc_bf16_f32(128, AT_N, 0, 0);  // A=Q K-major, B=K K-major
+constexpr uint32_t IDESC_PV = idesc_bf16_f32(128, AT_D, 0, 1);  // A=P (TMEM), B=V MN-major
+
+// loader geometry: 96 threads = 6 row groups x 16 chunks of 16 bytes
+constexpr int LD_ROWGROUPS = AT_LD_THREADS / 16;
+constexpr int LD_ROWS = (AT_N + LD_ROWGROUPS - 1) / LD_ROWGROUPS;  // 22
 
 struct __align__(1024) AttnSmem {
-  uint8_t q[TILE_BYTES];
-  uint8_t k[AT_STAGES][TILE_BYTES];
-  uint8_t v[AT_STAGES][TILE_BYTES];
-  uint8_t p[TILE_BYTES];
+  uint8_t q[2][TILE_BYTES];
+  uint8_t kv[AT_STAGES][2][TILE_BYTES];  // [stage][0 = K, 1 = V]
   uint64_t q_full;
   uint64_t kv_full[AT_STAGES];
   uint64_t kv_empty[AT_STAGES];
   uint64_t s_full[2];
-  uint64_t s_empty[2];
-  uint64_t p_full;
-  uint64_t o_done;
+  uint64_t p_full[2];
+  uint64_t o_final;
   uint64_t mma_done;
+  uint64_t xfer_free;   // (rank 1) rank 0's landing zone is free
+  uint64_t xfer_full;   // (rank 0) rank 1's partial results have landed
   uint32_t tmem_base;
   int abort;
 };
+// The split-KV landing zone in rank 0 reuses the K/V ring (partial O, fp32,
+// [tile][row][128] with a per-row chunk rotation) and the Q area (m, l).
+static_assert(sizeof(float) * 2 * 128 * AT_D <= AT_STAGES * 2 * TILE_BYTES, "landing zone");
 
-__device__ __forceinline__ void record_abort(AttnSmem& sm, int* status) {
+struct TileInfo {
+  int valid, h, t0;
+};
+
+// A wait gave up: stop the CTA's other roles and record the fault and the
+// waiting site (a small code naming the barrier).
+__device__ __forceinline__ void record_abort(AttnSmem& sm, int* status, int where) {
   sm.abort = 1;
   latch_status(status, 5 /* QUOKA_ERR_TIMEOUT */);
+  latch_where(status, where);
 }
 
 // Warp-uniform bounded wait (every lane polls; all lanes agree on the result).
-__device__ __forceinline__ bool warp_wait(uint64_t* bar, uint32_t parity, AttnSmem& sm, int* status) {
+__device__ __forceinline__ bool warp_wait(uint64_t* bar, uint32_t parity, AttnSmem& sm, int* status, int where) {
   const bool ok = mbar_wait(bar, parity, &sm.abort);
   const bool all_ok = __all_sync(0xffffffffu, ok);
-  if (!all_ok && (threadIdx.x & 31) == 0) record_abort(sm, status);
+  if (!all_ok && (threadIdx.x & 31) == 0) record_abort(sm, status, where);
   return all_ok;
 }
 
+// The same for a barrier that another CTA of the cluster arrives on.
+__device__ __forceinline__ bool warp_wait_cluster(uint64_t* bar, uint32_t parity, AttnSmem& sm, int* status,
+                                                  int where) {
+  bool ok = mbar_try_wait_cluster(bar, parity);
+  if (!ok) {
+    const uint64_t t0 = globaltimer_ns();
+    while (!ok && globaltimer_ns() - t0 < kWaitLimitNs) ok = mbar_try_wait_cluster(bar, parity);
+  }
+  const bool all_ok = __all_sync(0xffffffffu, ok);
+  if (!all_ok && (threadIdx.x & 31) == 0) record_abort(sm, status, where);
+  return all_ok;
+}
+
+__device__ __forceinline__ uint32_t pack_bf16x2(float a, float b) {
+  __nv_bfloat162 h = __floats2bfloat162_rn(a, b);
+  return *reinterpret_cast<uint32_t*>(&h);
+}
+
 __global__ void __launch_bounds__(AT_THREADS, 1)
-attn_tc_kernel(const AttnArgs a) {
+attn_tc_kernel(const AttnArgs a, int nsplit) {
   extern __shared__ uint8_t smem_raw[];
   AttnSmem& sm = *reinterpret_cast<AttnSmem*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-  const int h = blockIdx.y, bi = blockIdx.z;
-  const int G = a.nq / a.nkv, j = h / G;
-  const int t0 = blockIdx.x * AT_M;
+  const int j = blockIdx.y, bi = blockIdx.z;
+  const int G = a.nq / a.nkv;
+  const int split = nsplit > 1 ? (int)cluster_ctarank() : 0;
+  const int pair = blockIdx.x / nsplit;
+  const int ntt = (a.BCP + 127) / 128;  // row tiles per query head
+  const int R = G * ntt;                // row tiles per KV head
+
+  TileInfo ti[2];
+#pragma unroll
+  for (int w = 0; w < 2; ++w) {
+    const int r = 2 * pair + w;
+    ti[w].valid = r < R;
+    ti[w].h = j * G + (r < R ? r / ntt : 0);
+    ti[w].t0 = (r < R ? r % ntt : 0) * 128;
+  }
   const int64_t kvrow = (int64_t)bi * a.nkv + j;
   const int nsel = a.bsa > 0 ? max(0, min(a.kv_count[kvrow], a.bsa)) : 0;
-  const int nchunk = min(a.BCP, t0 + AT_M);
+  const int max_t0 = ti[1].valid ? max(ti[0].t0, ti[1].t0) : ti[0].t0;
+  const int nchunk = min(a.BCP, max_t0 + 128);
   const int total = nsel + nchunk;
   const int nT = (total + AT_N - 1) / AT_N;
+  const int per = (nT + nsplit - 1) / nsplit;
+  const int first = min(nT, split * per);
+  const int ntiles = min(nT, first + per) - first;  // key tiles of this CTA (may be 0)
 
   if (tid == 0) {
     mbar_init(&sm.q_full, AT_LD_THREADS);
@@ -103,13 +161,14 @@ attn_tc_kernel(const AttnArgs a) {
       mbar_init(&sm.kv_full[s], AT_LD_THREADS);
       mbar_init(&sm.kv_empty[s], 1);
     }
-    for (int s = 0; s < 2; ++s) {
-      mbar_init(&sm.s_full[s], 1);
-      mbar_init(&sm.s_empty[s], AT_SM_WARPS * 32);
+    for (int w = 0; w < 2; ++w) {
+      mbar_init(&sm.s_full[w], 1);
+      mbar_init(&sm.p_full[w], 128);
     }
-    mbar_init(&sm.p_full, AT_SM_WARPS * 32);
-    mbar_init(&sm.o_done, 1);
+    mbar_init(&sm.o_final, 1);
     mbar_init(&sm.mma_done, 1);
+    mbar_init(&sm.xfer_free, 1);
+    mbar_init(&sm.xfer_full, AT_SM_THREADS);
     sm.abort = 0;
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
   }
@@ -118,21 +177,20 @@ attn_tc_kernel(const AttnArgs a) {
     tmem_relinquish();
   }
   tc_fence_before();
-  __syncthreads();
+  if (nsplit > 1) {
+    // both CTAs' barriers must be initialised before any remote arrive
+    asm volatile("barrier.cluster.arrive.release.aligned;\n\tbarrier.cluster.wait.acquire.aligned;" ::: "memory");
+  } else {
+    __syncthreads();
+  }
   tc_fence_after();
   const uint32_t tmem = sm.tmem_base;
 
-  if (warp >= AT_MMA_WARP + 1) {
+  if (warp >= AT_LD_WARP0) {
     // ------------------------------------------------------------ loaders
-    // Two groups of 64 threads own alternating tiles (group g loads tiles
-    // i = g, g + 2, ... into stage g). Each group publishes a tile as soon as
-    // it has landed, so a group never waits for a free stage while holding
-    // back a tile the MMA needs first.
-    const int grp = (warp - (AT_MMA_WARP + 1)) / 2;
-    const int lt = tid - (AT_MMA_WARP + 1 + 2 * grp) * 32;  // 0..63
-    const int c = lt & 15;        // 16-byte chunk of a row (fixed per thread)
-    const int rsub = lt >> 4;     // row within a group of 4
-    const bf16* Qb = static_cast<const bf16*>(a.Q.data) + bi * a.Q.sb + h * a.Q.sh;
+    const int lt = tid - AT_LD_WARP0 * 32;  // 0..95
+    const int c = lt & 15;                   // 16-byte chunk of a row
+    const int rg = lt >> 4;                  // row group 0..5: rows rg, rg+6, ...
     const bf16* Kb = static_cast<const bf16*>(a.K.data) + bi * a.K.sb + j * a.K.sh;
     const bf16* Vb = static_cast<const bf16*>(a.V.data) + bi * a.V.sb + j * a.V.sh;
     const bf16* Kcb = static_cast<const bf16*>(a.Kc.data) + bi * a.Kc.sb + j * a.Kc.sh;
@@ -140,212 +198,307 @@ attn_tc_kernel(const AttnArgs a) {
     const int32_t* idx = a.kv_idx + kvrow * a.bsa;
     bool bad_index = false;
 
-    if (grp == 0) {
-      const uint32_t q_s = smem_u32(sm.q);
-#pragma unroll 4
-      for (int it = 0; it < 32; ++it) {
-        const int r = it * 4 + rsub;
-        const int t = t0 + r;
-        const bool ok = t < a.BCP;
-        const bf16* src = ok ? Qb + (int64_t)t * a.Q.st + c * 8 : Kcb;
-        cp_async_16(q_s + sw128_offset(r, c, 128), src, ok ? 16u : 0u);
+    // Q tiles (zero rows past the chunk or for a missing second tile)
+    for (int w = 0; w < 2; ++w) {
+      const bf16* Qb = static_cast<const bf16*>(a.Q.data) + bi * a.Q.sb + ti[w].h * a.Q.sh;
+      const uint32_t q_s = smem_u32(sm.q[w]);
+      for (int r = rg; r < 128; r += LD_ROWGROUPS) {
+        const int t = ti[w].t0 + r;
+        const bool ok = ti[w].valid && t < a.BCP;
+        cp_async_16(q_s + sw128_offset(r, c, 128), ok ? Qb + (int64_t)t * a.Q.st + c * 8 : Kcb, ok ? 16u : 0u);
       }
-      cp_async_commit();
     }
+    cp_async_arrive_noinc(&sm.q_full);
 
-    bool alive = true;
-    for (int i = grp; i < nT && alive; i += AT_STAGES) {
-      const int s = grp;
-      if (i >= AT_STAGES) alive = warp_wait(&sm.kv_empty[s], ((i / AT_STAGES) - 1) & 1, sm, a.status);
-      if (!alive) break;
-      const uint32_t k_s = smem_u32(sm.k[s]), v_s = smem_u32(sm.v[s]);
-#pragma unroll 4
-      for (int it = 0; it < 32; ++it) {
-        const int r = it * 4 + rsub;
-        const int n = i * AT_N + r;
-        const bf16* ks = Kcb;
-        const bf16* vs = Vcb;
-        uint32_t bytes = 0u;
-        if (n < nsel) {
-          const int32_t tau = __ldg(idx + n);
-          if (tau >= 0 && (int64_t)tau < a.T) {
-            ks = Kb + (int64_t)tau * a.K.st + c * 8;
-            vs = Vb + (int64_t)tau * a.V.st + c * 8;
-            bytes = 16u;
-          } else {
-            bad_index = true;
-          }
-        } else if (n < total) {
-          const int p = n - nsel;
-          ks = Kcb + (int64_t)p * a.Kc.st + c * 8;
-          vs = Vcb + (int64_t)p * a.Vc.st + c * 8;
-          bytes = 16u;
-        }
-        const uint32_t off = sw128_offset(r, c, 128);
-        cp_async_16(k_s + off, ks, bytes);
-        cp_async_16(v_s + off, vs, bytes);
+    // gather indices of this thread's rows of tile `gi` (-1: chunk key or past the end)
+    int32_t tau[LD_ROWS];
+    auto fetch_idx = [&](int gi) {
+#pragma unroll
+      for (int k = 0; k < LD_ROWS; ++k) {
+        const int r = rg + LD_ROWGROUPS * k;
+        const int n = gi * AT_N + r;
+        tau[k] = (r < AT_N && n < nsel) ? __ldg(idx + n) : -1;
       }
-      cp_async_commit();
-      cp_async_wait<0>();
-      fence_proxy_async_smem();
-      if (i == 0) mbar_arrive(&sm.q_full);
-      mbar_arrive(&sm.kv_full[s]);
+    };
+    if (ntiles > 0) fetch_idx(first);
+    bool alive = true;
+    for (int it = 0; it < ntiles && alive; ++it) {
+      const int s = it % AT_STAGES;
+      const int gi = first + it;
+      if (it >= AT_STAGES) alive = warp_wait(&sm.kv_empty[s], ((it / AT_STAGES) - 1) & 1, sm, a.status, 11);
+      if (!alive) break;
+      const uint32_t k_s = smem_u32(sm.kv[s][0]), v_s = smem_u32(sm.kv[s][1]);
+#pragma unroll
+      for (int k = 0; k < LD_ROWS; ++k) {
+        const int r = rg + LD_ROWGROUPS * k;
+        if (r < AT_N) {
+          const int n = gi * AT_N + r;
+          const bf16* ks = Kcb;
+          const bf16* vs = Vcb;
+          uint32_t bytes = 0u;
+          if (n < nsel) {
+            const int32_t tv = tau[k];
+            if (tv >= 0 && (int64_t)tv < a.T) {
+              ks = Kb + (int64_t)tv * a.K.st + c * 8;
+              vs = Vb + (int64_t)tv * a.V.st + c * 8;
+              bytes = 16u;
+            } else {
+              bad_index = true;
+            }
+          } else if (n < total) {
+            const int p = n - nsel;
+            ks = Kcb + (int64_t)p * a.Kc.st + c * 8;
+            vs = Vcb + (int64_t)p * a.Vc.st + c * 8;
+            bytes = 16u;
+          }
+          const uint32_t off = sw128_offset(r, c, 128);
+          cp_async_16(k_s + off, ks, bytes);
+          cp_async_16(v_s + off, vs, bytes);
+        }
+      }
+      cp_async_arrive_noinc(&sm.kv_full[s]);
+      if (it + 1 < ntiles) fetch_idx(gi + 1);
     }
     cp_async_wait<0>();
     if (bad_index) latch_status(a.status, 6 /* QUOKA_ERR_BOUNDS */);
   } else if (warp == AT_MMA_WARP) {
     // ------------------------------------------------------------ MMA issue
     if (lane == 0) {
-      const uint32_t q_s = smem_u32(sm.q), p_s = smem_u32(sm.p);
-      bool alive = mbar_wait(&sm.q_full, 0, &sm.abort);
-      auto issue_pv = [&](int jt) -> bool {
-        const int s = jt % AT_STAGES;
-        if (!mbar_wait(&sm.p_full, jt & 1, &sm.abort)) return false;
-        tc_fence_after();
-        const uint32_t v_s = smem_u32(sm.v[s]);
-#pragma unroll
-        for (int kk = 0; kk < AT_N / 16; ++kk) {
-          const uint64_t ad = sw128_desc(p_s + (kk >> 2) * ATOM_BYTES + (kk & 3) * 32, 16, 1024);
-          const uint64_t bd = sw128_desc(v_s + kk * 2048, ATOM_BYTES, 1024);
-          umma_bf16_ss(tmem + TM_O, ad, bd, IDESC_PV, (jt > 0 || kk > 0) ? 1u : 0u);
-        }
-        umma_commit(&sm.kv_empty[s]);
-        umma_commit(&sm.o_done);
-        return true;
-      };
-      for (int i = 0; i < nT && alive; ++i) {
-        const int s = i % AT_STAGES, sb = i & 1;
-        alive = mbar_wait(&sm.kv_full[s], (i / AT_STAGES) & 1, &sm.abort);
-        if (alive && i >= 2) alive = mbar_wait(&sm.s_empty[sb], ((i >> 1) - 1) & 1, &sm.abort);
-        if (!alive) break;
-        tc_fence_after();
-        const uint32_t k_s = smem_u32(sm.k[s]);
+      const uint32_t q0 = smem_u32(sm.q[0]), q1 = smem_u32(sm.q[1]);
+      const bool v0 = ti[0].valid, v1 = ti[1].valid;
+      auto qk = [&](int w, int s) {
+        const uint32_t qs = w ? q1 : q0, ks = smem_u32(sm.kv[s][0]);
 #pragma unroll
         for (int kk = 0; kk < AT_D / 16; ++kk) {
           const uint32_t koff = (kk >> 2) * ATOM_BYTES + (kk & 3) * 32;
-          const uint64_t ad = sw128_desc(q_s + koff, 16, 1024);
-          const uint64_t bd = sw128_desc(k_s + koff, 16, 1024);
-          umma_bf16_ss(tmem + (sb ? TM_S1 : TM_S0), ad, bd, IDESC_QK, kk > 0 ? 1u : 0u);
+          umma_bf16_ss(tmem + 128u * w, sw128_desc(qs + koff, 16, 1024), sw128_desc(ks + koff, 16, 1024),
+                       IDESC_QK, kk > 0 ? 1u : 0u);
         }
-        umma_commit(&sm.s_full[sb]);
-        if (i >= 1) alive = issue_pv(i - 1);
+        umma_commit(&sm.s_full[w]);
+      };
+      auto pv = [&](int w, int s, bool acc) {
+        const uint32_t vs = smem_u32(sm.kv[s][1]);
+#pragma unroll
+        for (int kk = 0; kk < AT_N / 16; ++kk)
+          umma_bf16_ts(tmem + 256u + 128u * w, tmem + 128u * w + kk * 8,
+                       sw128_desc(vs + kk * 2048, ATOM_BYTES, 1024), IDESC_PV, (acc || kk > 0) ? 1u : 0u);
+      };
+      int where = 21;
+      bool alive = mbar_wait(&sm.q_full, 0, &sm.abort);
+      for (int it = 0; it < ntiles && alive; ++it) {
+        const int s = it % AT_STAGES;
+        const int sp = (it + AT_STAGES - 1) % AT_STAGES;
+        where = 22;
+        alive = mbar_wait(&sm.kv_full[s], (it / AT_STAGES) & 1, &sm.abort);
+        if (!alive) break;
+        fence_proxy_async_smem();  // the cp.async writes become visible to the tensor core
+        tc_fence_after();
+        if (v0) qk(0, s);
+        if (it > 0) {
+          if (v1) {
+            where = 23;
+            alive = mbar_wait(&sm.p_full[1], (it - 1) & 1, &sm.abort);
+            if (!alive) break;
+            tc_fence_after();
+            pv(1, sp, it - 1 > 0);
+          }
+          umma_commit(&sm.kv_empty[sp]);
+        }
+        if (v1) qk(1, s);
+        if (v0) {
+          where = 24;
+          alive = mbar_wait(&sm.p_full[0], it & 1, &sm.abort);
+          if (!alive) break;
+          tc_fence_after();
+          pv(0, s, it > 0);
+        }
       }
-      if (alive && nT > 0) alive = issue_pv(nT - 1);
-      if (!alive) record_abort(sm, a.status);
-      // every MMA this thread issued has completed before TMEM is freed
+      if (alive && ntiles > 0 && v1) {
+        where = 25;
+        alive = mbar_wait(&sm.p_full[1], (ntiles - 1) & 1, &sm.abort);
+        if (alive) {
+          tc_fence_after();
+          pv(1, (ntiles - 1) % AT_STAGES, ntiles - 1 > 0);
+        }
+      }
+      if (!alive) record_abort(sm, a.status, where);
+      umma_commit(&sm.o_final);
       umma_commit(&sm.mma_done);
-      if (!mbar_drain(&sm.mma_done, 0)) latch_status(a.status, 5 /* QUOKA_ERR_TIMEOUT */);
+      if (!mbar_drain(&sm.mma_done, 0)) record_abort(sm, a.status, 26);
+      // rank 0: every MMA is done, so its K/V ring and Q area may now take
+      // rank 1's partial results
+      if (nsplit > 1 && split == 0) mbar_arrive_remote(mapa_shared(smem_u32(&sm.xfer_free), 1));
     }
     __syncwarp();
   } else {
     // ------------------------------------------------------------ softmax
-    const int r = tid;  // query row within the tile == TMEM lane
-    const int t = t0 + r;
-    const uint32_t lane_base = tmem + ((uint32_t)(warp * 32) << 16);
+    const int w = warp >> 2;           // query tile of this warpgroup
+    const int r = tid & 127;           // row == TMEM lane
+    const int t = ti[w].t0 + r;
+    const uint32_t lane_off = (uint32_t)((warp & 3) * 32) << 16;
+    const uint32_t S = tmem + lane_off + 128u * w;
+    const uint32_t O = tmem + lane_off + 256u + 128u * w;
     const float qscale = a.scale * 1.4426950408889634f;
     float m = -INFINITY, l = 0.f;
-    uint8_t* prow = sm.p;
     bool alive = true;
-    for (int i = 0; i < nT && alive; ++i) {
-      const int sb = i & 1;
-      alive = warp_wait(&sm.s_full[sb], (i >> 1) & 1, sm, a.status);
+    const bool active = ti[w].valid != 0;
+    for (int it = 0; it < ntiles && alive && active; ++it) {
+      alive = warp_wait(&sm.s_full[w], it & 1, sm, a.status, 31 + w);
       if (!alive) break;
       tc_fence_after();
-      float x[AT_N];
-#pragma unroll
-      for (int q4 = 0; q4 < AT_N / 32; ++q4)
-        tmem_ld32(lane_base + (sb ? TM_S1 : TM_S0) + q4 * 32, *reinterpret_cast<float(*)[32]>(&x[q4 * 32]));
-      tmem_wait_ld();
-      tc_fence_before();
-      mbar_arrive(&sm.s_empty[sb]);
-
-      // mask (keys past the list, and chunk keys after this row), scale, max
-      const int base_n = i * AT_N;
+      const int base_n = (first + it) * AT_N;
+      // pass 1: row max of the visible scaled scores
       float mx = -INFINITY;
+#pragma unroll 1
+      for (int c4 = 0; c4 < 4; ++c4) {
+        float v[32];
+        tmem_ld32(S + 32 * c4, v);
+        tmem_wait_ld();
 #pragma unroll
-      for (int cc = 0; cc < AT_N; ++cc) {
-        const int n = base_n + cc;
-        const bool vis = n < nsel || (n < total && n - nsel <= t);
-        x[cc] = vis ? x[cc] * qscale : -INFINITY;
-        mx = fmaxf(mx, x[cc]);
+        for (int u = 0; u < 32; ++u) {
+          const int n = base_n + 32 * c4 + u;
+          const bool vis = n < nsel || (n < total && n - nsel <= t);
+          mx = vis ? fmaxf(mx, v[u] * qscale) : mx;
+        }
       }
-      const float m_new = fmaxf(m, mx);
+      const float m_cand = fmaxf(m, mx);
+      const float m_new = (m_cand > m + RESCALE_THRESHOLD || m == -INFINITY) ? m_cand : m;
+      const float corr = (m_new == m) ? 1.f : ex2(m - m_new);
       const float m_use = m_new == -INFINITY ? 0.f : m_new;
-      const float corr = ex2(m - m_use);
+      // pass 2: P = 2^(s - m) in bf16, written over consumed S columns
       float rs = 0.f;
+#pragma unroll 1
+      for (int c4 = 0; c4 < 4; ++c4) {
+        float v[32];
+        tmem_ld32(S + 32 * c4, v);
+        tmem_wait_ld();
+        uint32_t pk[16];
 #pragma unroll
-      for (int cc = 0; cc < AT_N; ++cc) {
-        x[cc] = ex2(x[cc] - m_use);
-        rs += x[cc];
+        for (int u = 0; u < 32; u += 2) {
+          const int n = base_n + 32 * c4 + u;
+          const bool vis0 = n < nsel || (n < total && n - nsel <= t);
+          const bool vis1 = n + 1 < nsel || (n + 1 < total && n + 1 - nsel <= t);
+          const float p0 = vis0 ? ex2(v[u] * qscale - m_use) : 0.f;
+          const float p1 = vis1 ? ex2(v[u + 1] * qscale - m_use) : 0.f;
+          rs += p0 + p1;
+          pk[u >> 1] = pack_bf16x2(p0, p1);
+        }
+        tmem_st16(S + 16 * c4, pk);
       }
       l = l * corr + rs;
       m = m_new;
-
-      if (i > 0) {
-        // PV of the previous tile must be done before O is rescaled and the
-        // P buffer is overwritten
-        alive = warp_wait(&sm.o_done, (i - 1) & 1, sm, a.status);
-        if (!alive) break;
-        tc_fence_after();
-        if (__any_sync(0xffffffffu, corr != 1.f)) {
+      // O holds the products of the previous tiles (complete: they were
+      // issued before this tile's QK^T, whose completion we waited for)
+      if (it > 0 && __any_sync(0xffffffffu, corr != 1.f)) {
 #pragma unroll 1
-          for (int q4 = 0; q4 < AT_D / 32; ++q4) {
-            float o[32];
-            tmem_ld32(lane_base + TM_O + q4 * 32, o);
-            tmem_wait_ld();
+        for (int c4 = 0; c4 < 4; ++c4) {
+          float o[32];
+          tmem_ld32(O + 32 * c4, o);
+          tmem_wait_ld();
 #pragma unroll
-            for (int u = 0; u < 32; ++u) o[u] *= corr;
-            tmem_st32(lane_base + TM_O + q4 * 32, o);
-          }
-          tmem_wait_st();
+          for (int u = 0; u < 32; ++u) o[u] *= corr;
+          tmem_st32(O + 32 * c4, o);
         }
       }
-      // P row (bf16) into the swizzled K-major A-operand tile
-#pragma unroll
-      for (int c = 0; c < AT_N / 8; ++c) {
-        uint4 pk;
-        __nv_bfloat162 h0 = __floats2bfloat162_rn(x[8 * c + 0], x[8 * c + 1]);
-        __nv_bfloat162 h1 = __floats2bfloat162_rn(x[8 * c + 2], x[8 * c + 3]);
-        __nv_bfloat162 h2 = __floats2bfloat162_rn(x[8 * c + 4], x[8 * c + 5]);
-        __nv_bfloat162 h3 = __floats2bfloat162_rn(x[8 * c + 6], x[8 * c + 7]);
-        pk.x = *reinterpret_cast<uint32_t*>(&h0);
-        pk.y = *reinterpret_cast<uint32_t*>(&h1);
-        pk.z = *reinterpret_cast<uint32_t*>(&h2);
-        pk.w = *reinterpret_cast<uint32_t*>(&h3);
-        *reinterpret_cast<uint4*>(prow + sw128_offset(r, c, 128)) = pk;
-      }
-      fence_proxy_async_smem();
+      tmem_wait_st();
       tc_fence_before();
-      mbar_arrive(&sm.p_full);
+      mbar_arrive(&sm.p_full[w]);
     }
-    if (alive && nT > 0) alive = warp_wait(&sm.o_done, (nT - 1) & 1, sm, a.status);
-    if (alive) {
-      tc_fence_after();
-      const float inv = 1.f / l;
-      bf16* orow = static_cast<bf16*>(a.O) + (((int64_t)bi * a.nq + h) * a.BCP + t) * AT_D;
+
+    // ------------------------------------------------ epilogue / combine
+    const bool have = active && ntiles > 0;
+    if (alive) alive = warp_wait(&sm.o_final, 0, sm, a.status, 33);
+    tc_fence_after();
+    const float ln2 = 0.6931471805599453f;
+    float* land_o = reinterpret_cast<float*>(&sm.kv[0][0][0]) + (size_t)(w * 128 + r) * AT_D;
+    float* land_ml = reinterpret_cast<float*>(&sm.q[0][0]) + (size_t)(w * 128 + r) * 2;
+    if (nsplit > 1 && split == 1) {
+      // send (O, m, l) of this row to rank 0 once its landing zone is free
+      if (alive) alive = warp_wait_cluster(&sm.xfer_free, 0, sm, a.status, 41);
+      if (alive) {
+        const uint32_t ro = mapa_shared(smem_u32(land_o), 0);
 #pragma unroll 1
-      for (int q4 = 0; q4 < AT_D / 32; ++q4) {
-        float o[32];
-        tmem_ld32(lane_base + TM_O + q4 * 32, o);
-        tmem_wait_ld();
-        if (t < a.BCP) {
+        for (int c4 = 0; c4 < 4; ++c4) {
+          float o[32];
+          if (have) {
+            tmem_ld32(O + 32 * c4, o);
+            tmem_wait_ld();
+          } else {
+#pragma unroll
+            for (int u = 0; u < 32; ++u) o[u] = 0.f;
+          }
+#pragma unroll
+          for (int u = 0; u < 32; u += 4) {
+            const int chunk = (32 * c4 + u) >> 2;  // 16-byte chunk 0..31, rotated by row
+            st_cluster_v4(ro + (uint32_t)(((chunk + r) & 31) << 4), make_float4(o[u], o[u + 1], o[u + 2], o[u + 3]));
+          }
+        }
+        const uint32_t rml = mapa_shared(smem_u32(land_ml), 0);
+        st_cluster_f32(rml, have ? m : -INFINITY);
+        st_cluster_f32(rml + 4, have ? l : 0.f);
+      }
+      mbar_arrive_remote(mapa_shared(smem_u32(&sm.xfer_full), 0));
+    } else if (active) {
+      float m_o = -INFINITY, l_o = 0.f;
+      if (nsplit > 1) {
+        if (alive) alive = warp_wait_cluster(&sm.xfer_full, 0, sm, a.status, 42);
+        if (alive) {
+          m_o = land_ml[0];
+          l_o = land_ml[1];
+        }
+      }
+      // warp-uniform from here on (tcgen05.ld is a warp-collective); only
+      // the stores are predicated on the row being inside the chunk
+      if (alive) {
+        const bool row_ok = t < a.BCP;
+        const float mm = have ? m : -INFINITY;
+        const float ll = have ? l : 0.f;
+        const float M = fmaxf(mm, m_o);
+        const float f_me = mm == -INFINITY ? 0.f : ex2(mm - M);
+        const float f_ot = m_o == -INFINITY ? 0.f : ex2(m_o - M);
+        const float L = f_me * ll + f_ot * l_o;
+        const float inv = 1.f / L;
+        bf16* orow = static_cast<bf16*>(a.O) + (((int64_t)bi * a.nq + ti[w].h) * a.BCP + t) * AT_D;
+#pragma unroll 1
+        for (int c4 = 0; c4 < 4; ++c4) {
+          float o[32];
+          if (have) {
+            tmem_ld32(O + 32 * c4, o);
+            tmem_wait_ld();
+          } else {
+#pragma unroll
+            for (int u = 0; u < 32; ++u) o[u] = 0.f;
+          }
+          if (nsplit > 1) {
+#pragma unroll
+            for (int u = 0; u < 32; u += 4) {
+              const int chunk = (32 * c4 + u) >> 2;
+              const float4 p = *reinterpret_cast<const float4*>(land_o + 4 * ((chunk + r) & 31));
+              o[u] = o[u] * f_me + p.x * f_ot;
+              o[u + 1] = o[u + 1] * f_me + p.y * f_ot;
+              o[u + 2] = o[u + 2] * f_me + p.z * f_ot;
+              o[u + 3] = o[u + 3] * f_me + p.w * f_ot;
+            }
+          } else {
+#pragma unroll
+            for (int u = 0; u < 32; ++u) o[u] *= f_me;
+          }
 #pragma unroll
           for (int u = 0; u < 32; u += 8) {
             uint4 pk;
-            __nv_bfloat162 h0 = __floats2bfloat162_rn(o[u + 0] * inv, o[u + 1] * inv);
-            __nv_bfloat162 h1 = __floats2bfloat162_rn(o[u + 2] * inv, o[u + 3] * inv);
-            __nv_bfloat162 h2 = __floats2bfloat162_rn(o[u + 4] * inv, o[u + 5] * inv);
-            __nv_bfloat162 h3 = __floats2bfloat162_rn(o[u + 6] * inv, o[u + 7] * inv);
-            pk.x = *reinterpret_cast<uint32_t*>(&h0);
-            pk.y = *reinterpret_cast<uint32_t*>(&h1);
-            pk.z = *reinterpret_cast<uint32_t*>(&h2);
-            pk.w = *reinterpret_cast<uint32_t*>(&h3);
-            *reinterpret_cast<uint4*>(orow + q4 * 32 + u) = pk;
+            pk.x = pack_bf16x2(o[u] * inv, o[u + 1] * inv);
+            pk.y = pack_bf16x2(o[u + 2] * inv, o[u + 3] * inv);
+            pk.z = pack_bf16x2(o[u + 4] * inv, o[u + 5] * inv);
+            pk.w = pack_bf16x2(o[u + 6] * inv, o[u + 7] * inv);
+            if (row_ok) *reinterpret_cast<uint4*>(orow + 32 * c4 + u) = pk;
           }
         }
+        if (row_ok && a.lse != nullptr)
+          a.lse[((int64_t)bi * a.nq + ti[w].h) * a.BCP + t] = (M + __log2f(L)) * ln2;
       }
-      if (t < a.BCP && a.lse != nullptr)
-        a.lse[((int64_t)bi * a.nq + h) * a.BCP + t] = (m + __log2f(l)) * 0.6931471805599453f;
+    } else if (nsplit > 1) {
+      // an empty second tile on rank 0 still consumes its landing signal
+      warp_wait_cluster(&sm.xfer_full, 0, sm, a.status, 43);
     }
   }
 
@@ -364,9 +517,29 @@ cudaError_t launch_attn_tc(const AttnArgs& a, cudaStream_t stream) {
   const size_t smem = sizeof(AttnSmem) + 1024;
   cudaError_t e = cudaFuncSetAttribute(attn_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (e != cudaSuccess) return e;
-  dim3 grid((a.BCP + AT_M - 1) / AT_M, a.nq, a.b);
-  attn_tc_kernel<<<grid, AT_THREADS, smem, stream>>>(a);
-  return cudaGetLastError();
+  const int G = a.nq / a.nkv;
+  const int R = G * ((a.BCP + 127) / 128);
+  const int npairs = (R + 1) / 2;
+  const long ctas = (long)npairs * a.nkv * a.b;
+  int num_sms = 148;
+  {
+    int dev = 0;
+    if (cudaGetDevice(&dev) == cudaSuccess) cudaDeviceGetAttribute(&num_sms, cudaDevAttrMultiProcessorCount, dev);
+  }
+  const int nsplit = (2 * ctas <= num_sms) ? 2 : 1;
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(npairs * nsplit, a.nkv, a.b);
+  cfg.blockDim = dim3(AT_THREADS);
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = stream;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeClusterDimension;
+  attr[0].val.clusterDim.x = nsplit;
+  attr[0].val.clusterDim.y = 1;
+  attr[0].val.clusterDim.z = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, attn_tc_kernel, a, nsplit);
 }
 
 }  // namespace quoka

@@ -22,6 +22,12 @@ __device__ __forceinline__ void latch_status(int* status, int code) {
   if (status != nullptr) atomicCAS(status, 0, code);
 }
 
+// Record where the first device-side fault of a call happened (the word
+// after the status word; diagnostic only).
+__device__ __forceinline__ void latch_where(int* status, int where) {
+  if (status != nullptr) atomicCAS(status + 1, 0, where);
+}
+
 __device__ __forceinline__ float warp_sum(float v) {
 #pragma unroll
   for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);

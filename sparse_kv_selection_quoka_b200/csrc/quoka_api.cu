@@ -254,7 +254,7 @@ quoka_status quoka_select(const quoka_tensor* Q, const quoka_tensor* K, int NQ, 
   st = check_ws(ws, ws_bytes, L);
   if (st != QUOKA_OK) return st;
   cudaStream_t cs = static_cast<cudaStream_t>(stream);
-  if (cudaMemsetAsync(at<int>(ws, L.status), 0, sizeof(int), cs) != cudaSuccess) return QUOKA_ERR_CUDA;
+  if (cudaMemsetAsync(at<int>(ws, L.status), 0, 2 * sizeof(int), cs) != cudaSuccess) return QUOKA_ERR_CUDA;
   return run_select(Q, K, s, NQ, (int)bsa_eff, kv_idx, kv_count, q_idx, s_agg, ws, L, cs);
 }
 
@@ -275,9 +275,9 @@ quoka_status quoka_gather_kv(const quoka_tensor* K, const quoka_tensor* V, const
   cudaStream_t cs = static_cast<cudaStream_t>(stream);
   int* status = nullptr;
   if (ws != nullptr) {
-    if (((uintptr_t)ws % kAlign) != 0 || ws_bytes < sizeof(int)) return QUOKA_ERR_WORKSPACE;
+    if (((uintptr_t)ws % kAlign) != 0 || ws_bytes < 2 * sizeof(int)) return QUOKA_ERR_WORKSPACE;
     status = static_cast<int*>(ws);
-    if (cudaMemsetAsync(status, 0, sizeof(int), cs) != cudaSuccess) return QUOKA_ERR_CUDA;
+    if (cudaMemsetAsync(status, 0, 2 * sizeof(int), cs) != cudaSuccess) return QUOKA_ERR_CUDA;
   }
   cudaError_t e = quoka::launch_gather(K->dtype == QUOKA_BF16, (int)ks[3], strided(K), strided(V),
                                        (int)ks[0], (int)ks[1], ks[2], kv_idx, kv_count, BSA_eff, Ksel,
@@ -299,7 +299,7 @@ quoka_status quoka_sparse_gqa_attn(const quoka_tensor* Q, const quoka_tensor* K,
   if (ws == nullptr || ((uintptr_t)ws % kAlign) != 0 || ws_bytes < kAlign) return QUOKA_ERR_WORKSPACE;
   cudaStream_t cs = static_cast<cudaStream_t>(stream);
   int* status = static_cast<int*>(ws);
-  if (cudaMemsetAsync(status, 0, sizeof(int), cs) != cudaSuccess) return QUOKA_ERR_CUDA;
+  if (cudaMemsetAsync(status, 0, 2 * sizeof(int), cs) != cudaSuccess) return QUOKA_ERR_CUDA;
   return run_attn(Q, K, V, Kc, Vc, s, kv_idx, kv_count, BSA_eff, scale, O, lse, status, cs);
 }
 
@@ -322,7 +322,7 @@ quoka_status quoka_prefill_chunk(const quoka_tensor* Q, const quoka_tensor* K,
   if (st != QUOKA_OK) return st;
   cudaStream_t cs = static_cast<cudaStream_t>(stream);
   int* status = at<int>(ws, L.status);
-  if (cudaMemsetAsync(status, 0, sizeof(int), cs) != cudaSuccess) return QUOKA_ERR_CUDA;
+  if (cudaMemsetAsync(status, 0, 2 * sizeof(int), cs) != cudaSuccess) return QUOKA_ERR_CUDA;
   int32_t* kv_idx = kv_idx_out != nullptr ? kv_idx_out : at<int32_t>(ws, L.kvidx);
   int32_t* kv_count = at<int32_t>(ws, L.kvcount);
   st = run_select(Q, K, s, NQ, (int)bsa_eff, kv_idx, kv_count, nullptr, nullptr, ws, L, cs);
