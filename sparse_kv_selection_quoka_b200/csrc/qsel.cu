@@ -1,5 +1,9 @@
 // Query subselection and GQA group mean.
 //
+// Two variants of the selection kernel compute the same thing: the staged one
+// (the default) copies a head's query block into shared memory first; the
+// direct one reads global memory and serves chunks whose block does not fit.
+//
 // [QUOKA §2.1, Algorithm 1] MQ = mean of the chunk's queries over its tokens;
 // SQ = -cos(Q, MQ); the NQ queries with the largest SQ are kept, in rank
 // order. [QUOKA §2.3] the kept queries are L2-normalised and averaged over
@@ -107,6 +111,115 @@ qsel_kernel(const T* __restrict__ Q, int64_t sQb, int64_t sQh, int64_t sQt, int 
   }
 }
 
+constexpr int QSEL_STAGED_THREADS = 512;
+constexpr int QSEL_STAGED_WARPS = QSEL_STAGED_THREADS / 32;
+constexpr size_t QSEL_STAGED_MAX_BYTES = 192 * 1024;
+
+// The same computation with the head's whole (BCP, D) query block staged in
+// shared memory first (16-byte vector loads, all in flight at once), so that
+// the mean, the scores and the normalisation read shared memory. Dynamic
+// shared memory: the block (row-major, element type T), SQ[BCP], sel[NQ].
+template <typename T, int D>
+__global__ void __launch_bounds__(QSEL_STAGED_THREADS)
+qsel_staged_kernel(const T* __restrict__ Q, int64_t sQb, int64_t sQh, int64_t sQt, int BCP, int NQ,
+                   float* __restrict__ Qhat, int32_t* __restrict__ q_idx) {
+  extern __shared__ __align__(16) uint8_t qs_raw[];
+  T* blk = reinterpret_cast<T*>(qs_raw);
+  const size_t blk_bytes = ((size_t)BCP * D * sizeof(T) + 15) & ~size_t(15);
+  float* SQ = reinterpret_cast<float*>(qs_raw + blk_bytes);
+  int* sel = reinterpret_cast<int*>(SQ + BCP);
+  __shared__ float part[QSEL_STAGED_THREADS];
+  __shared__ float mq[D];
+  __shared__ float mq_norm;
+
+  const int h = blockIdx.x, bi = blockIdx.y, nq = gridDim.x;
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  const T* Qh = Q + bi * sQb + h * sQh;
+
+  // stage: row t, 16-byte vector v of the row
+  constexpr int VPR = D * (int)sizeof(T) / 16;  // vectors per row
+#pragma unroll 8
+  for (int e = tid; e < BCP * VPR; e += QSEL_STAGED_THREADS) {
+    const int t = e / VPR, v = e % VPR;
+    reinterpret_cast<uint4*>(blk + (size_t)t * D)[v] =
+        __ldg(reinterpret_cast<const uint4*>(Qh + (int64_t)t * sQt) + v);
+  }
+  for (int i = tid; i < NQ; i += QSEL_STAGED_THREADS) sel[i] = 0;
+  __syncthreads();
+
+  // (a) mean over tokens: column c = tid % D, token groups of 512 / D rows
+  constexpr int NGRP = QSEL_STAGED_THREADS / D;
+  {
+    const int c = tid % D, grp = tid / D;
+    float acc = 0.f;
+    for (int t = grp; t < BCP; t += NGRP) acc += to_f32(blk[(size_t)t * D + c]);
+    part[tid] = acc;
+  }
+  __syncthreads();
+  if (tid < D) {
+    float sum = 0.f;
+#pragma unroll
+    for (int g = 0; g < NGRP; ++g) sum += part[g * D + tid];
+    mq[tid] = sum / (float)BCP;
+  }
+  __syncthreads();
+  if (warp == 0) {
+    float sum = 0.f;
+    for (int k = lane; k < D; k += 32) sum += mq[k] * mq[k];
+    sum = warp_sum(sum);
+    if (lane == 0) mq_norm = sqrtf(sum);
+  }
+  __syncthreads();
+
+  // (a) SQ[t] = -(q_t . MQ) / max(|q_t| |MQ|, 1e-8), one warp per token
+  for (int t = warp; t < BCP; t += QSEL_STAGED_WARPS) {
+    const T* q = blk + (size_t)t * D;
+    float dot = 0.f, qq = 0.f;
+#pragma unroll
+    for (int k = lane; k < D; k += 32) {
+      const float v = to_f32(q[k]);
+      dot += v * mq[k];
+      qq += v * v;
+    }
+    dot = warp_sum(dot);
+    qq = warp_sum(qq);
+    if (lane == 0) SQ[t] = -dot / fmaxf(sqrtf(qq) * mq_norm, 1e-8f);
+  }
+  __syncthreads();
+
+  // (b) rank of token t = number of tokens that beat it (larger SQ, or equal
+  // SQ at a lower position)
+  for (int t = tid; t < BCP; t += QSEL_STAGED_THREADS) {
+    const float v = SQ[t];
+    int r = 0;
+    for (int u = 0; u < BCP; ++u) {
+      const float w = SQ[u];
+      r += (w > v) | ((w == v) & (u < t));
+    }
+    if (r < NQ) sel[r] = t;
+  }
+  __syncthreads();
+
+  // (c) L2-normalise the kept queries, one warp per rank
+  for (int i = warp; i < NQ; i += QSEL_STAGED_WARPS) {
+    const int t = sel[i];
+    const T* q = blk + (size_t)t * D;
+    float v[D / 32];
+    float qq = 0.f;
+#pragma unroll
+    for (int k = 0; k < D / 32; ++k) {
+      v[k] = to_f32(q[lane + 32 * k]);
+      qq += v[k] * v[k];
+    }
+    qq = warp_sum(qq);
+    const float nrm = fmaxf(sqrtf(qq), 1e-12f);
+    float* dst = Qhat + (((int64_t)bi * nq + h) * NQ + i) * D;
+#pragma unroll
+    for (int k = 0; k < D / 32; ++k) dst[lane + 32 * k] = v[k] / nrm;
+    if (lane == 0 && q_idx != nullptr) q_idx[((int64_t)bi * nq + h) * NQ + i] = t;
+  }
+}
+
 // Q_group[b, j, i, :] = (1/G) sum_{g<G} Qhat[b, jG+g, i, :], summed in head
 // order; optionally split into bf16 hi = rn(x) and lo = rn(x - hi).
 template <int D>
@@ -132,6 +245,16 @@ qgroup_kernel(const float* __restrict__ Qhat, int nq, int NQ, float* __restrict_
 template <typename T, int D>
 static cudaError_t qsel_typed(Strided Q, int b, int nq, int BCP, int NQ, float* Qhat,
                               int32_t* q_idx, cudaStream_t stream) {
+  const size_t blk_bytes = ((size_t)BCP * D * sizeof(T) + 15) & ~size_t(15);
+  const size_t staged = blk_bytes + (size_t)BCP * sizeof(float) + (size_t)NQ * sizeof(int);
+  if (staged <= QSEL_STAGED_MAX_BYTES) {
+    auto kern = qsel_staged_kernel<T, D>;
+    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)staged);
+    if (e != cudaSuccess) return e;
+    kern<<<dim3(nq, b), QSEL_STAGED_THREADS, staged, stream>>>(static_cast<const T*>(Q.data), Q.sb, Q.sh, Q.st,
+                                                               BCP, NQ, Qhat, q_idx);
+    return cudaGetLastError();
+  }
   const size_t smem = (size_t)BCP * sizeof(float) + (size_t)NQ * sizeof(int);
   auto kern = qsel_kernel<T, D>;
   if (smem > 48 * 1024) {

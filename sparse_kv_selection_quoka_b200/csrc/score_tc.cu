@@ -1,11 +1,306 @@
-// Key scoring on the tcgen05 tensor cores (placeholder until the kernel lands).
+// Key scoring on the tcgen05 tensor cores, K streamed from HBM once by TMA.
+//
+// [QUOKA §2.2] cosine score, [QUOKA §2.3] S = Q_group . K_norm^T reduced by a
+// max over the NQ chosen queries:
+//   S_agg[b, j, tau] = max_i (Q_group[b, j, i] . K[b, j, tau]) / |K[b, j, tau]|
+// The max commutes with the positive factor 1/|k|, so each key is divided
+// once, after the max. (QUOKA = the technical write-up "QUOKA: how it
+// reshapes LLM prefill efficiency", bqwf.cn news item 915859.)
+//
+// Precision: K is bf16 (exact on the tensor core); the fp32 group means are
+// split into bf16 hi + lo and both halves are multiplied, so the score
+// carries ~16 significant bits of the query instead of 8:
+//   D[key, i] = K . hi_i,  D[key, NQp + i] = K . lo_i  (NQp = NQ rounded up to 16),  s_i = D[key,i] + D[key,NQp+i]
+// with fp32 accumulation; |k| is summed in fp32 from the same shared-memory
+// tile the tensor core reads.
+//
+// Work split: each CTA owns a contiguous range of 128-key tiles of one
+// (batch, KV head); the grid has about one CTA per SM.
+// Warp roles (192 threads):
+//   warp 0      TMA producer: 4-D tensor map over the (possibly strided) K
+//               view, two 64-column boxes per tile in the 128-byte swizzle,
+//               into a ring of up to 6 stages (no multicast);
+//   warp 1      TMEM allocation and single-thread MMA issue,
+//               M=128 keys x N=2*NQp x K=128, into a double-buffered
+//               accumulator;
+//   warps 2-5   epilogue: thread = key (TMEM lane): max over the NQ
+//               columns, |k| from shared memory, S_agg store.
+// Every wait is bounded (see sm100.cuh); a wait that gives up records
+// QUOKA_ERR_TIMEOUT and the CTA unwinds.
+#include <cuda.h>
+#include <cudaTypedefs.h>
+
+#include "common.cuh"
 #include "kernels.h"
+#include "sm100.cuh"
 
 namespace quoka {
 
-cudaError_t launch_score_tc(int, Strided, int, int, int64_t, const uint16_t*, int, float*, int*,
-                            cudaStream_t) {
-  return cudaErrorNotSupported;
+using namespace sm100;
+
+namespace {
+
+constexpr int SC_D = 128;
+constexpr int SC_KEYS = 128;
+constexpr int SC_THREADS = 192;
+constexpr int SC_MAX_STAGES = 6;
+constexpr int SC_TILE_BYTES = SC_KEYS * SC_D * 2;  // 32 KiB
+constexpr int SC_ATOM = SC_KEYS * 128;             // one 64-column atom of a K tile
+
+struct ScoreBars {
+  uint64_t full[SC_MAX_STAGES];
+  uint64_t empty[SC_MAX_STAGES];
+  uint64_t tfull[2];
+  uint64_t tempty[2];
+  uint64_t done;
+  uint32_t tmem_base;
+  int abort;
+};
+
+struct ScoreArgs {
+  const uint16_t* qg_hilo;  // (b, nkv, 2*NQ, d) bf16: rows [0,NQ) hi, [NQ,2NQ) lo
+  float* s_agg;             // (b, nkv, T)
+  int* status;
+  int64_t T;
+  int NQ, NQp, nstages, tiles_per_cta, ntiles;
+  uint32_t tmem_cols;
+};
+
+__device__ __forceinline__ void sc_abort(ScoreBars& sb, int* status, int where) {
+  sb.abort = 1;
+  latch_status(status, 5 /* QUOKA_ERR_TIMEOUT */);
+  latch_where(status, where);
+}
+
+__device__ __forceinline__ bool sc_warp_wait(uint64_t* bar, uint32_t parity, ScoreBars& sb, int* status,
+                                             int where) {
+  const bool ok = mbar_wait(bar, parity, &sb.abort);
+  const bool all_ok = __all_sync(0xffffffffu, ok);
+  if (!all_ok && (threadIdx.x & 31) == 0) sc_abort(sb, status, where);
+  return all_ok;
+}
+
+__global__ void __launch_bounds__(SC_THREADS, 1)
+score_tc_kernel(const __grid_constant__ CUtensorMap tmap, const ScoreArgs a) {
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* base = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  const int N = 2 * a.NQp;                         // MMA N: hi rows then lo rows
+  uint8_t* qg_s = base;                            // [2 atoms][N rows][128 B]
+  const int qg_bytes = ((N * 256) + 1023) & ~1023;
+  uint8_t* ring = base + qg_bytes;                 // [nstages][32 KiB]
+  ScoreBars& sb = *reinterpret_cast<ScoreBars*>(ring + (size_t)a.nstages * SC_TILE_BYTES);
+
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int j = blockIdx.y, bi = blockIdx.z, nkv = gridDim.y;
+  const int64_t row = (int64_t)bi * nkv + j;
+  const int t_begin = blockIdx.x * a.tiles_per_cta;
+  const int n = max(0, min(a.ntiles, t_begin + a.tiles_per_cta) - t_begin);
+  const int NS = a.nstages;
+
+  if (tid == 0) {
+    for (int s = 0; s < NS; ++s) {
+      mbar_init(&sb.full[s], 1);
+      mbar_init(&sb.empty[s], 128);
+    }
+    for (int q = 0; q < 2; ++q) {
+      mbar_init(&sb.tfull[q], 1);
+      mbar_init(&sb.tempty[q], 128);
+    }
+    mbar_init(&sb.done, 1);
+    sb.abort = 0;
+    asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+    tma_prefetch_desc(&tmap);
+  }
+  if (warp == 1) {
+    tmem_alloc(&sb.tmem_base, a.tmem_cols);
+    tmem_relinquish();
+  }
+  // B operand: the group means (hi rows then lo rows, each padded to NQp
+  // with zero rows) in the K-major 128-byte-swizzled layout.
+  {
+    const uint16_t* src = a.qg_hilo + row * 2 * a.NQ * SC_D;
+    for (int e = tid; e < N * 16; e += SC_THREADS) {
+      const int r = e >> 4, c = e & 15;
+      const int half = r >= a.NQp;  // 0 = hi, 1 = lo
+      const int i = r - half * a.NQp;
+      uint4 v = make_uint4(0u, 0u, 0u, 0u);
+      if (i < a.NQ) v = *reinterpret_cast<const uint4*>(src + ((int64_t)(half * a.NQ + i)) * SC_D + c * 8);
+      *reinterpret_cast<uint4*>(qg_s + sw128_offset(r, c, N)) = v;
+    }
+    fence_proxy_async_smem();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = sb.tmem_base;
+
+  if (warp == 0) {
+    // ------------------------------------------------------------ TMA producer
+    if (lane == 0) {
+      for (int it = 0; it < n; ++it) {
+        const int s = it % NS;
+        if (it >= NS && !mbar_wait(&sb.empty[s], ((it / NS) - 1) & 1, &sb.abort)) {
+          sc_abort(sb, a.status, 51);
+          break;
+        }
+        const uint32_t dst = smem_u32(ring + (size_t)s * SC_TILE_BYTES);
+        mbar_arrive_expect_tx(&sb.full[s], SC_TILE_BYTES);
+        const int y = (t_begin + it) * SC_KEYS;
+        tma_load_4d(dst, &tmap, &sb.full[s], 0, y, j, bi);
+        tma_load_4d(dst + SC_ATOM, &tmap, &sb.full[s], 64, y, j, bi);
+      }
+    }
+    __syncwarp();
+  } else if (warp == 1) {
+    // ------------------------------------------------------------ MMA issue
+    if (lane == 0) {
+      const uint32_t idesc = idesc_bf16_f32(SC_KEYS, N, 0, 0);
+      const uint32_t qg = smem_u32(qg_s);
+      bool alive = true;
+      int where = 0;
+      for (int it = 0; it < n && alive; ++it) {
+        const int s = it % NS, acc = it & 1;
+        where = 52;
+        alive = mbar_wait(&sb.full[s], (it / NS) & 1, &sb.abort);
+        if (alive && it >= 2) {
+          where = 53;
+          alive = mbar_wait(&sb.tempty[acc], ((it >> 1) - 1) & 1, &sb.abort);
+        }
+        if (!alive) break;
+        tc_fence_after();
+        const uint32_t ks = smem_u32(ring + (size_t)s * SC_TILE_BYTES);
+#pragma unroll
+        for (int kk = 0; kk < SC_D / 16; ++kk) {
+          const uint64_t ad = sw128_desc(ks + (kk >> 2) * SC_ATOM + (kk & 3) * 32, 16, 1024);
+          const uint64_t bd = sw128_desc(qg + (kk >> 2) * (N * 128) + (kk & 3) * 32, 16, 1024);
+          umma_bf16_ss(tmem + (uint32_t)(acc * N), ad, bd, idesc, kk > 0 ? 1u : 0u);
+        }
+        umma_commit(&sb.tfull[acc]);
+      }
+      if (!alive) sc_abort(sb, a.status, where);
+      umma_commit(&sb.done);
+      if (!mbar_drain(&sb.done, 0)) sc_abort(sb, a.status, 54);
+    }
+    __syncwarp();
+  } else {
+    // ------------------------------------------------------------ epilogue
+    const int q = warp & 3;                  // TMEM lane quarter of this warp
+    const int r = q * 32 + lane;             // key within the tile
+    const uint32_t lane_off = (uint32_t)(q * 32) << 16;
+    float* out = a.s_agg + row * a.T;
+    for (int it = 0; it < n; ++it) {
+      const int s = it % NS, acc = it & 1;
+      if (!sc_warp_wait(&sb.tfull[acc], (it >> 1) & 1, sb, a.status, 55)) break;
+      tc_fence_after();
+      float mx = -INFINITY;
+      const uint32_t tbase = tmem + lane_off + (uint32_t)(acc * N);
+      for (int c0 = 0; c0 < a.NQp; c0 += 16) {
+        float hi[16], lo[16];
+        tmem_ld16(tbase + c0, hi);
+        tmem_ld16(tbase + a.NQp + c0, lo);
+        tmem_wait_ld();
+#pragma unroll
+        for (int u = 0; u < 16; ++u)
+          if (c0 + u < a.NQ) mx = fmaxf(mx, hi[u] + lo[u]);
+      }
+      tc_fence_before();
+      mbar_arrive(&sb.tempty[acc]);
+      // |k| from the tile in shared memory (the TMA writes are visible to
+      // threads that observe the stage's barrier)
+      if (!sc_warp_wait(&sb.full[s], (it / NS) & 1, sb, a.status, 56)) break;
+      const uint8_t* tile = ring + (size_t)s * SC_TILE_BYTES;
+      float ss = 0.f;
+#pragma unroll
+      for (int c = 0; c < 16; ++c) {
+        const uint4 raw = *reinterpret_cast<const uint4*>(tile + sw128_offset(r, c, SC_KEYS));
+        const __nv_bfloat162* h2 = reinterpret_cast<const __nv_bfloat162*>(&raw);
+#pragma unroll
+        for (int u = 0; u < 4; ++u) {
+          const float2 f = __bfloat1622float2(h2[u]);
+          ss = fmaf(f.x, f.x, ss);
+          ss = fmaf(f.y, f.y, ss);
+        }
+      }
+      mbar_arrive(&sb.empty[s]);
+      const int64_t key = (int64_t)(t_begin + it) * SC_KEYS + r;
+      if (key < a.T) out[key] = mx / fmaxf(sqrtf(ss), 1e-12f);
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc(tmem, a.tmem_cols);
+  }
+}
+
+PFN_cuTensorMapEncodeTiled_v12000 tensor_map_encoder() {
+  static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+  static bool tried = false;
+  if (!tried) {
+    tried = true;
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(p);
+  }
+  return fn;
+}
+
+}  // namespace
+
+cudaError_t launch_score_tc(int d, Strided K, int b, int nkv, int64_t T, const uint16_t* Qg_hilo, int NQ,
+                            float* S_agg, int* status, cudaStream_t stream) {
+  if (d != SC_D || NQ < 1 || NQ > 128 || T <= 0 || T > (int64_t)INT32_MAX - SC_KEYS) return cudaErrorNotSupported;
+  PFN_cuTensorMapEncodeTiled_v12000 encode = tensor_map_encoder();
+  if (encode == nullptr) return cudaErrorNotSupported;
+
+  CUtensorMap tmap;
+  const cuuint64_t dims[4] = {(cuuint64_t)SC_D, (cuuint64_t)T, (cuuint64_t)nkv, (cuuint64_t)b};
+  const cuuint64_t strides[3] = {(cuuint64_t)K.st * 2, (cuuint64_t)K.sh * 2, (cuuint64_t)K.sb * 2};
+  const cuuint32_t box[4] = {64, SC_KEYS, 1, 1};
+  const cuuint32_t estr[4] = {1, 1, 1, 1};
+  CUresult r = encode(&tmap, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, const_cast<void*>(K.data), dims, strides, box,
+                      estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                      CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  if (r != CUDA_SUCCESS) return cudaErrorNotSupported;
+
+  ScoreArgs a;
+  a.qg_hilo = Qg_hilo;
+  a.s_agg = S_agg;
+  a.status = status;
+  a.T = T;
+  a.NQ = NQ;
+  a.NQp = (NQ + 15) / 16 * 16;  // the epilogue reads 16-column groups
+  const int N = 2 * a.NQp;
+  uint32_t cols = 32;
+  while (cols < (uint32_t)(2 * N)) cols <<= 1;
+  a.tmem_cols = cols;
+  const int qg_bytes = ((N * 256) + 1023) & ~1023;
+  const int smem_cap = 227 * 1024;
+  const int bars = (int)sizeof(ScoreBars) + 1024;
+  a.nstages = (smem_cap - qg_bytes - bars) / SC_TILE_BYTES;
+  if (a.nstages > SC_MAX_STAGES) a.nstages = SC_MAX_STAGES;
+  if (a.nstages < 2) return cudaErrorNotSupported;
+  a.ntiles = (int)((T + SC_KEYS - 1) / SC_KEYS);
+
+  int num_sms = 148;
+  int dev = 0;
+  if (cudaGetDevice(&dev) == cudaSuccess) cudaDeviceGetAttribute(&num_sms, cudaDevAttrMultiProcessorCount, dev);
+  // at most one CTA per SM in total (one CTA fills an SM's shared memory)
+  int per_head = num_sms / (nkv * b);
+  if (per_head > a.ntiles) per_head = a.ntiles;
+  if (per_head < 1) per_head = 1;
+  a.tiles_per_cta = (a.ntiles + per_head - 1) / per_head;
+  per_head = (a.ntiles + a.tiles_per_cta - 1) / a.tiles_per_cta;
+
+  const size_t smem = (size_t)qg_bytes + (size_t)a.nstages * SC_TILE_BYTES + sizeof(ScoreBars) + 1024;
+  cudaError_t e = cudaFuncSetAttribute(score_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+  if (e != cudaSuccess) return e;
+  score_tc_kernel<<<dim3(per_head, nkv, b), SC_THREADS, smem, stream>>>(tmap, a);
+  return cudaGetLastError();
 }
 
 }  // namespace quoka

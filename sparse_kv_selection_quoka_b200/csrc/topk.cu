@@ -128,7 +128,22 @@ topk_cluster_kernel(const float* __restrict__ S, int64_t T, int bsa, int slice,
   const int n = (int)max((int64_t)0, min((int64_t)slice, T - lo));
   const int n_round = (n + TOPK_THREADS - 1) / TOPK_THREADS * TOPK_THREADS;
 
-  for (int e = tid; e < n; e += TOPK_THREADS) keys[e] = score_key(Sr[lo + e]);
+  // stage the slice as keys: 16-byte loads when the slice start is aligned
+  if ((((uintptr_t)(Sr + lo)) & 15u) == 0u) {
+    const int n4 = n >> 2;
+    const float4* src4 = reinterpret_cast<const float4*>(Sr + lo);
+#pragma unroll 4
+    for (int e = tid; e < n4; e += TOPK_THREADS) {
+      const float4 v = __ldg(src4 + e);
+      keys[4 * e] = score_key(v.x);
+      keys[4 * e + 1] = score_key(v.y);
+      keys[4 * e + 2] = score_key(v.z);
+      keys[4 * e + 3] = score_key(v.w);
+    }
+    for (int e = 4 * n4 + tid; e < n; e += TOPK_THREADS) keys[e] = score_key(Sr[lo + e]);
+  } else {
+    for (int e = tid; e < n; e += TOPK_THREADS) keys[e] = score_key(Sr[lo + e]);
+  }
 
   uint32_t prefix = 0u, pmask = 0u;
   uint32_t need = (uint32_t)bsa;  // rank (1-based, from the top) still to place
@@ -153,10 +168,22 @@ topk_cluster_kernel(const float* __restrict__ S, int64_t T, int bsa, int slice,
     uint32_t mine[4] = {0u, 0u, 0u, 0u};
     uint32_t tot = 0u;
     if (tid * q < nbins) {
-      for (int r = 0; r < C; ++r) {
-        const uint32_t* Hr = cluster.map_shared_rank(H, r);
-        for (int u = 0; u < q; ++u) mine[u] += Hr[nbins - 1 - (tid * q + u)];
+      // all remote loads are issued before any is used
+      uint32_t got[TOPK_MAX_CLUSTER][4];
+#pragma unroll
+      for (int r = 0; r < TOPK_MAX_CLUSTER; ++r) {
+        if (r < C) {
+          const uint32_t* Hr = cluster.map_shared_rank(H, r);
+#pragma unroll
+          for (int u = 0; u < 4; ++u) got[r][u] = u < q ? Hr[nbins - 1 - (tid * q + u)] : 0u;
+        }
       }
+#pragma unroll
+      for (int r = 0; r < TOPK_MAX_CLUSTER; ++r)
+        if (r < C) {
+#pragma unroll
+          for (int u = 0; u < 4; ++u) mine[u] += got[r][u];
+        }
       for (int u = 0; u < q; ++u) tot += mine[u];
     }
     uint32_t dummy;
