@@ -347,48 +347,75 @@ attn_tc_kernel(const AttnArgs a, int nsplit) {
       if (!alive) break;
       tc_fence_after();
       const int base_n = (first + it) * AT_N;
-      // pass 1: row max of the visible scaled scores
-      float mx = -INFINITY;
+      // Every key of this tile is visible to this row unless the tile runs
+      // past the key list or holds chunk keys after position t; such rows
+      // take the masked path, all others skip the per-key test.
+      const bool all_vis = (base_n + AT_N <= total) && (base_n + AT_N - 1 - nsel <= t);
+      // pass 1: row max of the visible scaled scores. The TMEM loads are
+      // warp-collective, so they stay outside the per-row branches.
+      float m4[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
+      float mxs = -INFINITY;
 #pragma unroll 1
       for (int c4 = 0; c4 < 4; ++c4) {
         float v[32];
+        __syncwarp();
         tmem_ld32(S + 32 * c4, v);
         tmem_wait_ld();
+        if (all_vis) {
 #pragma unroll
-        for (int u = 0; u < 32; ++u) {
-          const int n = base_n + 32 * c4 + u;
-          const bool vis = n < nsel || (n < total && n - nsel <= t);
-          mx = vis ? fmaxf(mx, v[u] * qscale) : mx;
+          for (int u = 0; u < 32; ++u) m4[u & 3] = fmaxf(m4[u & 3], v[u]);
+        } else {
+#pragma unroll
+          for (int u = 0; u < 32; ++u) {
+            const int n = base_n + 32 * c4 + u;
+            const bool vis = n < nsel || (n < total && n - nsel <= t);
+            mxs = vis ? fmaxf(mxs, v[u] * qscale) : mxs;
+          }
         }
       }
+      const float mx = all_vis ? fmaxf(fmaxf(m4[0], m4[1]), fmaxf(m4[2], m4[3])) * qscale : mxs;
       const float m_cand = fmaxf(m, mx);
       const float m_new = (m_cand > m + RESCALE_THRESHOLD || m == -INFINITY) ? m_cand : m;
       const float corr = (m_new == m) ? 1.f : ex2(m - m_new);
       const float m_use = m_new == -INFINITY ? 0.f : m_new;
       // pass 2: P = 2^(s - m) in bf16, written over consumed S columns
-      float rs = 0.f;
+      float rs4[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll 1
       for (int c4 = 0; c4 < 4; ++c4) {
         float v[32];
+        __syncwarp();
         tmem_ld32(S + 32 * c4, v);
         tmem_wait_ld();
         uint32_t pk[16];
+        if (all_vis) {
 #pragma unroll
-        for (int u = 0; u < 32; u += 2) {
-          const int n = base_n + 32 * c4 + u;
-          const bool vis0 = n < nsel || (n < total && n - nsel <= t);
-          const bool vis1 = n + 1 < nsel || (n + 1 < total && n + 1 - nsel <= t);
-          const float p0 = vis0 ? ex2(v[u] * qscale - m_use) : 0.f;
-          const float p1 = vis1 ? ex2(v[u + 1] * qscale - m_use) : 0.f;
-          rs += p0 + p1;
-          pk[u >> 1] = pack_bf16x2(p0, p1);
+          for (int u = 0; u < 32; u += 2) {
+            const float p0 = ex2(fmaf(v[u], qscale, -m_use));
+            const float p1 = ex2(fmaf(v[u + 1], qscale, -m_use));
+            rs4[(u >> 1) & 3] += p0 + p1;
+            pk[u >> 1] = pack_bf16x2(p0, p1);
+          }
+        } else {
+#pragma unroll
+          for (int u = 0; u < 32; u += 2) {
+            const int n = base_n + 32 * c4 + u;
+            const bool vis0 = n < nsel || (n < total && n - nsel <= t);
+            const bool vis1 = n + 1 < nsel || (n + 1 < total && n + 1 - nsel <= t);
+            const float p0 = vis0 ? ex2(fmaf(v[u], qscale, -m_use)) : 0.f;
+            const float p1 = vis1 ? ex2(fmaf(v[u + 1], qscale, -m_use)) : 0.f;
+            rs4[(u >> 1) & 3] += p0 + p1;
+            pk[u >> 1] = pack_bf16x2(p0, p1);
+          }
         }
+        __syncwarp();
         tmem_st16(S + 16 * c4, pk);
       }
+      const float rs = (rs4[0] + rs4[1]) + (rs4[2] + rs4[3]);
       l = l * corr + rs;
       m = m_new;
       // O holds the products of the previous tiles (complete: they were
       // issued before this tile's QK^T, whose completion we waited for)
+      // (warp-uniform condition: the rescale's TMEM traffic is collective)
       if (it > 0 && __any_sync(0xffffffffu, corr != 1.f)) {
 #pragma unroll 1
         for (int c4 = 0; c4 < 4; ++c4) {
