@@ -11,14 +11,14 @@
 // Work split. The query rows of one KV head j are cut into 128-row tiles
 // (one query head, 128 consecutive chunk positions each); a CTA takes two
 // such tiles (Q0, Q1) of the same KV head, so every K/V tile it brings in
-// feeds two 128x128x128 QK^T and two PV products. The key list of a CTA is
-// the selected prior rows (read in place through the sorted index list: the
-// gather is fused into the loads) followed by the chunk's keys, in tiles of
-// 128 keys. When the grid would fill less than half of the GPU, the key
+// feeds two 128x128x128 QK^T and two PV products. The key tiles of a CTA
+// are ceil(nsel/128) tiles of selected prior rows (read in place through the
+// sorted index list: the gather is fused into the loads; rows past nsel are
+// masked) followed by ceil(nchunk/128) tiles of the chunk's own keys. When the grid would fill less than half of the GPU, the key
 // tiles are split between the two CTAs of a cluster, and the partial results
 // are combined through distributed shared memory.
 //
-// Warp roles (384 threads):
+// Warp roles (544 threads):
 //   warps 0-3   softmax of Q0, warps 4-7 softmax of Q1: thread r owns query
 //               row r = TMEM lane r. Two passes over its S row in TMEM (row
 //               max, then exp2 on the MUFU); P is written back as bf16 over
@@ -29,17 +29,23 @@
 //   warp 8      TMEM allocation and the single-thread MMA issue, ordered
 //               QK0(i), PV1(i-1), QK1(i), PV0(i): while one softmax group
 //               works, the tensor core runs the other group's products.
-//   warps 9-11  loaders: cp.async 16-byte row chunks into a 2-stage K/V ring
-//               in the 128-byte-swizzled UMMA layout (zero-fill past the end
-//               of the key list); gather indices are prefetched a tile ahead;
-//               each thread's arrival on the stage barrier fires when its
-//               copies land.
+//   warps 9-16  loaders (256 threads): cp.async 16-byte row chunks, gathered
+//               by index, into a 2-stage K/V ring in the 128-byte-swizzled
+//               UMMA layout (zero-fill past the end of a list); each thread
+//               owns one 16-byte column chunk of 8 rows per tile, prefetches
+//               the next tile's gather indices, and its arrival on the stage
+//               barrier fires when its copies land. The Q tiles are 4-D TMA
+//               boxes (no multicast). Row gathers need many issuing threads:
+//               measured on B200, 16-byte cp.async gathers reach ~47 GB/s per
+//               SM from 256 threads but ~24 GB/s from 96, and TMA
+//               tile::gather4 ~16 GB/s.
 // TMEM: S0 | S1 | O0 | O1, 128 columns each (512).
 // Every wait is bounded: a wait that gives up records QUOKA_ERR_TIMEOUT and
 // the CTA unwinds (waits for in-flight copies and MMAs, frees TMEM).
 #include "common.cuh"
 #include "kernels.h"
 #include "sm100.cuh"
+#include "tmap.cuh"
 
 namespace quoka {
 
@@ -50,11 +56,12 @@ namespace {
 constexpr int AT_D = 128;        // head dim
 constexpr int AT_N = 128;        // keys per tile
 constexpr int AT_STAGES = 2;     // K/V ring depth
-constexpr int AT_THREADS = 384;
+constexpr int AT_THREADS = 544;
 constexpr int AT_MMA_WARP = 8;
 constexpr int AT_LD_WARP0 = 9;
-constexpr int AT_LD_THREADS = 96;
+constexpr int AT_LD_THREADS = 256;
 constexpr int AT_SM_THREADS = 256;
+constexpr int LD_ROWS = AT_N * 16 / AT_LD_THREADS;  // rows per loader thread per tile (8)
 constexpr int TILE_BYTES = 128 * AT_D * 2;  // 128 rows x 256 B
 constexpr int ATOM_BYTES = 128 * 128;       // one 64-column swizzle atom of a 128-row tile
 constexpr uint32_t TMEM_COLS = 512;
@@ -63,9 +70,10 @@ constexpr float RESCALE_THRESHOLD = 8.f;    // log2 units
 constexpr uint32_t IDESC_QK = idesc_bf16_f32(128, AT_N, 0, 0);  // A=Q K-major, B=K K-major
 constexpr uint32_t IDESC_PV = idesc_bf16_f32(128, AT_D, 0, 1);  // A=P (TMEM), B=V MN-major
 
-// loader geometry: 96 threads = 6 row groups x 16 chunks of 16 bytes
-constexpr int LD_ROWGROUPS = AT_LD_THREADS / 16;
-constexpr int LD_ROWS = (AT_N + LD_ROWGROUPS - 1) / LD_ROWGROUPS;  // 22
+// TMA tensor map of the queries (4-D boxes of 64 columns x 128 rows).
+struct AttnMaps {
+  CUtensorMap q;
+};
 
 struct __align__(1024) AttnSmem {
   uint8_t q[2][TILE_BYTES];
@@ -125,7 +133,7 @@ __device__ __forceinline__ uint32_t pack_bf16x2(float a, float b) {
 }
 
 __global__ void __launch_bounds__(AT_THREADS, 1)
-attn_tc_kernel(const AttnArgs a, int nsplit) {
+attn_tc_kernel(const __grid_constant__ AttnMaps maps, const AttnArgs a, int nsplit) {
   extern __shared__ uint8_t smem_raw[];
   AttnSmem& sm = *reinterpret_cast<AttnSmem*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
 
@@ -149,14 +157,15 @@ attn_tc_kernel(const AttnArgs a, int nsplit) {
   const int nsel = a.bsa > 0 ? max(0, min(a.kv_count[kvrow], a.bsa)) : 0;
   const int max_t0 = ti[1].valid ? max(ti[0].t0, ti[1].t0) : ti[0].t0;
   const int nchunk = min(a.BCP, max_t0 + 128);
-  const int total = nsel + nchunk;
-  const int nT = (total + AT_N - 1) / AT_N;
+  const int ntile_sel = (nsel + AT_N - 1) / AT_N;
+  const int ntile_chk = (nchunk + AT_N - 1) / AT_N;
+  const int nT = ntile_sel + ntile_chk;
   const int per = (nT + nsplit - 1) / nsplit;
   const int first = min(nT, split * per);
   const int ntiles = min(nT, first + per) - first;  // key tiles of this CTA (may be 0)
 
   if (tid == 0) {
-    mbar_init(&sm.q_full, AT_LD_THREADS);
+    mbar_init(&sm.q_full, 1);
     for (int s = 0; s < AT_STAGES; ++s) {
       mbar_init(&sm.kv_full[s], AT_LD_THREADS);
       mbar_init(&sm.kv_empty[s], 1);
@@ -188,39 +197,35 @@ attn_tc_kernel(const AttnArgs a, int nsplit) {
 
   if (warp >= AT_LD_WARP0) {
     // ------------------------------------------------------------ loaders
-    const int lt = tid - AT_LD_WARP0 * 32;  // 0..95
+    const int lt = tid - AT_LD_WARP0 * 32;  // 0..255
     const int c = lt & 15;                   // 16-byte chunk of a row
-    const int rg = lt >> 4;                  // row group 0..5: rows rg, rg+6, ...
-    const bf16* Kb = static_cast<const bf16*>(a.K.data) + bi * a.K.sb + j * a.K.sh;
-    const bf16* Vb = static_cast<const bf16*>(a.V.data) + bi * a.V.sb + j * a.V.sh;
-    const bf16* Kcb = static_cast<const bf16*>(a.Kc.data) + bi * a.Kc.sb + j * a.Kc.sh;
-    const bf16* Vcb = static_cast<const bf16*>(a.Vc.data) + bi * a.Vc.sb + j * a.Vc.sh;
-    const int32_t* idx = a.kv_idx + kvrow * a.bsa;
-    bool bad_index = false;
-
-    // Q tiles (zero rows past the chunk or for a missing second tile)
-    for (int w = 0; w < 2; ++w) {
-      const bf16* Qb = static_cast<const bf16*>(a.Q.data) + bi * a.Q.sb + ti[w].h * a.Q.sh;
-      const uint32_t q_s = smem_u32(sm.q[w]);
-      for (int r = rg; r < 128; r += LD_ROWGROUPS) {
-        const int t = ti[w].t0 + r;
-        const bool ok = ti[w].valid && t < a.BCP;
-        cp_async_16(q_s + sw128_offset(r, c, 128), ok ? Qb + (int64_t)t * a.Q.st + c * 8 : Kcb, ok ? 16u : 0u);
+    const int rg = lt >> 4;                  // rows rg, rg + 16, ... of a tile
+    if (lt == 0) {
+      tma_prefetch_desc(&maps.q);
+      mbar_arrive_expect_tx(&sm.q_full, (ti[1].valid ? 2 : 1) * TILE_BYTES);
+      for (int w = 0; w < 2; ++w) {
+        if (!ti[w].valid) continue;
+        const uint32_t q_s = smem_u32(sm.q[w]);
+        tma_load_4d(q_s, &maps.q, &sm.q_full, 0, ti[w].t0, ti[w].h, bi);
+        tma_load_4d(q_s + ATOM_BYTES, &maps.q, &sm.q_full, 64, ti[w].t0, ti[w].h, bi);
       }
     }
-    cp_async_arrive_noinc(&sm.q_full);
-
-    // gather indices of this thread's rows of tile `gi` (-1: chunk key or past the end)
+    const bf16* Kb = static_cast<const bf16*>(a.K.data) + bi * a.K.sb + j * a.K.sh + c * 8;
+    const bf16* Vb = static_cast<const bf16*>(a.V.data) + bi * a.V.sb + j * a.V.sh + c * 8;
+    const bf16* Kcb = static_cast<const bf16*>(a.Kc.data) + bi * a.Kc.sb + j * a.Kc.sh + c * 8;
+    const bf16* Vcb = static_cast<const bf16*>(a.Vc.data) + bi * a.Vc.sb + j * a.Vc.sh + c * 8;
+    const int32_t* idx = a.kv_idx + kvrow * a.bsa;
+    bool bad_index = false;
+    // gather indices of this thread's rows of selected tile `gi` (-1: past nsel)
     int32_t tau[LD_ROWS];
     auto fetch_idx = [&](int gi) {
 #pragma unroll
       for (int k = 0; k < LD_ROWS; ++k) {
-        const int r = rg + LD_ROWGROUPS * k;
-        const int n = gi * AT_N + r;
-        tau[k] = (r < AT_N && n < nsel) ? __ldg(idx + n) : -1;
+        const int n = gi * AT_N + rg + 16 * k;
+        tau[k] = n < nsel ? __ldg(idx + n) : -1;
       }
     };
-    if (ntiles > 0) fetch_idx(first);
+    if (ntiles > 0 && first < ntile_sel) fetch_idx(first);
     bool alive = true;
     for (int it = 0; it < ntiles && alive; ++it) {
       const int s = it % AT_STAGES;
@@ -228,36 +233,31 @@ attn_tc_kernel(const AttnArgs a, int nsplit) {
       if (it >= AT_STAGES) alive = warp_wait(&sm.kv_empty[s], ((it / AT_STAGES) - 1) & 1, sm, a.status, 11);
       if (!alive) break;
       const uint32_t k_s = smem_u32(sm.kv[s][0]), v_s = smem_u32(sm.kv[s][1]);
+      if (gi < ntile_sel) {
 #pragma unroll
-      for (int k = 0; k < LD_ROWS; ++k) {
-        const int r = rg + LD_ROWGROUPS * k;
-        if (r < AT_N) {
-          const int n = gi * AT_N + r;
-          const bf16* ks = Kcb;
-          const bf16* vs = Vcb;
-          uint32_t bytes = 0u;
-          if (n < nsel) {
-            const int32_t tv = tau[k];
-            if (tv >= 0 && (int64_t)tv < a.T) {
-              ks = Kb + (int64_t)tv * a.K.st + c * 8;
-              vs = Vb + (int64_t)tv * a.V.st + c * 8;
-              bytes = 16u;
-            } else {
-              bad_index = true;
-            }
-          } else if (n < total) {
-            const int p = n - nsel;
-            ks = Kcb + (int64_t)p * a.Kc.st + c * 8;
-            vs = Vcb + (int64_t)p * a.Vc.st + c * 8;
-            bytes = 16u;
-          }
+        for (int k = 0; k < LD_ROWS; ++k) {
+          const int r = rg + 16 * k;
+          const int32_t tv = tau[k];
+          const bool ok = tv >= 0 && (int64_t)tv < a.T;
+          bad_index |= (tv != -1) && !ok;
           const uint32_t off = sw128_offset(r, c, 128);
-          cp_async_16(k_s + off, ks, bytes);
-          cp_async_16(v_s + off, vs, bytes);
+          cp_async_16(k_s + off, ok ? Kb + (int64_t)tv * a.K.st : Kcb, ok ? 16u : 0u);
+          cp_async_16(v_s + off, ok ? Vb + (int64_t)tv * a.V.st : Vcb, ok ? 16u : 0u);
+        }
+        if (gi + 1 < ntile_sel && it + 1 < ntiles) fetch_idx(gi + 1);
+      } else {
+        const int p0 = (gi - ntile_sel) * AT_N;
+#pragma unroll
+        for (int k = 0; k < LD_ROWS; ++k) {
+          const int r = rg + 16 * k;
+          const int p = p0 + r;
+          const bool ok = p < nchunk;
+          const uint32_t off = sw128_offset(r, c, 128);
+          cp_async_16(k_s + off, Kcb + (int64_t)(ok ? p : 0) * a.Kc.st, ok ? 16u : 0u);
+          cp_async_16(v_s + off, Vcb + (int64_t)(ok ? p : 0) * a.Vc.st, ok ? 16u : 0u);
         }
       }
       cp_async_arrive_noinc(&sm.kv_full[s]);
-      if (it + 1 < ntiles) fetch_idx(gi + 1);
     }
     cp_async_wait<0>();
     if (bad_index) latch_status(a.status, 6 /* QUOKA_ERR_BOUNDS */);
@@ -346,69 +346,71 @@ attn_tc_kernel(const AttnArgs a, int nsplit) {
       alive = warp_wait(&sm.s_full[w], it & 1, sm, a.status, 31 + w);
       if (!alive) break;
       tc_fence_after();
-      const int base_n = (first + it) * AT_N;
-      // Every key of this tile is visible to this row unless the tile runs
-      // past the key list or holds chunk keys after position t; such rows
-      // take the masked path, all others skip the per-key test.
-      const bool all_vis = (base_n + AT_N <= total) && (base_n + AT_N - 1 - nsel <= t);
-      // pass 1: row max of the visible scaled scores. The TMEM loads are
-      // warp-collective, so they stay outside the per-row branches.
-      float m4[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
-      float mxs = -INFINITY;
+      const int gi = first + it;
+      const bool sel_tile = gi < ntile_sel;
+      // first key of the tile: selected-list index or chunk position
+      const int base_n = sel_tile ? gi * AT_N : (gi - ntile_sel) * AT_N;
+      // key c of the tile is visible to row t: a selected key below nsel, or
+      // a chunk key at a position p < nchunk with p <= t
+      const int lim = sel_tile ? nsel : min(nchunk, t + 1);
+      // rows whose every key of this tile is visible skip the per-key test
+      const bool all_vis = base_n + AT_N <= lim;
+      // pass 1: row max. TMEM loads are warp-collective, so they stay
+      // outside per-row branches; 64 columns per round trip.
+      float mx = -INFINITY;
 #pragma unroll 1
-      for (int c4 = 0; c4 < 4; ++c4) {
-        float v[32];
+      for (int h2 = 0; h2 < 2; ++h2) {
+        float v[64];
         __syncwarp();
-        tmem_ld32(S + 32 * c4, v);
+        tmem_ld32(S + 64 * h2, *reinterpret_cast<float(*)[32]>(&v[0]));
+        tmem_ld32(S + 64 * h2 + 32, *reinterpret_cast<float(*)[32]>(&v[32]));
         tmem_wait_ld();
         if (all_vis) {
+          float m4[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
 #pragma unroll
-          for (int u = 0; u < 32; ++u) m4[u & 3] = fmaxf(m4[u & 3], v[u]);
+          for (int u = 0; u < 64; ++u) m4[u & 3] = fmaxf(m4[u & 3], v[u]);
+          mx = fmaxf(mx, fmaxf(fmaxf(m4[0], m4[1]), fmaxf(m4[2], m4[3])) * qscale);
         } else {
 #pragma unroll
-          for (int u = 0; u < 32; ++u) {
-            const int n = base_n + 32 * c4 + u;
-            const bool vis = n < nsel || (n < total && n - nsel <= t);
-            mxs = vis ? fmaxf(mxs, v[u] * qscale) : mxs;
+          for (int u = 0; u < 64; ++u) {
+            const bool vis = base_n + 64 * h2 + u < lim;
+            mx = vis ? fmaxf(mx, v[u] * qscale) : mx;
           }
         }
       }
-      const float mx = all_vis ? fmaxf(fmaxf(m4[0], m4[1]), fmaxf(m4[2], m4[3])) * qscale : mxs;
       const float m_cand = fmaxf(m, mx);
       const float m_new = (m_cand > m + RESCALE_THRESHOLD || m == -INFINITY) ? m_cand : m;
       const float corr = (m_new == m) ? 1.f : ex2(m - m_new);
       const float m_use = m_new == -INFINITY ? 0.f : m_new;
-      // pass 2: P = 2^(s - m) in bf16, written over consumed S columns
+      // pass 2: P = 2^(s - m) in bf16, written over the S columns already read
       float rs4[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll 1
-      for (int c4 = 0; c4 < 4; ++c4) {
-        float v[32];
+      for (int h2 = 0; h2 < 2; ++h2) {
+        float v[64];
         __syncwarp();
-        tmem_ld32(S + 32 * c4, v);
+        tmem_ld32(S + 64 * h2, *reinterpret_cast<float(*)[32]>(&v[0]));
+        tmem_ld32(S + 64 * h2 + 32, *reinterpret_cast<float(*)[32]>(&v[32]));
         tmem_wait_ld();
-        uint32_t pk[16];
-        if (all_vis) {
+        if (!all_vis) {
 #pragma unroll
-          for (int u = 0; u < 32; u += 2) {
-            const float p0 = ex2(fmaf(v[u], qscale, -m_use));
-            const float p1 = ex2(fmaf(v[u + 1], qscale, -m_use));
-            rs4[(u >> 1) & 3] += p0 + p1;
-            pk[u >> 1] = pack_bf16x2(p0, p1);
-          }
-        } else {
-#pragma unroll
-          for (int u = 0; u < 32; u += 2) {
-            const int n = base_n + 32 * c4 + u;
-            const bool vis0 = n < nsel || (n < total && n - nsel <= t);
-            const bool vis1 = n + 1 < nsel || (n + 1 < total && n + 1 - nsel <= t);
-            const float p0 = vis0 ? ex2(fmaf(v[u], qscale, -m_use)) : 0.f;
-            const float p1 = vis1 ? ex2(fmaf(v[u + 1], qscale, -m_use)) : 0.f;
-            rs4[(u >> 1) & 3] += p0 + p1;
-            pk[u >> 1] = pack_bf16x2(p0, p1);
+          for (int u = 0; u < 64; ++u) {
+            const bool vis = base_n + 64 * h2 + u < lim;
+            v[u] = vis ? v[u] : -INFINITY;
           }
         }
-        __syncwarp();
-        tmem_st16(S + 16 * c4, pk);
+#pragma unroll
+        for (int c2 = 0; c2 < 2; ++c2) {
+          uint32_t pk[16];
+#pragma unroll
+          for (int u = 0; u < 32; u += 2) {
+            const float p0 = ex2(fmaf(v[32 * c2 + u], qscale, -m_use));
+            const float p1 = ex2(fmaf(v[32 * c2 + u + 1], qscale, -m_use));
+            rs4[(u >> 1) & 3] += p0 + p1;
+            pk[u >> 1] = pack_bf16x2(p0, p1);
+          }
+          __syncwarp();
+          tmem_st16(S + 32 * h2 + 16 * c2, pk);
+        }
       }
       const float rs = (rs4[0] + rs4[1]) + (rs4[2] + rs4[3]);
       l = l * corr + rs;
@@ -541,6 +543,9 @@ attn_tc_kernel(const AttnArgs a, int nsplit) {
 
 cudaError_t launch_attn_tc(const AttnArgs& a, cudaStream_t stream) {
   if (a.d != AT_D) return cudaErrorNotSupported;
+  AttnMaps maps;
+  if (!encode_bf16_4d(&maps.q, a.Q.data, AT_D, a.BCP, a.nq, a.b, a.Q.st, a.Q.sh, a.Q.sb, 128))
+    return cudaErrorNotSupported;
   const size_t smem = sizeof(AttnSmem) + 1024;
   cudaError_t e = cudaFuncSetAttribute(attn_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (e != cudaSuccess) return e;
@@ -566,7 +571,7 @@ cudaError_t launch_attn_tc(const AttnArgs& a, cudaStream_t stream) {
   attr[0].val.clusterDim.z = 1;
   cfg.attrs = attr;
   cfg.numAttrs = 1;
-  return cudaLaunchKernelEx(&cfg, attn_tc_kernel, a, nsplit);
+  return cudaLaunchKernelEx(&cfg, attn_tc_kernel, maps, a, nsplit);
 }
 
 }  // namespace quoka

@@ -27,12 +27,10 @@
 //               columns, |k| from shared memory, S_agg store.
 // Every wait is bounded (see sm100.cuh); a wait that gives up records
 // QUOKA_ERR_TIMEOUT and the CTA unwinds.
-#include <cuda.h>
-#include <cudaTypedefs.h>
-
 #include "common.cuh"
 #include "kernels.h"
 #include "sm100.cuh"
+#include "tmap.cuh"
 
 namespace quoka {
 
@@ -233,20 +231,6 @@ score_tc_kernel(const __grid_constant__ CUtensorMap tmap, const ScoreArgs a) {
     tc_fence_after();
     tmem_dealloc(tmem, a.tmem_cols);
   }
-}
-
-PFN_cuTensorMapEncodeTiled_v12000 tensor_map_encoder() {
-  static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
-  static bool tried = false;
-  if (!tried) {
-    tried = true;
-    void* p = nullptr;
-    cudaDriverEntryPointQueryResult q;
-    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
-        q == cudaDriverEntryPointSuccess)
-      fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(p);
-  }
-  return fn;
 }
 
 }  // namespace
