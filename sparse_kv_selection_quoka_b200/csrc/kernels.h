@@ -23,25 +23,35 @@ cudaError_t launch_qsel(bool bf16, int d, Strided Q, int b, int nq, int BCP, int
 // Step (c, second half): Q_group (b, nkv, NQ, d) fp32 = mean over the G
 // heads of each group of Qhat at the same rank; optionally also the bf16
 // hi/lo split (b, nkv, 2*NQ, d): rows [0, NQ) hi, rows [NQ, 2NQ) lo.
+// When `hist` is given, also zeroes the (b * nkv, TOPK_HIST_BINS) score
+// histogram that the tensor-core scoring kernel fills.
+constexpr int TOPK_HIST_BINS = 4096;
 cudaError_t launch_qgroup(int d, const float* Qhat, int b, int nq, int nkv, int NQ,
-                          float* Qg, uint16_t* Qg_hilo, cudaStream_t stream);
+                          float* Qg, uint16_t* Qg_hilo, uint32_t* hist, cudaStream_t stream);
 
 // Step (d) on the CUDA cores (fp32 arithmetic; any input dtype).
 cudaError_t launch_score_simt(bool bf16, int d, Strided K, int b, int nkv, int64_t T,
                               const float* Qg, int NQ, float* S_agg, cudaStream_t stream);
 
 // Step (d) on the tcgen05 tensor cores (bf16 K, Q_group as bf16 hi + lo).
+// Also accumulates, per (batch, KV head), the histogram of the top 12 bits
+// of the order-preserving score keys into `hist` (zeroed beforehand), the
+// first digit of the top-k radix select.
 // Returns cudaErrorNotSupported when the shape has no tensor-core variant.
 cudaError_t launch_score_tc(int d, Strided K, int b, int nkv, int64_t T,
-                            const uint16_t* Qg_hilo, int NQ, float* S_agg, int* status,
-                            cudaStream_t stream);
+                            const uint16_t* Qg_hilo, int NQ, float* S_agg, uint32_t* hist,
+                            int* status, cudaStream_t stream);
 
 // Step (e): per (batch, KV head) cluster radix select of the BSA_eff
 // largest scores, ties to the lower index, written in ascending key order.
 // Requires 1 <= bsa <= T and T <= topk_max_T().
 int64_t topk_max_T();
+// `hist`, when not null, is the (b * nkv, TOPK_HIST_BINS) histogram of the
+// top 12 key bits made by the scoring kernel; the first radix pass is then
+// skipped.
 cudaError_t launch_topk(const float* S_agg, int b, int nkv, int64_t T, int bsa,
-                        int32_t* kv_idx, int32_t* kv_count, cudaStream_t stream);
+                        const uint32_t* hist, int32_t* kv_idx, int32_t* kv_count,
+                        cudaStream_t stream);
 
 // Step (f): standalone gather of the selected K and V rows.
 cudaError_t launch_gather(bool bf16, int d, Strided K, Strided V, int b, int nkv, int64_t T,

@@ -358,7 +358,7 @@ qsel_cluster_kernel(const T* __restrict__ Q, int64_t sQb, int64_t sQh, int64_t s
 template <int D>
 __global__ void __launch_bounds__(D)
 qgroup_kernel(const float* __restrict__ Qhat, int nq, int NQ, float* __restrict__ Qg,
-              bf16* __restrict__ Qg_hilo) {
+              bf16* __restrict__ Qg_hilo, uint32_t* __restrict__ hist) {
   const int i = blockIdx.x, j = blockIdx.y, bi = blockIdx.z, nkv = gridDim.y;
   const int G = nq / nkv;
   const int k = threadIdx.x;
@@ -372,6 +372,11 @@ qgroup_kernel(const float* __restrict__ Qhat, int nq, int NQ, float* __restrict_
     const bf16 lo = __float2bfloat16_rn(v - __bfloat162float(hi));
     Qg_hilo[(row * 2 * NQ + i) * D + k] = hi;
     Qg_hilo[(row * 2 * NQ + NQ + i) * D + k] = lo;
+  }
+  if (hist != nullptr) {
+    // the NQ blocks of a row zero its histogram between them
+    uint32_t* h = hist + row * TOPK_HIST_BINS;
+    for (int e = i * D + k; e < TOPK_HIST_BINS; e += NQ * D) h[e] = 0u;
   }
 }
 
@@ -438,11 +443,11 @@ cudaError_t launch_qsel(bool is_bf16, int d, Strided Q, int b, int nq, int BCP, 
 }
 
 cudaError_t launch_qgroup(int d, const float* Qhat, int b, int nq, int nkv, int NQ, float* Qg,
-                          uint16_t* Qg_hilo, cudaStream_t stream) {
+                          uint16_t* Qg_hilo, uint32_t* hist, cudaStream_t stream) {
   dim3 grid(NQ, nkv, b);
   bf16* hl = reinterpret_cast<bf16*>(Qg_hilo);
-  if (d == 128) qgroup_kernel<128><<<grid, 128, 0, stream>>>(Qhat, nq, NQ, Qg, hl);
-  else if (d == 64) qgroup_kernel<64><<<grid, 64, 0, stream>>>(Qhat, nq, NQ, Qg, hl);
+  if (d == 128) qgroup_kernel<128><<<grid, 128, 0, stream>>>(Qhat, nq, NQ, Qg, hl, hist);
+  else if (d == 64) qgroup_kernel<64><<<grid, 64, 0, stream>>>(Qhat, nq, NQ, Qg, hl, hist);
   else return cudaErrorNotSupported;
   return cudaGetLastError();
 }

@@ -28,6 +28,7 @@ struct WsLayout {
   size_t sagg = 0;      // (b, nkv, T) fp32
   size_t kvidx = 0;     // (b, nkv, BSA_eff) int32
   size_t kvcount = 0;   // (b, nkv) int32
+  size_t hist = 0;      // (b, nkv, 4096) uint32: first-digit histogram of the score keys
   size_t total = 0;
 };
 
@@ -48,6 +49,7 @@ WsLayout ws_layout(int64_t b, int64_t nq, int64_t nkv, int64_t d, int64_t T, int
   L.sagg = take((size_t)(b * nkv * T) * 4);
   L.kvidx = take((size_t)(b * nkv * bsa_eff) * 4);
   L.kvcount = take((size_t)(b * nkv) * 4);
+  L.hist = take((size_t)(b * nkv) * quoka::TOPK_HIST_BINS * 4);
   L.total = off;
   return L;
 }
@@ -145,20 +147,25 @@ quoka_status run_select(const quoka_tensor* Q, const quoka_tensor* K, const Sele
   int32_t* qidx = q_idx != nullptr ? q_idx : at<int32_t>(ws, L.qidx);
   float* sagg = s_agg != nullptr ? s_agg : at<float>(ws, L.sagg);
   int* status = at<int>(ws, L.status);
+  uint32_t* hist = at<uint32_t>(ws, L.hist);
 
   cudaError_t e = quoka::launch_qsel(bf, d, strided(Q), b, nq, BCP, NQ, qhat, qidx, stream);
   if (e != cudaSuccess) return cuda_status(e);
-  e = quoka::launch_qgroup(d, qhat, b, nq, nkv, NQ, qg, bf ? qhilo : nullptr, stream);
+  e = quoka::launch_qgroup(d, qhat, b, nq, nkv, NQ, qg, bf ? qhilo : nullptr, bf ? hist : nullptr, stream);
   if (e != cudaSuccess) return cuda_status(e);
+  bool hist_made = false;
   if (s.T > 0) {
     e = cudaErrorNotSupported;
-    if (bf) e = quoka::launch_score_tc(d, strided(K), b, nkv, s.T, qhilo, NQ, sagg, status, stream);
+    if (bf) {
+      e = quoka::launch_score_tc(d, strided(K), b, nkv, s.T, qhilo, NQ, sagg, hist, status, stream);
+      hist_made = e == cudaSuccess;
+    }
     if (e == cudaErrorNotSupported)
       e = quoka::launch_score_simt(bf, d, strided(K), b, nkv, s.T, qg, NQ, sagg, stream);
     if (e != cudaSuccess) return cuda_status(e);
   }
   if (bsa_eff > 0) {
-    e = quoka::launch_topk(sagg, b, nkv, s.T, bsa_eff, kv_idx, kv_count, stream);
+    e = quoka::launch_topk(sagg, b, nkv, s.T, bsa_eff, hist_made ? hist : nullptr, kv_idx, kv_count, stream);
     if (e != cudaSuccess) return cuda_status(e);
   } else {
     e = cudaMemsetAsync(kv_count, 0, sizeof(int32_t) * b * nkv, stream);

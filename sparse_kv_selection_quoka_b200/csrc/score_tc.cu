@@ -58,6 +58,7 @@ struct ScoreBars {
 struct ScoreArgs {
   const uint16_t* qg_hilo;  // (b, nkv, 2*NQ, d) bf16: rows [0,NQ) hi, [NQ,2NQ) lo
   float* s_agg;             // (b, nkv, T)
+  uint32_t* hist;           // (b, nkv, TOPK_HIST_BINS): histogram of key >> 20
   int* status;
   int64_t T;
   int NQ, NQp, nstages, tiles_per_cta, ntiles;
@@ -85,7 +86,8 @@ score_tc_kernel(const __grid_constant__ CUtensorMap tmap, const ScoreArgs a) {
   const int N = 2 * a.NQp;                         // MMA N: hi rows then lo rows
   uint8_t* qg_s = base;                            // [2 atoms][N rows][128 B]
   const int qg_bytes = ((N * 256) + 1023) & ~1023;
-  uint8_t* ring = base + qg_bytes;                 // [nstages][32 KiB]
+  uint32_t* hist_s = reinterpret_cast<uint32_t*>(base + qg_bytes);  // [TOPK_HIST_BINS]
+  uint8_t* ring = base + qg_bytes + TOPK_HIST_BINS * 4;             // [nstages][32 KiB]
   ScoreBars& sb = *reinterpret_cast<ScoreBars*>(ring + (size_t)a.nstages * SC_TILE_BYTES);
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
@@ -113,6 +115,7 @@ score_tc_kernel(const __grid_constant__ CUtensorMap tmap, const ScoreArgs a) {
     tmem_alloc(&sb.tmem_base, a.tmem_cols);
     tmem_relinquish();
   }
+  for (int e = tid; e < TOPK_HIST_BINS; e += SC_THREADS) hist_s[e] = 0u;
   // B operand: the group means (hi rows then lo rows, each padded to NQp
   // with zero rows) in the K-major 128-byte-swizzled layout.
   {
@@ -190,7 +193,7 @@ score_tc_kernel(const __grid_constant__ CUtensorMap tmap, const ScoreArgs a) {
       const int s = it % NS, acc = it & 1;
       if (!sc_warp_wait(&sb.tfull[acc], (it >> 1) & 1, sb, a.status, 55)) break;
       tc_fence_after();
-      float mx = -INFINITY;
+      float mx4[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
       const uint32_t tbase = tmem + lane_off + (uint32_t)(acc * N);
       for (int c0 = 0; c0 < a.NQp; c0 += 16) {
         float hi[16], lo[16];
@@ -199,15 +202,17 @@ score_tc_kernel(const __grid_constant__ CUtensorMap tmap, const ScoreArgs a) {
         tmem_wait_ld();
 #pragma unroll
         for (int u = 0; u < 16; ++u)
-          if (c0 + u < a.NQ) mx = fmaxf(mx, hi[u] + lo[u]);
+          if (c0 + u < a.NQ) mx4[u & 3] = fmaxf(mx4[u & 3], hi[u] + lo[u]);
       }
+      const float mx = fmaxf(fmaxf(mx4[0], mx4[1]), fmaxf(mx4[2], mx4[3]));
       tc_fence_before();
       mbar_arrive(&sb.tempty[acc]);
       // |k| from the tile in shared memory (the TMA writes are visible to
       // threads that observe the stage's barrier)
       if (!sc_warp_wait(&sb.full[s], (it / NS) & 1, sb, a.status, 56)) break;
       const uint8_t* tile = ring + (size_t)s * SC_TILE_BYTES;
-      float ss = 0.f;
+      // eight independent partial sums keep the FMA chain short
+      float ss8[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
 #pragma unroll
       for (int c = 0; c < 16; ++c) {
         const uint4 raw = *reinterpret_cast<const uint4*>(tile + sw128_offset(r, c, SC_KEYS));
@@ -215,13 +220,24 @@ score_tc_kernel(const __grid_constant__ CUtensorMap tmap, const ScoreArgs a) {
 #pragma unroll
         for (int u = 0; u < 4; ++u) {
           const float2 f = __bfloat1622float2(h2[u]);
-          ss = fmaf(f.x, f.x, ss);
-          ss = fmaf(f.y, f.y, ss);
+          ss8[2 * u] = fmaf(f.x, f.x, ss8[2 * u]);
+          ss8[2 * u + 1] = fmaf(f.y, f.y, ss8[2 * u + 1]);
         }
       }
+      const float ss = ((ss8[0] + ss8[1]) + (ss8[2] + ss8[3])) + ((ss8[4] + ss8[5]) + (ss8[6] + ss8[7]));
       mbar_arrive(&sb.empty[s]);
       const int64_t key = (int64_t)(t_begin + it) * SC_KEYS + r;
-      if (key < a.T) out[key] = mx / fmaxf(sqrtf(ss), 1e-12f);
+      const float score = mx / fmaxf(sqrtf(ss), 1e-12f);
+      if (key < a.T) out[key] = score;
+      // first radix digit of the top-k: top 12 bits of the ordered key,
+      // counted once per distinct bin within the warp
+      const bool counted = key < a.T;
+      const uint32_t bin = score_key(score) >> 20;
+      const uint32_t act = __ballot_sync(0xffffffffu, counted);
+      if (counted) {
+        const uint32_t peers = __match_any_sync(act, bin);
+        if (lane == __ffs(peers) - 1) atomicAdd(&hist_s[bin], (uint32_t)__popc(peers));
+      }
     }
   }
 
@@ -231,12 +247,18 @@ score_tc_kernel(const __grid_constant__ CUtensorMap tmap, const ScoreArgs a) {
     tc_fence_after();
     tmem_dealloc(tmem, a.tmem_cols);
   }
+  // fold this CTA's histogram into the head's
+  uint32_t* gh = a.hist + row * TOPK_HIST_BINS;
+  for (int e = tid; e < TOPK_HIST_BINS; e += SC_THREADS) {
+    const uint32_t v = hist_s[e];
+    if (v != 0u) atomicAdd(gh + e, v);
+  }
 }
 
 }  // namespace
 
 cudaError_t launch_score_tc(int d, Strided K, int b, int nkv, int64_t T, const uint16_t* Qg_hilo, int NQ,
-                            float* S_agg, int* status, cudaStream_t stream) {
+                            float* S_agg, uint32_t* hist, int* status, cudaStream_t stream) {
   if (d != SC_D || NQ < 1 || NQ > 128 || T <= 0 || T > (int64_t)INT32_MAX - SC_KEYS) return cudaErrorNotSupported;
   PFN_cuTensorMapEncodeTiled_v12000 encode = tensor_map_encoder();
   if (encode == nullptr) return cudaErrorNotSupported;
@@ -254,6 +276,7 @@ cudaError_t launch_score_tc(int d, Strided K, int b, int nkv, int64_t T, const u
   ScoreArgs a;
   a.qg_hilo = Qg_hilo;
   a.s_agg = S_agg;
+  a.hist = hist;
   a.status = status;
   a.T = T;
   a.NQ = NQ;
@@ -265,7 +288,7 @@ cudaError_t launch_score_tc(int d, Strided K, int b, int nkv, int64_t T, const u
   const int qg_bytes = ((N * 256) + 1023) & ~1023;
   const int smem_cap = 227 * 1024;
   const int bars = (int)sizeof(ScoreBars) + 1024;
-  a.nstages = (smem_cap - qg_bytes - bars) / SC_TILE_BYTES;
+  a.nstages = (smem_cap - qg_bytes - TOPK_HIST_BINS * 4 - bars) / SC_TILE_BYTES;
   if (a.nstages > SC_MAX_STAGES) a.nstages = SC_MAX_STAGES;
   if (a.nstages < 2) return cudaErrorNotSupported;
   a.ntiles = (int)((T + SC_KEYS - 1) / SC_KEYS);
@@ -280,7 +303,8 @@ cudaError_t launch_score_tc(int d, Strided K, int b, int nkv, int64_t T, const u
   a.tiles_per_cta = (a.ntiles + per_head - 1) / per_head;
   per_head = (a.ntiles + a.tiles_per_cta - 1) / a.tiles_per_cta;
 
-  const size_t smem = (size_t)qg_bytes + (size_t)a.nstages * SC_TILE_BYTES + sizeof(ScoreBars) + 1024;
+  const size_t smem =
+      (size_t)qg_bytes + TOPK_HIST_BINS * 4 + (size_t)a.nstages * SC_TILE_BYTES + sizeof(ScoreBars) + 1024;
   cudaError_t e = cudaFuncSetAttribute(score_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (e != cudaSuccess) return e;
   score_tc_kernel<<<dim3(per_head, nkv, b), SC_THREADS, smem, stream>>>(tmap, a);
