@@ -40,7 +40,10 @@ import torch  # noqa: E402
 METRIC = "prefill chunk-tokens/sec at T=32K (keys-scored/sec, % HBM and tensor-pipe peak alongside)"
 UNIT = "chunk-tokens/s"
 FLUSH_BYTES = 256 << 20
-OUR_KERNELS_PER_STEP = 5  # qsel, qgroup, score, topk, attention
+def kernels_per_chunk(T, bsa_eff):
+    """Our kernel launches in one chunk's step: query select, group mean,
+    scoring (T > 0), top-k and gather (BSA_eff > 0), attention."""
+    return 2 + (1 if T > 0 else 0) + (2 if bsa_eff > 0 else 0) + 1
 
 
 def _peaks():
@@ -147,6 +150,12 @@ def select_bytes(b, nq, nkv, d, T, BCP, bsa_eff, es):
     return b * nkv * T * d * es + b * nq * BCP * d * es + b * nkv * bsa_eff * 4
 
 
+def gather_bytes(b, nkv, d, bsa_eff, es):
+    """Step (f): the selected K and V rows read once and written once, and
+    the index list read."""
+    return b * nkv * bsa_eff * (4 * d * es + 4)
+
+
 # ---------------------------------------------------------------- our arm
 
 def run_ours(args, rank, world, local_rank):
@@ -178,7 +187,8 @@ def run_ours(args, rank, world, local_rank):
             O = torch.empty((w.b, w.nq, L, w.d), dtype=tdt, device=dev)
             kv_idx = torch.empty((w.b, w.nkv, min(bsa, T)), dtype=torch.int32, device=dev)
             kv_count = torch.empty((w.b, w.nkv), dtype=torch.int32, device=dev)
-            chunks.append((views, bsa, ws, O, kv_idx, kv_count, T))
+            sel_kv = tuple(torch.empty((w.b, w.nkv, min(bsa, T), w.d), dtype=tdt, device=dev) for _ in range(2))
+            chunks.append((views, bsa, ws, O, kv_idx, kv_count, T, sel_kv))
     else:
         Q, K, V, Kc, Vc = (to_dev(a) for a in (x.Q, x.K, x.V, x.Kc, x.Vc))
         bsa_eff = min(w.BSA, w.T)
@@ -186,14 +196,22 @@ def run_ours(args, rank, world, local_rank):
         O = torch.empty((w.b, w.nq, w.BCP, w.d), dtype=tdt, device=dev)
         kv_idx = torch.empty((w.b, w.nkv, bsa_eff), dtype=torch.int32, device=dev)
         kv_count = torch.empty((w.b, w.nkv), dtype=torch.int32, device=dev)
-        chunks = [((Q, K, V, Kc, Vc), w.BSA, ws, O, kv_idx, kv_count, w.T)]
+        sel_kv = tuple(torch.empty((w.b, w.nkv, bsa_eff, w.d), dtype=tdt, device=dev) for _ in range(2))
+        chunks = [((Q, K, V, Kc, Vc), w.BSA, ws, O, kv_idx, kv_count, w.T, sel_kv)]
 
-    def one_chunk(ch, ev_mid=None):
-        (Qv, Kv, Vv, Kcv, Vcv), bsa, wsb, Ob, idx, cnt, _ = ch
+    def one_chunk(ch, evs=None):
+        """Steps (a)-(e) | (f) | (g) through the public calls; with `evs`
+        (three events) each boundary is recorded, so every part is timed on
+        its own: quoka_sparse_gqa_attn with a full workspace runs exactly
+        the gather and attention kernels below."""
+        (Qv, Kv, Vv, Kcv, Vcv), bsa, wsb, Ob, idx, cnt, _, (Ks, Vs) = ch
         q.quoka_select(Qv, Kv, w.NQ, bsa, kv_idx=idx, kv_count=cnt, ws=wsb, stream=stream)
-        if ev_mid is not None:
-            ev_mid.record(stream)
-        q.quoka_sparse_gqa_attn(Qv, Kv, Vv, idx, cnt, Kcv, Vcv, O=Ob, ws=wsb, stream=stream)
+        if evs is not None:
+            evs[0].record(stream)
+        q.quoka_gather_kv(Kv, Vv, idx, cnt, Ksel=Ks, Vsel=Vs, ws=wsb, stream=stream)
+        if evs is not None:
+            evs[1].record(stream)
+        q.quoka_sparse_gqa_attn_gathered(Qv, Ks, Vs, cnt, Kcv, Vcv, O=Ob, ws=wsb, stream=stream)
 
     for _ in range(args.warmup):
         for ch in chunks:
@@ -214,36 +232,37 @@ def run_ours(args, rank, world, local_rank):
         torch.distributed.barrier()
     torch.cuda.synchronize()
     n_ev = len(chunks)
-    t_step, t_sel, t_attn = 0.0, 0.0, 0.0
+    t_step, t_sel, t_gather, t_attn = 0.0, 0.0, 0.0, 0.0
     per_chunk = [0.0] * n_ev
     evs = []
     for _ in range(args.steps):
         flush.fill_(1)
         step_evs = []
         for ch in chunks:
-            e0, e1, e2 = (torch.cuda.Event(enable_timing=True) for _ in range(3))
-            e0.record(stream)
-            one_chunk(ch, ev_mid=e1)
-            e2.record(stream)
-            step_evs.append((e0, e1, e2))
+            e = [torch.cuda.Event(enable_timing=True) for _ in range(5)]
+            e[0].record(stream)
+            one_chunk(ch, evs=e[1:4])
+            e[4].record(stream)
+            step_evs.append(e)
         evs.append(step_evs)
     torch.cuda.synchronize()
     if world > 1:
         torch.distributed.barrier()
     for step_evs in evs:
-        for c, (e0, e1, e2) in enumerate(step_evs):
-            a, bms = e0.elapsed_time(e1), e1.elapsed_time(e2)
+        for c, e in enumerate(step_evs):
+            a, g, bms = e[0].elapsed_time(e[1]), e[1].elapsed_time(e[2]), e[2].elapsed_time(e[4])
             t_sel += a
+            t_gather += g
             t_attn += bms
-            t_step += a + bms
-            per_chunk[c] += a + bms
+            t_step += a + g + bms
+            per_chunk[c] += a + g + bms
     clocks = sampler.stop()
 
     K_ = args.steps
-    times = torch.tensor([t_step / K_, t_sel / K_, t_attn / K_], dtype=torch.float64, device=dev)
+    times = torch.tensor([t_step / K_, t_sel / K_, t_gather / K_, t_attn / K_], dtype=torch.float64, device=dev)
     if world > 1:
         torch.distributed.all_reduce(times, op=torch.distributed.ReduceOp.MAX)
-    ms_step, ms_sel, ms_attn = (float(v) for v in times.cpu())
+    ms_step, ms_sel, ms_gather, ms_attn = (float(v) for v in times.cpu())
 
     tokens_per_step = w.b * (w.T if sweep else w.BCP)
     if sweep:
@@ -254,10 +273,12 @@ def run_ours(args, rank, world, local_rank):
     if sweep:
         flops = sum(attn_flops(w.b, w.nq, w.d, x.BCP, min(ch[1], ch[6])) for ch in chunks)
         sbytes = sum(select_bytes(w.b, w.nq, w.nkv, w.d, ch[6], x.BCP, min(ch[1], ch[6]), es) for ch in chunks)
+        gbytes = sum(gather_bytes(w.b, w.nkv, w.d, min(ch[1], ch[6]), es) for ch in chunks)
         keys = sum(w.b * w.nkv * ch[6] for ch in chunks)
     else:
         flops = attn_flops(w.b, w.nq, w.d, w.BCP, min(w.BSA, w.T))
         sbytes = select_bytes(w.b, w.nq, w.nkv, w.d, w.T, w.BCP, min(w.BSA, w.T), es)
+        gbytes = gather_bytes(w.b, w.nkv, w.d, min(w.BSA, w.T), es)
         keys = w.b * w.nkv * w.T
     attn_tflops = flops / (ms_attn / 1e3) / 1e12
     sel_gbs = sbytes / (ms_sel / 1e3) / 1e9
@@ -280,6 +301,7 @@ def run_ours(args, rank, world, local_rank):
         "keys_scored_per_s": world * keys / (ms_sel / 1e3),
         "keys_scored_per_s_query_heads": world * keys * (w.nq // w.nkv) / (ms_sel / 1e3),
         "ms_select": ms_sel,
+        "ms_gather": ms_gather,
         "ms_attention": ms_attn,
         "roofline": {"kernel": "sparse GQA attention (tcgen05)" if w.dtype == "bf16" else "sparse GQA attention (fp32 CUDA cores)",
                      "bound": "tensor", "achieved": attn_tflops, "peak": tf_burst,
@@ -292,8 +314,11 @@ def run_ours(args, rank, world, local_rank):
         "roofline_select": {"steps": "(a)-(e)", "bound": "hbm", "achieved": sel_gbs, "peak": hbm,
                             "unit": "GB/s", "frac": sel_gbs / hbm, "frac_of_8TBs": sel_gbs / 8000.0,
                             "algorithmic_bytes_per_step": sbytes},
+        "roofline_gather": {"steps": "(f)", "bound": "hbm", "achieved": gbytes / (ms_gather / 1e3) / 1e9,
+                            "peak": hbm, "unit": "GB/s", "frac": gbytes / (ms_gather / 1e3) / 1e9 / hbm,
+                            "algorithmic_bytes_per_step": gbytes},
         "clocks": clocks,
-        "gpu_launches": OUR_KERNELS_PER_STEP * len(chunks) * K_,
+        "gpu_launches": sum(kernels_per_chunk(ch[6], min(ch[1], ch[6])) for ch in chunks) * K_,
     }
     if sweep:
         out["per_chunk_ms"] = [p / K_ for p in per_chunk]

@@ -74,10 +74,23 @@ typedef struct {
 } quoka_tensor;
 
 /* Bytes of workspace any call below needs for these sizes (the maximum over
- * the calls, so one workspace serves all of them). Returns 0 only for
- * invalid sizes. */
+ * the calls, so one workspace serves all of them; quoka_prefill_chunk needs
+ * exactly this much). Returns 0 only for invalid sizes. */
 size_t quoka_workspace_size(int b, int nq, int nkv, int d, int64_t T, int BCP,
                             int NQ, int BSA, quoka_dtype dtype);
+
+/* Bytes of workspace quoka_select (and quoka_select_static's scratch) needs
+ * for these sizes; at most quoka_workspace_size(). Returns 0 only for
+ * invalid sizes. */
+size_t quoka_select_workspace_size(int b, int nq, int nkv, int d, int64_t T,
+                                   int BCP, int NQ, int BSA, quoka_dtype dtype);
+
+/* Bytes of workspace with which quoka_sparse_gqa_attn takes its fastest path
+ * for these sizes: 256 (the status words) plus, for bf16 with d = 128 and
+ * BSA_eff > 0, two 256-byte-aligned buffers of b * nkv * BSA_eff * d bf16
+ * (the gathered selected K and V). Returns 0 only for invalid sizes. */
+size_t quoka_attn_workspace_size(int b, int nkv, int d, int BSA_eff,
+                                 quoka_dtype dtype);
 
 /* Steps (a)-(e), [QUOKA §2.1 Algorithm 1, §2.2, §2.3]:
  *   Q (b, nq, BCP, d), K (b, nkv, T, d), same dtype.
@@ -107,8 +120,8 @@ quoka_status quoka_select(const quoka_tensor* Q, const quoka_tensor* K, int NQ,
  *   Arguments, outputs and results are those of quoka_select, minus ws.
  *   Scratch comes from a file-scope device array of
  *   QUOKA_STATIC_SCRATCH_BYTES per device, held by every GPU that loads the
- *   library until the process exits. Shapes whose quoka_workspace_size()
- *   exceeds it are rejected with QUOKA_ERR_WORKSPACE before anything is
+ *   library until the process exits. Shapes whose
+ *   quoka_select_workspace_size() exceeds it are rejected with QUOKA_ERR_WORKSPACE before anything is
  *   enqueued. Nothing is allocated (no cudaMalloc or cudaFree, no allocating
  *   library call).
  *   The first call on each device looks up the array's device address (with
@@ -125,11 +138,12 @@ quoka_status quoka_select_static(const quoka_tensor* Q, const quoka_tensor* K, i
                                  int32_t* q_idx, float* s_agg, void* stream);
 
 /* Step (f), [QUOKA §4.2 problem 3]: Ksel[b, j, n] = K[b, j, kv_idx[b, j, n]]
- * and the same for V, for n < kv_count[b, j] (rows past the count are left
- * untouched).
+ * and the same for V, for n < kv_count[b, j]. Rows past the count, and rows
+ * whose index is out of range, are written as zeros (so the output can be
+ * handed to quoka_sparse_gqa_attn_gathered as it is).
  *   K, V (b, nkv, T, d); kv_idx (b, nkv, BSA_eff) int32; kv_count (b, nkv).
  *   Ksel, Vsel out (b, nkv, BSA_eff, d), contiguous, dtype of K.
- * An index outside [0, T) is skipped and latched as QUOKA_ERR_BOUNDS in
+ * An index outside [0, T) is not read and is latched as QUOKA_ERR_BOUNDS in
  * `ws` (which may be NULL, in which case it is only skipped). */
 quoka_status quoka_gather_kv(const quoka_tensor* K, const quoka_tensor* V,
                              const int32_t* kv_idx, const int32_t* kv_count,
@@ -140,8 +154,13 @@ quoka_status quoka_gather_kv(const quoka_tensor* K, const quoka_tensor* V,
  *   O[b,h,t] = sum_k softmax_k(scale * Q[b,h,t].k) v
  * over the selected prior keys k = K[b, j, kv_idx[b, j, n]] (n < kv_count,
  * no mask) and the chunk's own keys Kc[b, j, s] with s <= t (causal),
- * j = floor(h / G). The selected rows are read in place (fused gather).
+ * j = floor(h / G).
  *   Q (b, nq, BCP, d); K, V (b, nkv, T, d); Kc, Vc (b, nkv, BCP, d).
+ *   ws  at least 256 bytes. With ws_bytes >= quoka_attn_workspace_size()
+ *       (bf16, d = 128) the selected rows are first gathered into ws (step
+ *       (f) as its own kernel, the copy staying in L2) and the attention
+ *       streams them as dense tiles; with less, the bf16 attention gathers
+ *       the rows itself while loading them (slower, same results).
  *   O   out (b, nq, BCP, d), contiguous, dtype of Q.
  *   lse out (b, nq, BCP) float or NULL: natural-log partition function
  *       log sum_k exp(scale * q.k).
@@ -154,8 +173,29 @@ quoka_status quoka_sparse_gqa_attn(const quoka_tensor* Q, const quoka_tensor* K,
                                    float scale, void* O, float* lse, void* ws,
                                    size_t ws_bytes, void* stream);
 
+/* Step (g) on a selected KV that is already gathered, [QUOKA §4.2 problem 3]:
+ * the attention of quoka_sparse_gqa_attn with key n of KV head j being row
+ * n of Ksel[b, j] / Vsel[b, j] (n < kv_count[b, j]) instead of an indexed
+ * row of the cache. quoka_sparse_gqa_attn with a full workspace is exactly
+ * quoka_gather_kv followed by this call.
+ *   Ksel, Vsel (b, nkv, BSA_eff, d), dtype of Q, any 16-byte-aligned row
+ *   strides. Rows from kv_count to BSA_eff are masked out but are read: they
+ *   must hold finite values (quoka_gather_kv writes zeros there).
+ *   kv_count (b, nkv) int32, values above BSA_eff are clamped to it.
+ *   ws at least 256 bytes (the status words). Other arguments as in
+ *   quoka_sparse_gqa_attn. */
+quoka_status quoka_sparse_gqa_attn_gathered(const quoka_tensor* Q,
+                                            const quoka_tensor* Ksel,
+                                            const quoka_tensor* Vsel,
+                                            const int32_t* kv_count,
+                                            const quoka_tensor* Kc,
+                                            const quoka_tensor* Vc, float scale,
+                                            void* O, float* lse, void* ws,
+                                            size_t ws_bytes, void* stream);
+
 /* The whole step (a)-(g): quoka_select followed by quoka_sparse_gqa_attn on
- * one stream, with no host synchronisation in between.
+ * one stream, with no host synchronisation in between. ws must hold
+ * quoka_workspace_size() bytes.
  *   kv_idx_out (b, nkv, BSA_eff) int32 or NULL: the selected set (else kept
  *   in ws). lse may be NULL. */
 quoka_status quoka_prefill_chunk(const quoka_tensor* Q, const quoka_tensor* K,

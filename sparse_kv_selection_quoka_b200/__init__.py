@@ -11,9 +11,12 @@ without the built library.
 
 __all__ = [
     "quoka_workspace_size",
+    "quoka_select_workspace_size",
+    "quoka_attn_workspace_size",
     "quoka_select",
     "quoka_gather_kv",
     "quoka_sparse_gqa_attn",
+    "quoka_sparse_gqa_attn_gathered",
     "quoka_prefill_chunk",
     "quoka_get_device_status",
     "quoka_status_string",

@@ -37,9 +37,12 @@ STATUS_NAMES = {
 # names of every entry point include/quoka.h declares
 EXPORTS = (
     "quoka_workspace_size",
+    "quoka_select_workspace_size",
+    "quoka_attn_workspace_size",
     "quoka_select",
     "quoka_gather_kv",
     "quoka_sparse_gqa_attn",
+    "quoka_sparse_gqa_attn_gathered",
     "quoka_prefill_chunk",
     "quoka_get_device_status",
     "quoka_status_string",
@@ -86,12 +89,18 @@ def load() -> ctypes.CDLL:
         lib = ctypes.CDLL(LIB_PATH)
         lib.quoka_workspace_size.restype = _SZ
         lib.quoka_workspace_size.argtypes = [_I, _I, _I, _I, _I64, _I, _I, _I, _I]
+        lib.quoka_select_workspace_size.restype = _SZ
+        lib.quoka_select_workspace_size.argtypes = [_I, _I, _I, _I, _I64, _I, _I, _I, _I]
+        lib.quoka_attn_workspace_size.restype = _SZ
+        lib.quoka_attn_workspace_size.argtypes = [_I, _I, _I, _I, _I]
         lib.quoka_select.restype = _I
         lib.quoka_select.argtypes = [_T, _T, _I, _I, _P, _P, _P, _P, _P, _SZ, _P]
         lib.quoka_gather_kv.restype = _I
         lib.quoka_gather_kv.argtypes = [_T, _T, _P, _P, _I, _P, _P, _P, _SZ, _P]
         lib.quoka_sparse_gqa_attn.restype = _I
         lib.quoka_sparse_gqa_attn.argtypes = [_T, _T, _T, _P, _P, _I, _T, _T, _F, _P, _P, _P, _SZ, _P]
+        lib.quoka_sparse_gqa_attn_gathered.restype = _I
+        lib.quoka_sparse_gqa_attn_gathered.argtypes = [_T, _T, _T, _P, _T, _T, _F, _P, _P, _P, _SZ, _P]
         lib.quoka_prefill_chunk.restype = _I
         lib.quoka_prefill_chunk.argtypes = [_T, _T, _T, _T, _T, _I, _I, _F, _P, _P, _P, _P, _SZ, _P]
         lib.quoka_get_device_status.restype = _I
@@ -140,9 +149,20 @@ def _check(status: int, where: str) -> None:
         raise QuokaError(status, where)
 
 
+def _code(dtype) -> int:
+    return dtype if isinstance(dtype, int) else (QUOKA_BF16 if dtype == torch.bfloat16 else QUOKA_F32)
+
+
 def quoka_workspace_size(b, nq, nkv, d, T, BCP, NQ, BSA, dtype) -> int:
-    code = dtype if isinstance(dtype, int) else (QUOKA_BF16 if dtype == torch.bfloat16 else QUOKA_F32)
-    return int(load().quoka_workspace_size(b, nq, nkv, d, T, BCP, NQ, BSA, code))
+    return int(load().quoka_workspace_size(b, nq, nkv, d, T, BCP, NQ, BSA, _code(dtype)))
+
+
+def quoka_select_workspace_size(b, nq, nkv, d, T, BCP, NQ, BSA, dtype) -> int:
+    return int(load().quoka_select_workspace_size(b, nq, nkv, d, T, BCP, NQ, BSA, _code(dtype)))
+
+
+def quoka_attn_workspace_size(b, nkv, d, BSA_eff, dtype) -> int:
+    return int(load().quoka_attn_workspace_size(b, nkv, d, BSA_eff, _code(dtype)))
 
 
 def workspace_for(Q: torch.Tensor, K: torch.Tensor, NQ: int, BSA: int) -> torch.Tensor:
@@ -203,7 +223,35 @@ def quoka_gather_kv(K, V, kv_idx, kv_count, *, Ksel=None, Vsel=None, ws=None, st
 
 def quoka_sparse_gqa_attn(Q, K, V, kv_idx, kv_count, Kc, Vc, scale=None, *, O=None, lse=None,
                           want_lse=False, ws=None, stream=None):
-    """Steps (f)+(g). Returns (O (b,nq,BCP,d), lse or None)."""
+    """Steps (f)+(g). Returns (O (b,nq,BCP,d), lse or None). Without `ws`
+    a workspace of quoka_attn_workspace_size bytes is allocated (the path
+    that gathers the selected rows first); a 256-byte `ws` selects the path
+    that gathers them while loading."""
+    lib = load()
+    b, nq, BCP, d = Q.shape
+    if scale is None:
+        scale = d ** -0.5
+    if O is None:
+        O = torch.empty((b, nq, BCP, d), dtype=Q.dtype, device=Q.device)
+    if lse is None and want_lse:
+        lse = torch.empty((b, nq, BCP), dtype=torch.float32, device=Q.device)
+    if ws is None:
+        n = quoka_attn_workspace_size(b, K.shape[1], d, kv_idx.shape[2], Q.dtype)
+        ws = torch.empty(max(n, 256), dtype=torch.uint8, device=Q.device)
+    views = [tensor_view(x) for x in (Q, K, V, Kc, Vc)]
+    st = lib.quoka_sparse_gqa_attn(ctypes.byref(views[0]), ctypes.byref(views[1]), ctypes.byref(views[2]),
+                                   _ptr(kv_idx) if kv_idx.numel() else None, _ptr(kv_count),
+                                   kv_idx.shape[2], ctypes.byref(views[3]), ctypes.byref(views[4]),
+                                   float(scale), _ptr(O), _ptr(lse), _ptr(ws), ws.numel(),
+                                   _stream(stream))
+    _check(st, "quoka_sparse_gqa_attn")
+    return O, lse
+
+
+def quoka_sparse_gqa_attn_gathered(Q, Ksel, Vsel, kv_count, Kc, Vc, scale=None, *, O=None, lse=None,
+                                   want_lse=False, ws=None, stream=None):
+    """Step (g) on an already gathered selected KV (rows of Ksel / Vsel,
+    e.g. from quoka_gather_kv). Returns (O, lse or None)."""
     lib = load()
     b, nq, BCP, d = Q.shape
     if scale is None:
@@ -214,13 +262,12 @@ def quoka_sparse_gqa_attn(Q, K, V, kv_idx, kv_count, Kc, Vc, scale=None, *, O=No
         lse = torch.empty((b, nq, BCP), dtype=torch.float32, device=Q.device)
     if ws is None:
         ws = torch.empty(256, dtype=torch.uint8, device=Q.device)
-    views = [tensor_view(x) for x in (Q, K, V, Kc, Vc)]
-    st = lib.quoka_sparse_gqa_attn(ctypes.byref(views[0]), ctypes.byref(views[1]), ctypes.byref(views[2]),
-                                   _ptr(kv_idx) if kv_idx.numel() else None, _ptr(kv_count),
-                                   kv_idx.shape[2], ctypes.byref(views[3]), ctypes.byref(views[4]),
-                                   float(scale), _ptr(O), _ptr(lse), _ptr(ws), ws.numel(),
-                                   _stream(stream))
-    _check(st, "quoka_sparse_gqa_attn")
+    views = [tensor_view(x) for x in (Q, Ksel, Vsel, Kc, Vc)]
+    st = lib.quoka_sparse_gqa_attn_gathered(ctypes.byref(views[0]), ctypes.byref(views[1]),
+                                            ctypes.byref(views[2]), _ptr(kv_count), ctypes.byref(views[3]),
+                                            ctypes.byref(views[4]), float(scale), _ptr(O), _ptr(lse),
+                                            _ptr(ws), ws.numel(), _stream(stream))
+    _check(st, "quoka_sparse_gqa_attn_gathered")
     return O, lse
 
 

@@ -55,7 +55,8 @@ attn_simt_kernel(AttnArgs a) {
   const T* Vb = static_cast<const T*>(a.V.data) + bi * a.V.sb + j * a.V.sh;
   const T* Kcb = static_cast<const T*>(a.Kc.data) + bi * a.Kc.sb + j * a.Kc.sh;
   const T* Vcb = static_cast<const T*>(a.Vc.data) + bi * a.Vc.sb + j * a.Vc.sh;
-  const int32_t* idx = a.kv_idx + kvrow * a.bsa;
+  // no index list: the selected rows are already gathered (row n = key n)
+  const int32_t* idx = a.kv_idx != nullptr ? a.kv_idx + kvrow * a.bsa : nullptr;
 
   for (int kb = 0; kb < total; kb += AS_KT) {
     __syncthreads();
@@ -63,7 +64,7 @@ attn_simt_kernel(AttnArgs a) {
       const int n = kb + threadIdx.x;
       int vis = -2;
       if (n < nsel) {
-        const int32_t tau = idx[n];
+        const int32_t tau = idx != nullptr ? idx[n] : n;
         if (tau >= 0 && (int64_t)tau < a.T) vis = -1;
         else latch_status(a.status, 6 /* QUOKA_ERR_BOUNDS */);
       } else if (n < total) {
@@ -78,7 +79,7 @@ attn_simt_kernel(AttnArgs a) {
       const int vis = kvis[kr];
       float kv = 0.f, vv = 0.f;
       if (vis == -1) {
-        const int64_t tau = idx[n];
+        const int64_t tau = idx != nullptr ? idx[n] : n;
         kv = to_f32(Kb[tau * a.K.st + c]);
         vv = to_f32(Vb[tau * a.V.st + c]);
       } else if (vis >= 0) {

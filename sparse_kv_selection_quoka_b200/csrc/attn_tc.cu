@@ -12,13 +12,13 @@
 // (one query head, 128 consecutive chunk positions each); a CTA takes two
 // such tiles (Q0, Q1) of the same KV head, so every K/V tile it brings in
 // feeds two 128x128x128 QK^T and two PV products. The key tiles of a CTA
-// are ceil(nsel/128) tiles of selected prior rows (read in place through the
-// sorted index list: the gather is fused into the loads; rows past nsel are
-// masked) followed by ceil(nchunk/128) tiles of the chunk's own keys. When the grid would fill less than half of the GPU, the key
-// tiles are split between the two CTAs of a cluster, and the partial results
-// are combined through distributed shared memory.
+// are ceil(nsel/128) tiles of selected prior rows (rows past nsel are
+// masked) followed by ceil(nchunk/128) tiles of the chunk's own keys. When
+// the grid would fill less than half of the GPU, the key tiles are split
+// between the two CTAs of a cluster, and the partial results are combined
+// through distributed shared memory.
 //
-// Warp roles (544 threads):
+// Warp roles (320 or 544 threads):
 //   warps 0-3   softmax of Q0, warps 4-7 softmax of Q1: thread r owns query
 //               row r = TMEM lane r. Two passes over its S row in TMEM (row
 //               max, then exp2 on the MUFU); P is written back as bf16 over
@@ -29,7 +29,12 @@
 //   warp 8      TMEM allocation and the single-thread MMA issue, ordered
 //               QK0(i), PV1(i-1), QK1(i), PV0(i): while one softmax group
 //               works, the tensor core runs the other group's products.
-//   warps 9-16  loaders (256 threads): cp.async 16-byte row chunks, gathered
+//   Two loader variants (a template parameter):
+//   (TMA)       warp 9 issues TMA boxes: the selected keys come from a
+//               contiguous copy made by the gather kernel just before (so
+//               they are L2-resident), the chunk keys and Q from the inputs.
+//               320 threads. Used whenever the workspace holds the copy.
+//   (gather)    warps 9-16  loaders (256 threads): cp.async 16-byte row chunks, gathered
 //               by index, into a 2-stage K/V ring in the 128-byte-swizzled
 //               UMMA layout (zero-fill past the end of a list); each thread
 //               owns one 16-byte column chunk of 8 rows per tile, prefetches
@@ -56,7 +61,11 @@ namespace {
 constexpr int AT_D = 128;        // head dim
 constexpr int AT_N = 128;        // keys per tile
 constexpr int AT_STAGES = 2;     // K/V ring depth
-constexpr int AT_THREADS = 544;
+template <bool TMA_KV>
+struct AttnCfg {
+  static constexpr int threads = TMA_KV ? 320 : 544;
+  static constexpr int kv_arrivals = TMA_KV ? 1 : 256;  // arrivals per stage fill
+};
 constexpr int AT_MMA_WARP = 8;
 constexpr int AT_LD_WARP0 = 9;
 constexpr int AT_LD_THREADS = 256;
@@ -70,9 +79,11 @@ constexpr float RESCALE_THRESHOLD = 8.f;    // log2 units
 constexpr uint32_t IDESC_QK = idesc_bf16_f32(128, AT_N, 0, 0);  // A=Q K-major, B=K K-major
 constexpr uint32_t IDESC_PV = idesc_bf16_f32(128, AT_D, 0, 1);  // A=P (TMEM), B=V MN-major
 
-// TMA tensor map of the queries (4-D boxes of 64 columns x 128 rows).
+// TMA tensor maps (4-D boxes of 64 columns x 128 rows): the queries, and for
+// the TMA loader the gathered selected K/V (b, nkv, BSA, d) and the chunk's
+// K/V (b, nkv, BCP, d).
 struct AttnMaps {
-  CUtensorMap q;
+  CUtensorMap q, ks, vs, kc, vc;
 };
 
 struct __align__(1024) AttnSmem {
@@ -132,7 +143,8 @@ __device__ __forceinline__ uint32_t pack_bf16x2(float a, float b) {
   return *reinterpret_cast<uint32_t*>(&h);
 }
 
-__global__ void __launch_bounds__(AT_THREADS, 1)
+template <bool TMA_KV>
+__global__ void __launch_bounds__(AttnCfg<TMA_KV>::threads, 1)
 attn_tc_kernel(const __grid_constant__ AttnMaps maps, const AttnArgs a, int nsplit) {
   extern __shared__ uint8_t smem_raw[];
   AttnSmem& sm = *reinterpret_cast<AttnSmem*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -167,7 +179,7 @@ attn_tc_kernel(const __grid_constant__ AttnMaps maps, const AttnArgs a, int nspl
   if (tid == 0) {
     mbar_init(&sm.q_full, 1);
     for (int s = 0; s < AT_STAGES; ++s) {
-      mbar_init(&sm.kv_full[s], AT_LD_THREADS);
+      mbar_init(&sm.kv_full[s], AttnCfg<TMA_KV>::kv_arrivals);
       mbar_init(&sm.kv_empty[s], 1);
     }
     for (int w = 0; w < 2; ++w) {
@@ -195,7 +207,56 @@ attn_tc_kernel(const __grid_constant__ AttnMaps maps, const AttnArgs a, int nspl
   tc_fence_after();
   const uint32_t tmem = sm.tmem_base;
 
-  if (warp >= AT_LD_WARP0) {
+  if (TMA_KV && warp == AT_LD_WARP0) {
+    // ------------------------------------------------------------ TMA loads
+    bool alive = true;
+    int issued = 0;
+    if (lane == 0) {
+      tma_prefetch_desc(&maps.q);
+      tma_prefetch_desc(&maps.ks);
+      tma_prefetch_desc(&maps.vs);
+      tma_prefetch_desc(&maps.kc);
+      tma_prefetch_desc(&maps.vc);
+      mbar_arrive_expect_tx(&sm.q_full, (ti[1].valid ? 2 : 1) * TILE_BYTES);
+      for (int w = 0; w < 2; ++w) {
+        if (!ti[w].valid) continue;
+        const uint32_t q_s = smem_u32(sm.q[w]);
+        tma_load_4d(q_s, &maps.q, &sm.q_full, 0, ti[w].t0, ti[w].h, bi);
+        tma_load_4d(q_s + ATOM_BYTES, &maps.q, &sm.q_full, 64, ti[w].t0, ti[w].h, bi);
+      }
+      for (int it = 0; it < ntiles && alive; ++it) {
+        const int s = it % AT_STAGES;
+        const int gi = first + it;
+        if (it >= AT_STAGES && !mbar_wait(&sm.kv_empty[s], ((it / AT_STAGES) - 1) & 1, &sm.abort)) {
+          record_abort(sm, a.status, 11);
+          alive = false;
+          break;
+        }
+        const uint32_t k_s = smem_u32(sm.kv[s][0]), v_s = smem_u32(sm.kv[s][1]);
+        mbar_arrive_expect_tx(&sm.kv_full[s], 2 * TILE_BYTES);
+        // selected tiles read the gathered copy (rows past nsel are zero
+        // fill or stale copies, masked by the softmax); chunk tiles the chunk
+        const bool sel_tile = gi < ntile_sel;
+        const CUtensorMap* mk = sel_tile ? &maps.ks : &maps.kc;
+        const CUtensorMap* mv = sel_tile ? &maps.vs : &maps.vc;
+        const int y = sel_tile ? gi * AT_N : (gi - ntile_sel) * AT_N;
+        tma_load_4d(k_s, mk, &sm.kv_full[s], 0, y, j, bi);
+        tma_load_4d(k_s + ATOM_BYTES, mk, &sm.kv_full[s], 64, y, j, bi);
+        tma_load_4d(v_s, mv, &sm.kv_full[s], 0, y, j, bi);
+        tma_load_4d(v_s + ATOM_BYTES, mv, &sm.kv_full[s], 64, y, j, bi);
+        issued = it + 1;
+      }
+      // no copy may still be landing when the CTA exits (matters only when
+      // a consumer gave up early): wait, bounded, for the last fill of each
+      // stage and for Q
+      for (int s = 0; s < AT_STAGES; ++s) {
+        const int nf = issued > s ? (issued - s + AT_STAGES - 1) / AT_STAGES : 0;
+        if (nf > 0 && !mbar_drain(&sm.kv_full[s], (nf - 1) & 1)) record_abort(sm, a.status, 12);
+      }
+      if (!mbar_drain(&sm.q_full, 0)) record_abort(sm, a.status, 13);
+    }
+    __syncwarp();
+  } else if (!TMA_KV && warp >= AT_LD_WARP0) {
     // ------------------------------------------------------------ loaders
     const int lt = tid - AT_LD_WARP0 * 32;  // 0..255
     const int c = lt & 15;                   // 16-byte chunk of a row
@@ -543,11 +604,31 @@ attn_tc_kernel(const __grid_constant__ AttnMaps maps, const AttnArgs a, int nspl
 
 cudaError_t launch_attn_tc(const AttnArgs& a, cudaStream_t stream) {
   if (a.d != AT_D) return cudaErrorNotSupported;
+  // with no selected keys every tile is a chunk tile: TMA boxes as well
+  const bool tma_kv = a.kv_idx == nullptr || a.bsa == 0;
   AttnMaps maps;
   if (!encode_bf16_4d(&maps.q, a.Q.data, AT_D, a.BCP, a.nq, a.b, a.Q.st, a.Q.sh, a.Q.sb, 128))
     return cudaErrorNotSupported;
+  if (tma_kv) {
+    if (!encode_bf16_4d(&maps.kc, a.Kc.data, AT_D, a.BCP, a.nkv, a.b, a.Kc.st, a.Kc.sh, a.Kc.sb, 128) ||
+        !encode_bf16_4d(&maps.vc, a.Vc.data, AT_D, a.BCP, a.nkv, a.b, a.Vc.st, a.Vc.sh, a.Vc.sb, 128))
+      return cudaErrorNotSupported;
+    if (a.bsa > 0) {
+      // the gathered selected rows (b, nkv, bsa, d); rows past a list's
+      // count are masked in the softmax
+      if (!encode_bf16_4d(&maps.ks, a.K.data, AT_D, a.bsa, a.nkv, a.b, a.K.st, a.K.sh, a.K.sb, 128) ||
+          !encode_bf16_4d(&maps.vs, a.V.data, AT_D, a.bsa, a.nkv, a.b, a.V.st, a.V.sh, a.V.sb, 128))
+        return cudaErrorNotSupported;
+    } else {
+      maps.ks = maps.kc;  // never read: there are no selected tiles
+      maps.vs = maps.vc;
+    }
+  } else {
+    maps.ks = maps.vs = maps.kc = maps.vc = maps.q;  // unused by the gather loader
+  }
   const size_t smem = sizeof(AttnSmem) + 1024;
-  cudaError_t e = cudaFuncSetAttribute(attn_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+  auto kern = tma_kv ? attn_tc_kernel<true> : attn_tc_kernel<false>;
+  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (e != cudaSuccess) return e;
   const int G = a.nq / a.nkv;
   const int R = G * ((a.BCP + 127) / 128);
@@ -561,7 +642,7 @@ cudaError_t launch_attn_tc(const AttnArgs& a, cudaStream_t stream) {
   const int nsplit = (2 * ctas <= num_sms) ? 2 : 1;
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(npairs * nsplit, a.nkv, a.b);
-  cfg.blockDim = dim3(AT_THREADS);
+  cfg.blockDim = dim3(tma_kv ? AttnCfg<true>::threads : AttnCfg<false>::threads);
   cfg.dynamicSmemBytes = smem;
   cfg.stream = stream;
   cudaLaunchAttribute attr[1];
@@ -571,7 +652,7 @@ cudaError_t launch_attn_tc(const AttnArgs& a, cudaStream_t stream) {
   attr[0].val.clusterDim.z = 1;
   cfg.attrs = attr;
   cfg.numAttrs = 1;
-  return cudaLaunchKernelEx(&cfg, attn_tc_kernel, maps, a, nsplit);
+  return cudaLaunchKernelEx(&cfg, kern, maps, a, nsplit);
 }
 
 }  // namespace quoka

@@ -53,7 +53,10 @@ cudaError_t launch_topk(const float* S_agg, int b, int nkv, int64_t T, int bsa,
                         const uint32_t* hist, int32_t* kv_idx, int32_t* kv_count,
                         cudaStream_t stream);
 
-// Step (f): standalone gather of the selected K and V rows.
+// Step (f): gather of the selected K and V rows into contiguous
+// (b, nkv, bsa, d) buffers. Rows past kv_count, and rows whose index is out
+// of range (latched as QUOKA_ERR_BOUNDS when status is given), are written
+// as zeros.
 cudaError_t launch_gather(bool bf16, int d, Strided K, Strided V, int b, int nkv, int64_t T,
                           const int32_t* kv_idx, const int32_t* kv_count, int bsa,
                           void* Ksel, void* Vsel, int* status, cudaStream_t stream);
@@ -62,7 +65,7 @@ struct AttnArgs {
   Strided Q, K, V, Kc, Vc;
   int b, nq, nkv, d, BCP;
   int64_t T;
-  const int32_t* kv_idx;    // (b, nkv, bsa)
+  const int32_t* kv_idx;    // (b, nkv, bsa), or null: K/V hold the gathered rows (row n = key n)
   const int32_t* kv_count;  // (b, nkv)
   int bsa;
   float scale;
@@ -74,7 +77,10 @@ struct AttnArgs {
 // Steps (f)+(g) in fp32 on the CUDA cores (any input dtype).
 cudaError_t launch_attn_simt(bool bf16, const AttnArgs& a, cudaStream_t stream);
 
-// Steps (f)+(g) on the tcgen05 tensor cores (bf16 only).
+// Steps (f)+(g) on the tcgen05 tensor cores (bf16 only). With a.kv_idx
+// null, a.K / a.V are the gathered selected rows (b, nkv, >= bsa, d) and
+// every K/V tile is a TMA box; otherwise the kernel gathers the rows itself
+// while loading them.
 // Returns cudaErrorNotSupported when the shape has no tensor-core variant.
 cudaError_t launch_attn_tc(const AttnArgs& a, cudaStream_t stream);
 

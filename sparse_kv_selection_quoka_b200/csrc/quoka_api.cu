@@ -29,11 +29,20 @@ struct WsLayout {
   size_t kvidx = 0;     // (b, nkv, BSA_eff) int32
   size_t kvcount = 0;   // (b, nkv) int32
   size_t hist = 0;      // (b, nkv, 4096) uint32: first-digit histogram of the score keys
+  size_t select_total = 0;  // end of what quoka_select needs
+  size_t ksel = 0;      // (b, nkv, BSA_eff, d) bf16: gathered selected K (tensor-core attention)
+  size_t vsel = 0;      // (b, nkv, BSA_eff, d) bf16: gathered selected V
   size_t total = 0;
 };
 
+// The tensor-core attention (bf16, d = 128) streams the selected rows from a
+// contiguous gathered copy when the workspace holds one.
+bool uses_gather_buffers(quoka_dtype dtype, int64_t d, int64_t bsa_eff) {
+  return dtype == QUOKA_BF16 && d == 128 && bsa_eff > 0;
+}
+
 WsLayout ws_layout(int64_t b, int64_t nq, int64_t nkv, int64_t d, int64_t T, int64_t NQ,
-                   int64_t bsa_eff) {
+                   int64_t bsa_eff, bool gather_buffers) {
   WsLayout L;
   size_t off = 0;
   auto take = [&](size_t bytes) {
@@ -50,8 +59,21 @@ WsLayout ws_layout(int64_t b, int64_t nq, int64_t nkv, int64_t d, int64_t T, int
   L.kvidx = take((size_t)(b * nkv * bsa_eff) * 4);
   L.kvcount = take((size_t)(b * nkv) * 4);
   L.hist = take((size_t)(b * nkv) * quoka::TOPK_HIST_BINS * 4);
+  L.select_total = off;
+  if (gather_buffers) {
+    L.ksel = take((size_t)(b * nkv * bsa_eff * d) * 2);
+    L.vsel = take((size_t)(b * nkv * bsa_eff * d) * 2);
+  }
   L.total = off;
   return L;
+}
+
+// Workspace of quoka_sparse_gqa_attn alone: the status words, then (when
+// used) the gathered selected K and V.
+size_t attn_ws_bytes(int64_t b, int64_t nkv, int64_t d, int64_t bsa_eff, bool gather_buffers) {
+  size_t n = kAlign;
+  if (gather_buffers) n += 2 * align_up((size_t)(b * nkv * bsa_eff * d) * 2);
+  return n;
 }
 
 size_t elt_size(quoka_dtype t) { return t == QUOKA_BF16 ? 2 : 4; }
@@ -124,8 +146,8 @@ quoka_status validate_select(const quoka_tensor* Q, const quoka_tensor* K, int N
   return QUOKA_OK;
 }
 
-quoka_status check_ws(void* ws, size_t ws_bytes, const WsLayout& L) {
-  if (ws == nullptr || ((uintptr_t)ws % kAlign) != 0 || ws_bytes < L.total) return QUOKA_ERR_WORKSPACE;
+quoka_status check_ws(void* ws, size_t ws_bytes, size_t need) {
+  if (ws == nullptr || ((uintptr_t)ws % kAlign) != 0 || ws_bytes < need) return QUOKA_ERR_WORKSPACE;
   return QUOKA_OK;
 }
 
@@ -208,14 +230,16 @@ quoka_status validate_attn(const quoka_tensor* Q, const quoka_tensor* K, const q
   return QUOKA_OK;
 }
 
-quoka_status run_attn(const quoka_tensor* Q, const quoka_tensor* K, const quoka_tensor* V,
-                      const quoka_tensor* Kc, const quoka_tensor* Vc, const AttnShapes& s,
-                      const int32_t* kv_idx, const int32_t* kv_count, int bsa_eff, float scale,
-                      void* O, float* lse, int* status, cudaStream_t stream) {
+// Step (g) (with step (f) fused into the loads when kv_idx is given; with
+// kv_idx null, K / V are the gathered selected rows and T their row count).
+quoka_status run_attn(const quoka_tensor* Q, Strided K, Strided V, const quoka_tensor* Kc,
+                      const quoka_tensor* Vc, const AttnShapes& s, int64_t T, const int32_t* kv_idx,
+                      const int32_t* kv_count, int bsa_eff, float scale, void* O, float* lse,
+                      int* status, cudaStream_t stream) {
   quoka::AttnArgs a;
   a.Q = strided(Q);
-  a.K = strided(K);
-  a.V = strided(V);
+  a.K = K;
+  a.V = V;
   a.Kc = strided(Kc);
   a.Vc = strided(Vc);
   a.b = (int)s.b;
@@ -223,7 +247,7 @@ quoka_status run_attn(const quoka_tensor* Q, const quoka_tensor* K, const quoka_
   a.nkv = (int)s.nkv;
   a.d = (int)s.d;
   a.BCP = (int)s.BCP;
-  a.T = s.T;
+  a.T = T;
   a.kv_idx = kv_idx;
   a.kv_count = kv_count;
   a.bsa = bsa_eff;
@@ -237,6 +261,25 @@ quoka_status run_attn(const quoka_tensor* Q, const quoka_tensor* K, const quoka_
   return cuda_status(e);
 }
 
+// Steps (f)+(g) on the full cache K / V: when `gathered` (the workspace's
+// Ksel / Vsel buffers) is given, step (f) runs as its own kernel into it and
+// the attention streams the copy; otherwise the attention gathers in place.
+quoka_status gather_then_attn(const quoka_tensor* Q, const quoka_tensor* K, const quoka_tensor* V,
+                              const quoka_tensor* Kc, const quoka_tensor* Vc, const AttnShapes& s,
+                              const int32_t* kv_idx, const int32_t* kv_count, int bsa_eff, float scale,
+                              void* O, float* lse, void* ksel, void* vsel, int* status,
+                              cudaStream_t stream) {
+  if (ksel == nullptr || vsel == nullptr || bsa_eff == 0)
+    return run_attn(Q, strided(K), strided(V), Kc, Vc, s, s.T, kv_idx, kv_count, bsa_eff, scale, O, lse,
+                    status, stream);
+  cudaError_t e = quoka::launch_gather(Q->dtype == QUOKA_BF16, (int)s.d, strided(K), strided(V), (int)s.b,
+                                       (int)s.nkv, s.T, kv_idx, kv_count, bsa_eff, ksel, vsel, status, stream);
+  if (e != cudaSuccess) return cuda_status(e);
+  const int64_t sh = (int64_t)bsa_eff * s.d, sb = s.nkv * sh;
+  return run_attn(Q, Strided{ksel, sb, sh, s.d}, Strided{vsel, sb, sh, s.d}, Kc, Vc, s, bsa_eff, nullptr,
+                  kv_count, bsa_eff, scale, O, lse, status, stream);
+}
+
 }  // namespace
 
 extern "C" {
@@ -246,7 +289,20 @@ size_t quoka_workspace_size(int b, int nq, int nkv, int d, int64_t T, int BCP, i
   if (b < 1 || nq < 1 || nkv < 1 || d < 1 || T < 0 || BCP < 1 || NQ < 1 || BSA < 0) return 0;
   if (nq % nkv != 0 || (dtype != QUOKA_F32 && dtype != QUOKA_BF16)) return 0;
   const int64_t bsa_eff = std::min<int64_t>(BSA, T);
-  return ws_layout(b, nq, nkv, d, T, NQ, bsa_eff).total;
+  return ws_layout(b, nq, nkv, d, T, NQ, bsa_eff, uses_gather_buffers(dtype, d, bsa_eff)).total;
+}
+
+size_t quoka_select_workspace_size(int b, int nq, int nkv, int d, int64_t T, int BCP, int NQ, int BSA,
+                                   quoka_dtype dtype) {
+  if (quoka_workspace_size(b, nq, nkv, d, T, BCP, NQ, BSA, dtype) == 0) return 0;
+  const int64_t bsa_eff = std::min<int64_t>(BSA, T);
+  return ws_layout(b, nq, nkv, d, T, NQ, bsa_eff, false).select_total;
+}
+
+size_t quoka_attn_workspace_size(int b, int nkv, int d, int BSA_eff, quoka_dtype dtype) {
+  if (b < 1 || nkv < 1 || d < 1 || BSA_eff < 0) return 0;
+  if (dtype != QUOKA_F32 && dtype != QUOKA_BF16) return 0;
+  return attn_ws_bytes(b, nkv, d, BSA_eff, uses_gather_buffers(dtype, d, BSA_eff));
 }
 
 quoka_status quoka_select(const quoka_tensor* Q, const quoka_tensor* K, int NQ, int BSA,
@@ -257,8 +313,8 @@ quoka_status quoka_select(const quoka_tensor* Q, const quoka_tensor* K, int NQ, 
   if (st != QUOKA_OK) return st;
   const int64_t bsa_eff = std::min<int64_t>(BSA, s.T);
   if (kv_count == nullptr || (bsa_eff > 0 && kv_idx == nullptr)) return QUOKA_ERR_INVALID_ARG;
-  const WsLayout L = ws_layout(s.b, s.nq, s.nkv, s.d, s.T, NQ, bsa_eff);
-  st = check_ws(ws, ws_bytes, L);
+  const WsLayout L = ws_layout(s.b, s.nq, s.nkv, s.d, s.T, NQ, bsa_eff, false);
+  st = check_ws(ws, ws_bytes, L.select_total);
   if (st != QUOKA_OK) return st;
   cudaStream_t cs = static_cast<cudaStream_t>(stream);
   if (cudaMemsetAsync(at<int>(ws, L.status), 0, 2 * sizeof(int), cs) != cudaSuccess) return QUOKA_ERR_CUDA;
@@ -307,7 +363,36 @@ quoka_status quoka_sparse_gqa_attn(const quoka_tensor* Q, const quoka_tensor* K,
   cudaStream_t cs = static_cast<cudaStream_t>(stream);
   int* status = static_cast<int*>(ws);
   if (cudaMemsetAsync(status, 0, 2 * sizeof(int), cs) != cudaSuccess) return QUOKA_ERR_CUDA;
-  return run_attn(Q, K, V, Kc, Vc, s, kv_idx, kv_count, BSA_eff, scale, O, lse, status, cs);
+  // with room for the gathered copy, the selected rows are gathered first
+  void* ksel = nullptr;
+  void* vsel = nullptr;
+  const bool gb = uses_gather_buffers(Q->dtype, s.d, BSA_eff);
+  if (gb && ws_bytes >= attn_ws_bytes(s.b, s.nkv, s.d, BSA_eff, true)) {
+    ksel = static_cast<char*>(ws) + kAlign;
+    vsel = static_cast<char*>(ksel) + align_up((size_t)(s.b * s.nkv * BSA_eff * s.d) * 2);
+  }
+  return gather_then_attn(Q, K, V, Kc, Vc, s, kv_idx, kv_count, BSA_eff, scale, O, lse, ksel, vsel, status,
+                          cs);
+}
+
+quoka_status quoka_sparse_gqa_attn_gathered(const quoka_tensor* Q, const quoka_tensor* Ksel,
+                                            const quoka_tensor* Vsel, const int32_t* kv_count,
+                                            const quoka_tensor* Kc, const quoka_tensor* Vc, float scale,
+                                            void* O, float* lse, void* ws, size_t ws_bytes,
+                                            void* stream) {
+  AttnShapes s;
+  quoka_status st = validate_attn(Q, Ksel, Vsel, Kc, Vc, &s);
+  if (st != QUOKA_OK) return st;
+  if (kv_count == nullptr) return QUOKA_ERR_INVALID_ARG;
+  if (O == nullptr || !aligned16(O)) return QUOKA_ERR_INVALID_ARG;
+  if (!(scale > 0.f) || scale != scale) return QUOKA_ERR_INVALID_ARG;
+  if (ws == nullptr || ((uintptr_t)ws % kAlign) != 0 || ws_bytes < kAlign) return QUOKA_ERR_WORKSPACE;
+  cudaStream_t cs = static_cast<cudaStream_t>(stream);
+  int* status = static_cast<int*>(ws);
+  if (cudaMemsetAsync(status, 0, 2 * sizeof(int), cs) != cudaSuccess) return QUOKA_ERR_CUDA;
+  // the rows of Ksel / Vsel are the selected keys in list order: BSA_eff = T
+  return run_attn(Q, strided(Ksel), strided(Vsel), Kc, Vc, s, s.T, nullptr, kv_count, (int)s.T, scale, O,
+                  lse, status, cs);
 }
 
 quoka_status quoka_prefill_chunk(const quoka_tensor* Q, const quoka_tensor* K,
@@ -324,8 +409,9 @@ quoka_status quoka_prefill_chunk(const quoka_tensor* Q, const quoka_tensor* K,
   if (O == nullptr || !aligned16(O)) return QUOKA_ERR_INVALID_ARG;
   if (!(scale > 0.f) || scale != scale) return QUOKA_ERR_INVALID_ARG;
   const int64_t bsa_eff = std::min<int64_t>(BSA, s.T);
-  const WsLayout L = ws_layout(s.b, s.nq, s.nkv, s.d, s.T, NQ, bsa_eff);
-  st = check_ws(ws, ws_bytes, L);
+  const bool gb = uses_gather_buffers(Q->dtype, s.d, bsa_eff);
+  const WsLayout L = ws_layout(s.b, s.nq, s.nkv, s.d, s.T, NQ, bsa_eff, gb);
+  st = check_ws(ws, ws_bytes, L.total);
   if (st != QUOKA_OK) return st;
   cudaStream_t cs = static_cast<cudaStream_t>(stream);
   int* status = at<int>(ws, L.status);
@@ -334,7 +420,8 @@ quoka_status quoka_prefill_chunk(const quoka_tensor* Q, const quoka_tensor* K,
   int32_t* kv_count = at<int32_t>(ws, L.kvcount);
   st = run_select(Q, K, s, NQ, (int)bsa_eff, kv_idx, kv_count, nullptr, nullptr, ws, L, cs);
   if (st != QUOKA_OK) return st;
-  return run_attn(Q, K, V, Kc, Vc, as, kv_idx, kv_count, (int)bsa_eff, scale, O, lse, status, cs);
+  return gather_then_attn(Q, K, V, Kc, Vc, as, kv_idx, kv_count, (int)bsa_eff, scale, O, lse,
+                          gb ? at<void>(ws, L.ksel) : nullptr, gb ? at<void>(ws, L.vsel) : nullptr, status, cs);
 }
 
 quoka_status quoka_get_device_status(const void* ws, void* stream, int32_t* device_status) {

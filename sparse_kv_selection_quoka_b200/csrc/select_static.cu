@@ -50,7 +50,7 @@ extern "C" quoka_status quoka_select_static(const quoka_tensor* Q, const quoka_t
                                             int BSA, int32_t* kv_idx, int32_t* kv_count,
                                             int32_t* q_idx, float* s_agg, void* stream) {
   if (Q == nullptr || K == nullptr) return QUOKA_ERR_INVALID_ARG;
-  const size_t need = quoka_workspace_size((int)Q->shape[0], (int)Q->shape[1], (int)K->shape[1],
+  const size_t need = quoka_select_workspace_size((int)Q->shape[0], (int)Q->shape[1], (int)K->shape[1],
                                            (int)Q->shape[3], K->shape[2], (int)Q->shape[2], NQ, BSA,
                                            Q->dtype);
   if (need == 0) return QUOKA_ERR_INVALID_ARG;

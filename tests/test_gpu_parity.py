@@ -161,9 +161,14 @@ def test_sweep_chunks(c, sweep):
     run_prefill_and_check(x, ref, gi, rows=rows, dev=dev)
 
 
-def test_attention_on_given_selection_and_gather():
+@pytest.mark.parametrize("path", ["gathered", "fused", "split"])
+def test_attention_on_given_selection_and_gather(path):
     """quoka_sparse_gqa_attn and quoka_gather_kv on an externally given
-    sorted index set (the oracle's), independent of the selection kernels."""
+    sorted index set (the oracle's), independent of the selection kernels.
+    `gathered`: a workspace with room for the gathered copy (step (f) as its
+    own kernel, then dense tiles); `fused`: a 256-byte workspace (the
+    attention gathers the rows while loading them); `split`: quoka_gather_kv
+    then quoka_sparse_gqa_attn_gathered."""
     x = inputs.make_chunk(2, 8, 2, 128, 3000, 200, 8, 700, dtype="bf16", structure="qwen", seed=5)
     ref = orc.select(x.Q, x.K, x.NQ, x.BSA)
     sel = ref["sel"]
@@ -171,8 +176,12 @@ def test_attention_on_given_selection_and_gather():
     Q, K, V, Kc, Vc = (P.to_dev(a, dt) for a in (x.Q, x.K, x.V, x.Kc, x.Vc))
     kv_idx = torch.from_numpy(sel.astype(np.int32)).cuda()
     kv_count = torch.full((2, 2), sel.shape[2], dtype=torch.int32, device="cuda")
-    O, lse = q().quoka_sparse_gqa_attn(Q, K, V, kv_idx, kv_count, Kc, Vc, want_lse=True)
+    ws = None if path == "gathered" else torch.zeros(256, dtype=torch.uint8, device="cuda")
     Ks, Vs = q().quoka_gather_kv(K, V, kv_idx, kv_count)
+    if path == "split":
+        O, lse = q().quoka_sparse_gqa_attn_gathered(Q, Ks, Vs, kv_count, Kc, Vc, want_lse=True, ws=ws)
+    else:
+        O, lse = q().quoka_sparse_gqa_attn(Q, K, V, kv_idx, kv_count, Kc, Vc, want_lse=True, ws=ws)
     torch.cuda.synchronize()
     O_ref, L_ref = orc.sparse_attention(x.Q, x.K, x.V, sel, x.Kc, x.Vc)
     assert np.abs(O.float().cpu().numpy() - O_ref).max() <= P.O_TOL_BF16
@@ -203,6 +212,66 @@ def test_partial_count_uses_prefix_of_index_rows():
         Og = O.cpu().numpy()
         got = np.stack([Og[r] for r in rows])
         assert np.abs(got - O_ref).max() <= P.O_TOL_F32
+
+
+@pytest.mark.parametrize("path", ["gathered", "fused"])
+def test_partial_count_bf16_tensor_core_path(path):
+    """bf16, d = 128: kv_count below the row length on the tensor-core path.
+    The workspace starts as all-ones bytes (NaN as bf16), so rows of the
+    gathered copy past the count that were not zero-filled would poison the
+    output; the index tail holds out-of-range values that must not be read."""
+    x = inputs.make_chunk(1, 8, 2, 128, 3000, 200, 8, 600, dtype="bf16", structure="llama", seed=16)
+    rng = np.random.default_rng(16)
+    sel = np.stack([[np.sort(rng.choice(3000, 600, replace=False)) for _ in range(2)]])
+    counts = np.array([[1, 333]], dtype=np.int32)
+    idx = sel.copy()
+    idx[0, 0, 1:] = 10 ** 6
+    idx[0, 1, 333:] = -5
+    Q, K, V, Kc, Vc = (P.to_dev(a, "bf16") for a in (x.Q, x.K, x.V, x.Kc, x.Vc))
+    n = q().quoka_attn_workspace_size(1, 2, 128, 600, torch.bfloat16) if path == "gathered" else 256
+    ws = torch.full((n,), 255, dtype=torch.uint8, device="cuda")
+    O, lse = q().quoka_sparse_gqa_attn(Q, K, V, torch.from_numpy(idx.astype(np.int32)).cuda(),
+                                       torch.from_numpy(counts).cuda(), Kc, Vc, want_lse=True, ws=ws)
+    assert q().quoka_get_device_status(ws) == 0
+    Og = O.float().cpu().numpy()
+    for j, c in enumerate([1, 333]):
+        rows = [(0, h, t) for h in range(4 * j, 4 * j + 4) for t in range(200)]
+        sub = np.zeros((1, 2, c), dtype=np.int64)
+        sub[0, j] = sel[0, j, :c]
+        O_ref, _ = orc.sparse_attention_rows(x.Q, x.K, x.V, sub, x.Kc, x.Vc, rows)
+        got = np.stack([Og[r] for r in rows])
+        assert np.abs(got - O_ref).max() <= P.O_TOL_BF16
+
+
+def test_gathered_attention_fp32_and_partial_counts():
+    """quoka_gather_kv + quoka_sparse_gqa_attn_gathered in fp32 (CUDA-core
+    path), with counts below the row length: the gather writes zeros past the
+    count and the attention masks those rows."""
+    x = inputs.make_chunk(2, 6, 3, 64, 900, 70, 5, 200, dtype="f32", structure="llama", seed=17)
+    rng = np.random.default_rng(17)
+    sel = np.stack([[np.sort(rng.choice(900, 200, replace=False)) for _ in range(3)] for _ in range(2)])
+    counts = np.array([[200, 0, 17], [5, 199, 200]], dtype=np.int32)
+    Q, K, V, Kc, Vc = (P.to_dev(a, "f32") for a in (x.Q, x.K, x.V, x.Kc, x.Vc))
+    idx = torch.from_numpy(sel.astype(np.int32)).cuda()
+    cnt = torch.from_numpy(counts).cuda()
+    Ks = torch.full((2, 3, 200, 64), float("nan"), device="cuda")
+    Vs = torch.full((2, 3, 200, 64), float("nan"), device="cuda")
+    q().quoka_gather_kv(K, V, idx, cnt, Ksel=Ks, Vsel=Vs)
+    O, lse = q().quoka_sparse_gqa_attn_gathered(Q, Ks, Vs, cnt, Kc, Vc, want_lse=True)
+    torch.cuda.synchronize()
+    for bi in range(2):
+        for j in range(3):
+            c = counts[bi, j]
+            np.testing.assert_array_equal(Ks[bi, j, :c].cpu().numpy(), x.K[bi, j, sel[bi, j, :c]])
+            assert (Ks[bi, j, c:] == 0).all() and (Vs[bi, j, c:] == 0).all()
+    rows = [(bi, h, t) for bi in range(2) for h in range(6) for t in range(0, 70, 3)]
+    Og = O.cpu().numpy()
+    for (bi, h, t) in rows:
+        j = h // 2
+        sub = np.zeros((2, 3, counts[bi, j]), dtype=np.int64)
+        sub[bi, j] = sel[bi, j, :counts[bi, j]]
+        O_ref, _ = orc.sparse_attention_rows(x.Q, x.K, x.V, sub, x.Kc, x.Vc, [(bi, h, t)])
+        assert np.abs(Og[bi, h, t] - O_ref[0]).max() <= P.O_TOL_F32
 
 
 def test_planted_exact_ties_go_to_lower_index():
@@ -247,3 +316,16 @@ def test_out_of_range_index_is_latched_not_read():
     torch.cuda.synchronize()
     # the in-range rows were still gathered
     np.testing.assert_array_equal(Ks[0, 0, :3].cpu().numpy(), x.K[0, 0, [1, 5, 99]])
+
+
+@pytest.mark.parametrize("path", ["gathered", "fused"])
+def test_out_of_range_index_latched_bf16_tensor_core_path(path):
+    x = inputs.make_chunk(1, 4, 1, 128, 300, 64, 2, 10, dtype="bf16", structure="iid", seed=19)
+    Q, K, V, Kc, Vc = (P.to_dev(a, "bf16") for a in (x.Q, x.K, x.V, x.Kc, x.Vc))
+    idx = torch.tensor([[[1, 5, 99, 300, 2000]]], dtype=torch.int32, device="cuda")
+    cnt = torch.tensor([[5]], dtype=torch.int32, device="cuda")
+    n = q().quoka_attn_workspace_size(1, 1, 128, 5, torch.bfloat16) if path == "gathered" else 256
+    ws = torch.zeros(n, dtype=torch.uint8, device="cuda")
+    O, _ = q().quoka_sparse_gqa_attn(Q, K, V, idx, cnt, Kc, Vc, ws=ws)
+    assert q().quoka_get_device_status(ws) == 6
+    assert torch.isfinite(O.float()).all()

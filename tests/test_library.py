@@ -59,6 +59,31 @@ def test_workspace_size_host_only(lib):
     assert lib.quoka_workspace_size(1, 32, 8, 128, 100, 64, 4, 10, 7) == 0    # dtype
 
 
+def test_workspace_parts_host_only(lib):
+    # quoka_select needs only its own part; the full size adds the gathered
+    # selected K and V (bf16, d = 128) of the attention
+    full = lib.quoka_workspace_size(1, 32, 8, 128, 32768, 512, 32, 4096, 1)
+    sel = lib.quoka_select_workspace_size(1, 32, 8, 128, 32768, 512, 32, 4096, 1)
+    att = lib.quoka_attn_workspace_size(1, 8, 128, 4096, 1)
+    gathered = 2 * 8 * 4096 * 128 * 2
+    assert att == 256 + gathered
+    assert full == sel + gathered
+    # fp32, d = 64 and BSA_eff = 0 need no gathered copy
+    assert lib.quoka_attn_workspace_size(1, 8, 128, 4096, 0) == 256
+    assert lib.quoka_attn_workspace_size(1, 8, 64, 4096, 1) == 256
+    assert lib.quoka_attn_workspace_size(1, 8, 128, 0, 1) == 256
+    assert (lib.quoka_workspace_size(1, 32, 8, 128, 32768, 512, 32, 4096, 0)
+            == lib.quoka_select_workspace_size(1, 32, 8, 128, 32768, 512, 32, 4096, 0))
+    # BSA beyond T is clipped to BSA_eff = T
+    assert (lib.quoka_workspace_size(1, 4, 2, 128, 100, 64, 4, 1000, 1)
+            == lib.quoka_select_workspace_size(1, 4, 2, 128, 100, 64, 4, 1000, 1)
+            + 2 * ((2 * 100 * 128 * 2 + 255) // 256 * 256))
+    assert lib.quoka_select_workspace_size(1, 30, 8, 128, 100, 64, 4, 10, 1) == 0
+    assert lib.quoka_attn_workspace_size(0, 8, 128, 10, 1) == 0
+    assert lib.quoka_attn_workspace_size(1, 8, 128, -1, 1) == 0
+    assert lib.quoka_attn_workspace_size(1, 8, 128, 10, 7) == 0
+
+
 def _view(shape, dtype=1, data=0x10000, stride=None):
     from sparse_kv_selection_quoka_b200._lib import quoka_tensor
     v = quoka_tensor()
