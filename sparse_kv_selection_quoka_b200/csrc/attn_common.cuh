@@ -1,0 +1,187 @@
+// Pieces shared by the two tcgen05 attention kernels (the one that streams
+// gathered K/V tiles with TMA and the one that gathers rows while loading).
+//
+// Layout shared by both: a CTA owns two 128-row query tiles of one KV head;
+// TMEM holds S0 | S1 | O0 | O1 (128 fp32 columns each, 512 in all). Thread r
+// of softmax warpgroup w owns query row r of tile w, which is TMEM lane r.
+#pragma once
+
+#include "common.cuh"
+#include "sm100.cuh"
+
+namespace quoka {
+namespace attn {
+
+using namespace sm100;
+
+constexpr int D = 128;                    // head dim
+constexpr int N = 128;                    // keys per tile
+constexpr int TILE_BYTES = 128 * D * 2;   // one 128-row bf16 tile
+constexpr int ATOM_BYTES = 128 * 128;     // one 64-column swizzle atom of a 128-row tile
+constexpr uint32_t TMEM_COLS = 512;
+constexpr int SOFTMAX_THREADS = 256;      // warps 0-7
+constexpr float RESCALE_THRESHOLD = 8.f;  // log2 units
+
+constexpr uint32_t IDESC_QK = idesc_bf16_f32(128, N, 0, 0);  // A = Q K-major, B = K K-major
+constexpr uint32_t IDESC_PV = idesc_bf16_f32(128, D, 0, 1);  // A = P (TMEM), B = V MN-major
+
+struct TileInfo {
+  int valid, h, t0;
+};
+
+// Query tiles of pair `pair` of KV head j: row tile r = 2 * pair + w is query
+// head j * G + r / ntt, chunk rows [128 * (r % ntt), +128).
+__device__ __forceinline__ void pair_tiles(int pair, int j, int G, int ntt, TileInfo (&ti)[2]) {
+  const int R = G * ntt;
+#pragma unroll
+  for (int w = 0; w < 2; ++w) {
+    const int r = 2 * pair + w;
+    ti[w].valid = r < R;
+    ti[w].h = j * G + (r < R ? r / ntt : 0);
+    ti[w].t0 = (r < R ? r % ntt : 0) * 128;
+  }
+}
+
+// A wait gave up: stop the CTA's other roles and record the fault and the
+// waiting site (a small code naming the barrier).
+template <class Smem>
+__device__ __forceinline__ void record_abort(Smem& sm, int* status, int where) {
+  sm.abort = 1;
+  latch_status(status, 5 /* QUOKA_ERR_TIMEOUT */);
+  latch_where(status, where);
+}
+
+// Warp-uniform bounded wait (every lane polls; all lanes agree on the result).
+template <class Smem>
+__device__ __forceinline__ bool warp_wait(uint64_t* bar, uint32_t parity, Smem& sm, int* status, int where) {
+  const bool ok = mbar_wait(bar, parity, &sm.abort);
+  const bool all_ok = __all_sync(0xffffffffu, ok);
+  if (!all_ok && (threadIdx.x & 31) == 0) record_abort(sm, status, where);
+  return all_ok;
+}
+
+// Bounded wait on a local barrier that another CTA of the cluster completes.
+__device__ __forceinline__ bool wait_cluster(uint64_t* bar, uint32_t parity) {
+  bool ok = mbar_try_wait_cluster(bar, parity);
+  if (!ok) {
+    const uint64_t t0 = globaltimer_ns();
+    while (!ok && globaltimer_ns() - t0 < kWaitLimitNs) ok = mbar_try_wait_cluster(bar, parity);
+  }
+  return ok;
+}
+
+template <class Smem>
+__device__ __forceinline__ bool warp_wait_cluster(uint64_t* bar, uint32_t parity, Smem& sm, int* status, int where) {
+  const bool all_ok = __all_sync(0xffffffffu, wait_cluster(bar, parity));
+  if (!all_ok && (threadIdx.x & 31) == 0) record_abort(sm, status, where);
+  return all_ok;
+}
+
+__device__ __forceinline__ uint32_t pack_bf16x2(float a, float b) {
+  __nv_bfloat162 h = __floats2bfloat162_rn(a, b);
+  return *reinterpret_cast<uint32_t*>(&h);
+}
+
+// S[:, 0:128) = Q K^T for a 128-row Q tile and a 128-key K tile, both in
+// shared memory in the 128-byte-swizzled K-major layout (two 64-column atoms).
+__device__ __forceinline__ void issue_qk(uint32_t tmem_s, uint32_t q_smem, uint32_t k_smem) {
+#pragma unroll
+  for (int kk = 0; kk < D / 16; ++kk) {
+    const uint32_t koff = (kk >> 2) * ATOM_BYTES + (kk & 3) * 32;
+    umma_bf16_ss(tmem_s, sw128_desc(q_smem + koff, 16, 1024), sw128_desc(k_smem + koff, 16, 1024), IDESC_QK,
+                 kk > 0 ? 1u : 0u);
+  }
+}
+
+// O (+)= P V with P (bf16, packed two per column) in TMEM over the S columns
+// and V in shared memory in the 128-byte-swizzled MN-major layout.
+__device__ __forceinline__ void issue_pv(uint32_t tmem_o, uint32_t tmem_p, uint32_t v_smem, bool accumulate) {
+#pragma unroll
+  for (int kk = 0; kk < N / 16; ++kk)
+    umma_bf16_ts(tmem_o, tmem_p + kk * 8, sw128_desc(v_smem + kk * 2048, ATOM_BYTES, 1024), IDESC_PV,
+                 (accumulate || kk > 0) ? 1u : 0u);
+}
+
+// One key tile of the online softmax of this thread's query row, on S in
+// TMEM (this warp's lanes): key c of the tile (key number base_n + c) is
+// visible when base_n + c < lim. Two passes over the row (max, then
+// P = 2^(s * qscale - m) in bf16 over the consumed S columns); the running
+// max m moves only when it grows by more than RESCALE_THRESHOLD, in which
+// case the O accumulator (complete for the previous tiles) is rescaled in
+// TMEM. Updates m and l. Every TMEM access is warp-collective: no per-row
+// branch surrounds one.
+__device__ __forceinline__ void softmax_tile(uint32_t S, uint32_t O, bool have_o, int base_n, int lim, float qscale,
+                                             float& m, float& l) {
+  const bool all_vis = base_n + N <= lim;
+  float mx = -INFINITY;
+#pragma unroll 1
+  for (int h2 = 0; h2 < 2; ++h2) {
+    float v[64];
+    __syncwarp();
+    tmem_ld32(S + 64 * h2, *reinterpret_cast<float(*)[32]>(&v[0]));
+    tmem_ld32(S + 64 * h2 + 32, *reinterpret_cast<float(*)[32]>(&v[32]));
+    tmem_wait_ld();
+    if (all_vis) {
+      float m4[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
+#pragma unroll
+      for (int u = 0; u < 64; ++u) m4[u & 3] = fmaxf(m4[u & 3], v[u]);
+      mx = fmaxf(mx, fmaxf(fmaxf(m4[0], m4[1]), fmaxf(m4[2], m4[3])) * qscale);
+    } else {
+#pragma unroll
+      for (int u = 0; u < 64; ++u) {
+        const bool vis = base_n + 64 * h2 + u < lim;
+        mx = vis ? fmaxf(mx, v[u] * qscale) : mx;
+      }
+    }
+  }
+  const float m_cand = fmaxf(m, mx);
+  const float m_new = (m_cand > m + RESCALE_THRESHOLD || m == -INFINITY) ? m_cand : m;
+  const float corr = (m_new == m) ? 1.f : ex2(m - m_new);
+  const float m_use = m_new == -INFINITY ? 0.f : m_new;
+  float rs4[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll 1
+  for (int h2 = 0; h2 < 2; ++h2) {
+    float v[64];
+    __syncwarp();
+    tmem_ld32(S + 64 * h2, *reinterpret_cast<float(*)[32]>(&v[0]));
+    tmem_ld32(S + 64 * h2 + 32, *reinterpret_cast<float(*)[32]>(&v[32]));
+    tmem_wait_ld();
+    if (!all_vis) {
+#pragma unroll
+      for (int u = 0; u < 64; ++u) {
+        const bool vis = base_n + 64 * h2 + u < lim;
+        v[u] = vis ? v[u] : -INFINITY;
+      }
+    }
+#pragma unroll
+    for (int c2 = 0; c2 < 2; ++c2) {
+      uint32_t pk[16];
+#pragma unroll
+      for (int u = 0; u < 32; u += 2) {
+        const float p0 = ex2(fmaf(v[32 * c2 + u], qscale, -m_use));
+        const float p1 = ex2(fmaf(v[32 * c2 + u + 1], qscale, -m_use));
+        rs4[(u >> 1) & 3] += p0 + p1;
+        pk[u >> 1] = pack_bf16x2(p0, p1);
+      }
+      __syncwarp();
+      tmem_st16(S + 32 * h2 + 16 * c2, pk);
+    }
+  }
+  l = l * corr + ((rs4[0] + rs4[1]) + (rs4[2] + rs4[3]));
+  m = m_new;
+  // warp-uniform condition: the rescale's TMEM traffic is collective
+  if (have_o && __any_sync(0xffffffffu, corr != 1.f)) {
+#pragma unroll 1
+    for (int c4 = 0; c4 < 4; ++c4) {
+      float o[32];
+      tmem_ld32(O + 32 * c4, o);
+      tmem_wait_ld();
+#pragma unroll
+      for (int u = 0; u < 32; ++u) o[u] *= corr;
+      tmem_st32(O + 32 * c4, o);
+    }
+  }
+}
+
+}  // namespace attn
+}  // namespace quoka

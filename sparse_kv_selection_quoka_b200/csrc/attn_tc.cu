@@ -1,4 +1,5 @@
-// Sparse GQA attention on the tcgen05 tensor cores (bf16 in, fp32 accumulate).
+// Sparse GQA attention on the tcgen05 tensor cores, gathering the selected
+// K/V rows while loading them (bf16 in, fp32 accumulate).
 //
 // [QUOKA §4.2, problem 3] the selected KV is the attention's input, with no
 // causal mask over it; the chunk's own keys follow causally:
@@ -8,33 +9,25 @@
 // (QUOKA = the technical write-up "QUOKA: how it reshapes LLM prefill
 // efficiency", bqwf.cn news item 915859.)
 //
-// Work split. The query rows of one KV head j are cut into 128-row tiles
-// (one query head, 128 consecutive chunk positions each); a CTA takes two
-// such tiles (Q0, Q1) of the same KV head, so every K/V tile it brings in
-// feeds two 128x128x128 QK^T and two PV products. The key tiles of a CTA
-// are ceil(nsel/128) tiles of selected prior rows (rows past nsel are
-// masked) followed by ceil(nchunk/128) tiles of the chunk's own keys. When
-// the grid would fill less than half of the GPU, the key tiles are split
-// between the two CTAs of a cluster, and the partial results are combined
-// through distributed shared memory.
+// This variant serves callers whose workspace has no room for a gathered
+// copy of the selected rows; with one, the gather kernel runs first and the
+// TMA-streaming kernel (attn_tma.cu) does the attention, faster.
 //
-// Warp roles (320 or 544 threads):
-//   warps 0-3   softmax of Q0, warps 4-7 softmax of Q1: thread r owns query
-//               row r = TMEM lane r. Two passes over its S row in TMEM (row
-//               max, then exp2 on the MUFU); P is written back as bf16 over
-//               the S columns it has consumed, and is the A operand of PV
-//               straight from TMEM. The running max is only moved (and the O
-//               accumulator rescaled in TMEM) when it grows by more than 2^8,
-//               so rescales are rare. Final normalisation, combine and store.
+// Work split as in attn_tma.cu: a CTA takes two 128-row query tiles (Q0, Q1)
+// of one KV head; its key tiles are ceil(nsel/128) tiles of selected prior
+// rows (read in place through the sorted index list; rows past nsel are
+// zero-filled and masked) followed by ceil(nchunk/128) tiles of the chunk's
+// own keys. When the grid would fill less than half of the GPU, the key
+// tiles are split between the two CTAs of a cluster, and the partial results
+// are combined through distributed shared memory.
+//
+// Warp roles (544 threads):
+//   warps 0-7   softmax of Q0 (warps 0-3) and Q1 (warps 4-7), one query row
+//               per thread (attn_common.cuh); final normalisation, combine,
+//               store.
 //   warp 8      TMEM allocation and the single-thread MMA issue, ordered
-//               QK0(i), PV1(i-1), QK1(i), PV0(i): while one softmax group
-//               works, the tensor core runs the other group's products.
-//   Two loader variants (a template parameter):
-//   (TMA)       warp 9 issues TMA boxes: the selected keys come from a
-//               contiguous copy made by the gather kernel just before (so
-//               they are L2-resident), the chunk keys and Q from the inputs.
-//               320 threads. Used whenever the workspace holds the copy.
-//   (gather)    warps 9-16  loaders (256 threads): cp.async 16-byte row chunks, gathered
+//               QK0(i), PV1(i-1), QK1(i), PV0(i).
+//   warps 9-16  loaders (256 threads): cp.async 16-byte row chunks, gathered
 //               by index, into a 2-stage K/V ring in the 128-byte-swizzled
 //               UMMA layout (zero-fill past the end of a list); each thread
 //               owns one 16-byte column chunk of 8 rows per tile, prefetches
@@ -44,46 +37,29 @@
 //               measured on B200, 16-byte cp.async gathers reach ~47 GB/s per
 //               SM from 256 threads but ~24 GB/s from 96, and TMA
 //               tile::gather4 ~16 GB/s.
-// TMEM: S0 | S1 | O0 | O1, 128 columns each (512).
 // Every wait is bounded: a wait that gives up records QUOKA_ERR_TIMEOUT and
 // the CTA unwinds (waits for in-flight copies and MMAs, frees TMEM).
-#include "common.cuh"
+#include "attn_common.cuh"
 #include "kernels.h"
-#include "sm100.cuh"
 #include "tmap.cuh"
 
 namespace quoka {
 
 using namespace sm100;
+using namespace attn;
 
 namespace {
 
-constexpr int AT_D = 128;        // head dim
-constexpr int AT_N = 128;        // keys per tile
 constexpr int AT_STAGES = 2;     // K/V ring depth
-template <bool TMA_KV>
-struct AttnCfg {
-  static constexpr int threads = TMA_KV ? 320 : 544;
-  static constexpr int kv_arrivals = TMA_KV ? 1 : 256;  // arrivals per stage fill
-};
+constexpr int AT_THREADS = 544;
 constexpr int AT_MMA_WARP = 8;
 constexpr int AT_LD_WARP0 = 9;
 constexpr int AT_LD_THREADS = 256;
-constexpr int AT_SM_THREADS = 256;
-constexpr int LD_ROWS = AT_N * 16 / AT_LD_THREADS;  // rows per loader thread per tile (8)
-constexpr int TILE_BYTES = 128 * AT_D * 2;  // 128 rows x 256 B
-constexpr int ATOM_BYTES = 128 * 128;       // one 64-column swizzle atom of a 128-row tile
-constexpr uint32_t TMEM_COLS = 512;
-constexpr float RESCALE_THRESHOLD = 8.f;    // log2 units
+constexpr int LD_ROWS = N * 16 / AT_LD_THREADS;  // rows per loader thread per tile (8)
 
-constexpr uint32_t IDESC_QK = idesc_bf16_f32(128, AT_N, 0, 0);  // A=Q K-major, B=K K-major
-constexpr uint32_t IDESC_PV = idesc_bf16_f32(128, AT_D, 0, 1);  // A=P (TMEM), B=V MN-major
-
-// TMA tensor maps (4-D boxes of 64 columns x 128 rows): the queries, and for
-// the TMA loader the gathered selected K/V (b, nkv, BSA, d) and the chunk's
-// K/V (b, nkv, BCP, d).
+// TMA tensor map of the queries (4-D boxes of 64 columns x 128 rows).
 struct AttnMaps {
-  CUtensorMap q, ks, vs, kc, vc;
+  CUtensorMap q;
 };
 
 struct __align__(1024) AttnSmem {
@@ -103,49 +79,10 @@ struct __align__(1024) AttnSmem {
 };
 // The split-KV landing zone in rank 0 reuses the K/V ring (partial O, fp32,
 // [tile][row][128] with a per-row chunk rotation) and the Q area (m, l).
-static_assert(sizeof(float) * 2 * 128 * AT_D <= AT_STAGES * 2 * TILE_BYTES, "landing zone");
+static_assert(sizeof(float) * 2 * 128 * D <= AT_STAGES * 2 * TILE_BYTES, "landing zone");
 
-struct TileInfo {
-  int valid, h, t0;
-};
-
-// A wait gave up: stop the CTA's other roles and record the fault and the
-// waiting site (a small code naming the barrier).
-__device__ __forceinline__ void record_abort(AttnSmem& sm, int* status, int where) {
-  sm.abort = 1;
-  latch_status(status, 5 /* QUOKA_ERR_TIMEOUT */);
-  latch_where(status, where);
-}
-
-// Warp-uniform bounded wait (every lane polls; all lanes agree on the result).
-__device__ __forceinline__ bool warp_wait(uint64_t* bar, uint32_t parity, AttnSmem& sm, int* status, int where) {
-  const bool ok = mbar_wait(bar, parity, &sm.abort);
-  const bool all_ok = __all_sync(0xffffffffu, ok);
-  if (!all_ok && (threadIdx.x & 31) == 0) record_abort(sm, status, where);
-  return all_ok;
-}
-
-// The same for a barrier that another CTA of the cluster arrives on.
-__device__ __forceinline__ bool warp_wait_cluster(uint64_t* bar, uint32_t parity, AttnSmem& sm, int* status,
-                                                  int where) {
-  bool ok = mbar_try_wait_cluster(bar, parity);
-  if (!ok) {
-    const uint64_t t0 = globaltimer_ns();
-    while (!ok && globaltimer_ns() - t0 < kWaitLimitNs) ok = mbar_try_wait_cluster(bar, parity);
-  }
-  const bool all_ok = __all_sync(0xffffffffu, ok);
-  if (!all_ok && (threadIdx.x & 31) == 0) record_abort(sm, status, where);
-  return all_ok;
-}
-
-__device__ __forceinline__ uint32_t pack_bf16x2(float a, float b) {
-  __nv_bfloat162 h = __floats2bfloat162_rn(a, b);
-  return *reinterpret_cast<uint32_t*>(&h);
-}
-
-template <bool TMA_KV>
-__global__ void __launch_bounds__(AttnCfg<TMA_KV>::threads, 1)
-attn_tc_kernel(const __grid_constant__ AttnMaps maps, const AttnArgs a, int nsplit) {
+__global__ void __launch_bounds__(AT_THREADS, 1)
+attn_gather_kernel(const __grid_constant__ AttnMaps maps, const AttnArgs a, int nsplit) {
   extern __shared__ uint8_t smem_raw[];
   AttnSmem& sm = *reinterpret_cast<AttnSmem*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
 
@@ -155,22 +92,14 @@ attn_tc_kernel(const __grid_constant__ AttnMaps maps, const AttnArgs a, int nspl
   const int split = nsplit > 1 ? (int)cluster_ctarank() : 0;
   const int pair = blockIdx.x / nsplit;
   const int ntt = (a.BCP + 127) / 128;  // row tiles per query head
-  const int R = G * ntt;                // row tiles per KV head
-
   TileInfo ti[2];
-#pragma unroll
-  for (int w = 0; w < 2; ++w) {
-    const int r = 2 * pair + w;
-    ti[w].valid = r < R;
-    ti[w].h = j * G + (r < R ? r / ntt : 0);
-    ti[w].t0 = (r < R ? r % ntt : 0) * 128;
-  }
+  pair_tiles(pair, j, G, ntt, ti);
   const int64_t kvrow = (int64_t)bi * a.nkv + j;
   const int nsel = a.bsa > 0 ? max(0, min(a.kv_count[kvrow], a.bsa)) : 0;
   const int max_t0 = ti[1].valid ? max(ti[0].t0, ti[1].t0) : ti[0].t0;
   const int nchunk = min(a.BCP, max_t0 + 128);
-  const int ntile_sel = (nsel + AT_N - 1) / AT_N;
-  const int ntile_chk = (nchunk + AT_N - 1) / AT_N;
+  const int ntile_sel = (nsel + N - 1) / N;
+  const int ntile_chk = (nchunk + N - 1) / N;
   const int nT = ntile_sel + ntile_chk;
   const int per = (nT + nsplit - 1) / nsplit;
   const int first = min(nT, split * per);
@@ -179,7 +108,7 @@ attn_tc_kernel(const __grid_constant__ AttnMaps maps, const AttnArgs a, int nspl
   if (tid == 0) {
     mbar_init(&sm.q_full, 1);
     for (int s = 0; s < AT_STAGES; ++s) {
-      mbar_init(&sm.kv_full[s], AttnCfg<TMA_KV>::kv_arrivals);
+      mbar_init(&sm.kv_full[s], AT_LD_THREADS);
       mbar_init(&sm.kv_empty[s], 1);
     }
     for (int w = 0; w < 2; ++w) {
@@ -189,7 +118,7 @@ attn_tc_kernel(const __grid_constant__ AttnMaps maps, const AttnArgs a, int nspl
     mbar_init(&sm.o_final, 1);
     mbar_init(&sm.mma_done, 1);
     mbar_init(&sm.xfer_free, 1);
-    mbar_init(&sm.xfer_full, AT_SM_THREADS);
+    mbar_init(&sm.xfer_full, SOFTMAX_THREADS);
     sm.abort = 0;
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
   }
@@ -207,56 +136,7 @@ attn_tc_kernel(const __grid_constant__ AttnMaps maps, const AttnArgs a, int nspl
   tc_fence_after();
   const uint32_t tmem = sm.tmem_base;
 
-  if (TMA_KV && warp == AT_LD_WARP0) {
-    // ------------------------------------------------------------ TMA loads
-    bool alive = true;
-    int issued = 0;
-    if (lane == 0) {
-      tma_prefetch_desc(&maps.q);
-      tma_prefetch_desc(&maps.ks);
-      tma_prefetch_desc(&maps.vs);
-      tma_prefetch_desc(&maps.kc);
-      tma_prefetch_desc(&maps.vc);
-      mbar_arrive_expect_tx(&sm.q_full, (ti[1].valid ? 2 : 1) * TILE_BYTES);
-      for (int w = 0; w < 2; ++w) {
-        if (!ti[w].valid) continue;
-        const uint32_t q_s = smem_u32(sm.q[w]);
-        tma_load_4d(q_s, &maps.q, &sm.q_full, 0, ti[w].t0, ti[w].h, bi);
-        tma_load_4d(q_s + ATOM_BYTES, &maps.q, &sm.q_full, 64, ti[w].t0, ti[w].h, bi);
-      }
-      for (int it = 0; it < ntiles && alive; ++it) {
-        const int s = it % AT_STAGES;
-        const int gi = first + it;
-        if (it >= AT_STAGES && !mbar_wait(&sm.kv_empty[s], ((it / AT_STAGES) - 1) & 1, &sm.abort)) {
-          record_abort(sm, a.status, 11);
-          alive = false;
-          break;
-        }
-        const uint32_t k_s = smem_u32(sm.kv[s][0]), v_s = smem_u32(sm.kv[s][1]);
-        mbar_arrive_expect_tx(&sm.kv_full[s], 2 * TILE_BYTES);
-        // selected tiles read the gathered copy (rows past nsel are zero
-        // fill or stale copies, masked by the softmax); chunk tiles the chunk
-        const bool sel_tile = gi < ntile_sel;
-        const CUtensorMap* mk = sel_tile ? &maps.ks : &maps.kc;
-        const CUtensorMap* mv = sel_tile ? &maps.vs : &maps.vc;
-        const int y = sel_tile ? gi * AT_N : (gi - ntile_sel) * AT_N;
-        tma_load_4d(k_s, mk, &sm.kv_full[s], 0, y, j, bi);
-        tma_load_4d(k_s + ATOM_BYTES, mk, &sm.kv_full[s], 64, y, j, bi);
-        tma_load_4d(v_s, mv, &sm.kv_full[s], 0, y, j, bi);
-        tma_load_4d(v_s + ATOM_BYTES, mv, &sm.kv_full[s], 64, y, j, bi);
-        issued = it + 1;
-      }
-      // no copy may still be landing when the CTA exits (matters only when
-      // a consumer gave up early): wait, bounded, for the last fill of each
-      // stage and for Q
-      for (int s = 0; s < AT_STAGES; ++s) {
-        const int nf = issued > s ? (issued - s + AT_STAGES - 1) / AT_STAGES : 0;
-        if (nf > 0 && !mbar_drain(&sm.kv_full[s], (nf - 1) & 1)) record_abort(sm, a.status, 12);
-      }
-      if (!mbar_drain(&sm.q_full, 0)) record_abort(sm, a.status, 13);
-    }
-    __syncwarp();
-  } else if (!TMA_KV && warp >= AT_LD_WARP0) {
+  if (warp >= AT_LD_WARP0) {
     // ------------------------------------------------------------ loaders
     const int lt = tid - AT_LD_WARP0 * 32;  // 0..255
     const int c = lt & 15;                   // 16-byte chunk of a row
@@ -282,7 +162,7 @@ attn_tc_kernel(const __grid_constant__ AttnMaps maps, const AttnArgs a, int nspl
     auto fetch_idx = [&](int gi) {
 #pragma unroll
       for (int k = 0; k < LD_ROWS; ++k) {
-        const int n = gi * AT_N + rg + 16 * k;
+        const int n = gi * N + rg + 16 * k;
         tau[k] = n < nsel ? __ldg(idx + n) : -1;
       }
     };
@@ -307,7 +187,7 @@ attn_tc_kernel(const __grid_constant__ AttnMaps maps, const AttnArgs a, int nspl
         }
         if (gi + 1 < ntile_sel && it + 1 < ntiles) fetch_idx(gi + 1);
       } else {
-        const int p0 = (gi - ntile_sel) * AT_N;
+        const int p0 = (gi - ntile_sel) * N;
 #pragma unroll
         for (int k = 0; k < LD_ROWS; ++k) {
           const int r = rg + 16 * k;
@@ -328,21 +208,11 @@ attn_tc_kernel(const __grid_constant__ AttnMaps maps, const AttnArgs a, int nspl
       const uint32_t q0 = smem_u32(sm.q[0]), q1 = smem_u32(sm.q[1]);
       const bool v0 = ti[0].valid, v1 = ti[1].valid;
       auto qk = [&](int w, int s) {
-        const uint32_t qs = w ? q1 : q0, ks = smem_u32(sm.kv[s][0]);
-#pragma unroll
-        for (int kk = 0; kk < AT_D / 16; ++kk) {
-          const uint32_t koff = (kk >> 2) * ATOM_BYTES + (kk & 3) * 32;
-          umma_bf16_ss(tmem + 128u * w, sw128_desc(qs + koff, 16, 1024), sw128_desc(ks + koff, 16, 1024),
-                       IDESC_QK, kk > 0 ? 1u : 0u);
-        }
+        issue_qk(tmem + 128u * w, w ? q1 : q0, smem_u32(sm.kv[s][0]));
         umma_commit(&sm.s_full[w]);
       };
       auto pv = [&](int w, int s, bool acc) {
-        const uint32_t vs = smem_u32(sm.kv[s][1]);
-#pragma unroll
-        for (int kk = 0; kk < AT_N / 16; ++kk)
-          umma_bf16_ts(tmem + 256u + 128u * w, tmem + 128u * w + kk * 8,
-                       sw128_desc(vs + kk * 2048, ATOM_BYTES, 1024), IDESC_PV, (acc || kk > 0) ? 1u : 0u);
+        issue_pv(tmem + 256u + 128u * w, tmem + 128u * w, smem_u32(sm.kv[s][1]), acc);
       };
       int where = 21;
       bool alive = mbar_wait(&sm.q_full, 0, &sm.abort);
@@ -409,87 +279,12 @@ attn_tc_kernel(const __grid_constant__ AttnMaps maps, const AttnArgs a, int nspl
       tc_fence_after();
       const int gi = first + it;
       const bool sel_tile = gi < ntile_sel;
-      // first key of the tile: selected-list index or chunk position
-      const int base_n = sel_tile ? gi * AT_N : (gi - ntile_sel) * AT_N;
-      // key c of the tile is visible to row t: a selected key below nsel, or
-      // a chunk key at a position p < nchunk with p <= t
+      // first key of the tile: selected-list index or chunk position; key c
+      // of the tile is visible to row t when it is a selected key below
+      // nsel, or a chunk key at a position p < nchunk with p <= t
+      const int base_n = sel_tile ? gi * N : (gi - ntile_sel) * N;
       const int lim = sel_tile ? nsel : min(nchunk, t + 1);
-      // rows whose every key of this tile is visible skip the per-key test
-      const bool all_vis = base_n + AT_N <= lim;
-      // pass 1: row max. TMEM loads are warp-collective, so they stay
-      // outside per-row branches; 64 columns per round trip.
-      float mx = -INFINITY;
-#pragma unroll 1
-      for (int h2 = 0; h2 < 2; ++h2) {
-        float v[64];
-        __syncwarp();
-        tmem_ld32(S + 64 * h2, *reinterpret_cast<float(*)[32]>(&v[0]));
-        tmem_ld32(S + 64 * h2 + 32, *reinterpret_cast<float(*)[32]>(&v[32]));
-        tmem_wait_ld();
-        if (all_vis) {
-          float m4[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
-#pragma unroll
-          for (int u = 0; u < 64; ++u) m4[u & 3] = fmaxf(m4[u & 3], v[u]);
-          mx = fmaxf(mx, fmaxf(fmaxf(m4[0], m4[1]), fmaxf(m4[2], m4[3])) * qscale);
-        } else {
-#pragma unroll
-          for (int u = 0; u < 64; ++u) {
-            const bool vis = base_n + 64 * h2 + u < lim;
-            mx = vis ? fmaxf(mx, v[u] * qscale) : mx;
-          }
-        }
-      }
-      const float m_cand = fmaxf(m, mx);
-      const float m_new = (m_cand > m + RESCALE_THRESHOLD || m == -INFINITY) ? m_cand : m;
-      const float corr = (m_new == m) ? 1.f : ex2(m - m_new);
-      const float m_use = m_new == -INFINITY ? 0.f : m_new;
-      // pass 2: P = 2^(s - m) in bf16, written over the S columns already read
-      float rs4[4] = {0.f, 0.f, 0.f, 0.f};
-#pragma unroll 1
-      for (int h2 = 0; h2 < 2; ++h2) {
-        float v[64];
-        __syncwarp();
-        tmem_ld32(S + 64 * h2, *reinterpret_cast<float(*)[32]>(&v[0]));
-        tmem_ld32(S + 64 * h2 + 32, *reinterpret_cast<float(*)[32]>(&v[32]));
-        tmem_wait_ld();
-        if (!all_vis) {
-#pragma unroll
-          for (int u = 0; u < 64; ++u) {
-            const bool vis = base_n + 64 * h2 + u < lim;
-            v[u] = vis ? v[u] : -INFINITY;
-          }
-        }
-#pragma unroll
-        for (int c2 = 0; c2 < 2; ++c2) {
-          uint32_t pk[16];
-#pragma unroll
-          for (int u = 0; u < 32; u += 2) {
-            const float p0 = ex2(fmaf(v[32 * c2 + u], qscale, -m_use));
-            const float p1 = ex2(fmaf(v[32 * c2 + u + 1], qscale, -m_use));
-            rs4[(u >> 1) & 3] += p0 + p1;
-            pk[u >> 1] = pack_bf16x2(p0, p1);
-          }
-          __syncwarp();
-          tmem_st16(S + 32 * h2 + 16 * c2, pk);
-        }
-      }
-      const float rs = (rs4[0] + rs4[1]) + (rs4[2] + rs4[3]);
-      l = l * corr + rs;
-      m = m_new;
-      // O holds the products of the previous tiles (complete: they were
-      // issued before this tile's QK^T, whose completion we waited for)
-      // (warp-uniform condition: the rescale's TMEM traffic is collective)
-      if (it > 0 && __any_sync(0xffffffffu, corr != 1.f)) {
-#pragma unroll 1
-        for (int c4 = 0; c4 < 4; ++c4) {
-          float o[32];
-          tmem_ld32(O + 32 * c4, o);
-          tmem_wait_ld();
-#pragma unroll
-          for (int u = 0; u < 32; ++u) o[u] *= corr;
-          tmem_st32(O + 32 * c4, o);
-        }
-      }
+      softmax_tile(S, O, it > 0, base_n, lim, qscale, m, l);
       tmem_wait_st();
       tc_fence_before();
       mbar_arrive(&sm.p_full[w]);
@@ -500,7 +295,7 @@ attn_tc_kernel(const __grid_constant__ AttnMaps maps, const AttnArgs a, int nspl
     if (alive) alive = warp_wait(&sm.o_final, 0, sm, a.status, 33);
     tc_fence_after();
     const float ln2 = 0.6931471805599453f;
-    float* land_o = reinterpret_cast<float*>(&sm.kv[0][0][0]) + (size_t)(w * 128 + r) * AT_D;
+    float* land_o = reinterpret_cast<float*>(&sm.kv[0][0][0]) + (size_t)(w * 128 + r) * D;
     float* land_ml = reinterpret_cast<float*>(&sm.q[0][0]) + (size_t)(w * 128 + r) * 2;
     if (nsplit > 1 && split == 1) {
       // send (O, m, l) of this row to rank 0 once its landing zone is free
@@ -548,7 +343,7 @@ attn_tc_kernel(const __grid_constant__ AttnMaps maps, const AttnArgs a, int nspl
         const float f_ot = m_o == -INFINITY ? 0.f : ex2(m_o - M);
         const float L = f_me * ll + f_ot * l_o;
         const float inv = 1.f / L;
-        bf16* orow = static_cast<bf16*>(a.O) + (((int64_t)bi * a.nq + ti[w].h) * a.BCP + t) * AT_D;
+        bf16* orow = static_cast<bf16*>(a.O) + (((int64_t)bi * a.nq + ti[w].h) * a.BCP + t) * D;
 #pragma unroll 1
         for (int c4 = 0; c4 < 4; ++c4) {
           float o[32];
@@ -602,33 +397,13 @@ attn_tc_kernel(const __grid_constant__ AttnMaps maps, const AttnArgs a, int nspl
 
 }  // namespace
 
-cudaError_t launch_attn_tc(const AttnArgs& a, cudaStream_t stream) {
-  if (a.d != AT_D) return cudaErrorNotSupported;
-  // with no selected keys every tile is a chunk tile: TMA boxes as well
-  const bool tma_kv = a.kv_idx == nullptr || a.bsa == 0;
+cudaError_t launch_attn_tc_gather(const AttnArgs& a, cudaStream_t stream) {
+  if (a.d != D) return cudaErrorNotSupported;
   AttnMaps maps;
-  if (!encode_bf16_4d(&maps.q, a.Q.data, AT_D, a.BCP, a.nq, a.b, a.Q.st, a.Q.sh, a.Q.sb, 128))
+  if (!encode_bf16_4d(&maps.q, a.Q.data, D, a.BCP, a.nq, a.b, a.Q.st, a.Q.sh, a.Q.sb, 128))
     return cudaErrorNotSupported;
-  if (tma_kv) {
-    if (!encode_bf16_4d(&maps.kc, a.Kc.data, AT_D, a.BCP, a.nkv, a.b, a.Kc.st, a.Kc.sh, a.Kc.sb, 128) ||
-        !encode_bf16_4d(&maps.vc, a.Vc.data, AT_D, a.BCP, a.nkv, a.b, a.Vc.st, a.Vc.sh, a.Vc.sb, 128))
-      return cudaErrorNotSupported;
-    if (a.bsa > 0) {
-      // the gathered selected rows (b, nkv, bsa, d); rows past a list's
-      // count are masked in the softmax
-      if (!encode_bf16_4d(&maps.ks, a.K.data, AT_D, a.bsa, a.nkv, a.b, a.K.st, a.K.sh, a.K.sb, 128) ||
-          !encode_bf16_4d(&maps.vs, a.V.data, AT_D, a.bsa, a.nkv, a.b, a.V.st, a.V.sh, a.V.sb, 128))
-        return cudaErrorNotSupported;
-    } else {
-      maps.ks = maps.kc;  // never read: there are no selected tiles
-      maps.vs = maps.vc;
-    }
-  } else {
-    maps.ks = maps.vs = maps.kc = maps.vc = maps.q;  // unused by the gather loader
-  }
   const size_t smem = sizeof(AttnSmem) + 1024;
-  auto kern = tma_kv ? attn_tc_kernel<true> : attn_tc_kernel<false>;
-  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+  cudaError_t e = cudaFuncSetAttribute(attn_gather_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (e != cudaSuccess) return e;
   const int G = a.nq / a.nkv;
   const int R = G * ((a.BCP + 127) / 128);
@@ -642,7 +417,7 @@ cudaError_t launch_attn_tc(const AttnArgs& a, cudaStream_t stream) {
   const int nsplit = (2 * ctas <= num_sms) ? 2 : 1;
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(npairs * nsplit, a.nkv, a.b);
-  cfg.blockDim = dim3(tma_kv ? AttnCfg<true>::threads : AttnCfg<false>::threads);
+  cfg.blockDim = dim3(AT_THREADS);
   cfg.dynamicSmemBytes = smem;
   cfg.stream = stream;
   cudaLaunchAttribute attr[1];
@@ -652,7 +427,7 @@ cudaError_t launch_attn_tc(const AttnArgs& a, cudaStream_t stream) {
   attr[0].val.clusterDim.z = 1;
   cfg.attrs = attr;
   cfg.numAttrs = 1;
-  return cudaLaunchKernelEx(&cfg, kern, maps, a, nsplit);
+  return cudaLaunchKernelEx(&cfg, attn_gather_kernel, maps, a, nsplit);
 }
 
 }  // namespace quoka

@@ -77,11 +77,13 @@ struct AttnArgs {
 // Steps (f)+(g) in fp32 on the CUDA cores (any input dtype).
 cudaError_t launch_attn_simt(bool bf16, const AttnArgs& a, cudaStream_t stream);
 
-// Steps (f)+(g) on the tcgen05 tensor cores (bf16 only). With a.kv_idx
-// null, a.K / a.V are the gathered selected rows (b, nkv, >= bsa, d) and
-// every K/V tile is a TMA box; otherwise the kernel gathers the rows itself
-// while loading them.
-// Returns cudaErrorNotSupported when the shape has no tensor-core variant.
+// Steps (f)+(g) on the tcgen05 tensor cores (bf16, d = 128; O contiguous).
+// With a.kv_idx null (or bsa = 0), a.K / a.V are the gathered selected rows
+// (b, nkv, >= bsa, d) and every K/V tile is a TMA box (attn_tma.cu);
+// otherwise launch_attn_tc_gather runs, which gathers the rows by index
+// while loading them (attn_tc.cu).
+// Return cudaErrorNotSupported when the shape has no tensor-core variant.
 cudaError_t launch_attn_tc(const AttnArgs& a, cudaStream_t stream);
+cudaError_t launch_attn_tc_gather(const AttnArgs& a, cudaStream_t stream);
 
 }  // namespace quoka

@@ -37,18 +37,4 @@ inline bool encode_bf16_4d(CUtensorMap* m, const void* base, uint64_t d, uint64_
              CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
-// 2-D bf16 row map (d, rows) with a box of 64 columns x 1 row, the form
-// TMA row gathers (tile::gather4) take. Row stride in elements.
-inline bool encode_bf16_rows(CUtensorMap* m, const void* base, uint64_t d, uint64_t rows, int64_t s_row) {
-  auto enc = tensor_map_encoder();
-  if (enc == nullptr) return false;
-  const cuuint64_t dims[2] = {d, rows};
-  const cuuint64_t strides[1] = {(cuuint64_t)s_row * 2};
-  const cuuint32_t box[2] = {64, 1};
-  const cuuint32_t estr[2] = {1, 1};
-  return enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, strides, box, estr,
-             CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
-             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
-}
-
 }  // namespace quoka
