@@ -102,6 +102,109 @@ __device__ __forceinline__ void issue_pv(uint32_t tmem_o, uint32_t tmem_p, uint3
                  (accumulate || kk > 0) ? 1u : 0u);
 }
 
+// 2^x for two values on the FMA pipe instead of the MUFU: x = n + f with n
+// the nearest integer (adding 1.5 * 2^23 rounds to it) and f in [-1/2, 1/2];
+// 2^f from a cubic fitted to it by least squares on Chebyshev nodes of
+// [-1/2, 1/2] (relative error below 8e-5, far under bf16 resolution); 2^n
+// added straight into the exponent field. x is clamped at -126, where the
+// result (about 1e-38) is as good as the MUFU's flushed zero for a softmax.
+__device__ __forceinline__ void exp2_fma_pair(uint64_t x, float& p0, float& p1) {
+  constexpr float kRound = 12582912.f;  // 1.5 * 2^23
+  float x0, x1;
+  f2_unpack(x, x0, x1);
+  const uint64_t xc = f2_pack(fmaxf(x0, -126.f), fmaxf(x1, -126.f));
+  const uint64_t j = f2_add(xc, f2_pack(kRound, kRound));          // n in the low mantissa bits
+  const uint64_t n = f2_add(j, f2_pack(-kRound, -kRound));
+  const uint64_t f = f2_fma(n, f2_pack(-1.f, -1.f), xc);          // x - n, exact
+  uint64_t q = f2_fma(f2_pack(0.055088683807510905f, 0.055088683807510905f), f,
+                      f2_pack(0.24260405145947916f, 0.24260405145947916f));
+  q = f2_fma(q, f, f2_pack(0.6932762416819607f, 0.6932762416819607f));
+  q = f2_fma(q, f, f2_pack(0.9999289403695112f, 0.9999289403695112f));
+  float q0, q1, j0, j1;
+  f2_unpack(q, q0, q1);
+  f2_unpack(j, j0, j1);
+  p0 = __uint_as_float(__float_as_uint(q0) + (__float_as_uint(j0) << 23));
+  p1 = __uint_as_float(__float_as_uint(q1) + (__float_as_uint(j1) << 23));
+}
+
+// One key tile of the online softmax of this thread's query row, single
+// pass: the row's 128 scores are read from TMEM once into registers. Key c
+// of the tile (key number base_n + c) is visible when base_n + c < lim. Then
+// the row max (3-input max tree), and P = 2^(s * qscale - m) in bf16 over
+// the first 64 S columns (packed two per column), with the products and row
+// sums in paired fp32 arithmetic; of every 8 key pairs, FMA_PAIRS take the
+// FMA-pipe exp2 and the rest the MUFU, so both units share the work. The
+// running max m moves only when it grows by more than RESCALE_THRESHOLD, in
+// which case the O accumulator (complete for the previous tiles) is
+// rescaled in TMEM. Updates m and l. TMEM accesses are warp-collective: no
+// per-row branch surrounds one.
+template <int FMA_PAIRS>
+__device__ __forceinline__ void softmax_tile_1p(uint32_t S, uint32_t O, bool have_o, int base_n, int lim,
+                                                float qscale, float& m, float& l) {
+  float v[128];
+  __syncwarp();
+  tmem_ld64(S, v);
+  tmem_ld64(S + 64, v + 64);
+  tmem_wait_ld();
+  if (base_n + N > lim) {
+#pragma unroll
+    for (int u = 0; u < 128; ++u) v[u] = (base_n + u < lim) ? v[u] : -INFINITY;
+  }
+  float a[8];
+#pragma unroll
+  for (int k = 0; k < 8; ++k) a[k] = fmaxf(v[k], v[k + 8]);
+#pragma unroll
+  for (int u = 16; u < 128; u += 16)
+#pragma unroll
+    for (int k = 0; k < 8; ++k) a[k] = fmax3(a[k], v[u + k], v[u + 8 + k]);
+  const float mx = fmax3(fmax3(a[0], a[1], a[2]), fmax3(a[3], a[4], a[5]), fmaxf(a[6], a[7])) * qscale;
+  const float m_cand = fmaxf(m, mx);
+  const float m_new = (m_cand > m + RESCALE_THRESHOLD || m == -INFINITY) ? m_cand : m;
+  const float corr = (m_new == m) ? 1.f : ex2(m - m_new);
+  const float m_use = m_new == -INFINITY ? 0.f : m_new;
+  const uint64_t qs2 = f2_pack(qscale, qscale), nm2 = f2_pack(-m_use, -m_use);
+  uint64_t acc[4] = {0, 0, 0, 0};  // paired row sums (+0.0f halves)
+#pragma unroll
+  for (int c = 0; c < 4; ++c) {
+    uint32_t pk[16];
+#pragma unroll
+    for (int u = 0; u < 32; u += 2) {
+      const int e = 32 * c + u;
+      const uint64_t x = f2_fma(f2_pack(v[e], v[e + 1]), qs2, nm2);
+      float p0, p1;
+      if (((e >> 1) & 7) < FMA_PAIRS) {
+        exp2_fma_pair(x, p0, p1);
+      } else {
+        float x0, x1;
+        f2_unpack(x, x0, x1);
+        p0 = ex2(x0);
+        p1 = ex2(x1);
+      }
+      acc[(u >> 1) & 3] = f2_add(acc[(u >> 1) & 3], f2_pack(p0, p1));
+      pk[u >> 1] = pack_bf16x2(p0, p1);
+    }
+    __syncwarp();
+    tmem_st16(S + 16 * c, pk);
+  }
+  float r[8];
+#pragma unroll
+  for (int k = 0; k < 4; ++k) f2_unpack(acc[k], r[2 * k], r[2 * k + 1]);
+  l = l * corr + (((r[0] + r[1]) + (r[2] + r[3])) + ((r[4] + r[5]) + (r[6] + r[7])));
+  m = m_new;
+  // warp-uniform condition: the rescale's TMEM traffic is collective
+  if (have_o && __any_sync(0xffffffffu, corr != 1.f)) {
+#pragma unroll 1
+    for (int c4 = 0; c4 < 4; ++c4) {
+      float o[32];
+      tmem_ld32(O + 32 * c4, o);
+      tmem_wait_ld();
+#pragma unroll
+      for (int u = 0; u < 32; ++u) o[u] *= corr;
+      tmem_st32(O + 32 * c4, o);
+    }
+  }
+}
+
 // One key tile of the online softmax of this thread's query row, on S in
 // TMEM (this warp's lanes): key c of the tile (key number base_n + c) is
 // visible when base_n + c < lim. Two passes over the row (max, then

@@ -56,6 +56,10 @@ constexpr int THREADS = 352;
 constexpr int MMA_WARP = 8;
 constexpr int KLOAD_WARP = 9;
 constexpr int VLOAD_WARP = 10;
+// Of every 8 key pairs, how many take the FMA-pipe exp2 in the softmax.
+// Measured on B200 (Qwen-shaped layer): 0 and 2 run equally fast, more is
+// slower; 0 keeps the kernel free of register spills.
+constexpr int SOFTMAX_FMA_PAIRS = 0;
 // split-KV payload: partial O (fp32, 2 tiles x 128 rows x 128, each row's
 // 16-byte chunks rotated by the row index) followed by (m, l) per row
 constexpr uint32_t XFER_O_BYTES = 2 * 128 * D * 4;
@@ -136,9 +140,11 @@ attn_tma_kernel(const __grid_constant__ Maps maps, const AttnArgs a, int nsplit)
   const int ntile_sel = (nsel + N - 1) / N;
   const int ntile_chk = (nchunk + N - 1) / N;
   const int nT = ntile_sel + ntile_chk;
-  const int per = (nT + nsplit - 1) / nsplit;
-  const int first = min(nT, split * per);
-  const int ntiles = min(nT, first + per) - first;  // key tiles of this CTA (may be 0)
+  // split: rank 0 takes one or two tiles more than rank 1, so that rank 1's
+  // payload transfer overlaps rank 0's last tiles
+  const int n0 = nsplit > 1 ? min(nT, (nT + 3) / 2) : nT;
+  const int first = split == 0 ? 0 : n0;
+  const int ntiles = split == 0 ? n0 : nT - n0;  // key tiles of this CTA (may be 0)
 
   if (tid == 0) {
     mbar_init(&sm.q_full, 1);
@@ -285,7 +291,7 @@ attn_tma_kernel(const __grid_constant__ Maps maps, const AttnArgs a, int nsplit)
       // key at a position p < nchunk with p <= t
       const int base_n = (sel_tile ? gi : gi - ntile_sel) * N;
       const int lim = sel_tile ? nsel : min(nchunk, t + 1);
-      softmax_tile(S, O, it > 0, base_n, lim, qscale, m, l);
+      softmax_tile_1p<SOFTMAX_FMA_PAIRS>(S, O, it > 0, base_n, lim, qscale, m, l);
       tmem_wait_st();
       tc_fence_before();
       mbar_arrive(&sm.p_full[w]);
@@ -296,8 +302,9 @@ attn_tma_kernel(const __grid_constant__ Maps maps, const AttnArgs a, int nsplit)
     if (alive) alive = warp_wait(&sm.o_final, 0, sm, a.status, 33);
     tc_fence_after();
     const int row = w * 128 + r;
-    float* pay_o = reinterpret_cast<float*>(sm.k[0]) + (size_t)row * D;
-    float* pay_ml = reinterpret_cast<float*>(sm.k[0] + XFER_O_BYTES) + (size_t)row * 2;
+    uint8_t* span = reinterpret_cast<uint8_t*>(&sm) + offsetof(Smem, k);  // K ring, then V ring
+    float* pay_o = reinterpret_cast<float*>(span) + (size_t)row * D;
+    float* pay_ml = reinterpret_cast<float*>(span + XFER_O_BYTES) + (size_t)row * 2;
     if (nsplit > 1 && split == 1) {
       // stage this row's (O, m, l) in the own K/V span (free: every MMA is
       // done), then one thread sends the whole payload to rank 0
