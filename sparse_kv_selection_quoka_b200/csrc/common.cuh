@@ -62,4 +62,19 @@ __device__ __forceinline__ uint32_t score_key(float f) {
   return (u & 0x80000000u) ? ~u : (u | 0x80000000u);
 }
 
+// 12-bit bucket of a score, linear over [-1, 1] (cosine-type scores lie
+// there): floor((s + 1) * 2048) clamped to [0, 4095]. Non-decreasing in the
+// score's key order (every step rounds monotonically; a NaN goes to the end
+// its key sorts to), so keys in a higher bucket are always larger.
+__device__ __forceinline__ uint32_t score_bin(float s) {
+  if (s != s) return (__float_as_uint(s) >> 31) ? 0u : 4095u;
+  const float x = fminf(fmaxf((s + 1.f) * 2048.f, 0.f), 4095.f);
+  return (uint32_t)x;
+}
+
+// The score an order-preserving key stands for (inverse of score_key).
+__device__ __forceinline__ float key_score(uint32_t k) {
+  return __uint_as_float((k & 0x80000000u) ? (k & 0x7FFFFFFFu) : ~k);
+}
+
 }  // namespace quoka

@@ -34,9 +34,9 @@ cudaError_t launch_score_simt(bool bf16, int d, Strided K, int b, int nkv, int64
                               const float* Qg, int NQ, float* S_agg, cudaStream_t stream);
 
 // Step (d) on the tcgen05 tensor cores (bf16 K, Q_group as bf16 hi + lo).
-// Also accumulates, per (batch, KV head), the histogram of the top 12 bits
-// of the order-preserving score keys into `hist` (zeroed beforehand), the
-// first digit of the top-k radix select.
+// Also accumulates, per (batch, KV head), the histogram of the scores'
+// 12-bit value buckets (score_bin) into `hist` (zeroed beforehand), the
+// first digit of the top-k select.
 // Returns cudaErrorNotSupported when the shape has no tensor-core variant.
 cudaError_t launch_score_tc(int d, Strided K, int b, int nkv, int64_t T,
                             const uint16_t* Qg_hilo, int NQ, float* S_agg, uint32_t* hist,
@@ -47,10 +47,10 @@ cudaError_t launch_score_tc(int d, Strided K, int b, int nkv, int64_t T,
 // Requires 1 <= bsa <= T and T <= topk_max_T().
 int64_t topk_max_T();
 // `hist`, when not null, is the (b * nkv, TOPK_HIST_BINS) histogram of the
-// top 12 key bits made by the scoring kernel; the first radix pass is then
+// scores' value buckets made by the scoring kernel; the first pass is then
 // skipped.
 cudaError_t launch_topk(const float* S_agg, int b, int nkv, int64_t T, int bsa,
-                        const uint32_t* hist, int32_t* kv_idx, int32_t* kv_count,
+                        const uint32_t* hist, int32_t* kv_idx, int32_t* kv_count, int* status,
                         cudaStream_t stream);
 
 // Step (f): gather of the selected K and V rows into contiguous

@@ -187,7 +187,8 @@ quoka_status run_select(const quoka_tensor* Q, const quoka_tensor* K, const Sele
     if (e != cudaSuccess) return cuda_status(e);
   }
   if (bsa_eff > 0) {
-    e = quoka::launch_topk(sagg, b, nkv, s.T, bsa_eff, hist_made ? hist : nullptr, kv_idx, kv_count, stream);
+    e = quoka::launch_topk(sagg, b, nkv, s.T, bsa_eff, hist_made ? hist : nullptr, kv_idx, kv_count, status,
+                           stream);
     if (e != cudaSuccess) return cuda_status(e);
   } else {
     e = cudaMemsetAsync(kv_count, 0, sizeof(int32_t) * b * nkv, stream);

@@ -58,7 +58,7 @@ struct ScoreBars {
 struct ScoreArgs {
   const uint16_t* qg_hilo;  // (b, nkv, 2*NQ, d) bf16: rows [0,NQ) hi, [NQ,2NQ) lo
   float* s_agg;             // (b, nkv, T)
-  uint32_t* hist;           // (b, nkv, TOPK_HIST_BINS): histogram of key >> 20
+  uint32_t* hist;           // (b, nkv, TOPK_HIST_BINS): histogram of score_bin(S_agg)
   int* status;
   int64_t T;
   int NQ, NQp, nstages, tiles_per_cta, ntiles;
@@ -229,10 +229,10 @@ score_tc_kernel(const __grid_constant__ CUtensorMap tmap, const ScoreArgs a) {
       const int64_t key = (int64_t)(t_begin + it) * SC_KEYS + r;
       const float score = mx / fmaxf(sqrtf(ss), 1e-12f);
       if (key < a.T) out[key] = score;
-      // first radix digit of the top-k: top 12 bits of the ordered key,
-      // counted once per distinct bin within the warp
+      // first digit of the top-k select: the score's 12-bit value bucket,
+      // counted once per distinct bucket within the warp
       const bool counted = key < a.T;
-      const uint32_t bin = score_key(score) >> 20;
+      const uint32_t bin = score_bin(score);
       const uint32_t act = __ballot_sync(0xffffffffu, counted);
       if (counted) {
         const uint32_t peers = __match_any_sync(act, bin);

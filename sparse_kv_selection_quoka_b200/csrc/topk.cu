@@ -6,21 +6,28 @@
 // write-up "QUOKA: how it reshapes LLM prefill efficiency", bqwf.cn news item
 // 915859.)
 //
-// One CTA per (batch, KV head) when the head's T scores fit in shared memory,
-// else one thread-block cluster of C CTAs, each owning a contiguous slice.
-// The scores are converted once into order-preserving 32-bit keys held in
-// shared memory, and an exact MSB-first radix select with 12-, 12- and 8-bit
-// digits finds the BSA-th largest key u*: the first digit's histogram comes
-// from the scoring kernel when it made one (else it is built here); per
-// later pass every CTA builds a histogram (warp-aggregated shared-memory
-// atomics) of the keys that still match the known prefix; in a cluster the histograms are summed through
-// distributed shared memory; a block scan finds the bin holding the BSA-th
-// largest key. A final pass keeps the keys > u* and the first (in index
-// order) keys == u* needed to reach BSA: each warp owns a contiguous segment
-// of its CTA's slice, counts its picks, one block scan (plus a cluster
-// exchange of CTA totals) gives every warp its output offset, and the warp
-// writes its picks in order with ballots. Nothing is written to global memory
-// but the result.
+// A thread-block cluster of C CTAs per (batch, KV head) (C = 1 for short
+// rows), each owning a contiguous slice of the row, staged in shared memory
+// as order-preserving 32-bit keys. The select finds the BSA-th largest key
+// u* most significant part first:
+//   1. The score's 12-bit value bucket (linear over [-1, 1], where the
+//      scores lie; the bit pattern's top bits would put nearly all of them
+//      in a few bins). Its histogram comes from the scoring kernel when it
+//      made one (else it is built here, summed over the cluster); a block
+//      scan finds the threshold bucket b0.
+//   2. One pass over the slice counts the keys above b0 and lists the keys
+//      in b0 (the candidates). After one cluster barrier every CTA reads all
+//      ranks' counts and candidate lists (small: a bucket is 1/2048 of the
+//      score range) and resolves u* among the candidates on its own (direct
+//      ranking, or radix passes over the gathered list), and from the same
+//      data its output offset: nothing else crosses between the CTAs.
+//   3. The final pass keeps the keys > u* and the first (in index order)
+//      keys == u* needed to reach BSA: each warp owns a contiguous segment of
+//      the slice, counts its picks, one block scan gives every warp its
+//      offset, and the warp writes its picks in order with ballots.
+// When a bucket holds more candidates than the gathered list can take, the
+// exact passes run over every slice instead, their histograms summed over
+// the cluster through distributed shared memory.
 #include <cooperative_groups.h>
 
 #include "common.cuh"
@@ -30,27 +37,33 @@ namespace cg = cooperative_groups;
 
 namespace quoka {
 
+namespace {
+
 constexpr int TOPK_THREADS = 1024;
 constexpr int TOPK_WARPS = TOPK_THREADS / 32;
 constexpr int TOPK_MAX_CLUSTER = 8;
-constexpr int TOPK_MAX_SLICE = 44 * 1024;       // keys per CTA (176 KiB of shared memory)
-constexpr int TOPK_SLICE_TARGET = 40 * 1024;    // one CTA per head up to this many keys
-constexpr int TOPK_BINS = 4096;                 // widest digit: 12 bits
-constexpr int TOPK_PASSES = 3;
-// Digits, most significant first: bits [31:20], [19:8], [7:0]. Scores lie in
-// [-1, 1], so the top 12 bits (sign, exponent, 3 mantissa bits) already
-// spread them over a few dozen bins.
-__constant__ int kTopkShift[TOPK_PASSES] = {20, 8, 0};
-__constant__ int kTopkBits[TOPK_PASSES] = {12, 12, 8};
-
-int64_t topk_max_T() { return (int64_t)TOPK_MAX_CLUSTER * TOPK_MAX_SLICE; }
+constexpr int TOPK_MAX_SLICE = 36 * 1024;  // keys per CTA (144 KiB of shared memory; 208 KiB in all)
+constexpr int TOPK_SLICE_TARGET = 4096;    // keys per CTA while the cluster can spread them
+constexpr int TOPK_LIST_MAX = 4096;        // candidates gathered in every CTA
+constexpr int TOPK_BINS = 4096;            // widest digit: 12 bits
+static_assert(TOPK_BINS / TOPK_THREADS <= 4, "bins per thread in a pick");
 
 struct TopkShared {
   uint32_t hist[2][TOPK_BINS];
   uint32_t wsum[TOPK_WARPS];
   uint32_t woff[TOPK_WARPS];
-  uint32_t counts[2];  // keys > u*, keys == u* in this CTA's slice
-  uint32_t bin, above, total;
+  uint32_t bin, above, total, bincount;
+  uint32_t kmin, kmax;       // smallest / largest candidate key (this CTA)
+  uint32_t gt0;              // keys of this slice above the threshold bucket
+  uint32_t ncand;            // candidates of this slice (keys in the bucket)
+  uint32_t rank_base[TOPK_MAX_CLUSTER + 1];  // gathered list: where each rank's part starts
+  uint32_t rc_gt[TOPK_MAX_CLUSTER];   // per rank: keys above the threshold bucket
+  uint32_t rc_n[TOPK_MAX_CLUSTER];    // per rank: candidates
+  uint32_t rc_gtc[TOPK_MAX_CLUSTER];  // per rank: candidates > u*
+  uint32_t rc_eqc[TOPK_MAX_CLUSTER];  // per rank: candidates == u*
+  uint32_t cgt[TOPK_THREADS], ceq[TOPK_THREADS];  // direct ranking: per candidate, #greater / #equal
+  uint8_t grank[TOPK_LIST_MAX];       // gathered list: the rank each candidate came from
+  uint32_t ustar, need_eq;   // the BSA-th largest key; how many keys == u* the row keeps
   uint32_t sel_base, take_eq;
 };
 
@@ -98,11 +111,21 @@ __device__ __forceinline__ void hist_add(uint32_t* H, uint32_t bin, bool active)
   if (lane == __ffs(peers) - 1) atomicAdd(&H[bin], (uint32_t)__popc(peers));
 }
 
+// Split cluster barrier: every thread of every CTA arrives, then waits;
+// work placed in between overlaps the barrier.
+__device__ __forceinline__ void cluster_arrive() {
+  asm volatile("barrier.cluster.arrive.release.aligned;" ::: "memory");
+}
+__device__ __forceinline__ void cluster_wait() { asm volatile("barrier.cluster.wait.acquire.aligned;" ::: "memory"); }
+
 template <bool CLUSTER>
 __global__ void __launch_bounds__(TOPK_THREADS)
 topk_kernel(const float* __restrict__ S, int64_t T, int bsa, int slice, const uint32_t* __restrict__ ghist,
             int32_t* __restrict__ kv_idx, int32_t* __restrict__ kv_count) {
-  extern __shared__ uint32_t keys[];
+  extern __shared__ uint32_t smem_dyn[];
+  uint32_t* keys = smem_dyn;          // [slice]: this CTA's keys
+  uint32_t* glist = smem_dyn + slice;  // [TOPK_LIST_MAX]: all ranks' candidates, in rank order
+  uint32_t* clist = glist + TOPK_LIST_MAX;  // [TOPK_LIST_MAX]: this slice's candidates
   __shared__ TopkShared sh;
   cg::cluster_group cluster = cg::this_cluster();
   const int C = CLUSTER ? (int)cluster.num_blocks() : 1;
@@ -116,6 +139,27 @@ topk_kernel(const float* __restrict__ S, int64_t T, int bsa, int slice, const ui
   const int n = (int)max((int64_t)0, min((int64_t)slice, T - lo));
   const int n_round = (n + TOPK_THREADS - 1) / TOPK_THREADS * TOPK_THREADS;
 
+  if (tid == 0) {
+    sh.kmin = 0xFFFFFFFFu;
+    sh.kmax = 0u;
+    sh.gt0 = 0u;
+    sh.ncand = 0u;
+  }
+  if (tid < TOPK_MAX_CLUSTER) {
+    sh.rc_gtc[tid] = 0u;
+    sh.rc_eqc[tid] = 0u;
+  }
+  sh.cgt[tid] = 0u;
+  sh.ceq[tid] = 0u;
+  // the scoring kernel's histogram bins this thread owns in the first pick
+  // (loaded first: the loads overlap the staging below)
+  uint32_t g0[4] = {0u, 0u, 0u, 0u};
+  if (ghist != nullptr) {
+    const uint32_t* Hg = ghist + row * TOPK_BINS;
+    constexpr int q0 = TOPK_BINS / TOPK_THREADS;
+#pragma unroll
+    for (int u = 0; u < q0; ++u) g0[u] = __ldg(Hg + TOPK_BINS - 1 - (tid * q0 + u));
+  }
   // stage the slice as keys (16-byte loads when the slice start is aligned)
   if ((((uintptr_t)(Sr + lo)) & 15u) == 0u) {
     const int n4 = n >> 2;
@@ -123,50 +167,28 @@ topk_kernel(const float* __restrict__ S, int64_t T, int bsa, int slice, const ui
 #pragma unroll 4
     for (int e = tid; e < n4; e += TOPK_THREADS) {
       const float4 v = __ldg(src4 + e);
-      keys[4 * e] = score_key(v.x);
-      keys[4 * e + 1] = score_key(v.y);
-      keys[4 * e + 2] = score_key(v.z);
-      keys[4 * e + 3] = score_key(v.w);
+      reinterpret_cast<uint4*>(keys)[e] = make_uint4(score_key(v.x), score_key(v.y), score_key(v.z), score_key(v.w));
     }
     for (int e = 4 * n4 + tid; e < n; e += TOPK_THREADS) keys[e] = score_key(Sr[lo + e]);
   } else {
     for (int e = tid; e < n; e += TOPK_THREADS) keys[e] = score_key(Sr[lo + e]);
   }
 
-  uint32_t prefix = 0u, pmask = 0u;
-  uint32_t need = (uint32_t)bsa;  // rank (1-based, from the top) still to place
-#pragma unroll 1
-  for (int p = 0; p < TOPK_PASSES; ++p) {
-    const int shift = kTopkShift[p];
-    const int nbins = 1 << kTopkBits[p];
-    const uint32_t dmask = (uint32_t)nbins - 1u;
-    uint32_t* H = sh.hist[p & 1];
-    // the first digit's histogram may come precomputed (whole head, global)
-    const bool from_global = p == 0 && ghist != nullptr;
-    if (!from_global) {
-      for (int i = tid; i < nbins; i += TOPK_THREADS) H[i] = 0u;
-      __syncthreads();
-      for (int e = tid; e < n_round; e += TOPK_THREADS) {
-        const uint32_t k = e < n ? keys[e] : 0u;
-        hist_add(H, (k >> shift) & dmask, e < n && (k & pmask) == prefix);
-      }
-      if (CLUSTER) cluster.sync();  // every CTA's histogram of this pass is complete
-      else __syncthreads();
-    }
-
-    // Thread t owns bins nbins-1-q*t .. nbins-q*(t+1) (largest keys first,
-    // q = nbins / TOPK_THREADS bins each), summed over the cluster; the
-    // inclusive scan gives the count of matching keys at or above each bin.
+  // From a histogram over `nbins` bins (this CTA's H, optionally summed over
+  // the cluster, or the preloaded global one), the bin holding the need-th
+  // largest of the counted keys, the count of counted keys in higher bins,
+  // and the bin's own count. Thread t owns bins nbins-1-q*t .. nbins-q*(t+1)
+  // (largest first, q = nbins / TOPK_THREADS bins each); an inclusive block
+  // scan gives the count at or above each bin.
+  auto pick_bin = [&](const uint32_t* H, int nbins, bool global, bool sum_cluster, uint32_t need_,
+                      uint32_t* bin_out, uint32_t* above_out) {
     const int q = nbins >= TOPK_THREADS ? nbins / TOPK_THREADS : 1;
     uint32_t mine[4] = {0u, 0u, 0u, 0u};
-    uint32_t tot = 0u;
-    if (tid * q < nbins && from_global) {
-      const uint32_t* Hg = ghist + row * TOPK_BINS;
+    if (global) {
 #pragma unroll
-      for (int u = 0; u < 4; ++u) mine[u] = u < q ? __ldg(Hg + nbins - 1 - (tid * q + u)) : 0u;
-      for (int u = 0; u < q; ++u) tot += mine[u];
+      for (int u = 0; u < 4; ++u) mine[u] = g0[u];
     } else if (tid * q < nbins) {
-      if (CLUSTER) {
+      if (CLUSTER && sum_cluster) {
         uint32_t got[TOPK_MAX_CLUSTER][4];
 #pragma unroll
         for (int r = 0; r < TOPK_MAX_CLUSTER; ++r) {
@@ -186,32 +208,305 @@ topk_kernel(const float* __restrict__ S, int64_t T, int bsa, int slice, const ui
 #pragma unroll
         for (int u = 0; u < 4; ++u) mine[u] = u < q ? H[nbins - 1 - (tid * q + u)] : 0u;
       }
-      for (int u = 0; u < q; ++u) tot += mine[u];
     }
+    const uint32_t tot = (mine[0] + mine[1]) + (mine[2] + mine[3]);
     uint32_t dummy;
     const uint32_t incl = block_scan_incl(tot, sh, &dummy);
-    if (tid * q < nbins && incl >= need && incl - tot < need) {
+    if (tid * q < nbins && incl >= need_ && incl - tot < need_) {
       uint32_t acc = incl - tot;
       for (int u = 0; u < q; ++u) {
-        if (acc + mine[u] >= need) {
+        if (acc + mine[u] >= need_) {
           sh.bin = (uint32_t)(nbins - 1 - (tid * q + u));
           sh.above = acc;
+          sh.bincount = mine[u];
           break;
         }
         acc += mine[u];
       }
     }
     __syncthreads();
-    need -= sh.above;
-    prefix |= sh.bin << shift;
-    pmask |= dmask << shift;
-    // This histogram buffer is next cleared two passes later, after another
-    // cluster-wide barrier, by which time every CTA has finished reading it.
-  }
-  const uint32_t ustar = prefix;
+    *bin_out = sh.bin;
+    *above_out = sh.above;
+  };
 
-  // Warp w owns the contiguous segment [w*seg, (w+1)*seg) of the slice and
-  // counts its keys > u* and == u* (lane-strided reads: no bank conflicts).
+  // Exact passes over candidate keys: 12-bit digits of the key from the
+  // highest bit where the smallest and largest candidate differ (the bits
+  // above it are common to all candidates). `full_scan`: walk the slice,
+  // testing the bucket (histograms summed over the cluster); else walk
+  // list[0 .. nlist) (this CTA alone). Returns u*; `need` becomes the
+  // number of keys == u* to keep.
+  uint32_t need = (uint32_t)bsa;  // rank (1-based, from the top) still to place
+  uint32_t b0 = 0u, above = 0u;
+  auto exact_passes = [&](uint32_t kmin, uint32_t kmax, bool full_scan, const uint32_t* list, int nlist) {
+    uint32_t prefix = kmin;  // all candidates equal: u* is their key
+    if (kmin == kmax) return prefix;
+    int hb = 31 - __clz(kmin ^ kmax);
+    uint32_t pmask = hb == 31 ? 0u : ~((2u << hb) - 1u);
+    prefix = kmax & pmask;
+    const int nlist_round = (nlist + TOPK_THREADS - 1) / TOPK_THREADS * TOPK_THREADS;
+#pragma unroll 1
+    for (int p = 1;; ++p) {
+      const int width = min(12, hb + 1), shift = hb + 1 - width;
+      const int nbins = 1 << width;
+      const uint32_t dmask = (uint32_t)nbins - 1u;
+      // this buffer was last read (remotely too) two passes ago, before a
+      // cluster-wide barrier every CTA has since passed
+      uint32_t* H = sh.hist[p & 1];
+      for (int i = tid; i < nbins; i += TOPK_THREADS) H[i] = 0u;
+      __syncthreads();
+      if (full_scan) {
+        for (int e = tid; e < n_round; e += TOPK_THREADS) {
+          const uint32_t k = e < n ? keys[e] : 0u;
+          const bool cand = e < n && (k & pmask) == prefix && score_bin(key_score(k)) == b0;
+          hist_add(H, (k >> shift) & dmask, cand);
+        }
+        if (CLUSTER) cluster.sync();
+        else __syncthreads();
+      } else {
+        for (int i = tid; i < nlist_round; i += TOPK_THREADS) {
+          const uint32_t k = i < nlist ? list[i] : 0u;
+          hist_add(H, (k >> shift) & dmask, i < nlist && (k & pmask) == prefix);
+        }
+        __syncthreads();
+      }
+      uint32_t bin;
+      pick_bin(H, nbins, false, full_scan, need, &bin, &above);
+      need -= above;
+      prefix |= bin << shift;
+      pmask |= dmask << shift;
+      if (shift == 0) break;
+      hb = shift - 1;
+    }
+    return prefix;
+  };
+
+  // 1. the value bucket b0 holding the BSA-th largest score
+  {
+    uint32_t* H = sh.hist[0];
+    if (ghist == nullptr) {
+      for (int i = tid; i < TOPK_BINS; i += TOPK_THREADS) H[i] = 0u;
+      __syncthreads();
+      for (int e = tid; e < n_round; e += TOPK_THREADS) {
+        const uint32_t k = e < n ? keys[e] : 0u;
+        hist_add(H, score_bin(key_score(k)), e < n);
+      }
+      if (CLUSTER) cluster.sync();  // every CTA's histogram is complete
+      else __syncthreads();
+    }
+    pick_bin(H, TOPK_BINS, ghist != nullptr, true, need, &b0, &above);
+    need -= above;
+  }
+  const uint32_t cnt0 = sh.bincount;  // keys of the whole row in bucket b0
+  const bool gathered = cnt0 <= (uint32_t)TOPK_LIST_MAX;  // the same in every CTA
+
+  uint32_t ustar;
+  if (gathered) {
+    // 2a. count this slice's keys above b0 and list its keys in b0
+    uint32_t gt = 0u;
+    for (int e0 = 0; e0 < n_round; e0 += TOPK_THREADS) {
+      const int e = e0 + tid;
+      const uint32_t k = e < n ? keys[e] : 0u;
+      const uint32_t bk = score_bin(key_score(k));
+      gt += (e < n && bk > b0) ? 1u : 0u;
+      const bool cand = e < n && bk == b0;
+      const uint32_t cb = __ballot_sync(0xffffffffu, cand);
+      if (cb != 0u) {
+        uint32_t base = 0u;
+        if (lane == 0) base = atomicAdd(&sh.ncand, (uint32_t)__popc(cb));
+        base = __shfl_sync(0xffffffffu, base, 0);
+        const uint32_t pos = base + (uint32_t)__popc(cb & ((1u << lane) - 1u));
+        if (cand) clist[pos] = k;  // pos < cnt0 <= TOPK_LIST_MAX
+      }
+    }
+    gt = __reduce_add_sync(0xffffffffu, gt);
+    if (lane == 0 && gt != 0u) atomicAdd(&sh.gt0, gt);
+    // 2b. every rank's counts and candidates, gathered in rank order
+    if (CLUSTER) {
+      cluster_arrive();
+      cluster_wait();
+    } else {
+      __syncthreads();
+    }
+    // warp 0: every rank's counts, and where its part of the gathered list
+    // starts (exclusive scan over the ranks)
+    if (warp == 0) {
+      uint32_t gtr = 0u, nr = 0u;
+      if (lane < C) {
+        const TopkShared* shr = CLUSTER ? cluster.map_shared_rank(&sh, lane) : &sh;
+        gtr = shr->gt0;
+        nr = shr->ncand;
+      }
+      uint32_t incl = nr;
+#pragma unroll
+      for (int o = 1; o < TOPK_MAX_CLUSTER; o <<= 1) {
+        const uint32_t v = __shfl_up_sync(0xffffffffu, incl, o);
+        if (lane >= o) incl += v;
+      }
+      if (lane < C) {
+        sh.rc_gt[lane] = gtr;
+        sh.rank_base[lane] = incl - nr;
+      }
+      if (lane == C - 1) sh.rank_base[C] = incl;
+    }
+    __syncthreads();
+    const int nl = (int)sh.rank_base[C];  // == cnt0
+    for (int g = tid; g < nl; g += TOPK_THREADS) {
+      int r = 0;
+      while (r + 1 < C && (uint32_t)g >= sh.rank_base[r + 1]) ++r;
+      const uint32_t* cl = CLUSTER ? cluster.map_shared_rank(clist, r) : clist;
+      glist[g] = cl[g - sh.rank_base[r]];
+      sh.grank[g] = (uint8_t)r;
+    }
+    // done reading the other CTAs' shared memory (their wait at the end
+    // keeps every CTA alive until all have read)
+    if (CLUSTER) cluster_arrive();
+    __syncthreads();
+    // 2c. u* among the gathered candidates, and how many candidates of each
+    // rank lie above it / equal it
+    if (nl <= TOPK_THREADS) {
+      // Direct ranking: candidate i counts the candidates greater than /
+      // equal to it (the comparisons split over the idle warps, partial
+      // counts summed in shared memory). u* is the key whose rank range
+      // [#greater, #greater + #equal) holds `need`; a candidate is above u*
+      // exactly when its whole range lies before `need`.
+      const int ncw = (nl + 31) / 32;      // warps of candidates
+      const int nsplit = TOPK_WARPS / ncw;  // comparison groups
+      const int grp = warp / ncw;
+      if (grp < nsplit) {
+        const int i = (warp % ncw) * 32 + lane;
+        const uint32_t k = i < nl ? glist[i] : 0u;
+        const int jlen = (nl + nsplit - 1) / nsplit;
+        const int j0 = grp * jlen, j1 = min(nl, j0 + jlen);
+        uint32_t ngt = 0u, neq = 0u;
+#pragma unroll 4
+        for (int jj = j0; jj < j1; ++jj) {
+          const uint32_t o = glist[jj];
+          ngt += o > k;
+          neq += o == k;
+        }
+        if (i < nl && (ngt | neq) != 0u) {
+          atomicAdd(&sh.cgt[i], ngt);
+          atomicAdd(&sh.ceq[i], neq);
+        }
+      }
+      __syncthreads();
+      if (tid < nl) {
+        const uint32_t ngt = sh.cgt[tid], neq = sh.ceq[tid];
+        const int r = sh.grank[tid];
+        if (ngt + neq < need) {
+          atomicAdd(&sh.rc_gtc[r], 1u);
+        } else if (ngt < need) {  // equal keys agree
+          sh.ustar = glist[tid];
+          sh.need_eq = need - ngt;
+          atomicAdd(&sh.rc_eqc[r], 1u);
+        }
+      }
+      __syncthreads();
+      ustar = sh.ustar;
+      need = sh.need_eq;
+    } else {
+      uint32_t lo_k = 0xFFFFFFFFu, hi_k = 0u;
+      for (int i = tid; i < nl; i += TOPK_THREADS) {
+        lo_k = min(lo_k, glist[i]);
+        hi_k = max(hi_k, glist[i]);
+      }
+      lo_k = __reduce_min_sync(0xffffffffu, lo_k);
+      hi_k = __reduce_max_sync(0xffffffffu, hi_k);
+      if (lane == 0) {
+        atomicMin(&sh.kmin, lo_k);
+        atomicMax(&sh.kmax, hi_k);
+      }
+      __syncthreads();
+      ustar = exact_passes(sh.kmin, sh.kmax, false, glist, nl);
+      for (int g = tid; g < nl; g += TOPK_THREADS) {
+        const uint32_t k = glist[g];
+        const int r = sh.grank[g];
+        if (k > ustar) atomicAdd(&sh.rc_gtc[r], 1u);
+        if (k == ustar) atomicAdd(&sh.rc_eqc[r], 1u);
+      }
+      __syncthreads();
+    }
+    // 2d. this CTA's output offset: per lower rank, its keys > u* and its
+    // share (in rank order) of the keys == u*
+    uint32_t* rc_gt = sh.rc_gt;
+    uint32_t* rc_gtc = sh.rc_gtc;
+    uint32_t* rc_eqc = sh.rc_eqc;
+    if (tid == 0) {
+      uint32_t sel_base = 0u, eq_seen = 0u, my_take = 0u;
+      for (int r = 0; r <= c; ++r) {
+        const uint32_t er = rc_eqc[r];
+        const uint32_t take = need > eq_seen ? min(er, need - eq_seen) : 0u;
+        if (r < c) sel_base += rc_gt[r] + rc_gtc[r] + take;
+        if (r == c) my_take = take;
+        eq_seen += er;
+      }
+      sh.sel_base = sel_base;
+      sh.take_eq = my_take;
+    }
+    __syncthreads();
+  }
+  else {
+    // Many candidates: their smallest / largest key over the cluster, then
+    // exact passes over every slice with cluster-summed histograms.
+    uint32_t kmin = 0xFFFFFFFFu, kmax = 0u;
+    for (int e = tid; e < n; e += TOPK_THREADS) {
+      const uint32_t k = keys[e];
+      if (score_bin(key_score(k)) == b0) {
+        kmin = min(kmin, k);
+        kmax = max(kmax, k);
+      }
+    }
+    kmin = __reduce_min_sync(0xffffffffu, kmin);
+    kmax = __reduce_max_sync(0xffffffffu, kmax);
+    if (lane == 0) {
+      atomicMin(&sh.kmin, kmin);
+      atomicMax(&sh.kmax, kmax);
+    }
+    if (CLUSTER) cluster.sync();
+    else __syncthreads();
+    kmin = 0xFFFFFFFFu;
+    kmax = 0u;
+    for (int r = 0; r < C; ++r) {
+      const TopkShared* shr = CLUSTER ? cluster.map_shared_rank(&sh, r) : &sh;
+      kmin = min(kmin, shr->kmin);
+      kmax = max(kmax, shr->kmax);
+    }
+    ustar = exact_passes(kmin, kmax, true, nullptr, 0);
+    // this slice's keys > u* and == u*, exchanged for the output offsets
+    uint32_t g = 0u, q_eq = 0u;
+    for (int e = tid; e < n; e += TOPK_THREADS) {
+      const uint32_t k = keys[e];
+      g += k > ustar;
+      q_eq += k == ustar;
+    }
+    g = __reduce_add_sync(0xffffffffu, g);
+    q_eq = __reduce_add_sync(0xffffffffu, q_eq);
+    if (lane == 0) {
+      atomicAdd(&sh.rc_gtc[c], g);
+      atomicAdd(&sh.rc_eqc[c], q_eq);
+    }
+    if (CLUSTER) cluster.sync();
+    else __syncthreads();
+    if (tid == 0) {
+      uint32_t sel_base = 0u, eq_seen = 0u, my_take = 0u;
+      for (int r = 0; r <= c; ++r) {
+        const TopkShared* shr = CLUSTER ? cluster.map_shared_rank(&sh, r) : &sh;
+        const uint32_t gr = shr->rc_gtc[r], er = shr->rc_eqc[r];
+        const uint32_t take = need > eq_seen ? min(er, need - eq_seen) : 0u;
+        if (r < c) sel_base += gr + take;
+        if (r == c) my_take = take;
+        eq_seen += er;
+      }
+      sh.sel_base = sel_base;
+      sh.take_eq = my_take;
+    }
+    __syncthreads();
+  }
+
+  // 3. Warp w owns the contiguous segment [w*seg, (w+1)*seg) of the slice:
+  // it counts its keys > u* and == u* (lane-strided reads: no bank
+  // conflicts), one block scan places the warps, and each writes its picks
+  // in index order.
   const int seg = (n + TOPK_WARPS - 1) / TOPK_WARPS;
   const int s0 = min(n, warp * seg), s1 = min(n, s0 + seg);
   uint32_t g = 0u, q_eq = 0u;
@@ -222,34 +517,13 @@ topk_kernel(const float* __restrict__ S, int64_t T, int bsa, int slice, const ui
   }
   // both counts in one scan: (gt << 16) | eq (per-CTA counts < 65536)
   uint32_t packed = (g << 16) | q_eq;
-#pragma unroll
-  for (int o = 16; o > 0; o >>= 1) packed += __shfl_xor_sync(0xffffffffu, packed, o);
+  packed = __reduce_add_sync(0xffffffffu, packed);
   uint32_t cta_total;
   const uint32_t wincl = block_scan_incl(lane == 0 ? packed : 0u, sh, &cta_total);
   const uint32_t wex = wincl - (lane == 0 ? packed : 0u);  // valid in lane 0
   const uint32_t w_gt_before = __shfl_sync(0xffffffffu, wex >> 16, 0);
   const uint32_t w_eq_before = __shfl_sync(0xffffffffu, wex & 0xFFFFu, 0);
   const uint32_t w_eq = packed & 0xFFFFu;  // warp sums are replicated in every lane
-  if (tid == 0) {
-    sh.counts[0] = cta_total >> 16;
-    sh.counts[1] = cta_total & 0xFFFFu;
-  }
-  if (CLUSTER) cluster.sync();
-  else __syncthreads();
-  if (tid == 0) {
-    uint32_t sel_base = 0u, eq_seen = 0u, my_take = 0u;
-    for (int r = 0; r < C; ++r) {
-      const uint32_t* cr = CLUSTER ? cluster.map_shared_rank(sh.counts, r) : sh.counts;
-      const uint32_t gr = cr[0], er = cr[1];
-      const uint32_t take = need > eq_seen ? min(er, need - eq_seen) : 0u;
-      if (r < c) sel_base += gr + take;
-      if (r == c) my_take = take;
-      eq_seen += er;
-    }
-    sh.sel_base = sel_base;
-    sh.take_eq = my_take;
-  }
-  __syncthreads();
   // this warp's share of the tied keys, and its first output position
   const uint32_t take_cta = sh.take_eq;
   const uint32_t w_take = take_cta > w_eq_before ? min(w_eq, take_cta - w_eq_before) : 0u;
@@ -273,28 +547,35 @@ topk_kernel(const float* __restrict__ S, int64_t T, int bsa, int slice, const ui
     eq_used += (uint32_t)__popc(eqb);
   }
   if (c == 0 && tid == 0) kv_count[row] = bsa;
-  if (CLUSTER) cluster.sync();  // keep this CTA's shared memory alive for remote readers
+  // every CTA stays until the others are done reading its shared memory
+  if (CLUSTER) {
+    if (gathered) cluster_wait();
+    else cluster.sync();
+  }
 }
 
+}  // namespace
+
+int64_t topk_max_T() { return (int64_t)TOPK_MAX_CLUSTER * TOPK_MAX_SLICE; }
+
 cudaError_t launch_topk(const float* S_agg, int b, int nkv, int64_t T, int bsa, const uint32_t* hist,
-                        int32_t* kv_idx, int32_t* kv_count, cudaStream_t stream) {
+                        int32_t* kv_idx, int32_t* kv_count, int* status, cudaStream_t stream) {
+  (void)status;  // every wait in the kernel is a hardware barrier phase that all threads reach
   if (bsa <= 0 || T <= 0 || bsa > T || T > topk_max_T()) return cudaErrorInvalidValue;
   int C = (int)((T + TOPK_SLICE_TARGET - 1) / TOPK_SLICE_TARGET);
   if (C > TOPK_MAX_CLUSTER) C = TOPK_MAX_CLUSTER;
   if (C < 1) C = 1;
   const int slice = (int)((T + C - 1) / C);
   if (slice > TOPK_MAX_SLICE) return cudaErrorInvalidValue;
-  const size_t smem = (size_t)slice * sizeof(uint32_t);
+  const size_t smem = ((size_t)slice + 2 * TOPK_LIST_MAX) * sizeof(uint32_t);
   if (C == 1) {
-    cudaError_t e = cudaFuncSetAttribute(topk_kernel<false>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                         (int)(smem < 1024 ? 1024 : smem));
+    cudaError_t e = cudaFuncSetAttribute(topk_kernel<false>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return e;
     topk_kernel<false><<<dim3(1, nkv, b), TOPK_THREADS, smem, stream>>>(S_agg, T, bsa, slice, hist, kv_idx,
                                                                         kv_count);
     return cudaGetLastError();
   }
-  cudaError_t e = cudaFuncSetAttribute(topk_kernel<true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                       (int)(smem < 1024 ? 1024 : smem));
+  cudaError_t e = cudaFuncSetAttribute(topk_kernel<true>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (e != cudaSuccess) return e;
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(C, nkv, b);
