@@ -16,15 +16,22 @@
 //
 // Work split: each CTA owns a contiguous range of 128-key tiles of one
 // (batch, KV head); the grid has about one CTA per SM.
-// Warp roles (192 threads):
+// Warp roles (448 threads):
 //   warp 0      TMA producer: 4-D tensor map over the (possibly strided) K
 //               view, two 64-column boxes per tile in the 128-byte swizzle,
-//               into a ring of up to 6 stages (no multicast);
+//               into a ring of up to 6 stages (no multicast); it starts
+//               before the query groups are staged;
 //   warp 1      TMEM allocation and single-thread MMA issue,
-//               M=128 keys x N=2*NQp x K=128, into a double-buffered
-//               accumulator;
-//   warps 2-5   epilogue: thread = key (TMEM lane): max over the NQ
-//               columns, |k| from shared memory, S_agg store.
+//               M=128 keys x N=2*NQp x K=128, into accumulator tile % 3;
+//   warps 2-13  epilogue, three warpgroups taking the tiles round-robin,
+//               each with its own TMEM accumulator (one warpgroup alone is
+//               latency-bound well below the HBM rate): thread = key (TMEM
+//               lane): max over the NQ columns, |k| from shared memory,
+//               S_agg store, histogram of the value buckets. A stage is
+//               released once its warpgroup has read |k| from it.
+// Measured on B200 (Qwen-shaped layer): computing |k|^2 on the tensor core
+// instead (the diagonal of a K K^T product) costs more MMA time per tile
+// than it saves.
 // Every wait is bounded (see sm100.cuh); a wait that gives up records
 // QUOKA_ERR_TIMEOUT and the CTA unwinds.
 #include "common.cuh"
@@ -40,7 +47,8 @@ namespace {
 
 constexpr int SC_D = 128;
 constexpr int SC_KEYS = 128;
-constexpr int SC_THREADS = 192;
+constexpr int SC_EPI = 3;                        // epilogue warpgroups (tiles round-robin)
+constexpr int SC_THREADS = 64 + 128 * SC_EPI;
 constexpr int SC_MAX_STAGES = 6;
 constexpr int SC_TILE_BYTES = SC_KEYS * SC_D * 2;  // 32 KiB
 constexpr int SC_ATOM = SC_KEYS * 128;             // one 64-column atom of a K tile
@@ -48,8 +56,8 @@ constexpr int SC_ATOM = SC_KEYS * 128;             // one 64-column atom of a K 
 struct ScoreBars {
   uint64_t full[SC_MAX_STAGES];
   uint64_t empty[SC_MAX_STAGES];
-  uint64_t tfull[2];
-  uint64_t tempty[2];
+  uint64_t tfull[SC_EPI];   // accumulator g holds a finished tile (g = tile % SC_EPI)
+  uint64_t tempty[SC_EPI];  // epilogue warpgroup g has read accumulator g
   uint64_t done;
   uint32_t tmem_base;
   int abort;
@@ -62,6 +70,7 @@ struct ScoreArgs {
   int* status;
   int64_t T;
   int NQ, NQp, nstages, tiles_per_cta, ntiles;
+  int nepi;                 // epilogue warpgroups in use (TMEM holds one accumulator each)
   uint32_t tmem_cols;
 };
 
@@ -84,6 +93,7 @@ score_tc_kernel(const __grid_constant__ CUtensorMap tmap, const ScoreArgs a) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t* base = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   const int N = 2 * a.NQp;                         // MMA N: hi rows then lo rows
+  const int ACC = N;                               // columns of one accumulator
   uint8_t* qg_s = base;                            // [2 atoms][N rows][128 B]
   const int qg_bytes = ((N * 256) + 1023) & ~1023;
   uint32_t* hist_s = reinterpret_cast<uint32_t*>(base + qg_bytes);  // [TOPK_HIST_BINS]
@@ -100,9 +110,9 @@ score_tc_kernel(const __grid_constant__ CUtensorMap tmap, const ScoreArgs a) {
   if (tid == 0) {
     for (int s = 0; s < NS; ++s) {
       mbar_init(&sb.full[s], 1);
-      mbar_init(&sb.empty[s], 128);
+      mbar_init(&sb.empty[s], 128);  // released by the epilogue warpgroup that read |k|
     }
-    for (int q = 0; q < 2; ++q) {
+    for (int q = 0; q < SC_EPI; ++q) {
       mbar_init(&sb.tfull[q], 1);
       mbar_init(&sb.tempty[q], 128);
     }
@@ -115,28 +125,14 @@ score_tc_kernel(const __grid_constant__ CUtensorMap tmap, const ScoreArgs a) {
     tmem_alloc(&sb.tmem_base, a.tmem_cols);
     tmem_relinquish();
   }
-  for (int e = tid; e < TOPK_HIST_BINS; e += SC_THREADS) hist_s[e] = 0u;
-  // B operand: the group means (hi rows then lo rows, each padded to NQp
-  // with zero rows) in the K-major 128-byte-swizzled layout.
-  {
-    const uint16_t* src = a.qg_hilo + row * 2 * a.NQ * SC_D;
-    for (int e = tid; e < N * 16; e += SC_THREADS) {
-      const int r = e >> 4, c = e & 15;
-      const int half = r >= a.NQp;  // 0 = hi, 1 = lo
-      const int i = r - half * a.NQp;
-      uint4 v = make_uint4(0u, 0u, 0u, 0u);
-      if (i < a.NQ) v = *reinterpret_cast<const uint4*>(src + ((int64_t)(half * a.NQ + i)) * SC_D + c * 8);
-      *reinterpret_cast<uint4*>(qg_s + sw128_offset(r, c, N)) = v;
-    }
-    fence_proxy_async_smem();
-  }
   tc_fence_before();
-  __syncthreads();
+  __syncthreads();  // barriers initialised, TMEM allocated
   tc_fence_after();
   const uint32_t tmem = sb.tmem_base;
 
   if (warp == 0) {
     // ------------------------------------------------------------ TMA producer
+    // (starts at once: the K stream does not depend on the query groups)
     if (lane == 0) {
       for (int it = 0; it < n; ++it) {
         const int s = it % NS;
@@ -152,6 +148,32 @@ score_tc_kernel(const __grid_constant__ CUtensorMap tmap, const ScoreArgs a) {
       }
     }
     __syncwarp();
+  }
+  const int nstage_threads = SC_THREADS - 32;  // everyone but the producer
+  const int st = tid - 32;
+  if (warp != 0) {
+  for (int e = st; e < TOPK_HIST_BINS; e += nstage_threads) hist_s[e] = 0u;
+  // B operand: the group means (hi rows then lo rows, each padded to NQp
+  // with zero rows) in the K-major 128-byte-swizzled layout.
+  {
+    const uint16_t* src = a.qg_hilo + row * 2 * a.NQ * SC_D;
+    for (int e = st; e < N * 16; e += nstage_threads) {
+      const int r = e >> 4, c = e & 15;
+      const int half = r >= a.NQp;  // 0 = hi, 1 = lo
+      const int i = r - half * a.NQp;
+      uint4 v = make_uint4(0u, 0u, 0u, 0u);
+      if (i < a.NQ) v = *reinterpret_cast<const uint4*>(src + ((int64_t)(half * a.NQ + i)) * SC_D + c * 8);
+      *reinterpret_cast<uint4*>(qg_s + sw128_offset(r, c, N)) = v;
+    }
+    fence_proxy_async_smem();
+  }
+  // the query groups and the zeroed histogram are in place (the producer
+  // does not take part)
+  named_barrier_sync(1, nstage_threads);
+  }
+
+  if (warp == 0) {
+    // (the producer ran above)
   } else if (warp == 1) {
     // ------------------------------------------------------------ MMA issue
     if (lane == 0) {
@@ -159,22 +181,24 @@ score_tc_kernel(const __grid_constant__ CUtensorMap tmap, const ScoreArgs a) {
       const uint32_t qg = smem_u32(qg_s);
       bool alive = true;
       int where = 0;
+      const int NE = a.nepi;
       for (int it = 0; it < n && alive; ++it) {
-        const int s = it % NS, acc = it & 1;
+        const int s = it % NS, acc = it % NE;
         where = 52;
         alive = mbar_wait(&sb.full[s], (it / NS) & 1, &sb.abort);
-        if (alive && it >= 2) {
+        if (alive && it >= NE) {
           where = 53;
-          alive = mbar_wait(&sb.tempty[acc], ((it >> 1) - 1) & 1, &sb.abort);
+          alive = mbar_wait(&sb.tempty[acc], ((it / NE) - 1) & 1, &sb.abort);
         }
         if (!alive) break;
         tc_fence_after();
         const uint32_t ks = smem_u32(ring + (size_t)s * SC_TILE_BYTES);
+        const uint32_t d = tmem + (uint32_t)(acc * ACC);
 #pragma unroll
         for (int kk = 0; kk < SC_D / 16; ++kk) {
           const uint64_t ad = sw128_desc(ks + (kk >> 2) * SC_ATOM + (kk & 3) * 32, 16, 1024);
           const uint64_t bd = sw128_desc(qg + (kk >> 2) * (N * 128) + (kk & 3) * 32, 16, 1024);
-          umma_bf16_ss(tmem + (uint32_t)(acc * N), ad, bd, idesc, kk > 0 ? 1u : 0u);
+          umma_bf16_ss(d, ad, bd, idesc, kk > 0 ? 1u : 0u);
         }
         umma_commit(&sb.tfull[acc]);
       }
@@ -185,16 +209,18 @@ score_tc_kernel(const __grid_constant__ CUtensorMap tmap, const ScoreArgs a) {
     __syncwarp();
   } else {
     // ------------------------------------------------------------ epilogue
+    const int g = (warp - 2) >> 2;           // epilogue warpgroup: tiles g, g + SC_EPI, ...
     const int q = warp & 3;                  // TMEM lane quarter of this warp
     const int r = q * 32 + lane;             // key within the tile
     const uint32_t lane_off = (uint32_t)(q * 32) << 16;
     float* out = a.s_agg + row * a.T;
-    for (int it = 0; it < n; ++it) {
-      const int s = it % NS, acc = it & 1;
-      if (!sc_warp_wait(&sb.tfull[acc], (it >> 1) & 1, sb, a.status, 55)) break;
+    const int NE = a.nepi;  // warpgroups g >= NE stay idle
+    for (int it = g; it < n && g < NE; it += NE) {
+      const int s = it % NS, acc = g;
+      if (!sc_warp_wait(&sb.tfull[acc], (it / NE) & 1, sb, a.status, 55)) break;
       tc_fence_after();
       float mx4[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
-      const uint32_t tbase = tmem + lane_off + (uint32_t)(acc * N);
+      const uint32_t tbase = tmem + lane_off + (uint32_t)(acc * ACC);
       for (int c0 = 0; c0 < a.NQp; c0 += 16) {
         float hi[16], lo[16];
         tmem_ld16(tbase + c0, hi);
@@ -282,8 +308,10 @@ cudaError_t launch_score_tc(int d, Strided K, int b, int nkv, int64_t T, const u
   a.NQ = NQ;
   a.NQp = (NQ + 15) / 16 * 16;  // the epilogue reads 16-column groups
   const int N = 2 * a.NQp;
+  const int acc_cols = N;
+  a.nepi = 512 / acc_cols < SC_EPI ? 512 / acc_cols : SC_EPI;  // N <= 256: at least 1
   uint32_t cols = 32;
-  while (cols < (uint32_t)(2 * N)) cols <<= 1;
+  while (cols < (uint32_t)(a.nepi * acc_cols)) cols <<= 1;
   a.tmem_cols = cols;
   const int qg_bytes = ((N * 256) + 1023) & ~1023;
   const int smem_cap = 227 * 1024;
