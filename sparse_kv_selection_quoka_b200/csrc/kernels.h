@@ -29,6 +29,13 @@ constexpr int TOPK_HIST_BINS = 4096;
 cudaError_t launch_qgroup(int d, const float* Qhat, int b, int nq, int nkv, int NQ,
                           float* Qg, uint16_t* Qg_hilo, uint32_t* hist, cudaStream_t stream);
 
+// Steps (a)-(c) fused (query selection and group mean in one kernel) for
+// bf16, d = 128, BCP <= 512, NQ <= 32, G <= 8: writes q_idx (rank order,
+// when not null), Qg and Qg_hilo as launch_qgroup does, and zeroes `hist`
+// when given. Returns cudaErrorNotSupported for other shapes.
+cudaError_t launch_qsel_group_fast(Strided Q, int b, int nq, int nkv, int BCP, int NQ, int32_t* q_idx,
+                                   float* Qg, uint16_t* Qg_hilo, uint32_t* hist, cudaStream_t stream);
+
 // Step (d) on the CUDA cores (fp32 arithmetic; any input dtype).
 cudaError_t launch_score_simt(bool bf16, int d, Strided K, int b, int nkv, int64_t T,
                               const float* Qg, int NQ, float* S_agg, cudaStream_t stream);

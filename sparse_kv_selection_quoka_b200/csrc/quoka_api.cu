@@ -171,9 +171,14 @@ quoka_status run_select(const quoka_tensor* Q, const quoka_tensor* K, const Sele
   int* status = at<int>(ws, L.status);
   uint32_t* hist = at<uint32_t>(ws, L.hist);
 
-  cudaError_t e = quoka::launch_qsel(bf, d, strided(Q), b, nq, BCP, NQ, qhat, qidx, stream);
-  if (e != cudaSuccess) return cuda_status(e);
-  e = quoka::launch_qgroup(d, qhat, b, nq, nkv, NQ, qg, bf ? qhilo : nullptr, bf ? hist : nullptr, stream);
+  cudaError_t e = cudaErrorNotSupported;
+  if (bf && d == 128)
+    e = quoka::launch_qsel_group_fast(strided(Q), b, nq, nkv, BCP, NQ, qidx, qg, qhilo, hist, stream);
+  if (e == cudaErrorNotSupported) {
+    e = quoka::launch_qsel(bf, d, strided(Q), b, nq, BCP, NQ, qhat, qidx, stream);
+    if (e != cudaSuccess) return cuda_status(e);
+    e = quoka::launch_qgroup(d, qhat, b, nq, nkv, NQ, qg, bf ? qhilo : nullptr, bf ? hist : nullptr, stream);
+  }
   if (e != cudaSuccess) return cuda_status(e);
   bool hist_made = false;
   if (s.T > 0) {
