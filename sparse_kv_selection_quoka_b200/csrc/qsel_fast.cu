@@ -45,11 +45,12 @@ constexpr int QF_MAX_BCP = 512;
 constexpr int QF_MAX_NQ = 32;
 constexpr int QF_MAX_G = 8;
 constexpr int QF_CHUNKS = QF_D / 8;  // 16-byte chunks per bf16 row
+static_assert(QF_MAX_NQ * (QF_D / 4) % QF_THREADS == 0, "group-mean units per thread");
 
 struct __align__(16) QfShared {
   alignas(16) float qhat[QF_MAX_NQ][QF_D];  // the normalised winners, rank order (read as float4)
   alignas(16) float colpart[QF_WARPS][QF_D];  // per-warp column sums
-  float mq[QF_D];
+  alignas(16) float mq[QF_D];
   float nrm[QF_MAX_BCP];             // |Q[t]| (clamped)
   uint64_t lists[QF_WARPS][32];       // sorted (key, position) lists of the merge tree
   float mq_norm;
@@ -173,11 +174,14 @@ qsel_fast_kernel(const bf16* __restrict__ Q, int64_t sQb, int64_t sQh, int64_t s
       for (int c = 0; c < QF_CHUNKS; ++c) {
         const uint4 raw = row[c ^ (t & 15)];
         const __nv_bfloat162* h2 = reinterpret_cast<const __nv_bfloat162*>(&raw);
+        const float4 ma = reinterpret_cast<const float4*>(sh.mq)[2 * c];
+        const float4 mb = reinterpret_cast<const float4*>(sh.mq)[2 * c + 1];
+        const float mv[8] = {ma.x, ma.y, ma.z, ma.w, mb.x, mb.y, mb.z, mb.w};
 #pragma unroll
         for (int u = 0; u < 4; ++u) {
           const float2 f = __bfloat1622float2(h2[u]);
-          dot4[u] = fmaf(f.x, sh.mq[c * 8 + 2 * u], dot4[u]);
-          dot4[u] = fmaf(f.y, sh.mq[c * 8 + 2 * u + 1], dot4[u]);
+          dot4[u] = fmaf(f.x, mv[2 * u], dot4[u]);
+          dot4[u] = fmaf(f.y, mv[2 * u + 1], dot4[u]);
           qq4[u] = fmaf(f.x, f.x, qq4[u]);
           qq4[u] = fmaf(f.y, f.y, qq4[u]);
         }
@@ -193,14 +197,24 @@ qsel_fast_kernel(const bf16* __restrict__ Q, int64_t sQb, int64_t sQh, int64_t s
   key = warp_sort_desc(key, lane);
   sh.lists[warp][lane] = key;
   __syncthreads();
+  // warps 0-3 fold lists 4w+1 .. 4w+3 into list 4w; then warp 0 folds the
+  // four results into list 0
+  if (warp < 4) {
+    uint64_t m = sh.lists[4 * warp][lane];
 #pragma unroll 1
-  for (int width = QF_WARPS / 2; width >= 1; width >>= 1) {
-    uint64_t merged = 0u;
-    if (warp < width) merged = warp_merge_top(sh.lists[2 * warp][lane], sh.lists[2 * warp + 1], lane);
-    __syncthreads();
-    if (warp < width) sh.lists[warp][lane] = merged;
-    __syncthreads();
+    for (int u = 1; u < 4; ++u) m = warp_merge_top(m, sh.lists[4 * warp + u], lane);
+    __syncwarp();
+    sh.lists[4 * warp][lane] = m;
   }
+  __syncthreads();
+  if (warp == 0) {
+    uint64_t m = sh.lists[0][lane];
+#pragma unroll 1
+    for (int u = 1; u < 4; ++u) m = warp_merge_top(m, sh.lists[4 * u], lane);
+    __syncwarp();
+    sh.lists[0][lane] = m;
+  }
+  __syncthreads();
   // 5. normalise the winners (thread = rank i, chunk cc), rank order
   {
     const int i = tid >> 4, cc = tid & 15;
@@ -223,29 +237,44 @@ qsel_fast_kernel(const bf16* __restrict__ Q, int64_t sQb, int64_t sQh, int64_t s
   cl_wait();
   const int64_t row = (int64_t)bi * nkv + j;
   const int units = ((NQ - g + G - 1) / G) * (QF_D / 4);  // float4 units of this CTA's ranks
-  for (int e = tid; e < units; e += QF_THREADS) {
-    const int i = g + G * (e / (QF_D / 4)), c4 = e % (QF_D / 4);
-    float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
-    for (int hh = 0; hh < G; ++hh) {
-      const QfShared* rs = cluster.map_shared_rank(&sh, hh);
-      const float4 v = reinterpret_cast<const float4*>(rs->qhat[i])[c4];
-      acc.x += v.x;
-      acc.y += v.y;
-      acc.z += v.z;
-      acc.w += v.w;
+  constexpr int UPT = QF_MAX_NQ * (QF_D / 4) / QF_THREADS;  // units per thread at most (2)
+  float4 acc[UPT];
+#pragma unroll
+  for (int u = 0; u < UPT; ++u) {
+    const int e = tid + u * QF_THREADS;
+    acc[u] = make_float4(0.f, 0.f, 0.f, 0.f);
+    if (e < units) {
+      const int i = g + G * (e / (QF_D / 4)), c4 = e % (QF_D / 4);
+      for (int hh = 0; hh < G; ++hh) {
+        const QfShared* rs = cluster.map_shared_rank(&sh, hh);
+        const float4 v = reinterpret_cast<const float4*>(rs->qhat[i])[c4];
+        acc[u].x += v.x;
+        acc[u].y += v.y;
+        acc[u].z += v.z;
+        acc[u].w += v.w;
+      }
     }
+  }
+  // done reading the other CTAs' winners; the wait at the end keeps every
+  // CTA alive until all have read
+  cl_arrive();
+#pragma unroll
+  for (int u = 0; u < UPT; ++u) {
+    const int e = tid + u * QF_THREADS;
+    if (e >= units) continue;
+    const int i = g + G * (e / (QF_D / 4)), c4 = e % (QF_D / 4);
     const float inv = 1.f / (float)G;
-    const float o[4] = {acc.x * inv, acc.y * inv, acc.z * inv, acc.w * inv};
+    const float o[4] = {acc[u].x * inv, acc[u].y * inv, acc[u].z * inv, acc[u].w * inv};
     reinterpret_cast<float4*>(Qg + (row * NQ + i) * QF_D)[c4] = make_float4(o[0], o[1], o[2], o[3]);
     if (Qg_hilo != nullptr) {
       uint32_t hw[2], lw[2];
 #pragma unroll
-      for (int u = 0; u < 2; ++u) {
-        const bf16 h0 = __float2bfloat16_rn(o[2 * u]), h1 = __float2bfloat16_rn(o[2 * u + 1]);
-        const bf16 l0 = __float2bfloat16_rn(o[2 * u] - __bfloat162float(h0));
-        const bf16 l1 = __float2bfloat16_rn(o[2 * u + 1] - __bfloat162float(h1));
-        hw[u] = (uint32_t)__bfloat16_as_ushort(h0) | ((uint32_t)__bfloat16_as_ushort(h1) << 16);
-        lw[u] = (uint32_t)__bfloat16_as_ushort(l0) | ((uint32_t)__bfloat16_as_ushort(l1) << 16);
+      for (int v2 = 0; v2 < 2; ++v2) {
+        const bf16 h0 = __float2bfloat16_rn(o[2 * v2]), h1 = __float2bfloat16_rn(o[2 * v2 + 1]);
+        const bf16 l0 = __float2bfloat16_rn(o[2 * v2] - __bfloat162float(h0));
+        const bf16 l1 = __float2bfloat16_rn(o[2 * v2 + 1] - __bfloat162float(h1));
+        hw[v2] = (uint32_t)__bfloat16_as_ushort(h0) | ((uint32_t)__bfloat16_as_ushort(h1) << 16);
+        lw[v2] = (uint32_t)__bfloat16_as_ushort(l0) | ((uint32_t)__bfloat16_as_ushort(l1) << 16);
       }
       // 8-byte stores: element offsets are multiples of 4
       *reinterpret_cast<uint2*>(Qg_hilo + (row * 2 * NQ + i) * QF_D + 4 * c4) = make_uint2(hw[0], hw[1]);
@@ -254,10 +283,8 @@ qsel_fast_kernel(const bf16* __restrict__ Q, int64_t sQb, int64_t sQh, int64_t s
   }
   if (hist != nullptr) {
     uint32_t* hr = hist + row * TOPK_HIST_BINS;
-    for (int e = g * QF_THREADS + tid; e < TOPK_HIST_BINS; e += G * QF_THREADS) hr[e] = 0u;
+    for (int z = g * QF_THREADS + tid; z < TOPK_HIST_BINS; z += G * QF_THREADS) hr[z] = 0u;
   }
-  // every CTA stays until the others have read its winners
-  cl_arrive();
   cl_wait();
 }
 
