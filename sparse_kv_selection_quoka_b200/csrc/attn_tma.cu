@@ -127,6 +127,7 @@ attn_tma_kernel(const __grid_constant__ Maps maps, const AttnArgs a, int nsplit)
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int j = blockIdx.y, bi = blockIdx.z;
+  pdl_wait();  // the gathered rows and their counts come from the previous kernel
   const int G = a.nq / a.nkv;
   const int split = nsplit > 1 ? (int)cluster_ctarank() : 0;
   const int pair = blockIdx.x / nsplit;
@@ -134,7 +135,7 @@ attn_tma_kernel(const __grid_constant__ Maps maps, const AttnArgs a, int nsplit)
   TileInfo ti[2];
   pair_tiles(pair, j, G, ntt, ti);      // ti[0] is always valid
   const int64_t kvrow = (int64_t)bi * a.nkv + j;
-  const int nsel = a.bsa > 0 ? max(0, min(a.kv_count[kvrow], a.bsa)) : 0;
+  const int nsel = a.bsa > 0 ? max(0, min(__ldcg(a.kv_count + kvrow), a.bsa)) : 0;
   const int max_t0 = ti[1].valid ? max(ti[0].t0, ti[1].t0) : ti[0].t0;
   const int nchunk = min(a.BCP, max_t0 + 128);
   const int ntile_sel = (nsel + N - 1) / N;
@@ -421,7 +422,7 @@ attn_tma_kernel(const __grid_constant__ Maps maps, const AttnArgs a, int nsplit)
 
 }  // namespace
 
-cudaError_t launch_attn_tc(const AttnArgs& a, cudaStream_t stream) {
+cudaError_t launch_attn_tc(const AttnArgs& a, bool pdl, cudaStream_t stream) {
   if (a.d != D) return cudaErrorNotSupported;
   // rows gathered by index while loading: the other kernel
   if (a.kv_idx != nullptr && a.bsa > 0) return launch_attn_tc_gather(a, stream);
@@ -459,13 +460,15 @@ cudaError_t launch_attn_tc(const AttnArgs& a, cudaStream_t stream) {
   cfg.blockDim = dim3(THREADS);
   cfg.dynamicSmemBytes = smem;
   cfg.stream = stream;
-  cudaLaunchAttribute attr[1];
+  cudaLaunchAttribute attr[2];
   attr[0].id = cudaLaunchAttributeClusterDimension;
   attr[0].val.clusterDim.x = nsplit;
   attr[0].val.clusterDim.y = 1;
   attr[0].val.clusterDim.z = 1;
+  attr[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[1].val.programmaticStreamSerializationAllowed = 1;
   cfg.attrs = attr;
-  cfg.numAttrs = 1;
+  cfg.numAttrs = pdl ? 2 : 1;
   return cudaLaunchKernelEx(&cfg, attn_tma_kernel, maps, a, nsplit);
 }
 

@@ -62,6 +62,15 @@ __device__ __forceinline__ uint32_t score_key(float f) {
   return (u & 0x80000000u) ? ~u : (u | 0x80000000u);
 }
 
+// Programmatic dependent launch: a kernel launched with the programmatic
+// stream serialisation attribute may start while its predecessor in the
+// stream still runs; pdl_wait() blocks the calling thread until the
+// predecessor grid has completed and its memory is visible (a no-op for a
+// normal launch). pdl_trigger() lets the dependent grid launch once every
+// CTA of this grid has called it or exited.
+__device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+__device__ __forceinline__ void pdl_trigger() { asm volatile("griddepcontrol.launch_dependents;" ::: "memory"); }
+
 // 12-bit bucket of a score, linear over [-1, 1] (cosine-type scores lie
 // there): floor((s + 1) * 2048) clamped to [0, 4095]. Non-decreasing in the
 // score's key order (every step rounds monotonically; a NaN goes to the end

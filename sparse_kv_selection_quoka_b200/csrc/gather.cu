@@ -40,7 +40,10 @@ gather_kernel(const char* __restrict__ K, int64_t sKb, int64_t sKh, int64_t sKt,
               int cpr_log2, char* __restrict__ Ksel, char* __restrict__ Vsel, int* status) {
   const int j = blockIdx.y, bi = blockIdx.z, nkv = gridDim.y;
   const int64_t row = (int64_t)bi * nkv + j;
-  const int cnt = max(0, min(__ldg(kv_count + row), bsa));
+  pdl_trigger();  // the attention may launch once every CTA has started
+  pdl_wait();     // the indices may come from the previous kernel
+  // (indices possibly written by the previous kernel: L2-coherent loads)
+  const int cnt = max(0, min(__ldcg(kv_count + row), bsa));
   const int64_t nitems = (int64_t)bsa << cpr_log2;
   const int64_t i0 = (int64_t)blockIdx.x * (kThreads * kItems) + threadIdx.x;
   const int cmask = (1 << cpr_log2) - 1;
@@ -60,7 +63,7 @@ gather_kernel(const char* __restrict__ K, int64_t sKb, int64_t sKh, int64_t sKt,
     vv[u] = kv[u];
     if (i >= nitems) continue;
     if (n < cnt) {
-      const int32_t tau = __ldg(kv_idx + row * bsa + n);
+      const int32_t tau = __ldcg(kv_idx + row * bsa + n);
       if (tau >= 0 && (int64_t)tau < T) {
         kv[u] = ld_stream(reinterpret_cast<const uint4*>(Kb + tau * sKt) + c);
         vv[u] = ld_stream(reinterpret_cast<const uint4*>(Vb + tau * sVt) + c);

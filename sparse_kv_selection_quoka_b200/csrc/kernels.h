@@ -45,9 +45,11 @@ cudaError_t launch_score_simt(bool bf16, int d, Strided K, int b, int nkv, int64
 // 12-bit value buckets (score_bin) into `hist` (zeroed beforehand), the
 // first digit of the top-k select.
 // Returns cudaErrorNotSupported when the shape has no tensor-core variant.
+// pdl: launch with programmatic stream serialisation (the kernel starts its
+// K stream while the previous kernel in the stream still runs).
 cudaError_t launch_score_tc(int d, Strided K, int b, int nkv, int64_t T,
                             const uint16_t* Qg_hilo, int NQ, float* S_agg, uint32_t* hist,
-                            int* status, cudaStream_t stream);
+                            int* status, bool pdl, cudaStream_t stream);
 
 // Step (e): per (batch, KV head) cluster radix select of the BSA_eff
 // largest scores, ties to the lower index, written in ascending key order.
@@ -58,7 +60,7 @@ int64_t topk_max_T();
 // skipped.
 cudaError_t launch_topk(const float* S_agg, int b, int nkv, int64_t T, int bsa,
                         const uint32_t* hist, int32_t* kv_idx, int32_t* kv_count, int* status,
-                        cudaStream_t stream);
+                        bool pdl, cudaStream_t stream);
 
 // Step (f): gather of the selected K and V rows into contiguous
 // (b, nkv, bsa, d) buffers. Rows past kv_count, and rows whose index is out
@@ -90,7 +92,7 @@ cudaError_t launch_attn_simt(bool bf16, const AttnArgs& a, cudaStream_t stream);
 // otherwise launch_attn_tc_gather runs, which gathers the rows by index
 // while loading them (attn_tc.cu).
 // Return cudaErrorNotSupported when the shape has no tensor-core variant.
-cudaError_t launch_attn_tc(const AttnArgs& a, cudaStream_t stream);
+cudaError_t launch_attn_tc(const AttnArgs& a, bool pdl, cudaStream_t stream);
 cudaError_t launch_attn_tc_gather(const AttnArgs& a, cudaStream_t stream);
 
 }  // namespace quoka

@@ -115,6 +115,7 @@ qsel_fast_kernel(const bf16* __restrict__ Q, int64_t sQb, int64_t sQh, int64_t s
   const int h = j * G + g;
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const bf16* Qh = Q + bi * sQb + h * sQh;
+  pdl_trigger();  // the scoring kernel may launch and start streaming K
 
   // 1. stage the rows; thread (rg, cc) handles chunk cc of rows rg, rg + 32, ...
   {

@@ -184,7 +184,7 @@ quoka_status run_select(const quoka_tensor* Q, const quoka_tensor* K, const Sele
   if (s.T > 0) {
     e = cudaErrorNotSupported;
     if (bf) {
-      e = quoka::launch_score_tc(d, strided(K), b, nkv, s.T, qhilo, NQ, sagg, hist, status, stream);
+      e = quoka::launch_score_tc(d, strided(K), b, nkv, s.T, qhilo, NQ, sagg, hist, status, true, stream);
       hist_made = e == cudaSuccess;
     }
     if (e == cudaErrorNotSupported)
@@ -193,7 +193,7 @@ quoka_status run_select(const quoka_tensor* Q, const quoka_tensor* K, const Sele
   }
   if (bsa_eff > 0) {
     e = quoka::launch_topk(sagg, b, nkv, s.T, bsa_eff, hist_made ? hist : nullptr, kv_idx, kv_count, status,
-                           stream);
+                           true, stream);
     if (e != cudaSuccess) return cuda_status(e);
   } else {
     e = cudaMemsetAsync(kv_count, 0, sizeof(int32_t) * b * nkv, stream);
@@ -241,7 +241,7 @@ quoka_status validate_attn(const quoka_tensor* Q, const quoka_tensor* K, const q
 quoka_status run_attn(const quoka_tensor* Q, Strided K, Strided V, const quoka_tensor* Kc,
                       const quoka_tensor* Vc, const AttnShapes& s, int64_t T, const int32_t* kv_idx,
                       const int32_t* kv_count, int bsa_eff, float scale, void* O, float* lse,
-                      int* status, cudaStream_t stream) {
+                      int* status, cudaStream_t stream, bool pdl = false) {
   quoka::AttnArgs a;
   a.Q = strided(Q);
   a.K = K;
@@ -262,7 +262,7 @@ quoka_status run_attn(const quoka_tensor* Q, Strided K, Strided V, const quoka_t
   a.lse = lse;
   a.status = status;
   cudaError_t e = cudaErrorNotSupported;
-  if (Q->dtype == QUOKA_BF16) e = quoka::launch_attn_tc(a, stream);
+  if (Q->dtype == QUOKA_BF16) e = quoka::launch_attn_tc(a, pdl, stream);
   if (e == cudaErrorNotSupported) e = quoka::launch_attn_simt(Q->dtype == QUOKA_BF16, a, stream);
   return cuda_status(e);
 }
@@ -282,8 +282,9 @@ quoka_status gather_then_attn(const quoka_tensor* Q, const quoka_tensor* K, cons
                                        (int)s.nkv, s.T, kv_idx, kv_count, bsa_eff, ksel, vsel, status, stream);
   if (e != cudaSuccess) return cuda_status(e);
   const int64_t sh = (int64_t)bsa_eff * s.d, sb = s.nkv * sh;
+  // the attention may launch while the gather finishes (it waits for it)
   return run_attn(Q, Strided{ksel, sb, sh, s.d}, Strided{vsel, sb, sh, s.d}, Kc, Vc, s, bsa_eff, nullptr,
-                  kv_count, bsa_eff, scale, O, lse, status, stream);
+                  kv_count, bsa_eff, scale, O, lse, status, stream, true);
 }
 
 }  // namespace

@@ -103,6 +103,7 @@ score_tc_kernel(const __grid_constant__ CUtensorMap tmap, const ScoreArgs a) {
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int j = blockIdx.y, bi = blockIdx.z, nkv = gridDim.y;
   const int64_t row = (int64_t)bi * nkv + j;
+  pdl_trigger();
   const int t_begin = blockIdx.x * a.tiles_per_cta;
   const int n = max(0, min(a.ntiles, t_begin + a.tiles_per_cta) - t_begin);
   const int NS = a.nstages;
@@ -152,6 +153,8 @@ score_tc_kernel(const __grid_constant__ CUtensorMap tmap, const ScoreArgs a) {
   const int nstage_threads = SC_THREADS - 32;  // everyone but the producer
   const int st = tid - 32;
   if (warp != 0) {
+  // the query groups (and the zeroed histogram) come from the previous kernel
+  pdl_wait();
   for (int e = st; e < TOPK_HIST_BINS; e += nstage_threads) hist_s[e] = 0u;
   // B operand: the group means (hi rows then lo rows, each padded to NQp
   // with zero rows) in the K-major 128-byte-swizzled layout.
@@ -162,7 +165,8 @@ score_tc_kernel(const __grid_constant__ CUtensorMap tmap, const ScoreArgs a) {
       const int half = r >= a.NQp;  // 0 = hi, 1 = lo
       const int i = r - half * a.NQp;
       uint4 v = make_uint4(0u, 0u, 0u, 0u);
-      if (i < a.NQ) v = *reinterpret_cast<const uint4*>(src + ((int64_t)(half * a.NQ + i)) * SC_D + c * 8);
+      // (written by the previous kernel: L2-coherent load)
+      if (i < a.NQ) v = __ldcg(reinterpret_cast<const uint4*>(src + ((int64_t)(half * a.NQ + i)) * SC_D + c * 8));
       *reinterpret_cast<uint4*>(qg_s + sw128_offset(r, c, N)) = v;
     }
     fence_proxy_async_smem();
@@ -273,7 +277,8 @@ score_tc_kernel(const __grid_constant__ CUtensorMap tmap, const ScoreArgs a) {
     tc_fence_after();
     tmem_dealloc(tmem, a.tmem_cols);
   }
-  // fold this CTA's histogram into the head's
+  // fold this CTA's histogram into the head's (zeroed by the previous kernel)
+  pdl_wait();
   uint32_t* gh = a.hist + row * TOPK_HIST_BINS;
   for (int e = tid; e < TOPK_HIST_BINS; e += SC_THREADS) {
     const uint32_t v = hist_s[e];
@@ -284,7 +289,7 @@ score_tc_kernel(const __grid_constant__ CUtensorMap tmap, const ScoreArgs a) {
 }  // namespace
 
 cudaError_t launch_score_tc(int d, Strided K, int b, int nkv, int64_t T, const uint16_t* Qg_hilo, int NQ,
-                            float* S_agg, uint32_t* hist, int* status, cudaStream_t stream) {
+                            float* S_agg, uint32_t* hist, int* status, bool pdl, cudaStream_t stream) {
   if (d != SC_D || NQ < 1 || NQ > 128 || T <= 0 || T > (int64_t)INT32_MAX - SC_KEYS) return cudaErrorNotSupported;
   PFN_cuTensorMapEncodeTiled_v12000 encode = tensor_map_encoder();
   if (encode == nullptr) return cudaErrorNotSupported;
@@ -335,8 +340,17 @@ cudaError_t launch_score_tc(int d, Strided K, int b, int nkv, int64_t T, const u
       (size_t)qg_bytes + TOPK_HIST_BINS * 4 + (size_t)a.nstages * SC_TILE_BYTES + sizeof(ScoreBars) + 1024;
   cudaError_t e = cudaFuncSetAttribute(score_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (e != cudaSuccess) return e;
-  score_tc_kernel<<<dim3(per_head, nkv, b), SC_THREADS, smem, stream>>>(tmap, a);
-  return cudaGetLastError();
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(per_head, nkv, b);
+  cfg.blockDim = dim3(SC_THREADS);
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = stream;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = pdl ? 1 : 0;
+  return cudaLaunchKernelEx(&cfg, score_tc_kernel, tmap, a);
 }
 
 }  // namespace quoka

@@ -139,6 +139,7 @@ topk_kernel(const float* __restrict__ S, int64_t T, int bsa, int slice, const ui
   const int n = (int)max((int64_t)0, min((int64_t)slice, T - lo));
   const int n_round = (n + TOPK_THREADS - 1) / TOPK_THREADS * TOPK_THREADS;
 
+  pdl_trigger();
   if (tid == 0) {
     sh.kmin = 0xFFFFFFFFu;
     sh.kmax = 0u;
@@ -154,11 +155,15 @@ topk_kernel(const float* __restrict__ S, int64_t T, int bsa, int slice, const ui
   // the scoring kernel's histogram bins this thread owns in the first pick
   // (loaded first: the loads overlap the staging below)
   uint32_t g0[4] = {0u, 0u, 0u, 0u};
+  // The scores and their histogram come from the previous kernel, which may
+  // still run until this wait returns: they are read with L2-coherent loads
+  // (never the read-only path, which assumes data fixed for the kernel's life).
+  pdl_wait();
   if (ghist != nullptr) {
     const uint32_t* Hg = ghist + row * TOPK_BINS;
     constexpr int q0 = TOPK_BINS / TOPK_THREADS;
 #pragma unroll
-    for (int u = 0; u < q0; ++u) g0[u] = __ldg(Hg + TOPK_BINS - 1 - (tid * q0 + u));
+    for (int u = 0; u < q0; ++u) g0[u] = __ldcg(Hg + TOPK_BINS - 1 - (tid * q0 + u));
   }
   // stage the slice as keys (16-byte loads when the slice start is aligned)
   if ((((uintptr_t)(Sr + lo)) & 15u) == 0u) {
@@ -166,12 +171,12 @@ topk_kernel(const float* __restrict__ S, int64_t T, int bsa, int slice, const ui
     const float4* src4 = reinterpret_cast<const float4*>(Sr + lo);
 #pragma unroll 4
     for (int e = tid; e < n4; e += TOPK_THREADS) {
-      const float4 v = __ldg(src4 + e);
+      const float4 v = __ldcg(src4 + e);
       reinterpret_cast<uint4*>(keys)[e] = make_uint4(score_key(v.x), score_key(v.y), score_key(v.z), score_key(v.w));
     }
-    for (int e = 4 * n4 + tid; e < n; e += TOPK_THREADS) keys[e] = score_key(Sr[lo + e]);
+    for (int e = 4 * n4 + tid; e < n; e += TOPK_THREADS) keys[e] = score_key(__ldcg(Sr + lo + e));
   } else {
-    for (int e = tid; e < n; e += TOPK_THREADS) keys[e] = score_key(Sr[lo + e]);
+    for (int e = tid; e < n; e += TOPK_THREADS) keys[e] = score_key(__ldcg(Sr + lo + e));
   }
 
   // From a histogram over `nbins` bins (this CTA's H, optionally summed over
@@ -559,7 +564,7 @@ topk_kernel(const float* __restrict__ S, int64_t T, int bsa, int slice, const ui
 int64_t topk_max_T() { return (int64_t)TOPK_MAX_CLUSTER * TOPK_MAX_SLICE; }
 
 cudaError_t launch_topk(const float* S_agg, int b, int nkv, int64_t T, int bsa, const uint32_t* hist,
-                        int32_t* kv_idx, int32_t* kv_count, int* status, cudaStream_t stream) {
+                        int32_t* kv_idx, int32_t* kv_count, int* status, bool pdl, cudaStream_t stream) {
   (void)status;  // every wait in the kernel is a hardware barrier phase that all threads reach
   if (bsa <= 0 || T <= 0 || bsa > T || T > topk_max_T()) return cudaErrorInvalidValue;
   int C = (int)((T + TOPK_SLICE_TARGET - 1) / TOPK_SLICE_TARGET);
@@ -568,28 +573,31 @@ cudaError_t launch_topk(const float* S_agg, int b, int nkv, int64_t T, int bsa, 
   const int slice = (int)((T + C - 1) / C);
   if (slice > TOPK_MAX_SLICE) return cudaErrorInvalidValue;
   const size_t smem = ((size_t)slice + 2 * TOPK_LIST_MAX) * sizeof(uint32_t);
-  if (C == 1) {
-    cudaError_t e = cudaFuncSetAttribute(topk_kernel<false>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-    if (e != cudaSuccess) return e;
-    topk_kernel<false><<<dim3(1, nkv, b), TOPK_THREADS, smem, stream>>>(S_agg, T, bsa, slice, hist, kv_idx,
-                                                                        kv_count);
-    return cudaGetLastError();
-  }
-  cudaError_t e = cudaFuncSetAttribute(topk_kernel<true>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+  auto kern = C == 1 ? topk_kernel<false> : topk_kernel<true>;
+  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (e != cudaSuccess) return e;
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(C, nkv, b);
   cfg.blockDim = dim3(TOPK_THREADS);
   cfg.dynamicSmemBytes = smem;
   cfg.stream = stream;
-  cudaLaunchAttribute attr[1];
-  attr[0].id = cudaLaunchAttributeClusterDimension;
-  attr[0].val.clusterDim.x = C;
-  attr[0].val.clusterDim.y = 1;
-  attr[0].val.clusterDim.z = 1;
+  cudaLaunchAttribute attr[2];
+  int na = 0;
+  if (C > 1) {
+    attr[na].id = cudaLaunchAttributeClusterDimension;
+    attr[na].val.clusterDim.x = C;
+    attr[na].val.clusterDim.y = 1;
+    attr[na].val.clusterDim.z = 1;
+    ++na;
+  }
+  if (pdl) {
+    attr[na].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[na].val.programmaticStreamSerializationAllowed = 1;
+    ++na;
+  }
   cfg.attrs = attr;
-  cfg.numAttrs = 1;
-  return cudaLaunchKernelEx(&cfg, topk_kernel<true>, S_agg, T, bsa, slice, hist, kv_idx, kv_count);
+  cfg.numAttrs = na;
+  return cudaLaunchKernelEx(&cfg, kern, S_agg, T, bsa, slice, hist, kv_idx, kv_count);
 }
 
 }  // namespace quoka
