@@ -55,14 +55,14 @@ def _peaks():
     return 6650.0, 1590.0, 1400.0, "fallback"
 
 
-def _profiled_traffic(profile_name: str, source_rel: str):
+def _profiled_traffic(profile_name: str, *source_rel: str):
     """DRAM bytes per launch from a committed ncu summary, if the kernel's
-    source still hashes to the value recorded with the counters (else None:
-    the counters describe an older kernel)."""
+    sources (hashed in the given order) still match the value recorded with
+    the counters (else None: the counters describe an older kernel)."""
     import hashlib
     prof = os.path.join(ROOT, "profiles", profile_name)
-    src = os.path.join(ROOT, source_rel)
-    if not (os.path.exists(prof) and os.path.exists(src)):
+    srcs = [os.path.join(ROOT, r) for r in source_rel]
+    if not (os.path.exists(prof) and all(os.path.exists(x) for x in srcs)):
         return None
     want, traffic = None, None
     with open(prof) as f:
@@ -72,8 +72,11 @@ def _profiled_traffic(profile_name: str, source_rel: str):
                 traffic = int(line.split(":")[1])
             elif line.startswith("source_sha256_16:"):
                 want = line.split(":")[1].strip()
-    with open(src, "rb") as f:
-        have = hashlib.sha256(f.read()).hexdigest()[:16]
+    m = hashlib.sha256()
+    for x in srcs:
+        with open(x, "rb") as f:
+            m.update(f.read())
+    have = m.hexdigest()[:16]
     return traffic if (want is not None and have == want) else None
 
 
@@ -306,9 +309,10 @@ def run_ours(args, rank, world, local_rank):
         "roofline": {"kernel": "sparse GQA attention (tcgen05)" if w.dtype == "bf16" else "sparse GQA attention (fp32 CUDA cores)",
                      "bound": "tensor", "achieved": attn_tflops, "peak": tf_burst,
                      "unit": "TFLOP/s", "frac": attn_tflops / tf_burst,
-                     "traffic": (_profiled_traffic("attn_tc_qwen3-4b_T32k.md",
-                                                   "sparse_kv_selection_quoka_b200/csrc/attn_tc.cu")
-                                 if w.name == "qwen3-4b_T32k" else None),
+                     "traffic": (_profiled_traffic("attn_tma_qwen3-4b_T32k.md",
+                                                   "sparse_kv_selection_quoka_b200/csrc/attn_tma.cu",
+                                                   "sparse_kv_selection_quoka_b200/csrc/attn_common.cuh")
+                                 if w.name == "qwen3-4b_T32k" and w.dtype == "bf16" else None),
                      "peak_kind": f"bf16 dense, burst, {peak_src}",
                      "algorithmic_flops_per_launch": flops / max(1, len(chunks))},
         "roofline_select": {"steps": "(a)-(e)", "bound": "hbm", "achieved": sel_gbs, "peak": hbm,
