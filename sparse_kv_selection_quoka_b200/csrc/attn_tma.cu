@@ -18,8 +18,9 @@
 // ceil(nsel/128) tiles of selected rows (rows past nsel are masked)
 // followed by ceil(nchunk/128) tiles of the chunk's own keys. When the grid
 // would fill less than half of the GPU, the key tiles are split between the
-// two CTAs of a cluster; rank 1 sends its partial (O, m, l) to rank 0 with
-// one bulk shared-to-shared copy over the cluster, and rank 0 combines.
+// two CTAs of a cluster: rank r finalises query tile r, and each rank sends
+// its partial (O, m, l) of the other tile to the peer with bulk
+// shared-to-shared copies over the cluster (both directions at once).
 //
 // Warp roles (352 threads):
 //   warps 0-7   softmax of Q0 (warps 0-3) and Q1 (warps 4-7), one query row
@@ -60,10 +61,13 @@ constexpr int VLOAD_WARP = 10;
 // Measured on B200 (Qwen-shaped layer): 0 and 2 run equally fast, more is
 // slower; 0 keeps the kernel free of register spills.
 constexpr int SOFTMAX_FMA_PAIRS = 0;
-// split-KV payload: partial O (fp32, 2 tiles x 128 rows x 128, each row's
-// 16-byte chunks rotated by the row index) followed by (m, l) per row
-constexpr uint32_t XFER_O_BYTES = 2 * 128 * D * 4;
-constexpr uint32_t XFER_BYTES = XFER_O_BYTES + 2 * 128 * 2 * 4;
+// split-KV payload of one query tile: partial O (fp32, 128 rows x 128, each
+// row's 16-byte chunks rotated by the row index) followed by (m, l) per row;
+// staged at OUT_OFF of the K/V span, received at IN_OFF
+constexpr uint32_t XFER_O_BYTES = 128 * D * 4;
+constexpr uint32_t XFER_BYTES = XFER_O_BYTES + 128 * 2 * 4;
+constexpr uint32_t XFER_OUT_OFF = 0;
+constexpr uint32_t XFER_IN_OFF = 80 * 1024;
 constexpr uint32_t XFER_PIECE = 32768;  // bytes per bulk copy
 
 struct Maps {
@@ -79,13 +83,14 @@ struct __align__(1024) Smem {
   uint64_t v_full[VST], v_empty[VST];
   uint64_t s_full[2], p_full[2];
   uint64_t o_final, mma_done;
-  uint64_t xfer_free;  // (rank 1) rank 0's landing zone is free
-  uint64_t xfer_full;  // (rank 0) the payload has landed
-  uint64_t xfer_done;  // (rank 1) rank 0 has the payload: the source may go
+  uint64_t xfer_free;  // the peer's landing zone is free (its MMAs are done)
+  uint64_t xfer_full;  // the peer's partial of this rank's tile has landed
+  uint64_t xfer_done;  // the peer holds this rank's payload: the source may go
   uint32_t tmem_base;
   int abort;
 };
-static_assert(XFER_BYTES <= (KST + VST) * TILE_BYTES, "split-KV payload");
+static_assert(XFER_OUT_OFF + XFER_BYTES <= XFER_IN_OFF && XFER_IN_OFF + XFER_BYTES <= (KST + VST) * TILE_BYTES,
+              "split-KV payloads");
 static_assert(offsetof(Smem, v) == offsetof(Smem, k) + KST * TILE_BYTES, "K and V rings adjacent");
 
 // Loader of one ring: TMA boxes of the key tiles [first, first + ntiles)
@@ -168,8 +173,9 @@ attn_tma_kernel(const __grid_constant__ Maps maps, const AttnArgs a, int nsplit)
     mbar_init(&sm.xfer_done, 1);
     sm.abort = 0;
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
-    // rank 0 expects the payload bytes before rank 1 can send anything
-    if (nsplit > 1 && split == 0) mbar_arrive_expect_tx(&sm.xfer_full, XFER_BYTES);
+    // rank r finalises query tile r: it expects the peer's partial of that
+    // tile before the peer can send anything
+    if (nsplit > 1 && ti[split].valid) mbar_arrive_expect_tx(&sm.xfer_full, XFER_BYTES);
   }
   if (warp == MMA_WARP) {
     tmem_alloc(&sm.tmem_base, TMEM_COLS);
@@ -264,9 +270,9 @@ attn_tma_kernel(const __grid_constant__ Maps maps, const AttnArgs a, int nsplit)
       umma_commit(&sm.o_final);
       umma_commit(&sm.mma_done);
       if (!mbar_drain(&sm.mma_done, 0)) record_abort(sm, a.status, 27);
-      // rank 0: every MMA is done (and every load they waited for has
-      // landed), so its K/V span may now take rank 1's payload
-      if (nsplit > 1 && split == 0) mbar_arrive_remote(mapa_shared(smem_u32(&sm.xfer_free), 1));
+      // every MMA is done (and every load they waited for has landed), so
+      // this rank's K/V span may now take the peer's payload
+      if (nsplit > 1) mbar_arrive_remote(mapa_shared(smem_u32(&sm.xfer_free), (uint32_t)(split ^ 1)));
     }
     __syncwarp();
   } else {
@@ -302,67 +308,16 @@ attn_tma_kernel(const __grid_constant__ Maps maps, const AttnArgs a, int nsplit)
     const bool have = active && ntiles > 0;  // warp-uniform: TMEM loads below are collective
     if (alive) alive = warp_wait(&sm.o_final, 0, sm, a.status, 33);
     tc_fence_after();
-    const int row = w * 128 + r;
     uint8_t* span = reinterpret_cast<uint8_t*>(&sm) + offsetof(Smem, k);  // K ring, then V ring
-    float* pay_o = reinterpret_cast<float*>(span) + (size_t)row * D;
-    float* pay_ml = reinterpret_cast<float*>(span + XFER_O_BYTES) + (size_t)row * 2;
-    if (nsplit > 1 && split == 1) {
-      // stage this row's (O, m, l) in the own K/V span (free: every MMA is
-      // done), then one thread sends the whole payload to rank 0
-#pragma unroll 1
-      for (int c4 = 0; c4 < 4; ++c4) {
-        float o[32];
-        if (have) {
-          tmem_ld32(O + 32 * c4, o);
-          tmem_wait_ld();
-        } else {
-#pragma unroll
-          for (int u = 0; u < 32; ++u) o[u] = 0.f;
-        }
-#pragma unroll
-        for (int u = 0; u < 32; u += 4) {
-          const int chunk = (32 * c4 + u) >> 2;  // 16-byte chunk 0..31, rotated by row
-          *reinterpret_cast<float4*>(pay_o + 4 * ((chunk + r) & 31)) =
-              make_float4(o[u], o[u + 1], o[u + 2], o[u + 3]);
-        }
-      }
-      pay_ml[0] = have ? m : -INFINITY;
-      pay_ml[1] = have ? l : 0.f;
-      fence_proxy_async_smem();  // the staged payload becomes visible to the bulk copy
-      named_barrier_sync(1, SOFTMAX_THREADS);
-      if (tid == 0) {
-        bool ok = wait_cluster(&sm.xfer_free, 0);
-        if (ok) {
-          const uint32_t src = smem_u32(sm.k[0]);
-          const uint32_t dst = mapa_shared(src, 0), bar = mapa_shared(smem_u32(&sm.xfer_full), 0);
-          for (uint32_t off = 0; off < XFER_BYTES; off += XFER_PIECE)
-            bulk_copy_to_cluster(dst + off, src + off, min(XFER_PIECE, XFER_BYTES - off), bar);
-          // the source must stay in place until rank 0 holds the payload
-          ok = wait_cluster(&sm.xfer_done, 0);
-        }
-        if (!ok) record_abort(sm, a.status, 41);
-      }
-    } else {
-      float m_o = -INFINITY, l_o = 0.f;  // the other rank's part
-      if (nsplit > 1) {
-        if (alive) alive = warp_wait_cluster(&sm.xfer_full, 0, sm, a.status, 42);
-        if (alive) {
-          m_o = pay_ml[0];
-          l_o = pay_ml[1];
-        }
-        if (tid == 0) mbar_arrive_remote(mapa_shared(smem_u32(&sm.xfer_done), 1));
-      }
+    const uint32_t peer = (uint32_t)(split ^ 1);
+    // Split-KV: rank `split` finalises query tile `split`; the warpgroup of
+    // the other tile stages its partial and sends it to the peer, so both
+    // directions move at once and both warpgroups work.
+    const bool send = nsplit > 1 && w != split;
+    if (send) {
       if (active) {
-        const float mm = have ? m : -INFINITY;
-        const float ll = have ? l : 0.f;
-        const float M = fmaxf(mm, m_o);
-        const float f_me = mm == -INFINITY ? 0.f : ex2(mm - M);
-        const float f_ot = m_o == -INFINITY ? 0.f : ex2(m_o - M);
-        const float L = f_me * ll + f_ot * l_o;
-        const float inv = 1.f / L;
-        // the normalised row, bf16, into the tile's 128-byte-swizzled
-        // output staging (the Q area: every MMA is done)
-        uint8_t* ot = sm.q[w];
+        float* out_o = reinterpret_cast<float*>(span + XFER_OUT_OFF) + (size_t)r * D;
+        float* out_ml = reinterpret_cast<float*>(span + XFER_OUT_OFF + XFER_O_BYTES) + (size_t)r * 2;
 #pragma unroll 1
         for (int c4 = 0; c4 < 4; ++c4) {
           float o[32];
@@ -373,41 +328,97 @@ attn_tma_kernel(const __grid_constant__ Maps maps, const AttnArgs a, int nsplit)
 #pragma unroll
             for (int u = 0; u < 32; ++u) o[u] = 0.f;
           }
-          if (nsplit > 1) {
 #pragma unroll
-            for (int u = 0; u < 32; u += 4) {
-              const int chunk = (32 * c4 + u) >> 2;
-              const float4 p = *reinterpret_cast<const float4*>(pay_o + 4 * ((chunk + r) & 31));
-              o[u] = o[u] * f_me + p.x * f_ot;
-              o[u + 1] = o[u + 1] * f_me + p.y * f_ot;
-              o[u + 2] = o[u + 2] * f_me + p.z * f_ot;
-              o[u + 3] = o[u + 3] * f_me + p.w * f_ot;
-            }
-          } else {
-#pragma unroll
-            for (int u = 0; u < 32; ++u) o[u] *= f_me;
-          }
-#pragma unroll
-          for (int u = 0; u < 32; u += 8) {
-            uint4 pk;
-            pk.x = pack_bf16x2(o[u] * inv, o[u + 1] * inv);
-            pk.y = pack_bf16x2(o[u + 2] * inv, o[u + 3] * inv);
-            pk.z = pack_bf16x2(o[u + 4] * inv, o[u + 5] * inv);
-            pk.w = pack_bf16x2(o[u + 6] * inv, o[u + 7] * inv);
-            *reinterpret_cast<uint4*>(ot + sw128_offset(r, (32 * c4 + u) >> 3, 128)) = pk;
+          for (int u = 0; u < 32; u += 4) {
+            const int chunk = (32 * c4 + u) >> 2;  // 16-byte chunk 0..31, rotated by row
+            *reinterpret_cast<float4*>(out_o + 4 * ((chunk + r) & 31)) =
+                make_float4(o[u], o[u + 1], o[u + 2], o[u + 3]);
           }
         }
-        if (t < a.BCP && a.lse != nullptr)
-          a.lse[((int64_t)bi * a.nq + ti[w].h) * a.BCP + t] = (M + __log2f(L)) * 0.6931471805599453f;
-        // rows past the chunk are clipped by the store
-        fence_proxy_async_smem();
+        out_ml[0] = have ? m : -INFINITY;
+        out_ml[1] = have ? l : 0.f;
+        fence_proxy_async_smem();  // the staged payload becomes visible to the bulk copy
         named_barrier_sync(2 + w, 128);
         if (r == 0) {
-          tma_store_4d(&maps.o, smem_u32(ot), 0, ti[w].t0, ti[w].h, bi);
-          tma_store_4d(&maps.o, smem_u32(ot) + ATOM_BYTES, 64, ti[w].t0, ti[w].h, bi);
-          bulk_commit_group();
-          bulk_wait_group_0();
+          bool ok = wait_cluster(&sm.xfer_free, 0);
+          if (ok) {
+            const uint32_t src = smem_u32(span + XFER_OUT_OFF);
+            const uint32_t dst = mapa_shared(smem_u32(span + XFER_IN_OFF), peer);
+            const uint32_t bar = mapa_shared(smem_u32(&sm.xfer_full), peer);
+            for (uint32_t off = 0; off < XFER_BYTES; off += XFER_PIECE)
+              bulk_copy_to_cluster(dst + off, src + off, min(XFER_PIECE, XFER_BYTES - off), bar);
+            // the source must stay in place until the peer holds the payload
+            ok = wait_cluster(&sm.xfer_done, 0);
+          }
+          if (!ok) record_abort(sm, a.status, 41);
         }
+      }
+    } else if (active) {
+      float m_o = -INFINITY, l_o = 0.f;  // the peer's part
+      const float* in_o = reinterpret_cast<const float*>(span + XFER_IN_OFF) + (size_t)r * D;
+      const float* in_ml = reinterpret_cast<const float*>(span + XFER_IN_OFF + XFER_O_BYTES) + (size_t)r * 2;
+      if (nsplit > 1) {
+        if (alive) alive = warp_wait_cluster(&sm.xfer_full, 0, sm, a.status, 42);
+        if (alive) {
+          m_o = in_ml[0];
+          l_o = in_ml[1];
+        }
+        if (r == 0) mbar_arrive_remote(mapa_shared(smem_u32(&sm.xfer_done), peer));
+      }
+      const float mm = have ? m : -INFINITY;
+      const float ll = have ? l : 0.f;
+      const float M = fmaxf(mm, m_o);
+      const float f_me = mm == -INFINITY ? 0.f : ex2(mm - M);
+      const float f_ot = m_o == -INFINITY ? 0.f : ex2(m_o - M);
+      const float L = f_me * ll + f_ot * l_o;
+      const float inv = 1.f / L;
+      // the normalised row, bf16, into the tile's 128-byte-swizzled output
+      // staging (the Q area: every MMA is done)
+      uint8_t* ot = sm.q[w];
+#pragma unroll 1
+      for (int c4 = 0; c4 < 4; ++c4) {
+        float o[32];
+        if (have) {
+          tmem_ld32(O + 32 * c4, o);
+          tmem_wait_ld();
+        } else {
+#pragma unroll
+          for (int u = 0; u < 32; ++u) o[u] = 0.f;
+        }
+        if (nsplit > 1) {
+#pragma unroll
+          for (int u = 0; u < 32; u += 4) {
+            const int chunk = (32 * c4 + u) >> 2;
+            const float4 p = *reinterpret_cast<const float4*>(in_o + 4 * ((chunk + r) & 31));
+            o[u] = o[u] * f_me + p.x * f_ot;
+            o[u + 1] = o[u + 1] * f_me + p.y * f_ot;
+            o[u + 2] = o[u + 2] * f_me + p.z * f_ot;
+            o[u + 3] = o[u + 3] * f_me + p.w * f_ot;
+          }
+        } else {
+#pragma unroll
+          for (int u = 0; u < 32; ++u) o[u] *= f_me;
+        }
+#pragma unroll
+        for (int u = 0; u < 32; u += 8) {
+          uint4 pk;
+          pk.x = pack_bf16x2(o[u] * inv, o[u + 1] * inv);
+          pk.y = pack_bf16x2(o[u + 2] * inv, o[u + 3] * inv);
+          pk.z = pack_bf16x2(o[u + 4] * inv, o[u + 5] * inv);
+          pk.w = pack_bf16x2(o[u + 6] * inv, o[u + 7] * inv);
+          *reinterpret_cast<uint4*>(ot + sw128_offset(r, (32 * c4 + u) >> 3, 128)) = pk;
+        }
+      }
+      if (t < a.BCP && a.lse != nullptr)
+        a.lse[((int64_t)bi * a.nq + ti[w].h) * a.BCP + t] = (M + __log2f(L)) * 0.6931471805599453f;
+      // rows past the chunk are clipped by the store
+      fence_proxy_async_smem();
+      named_barrier_sync(2 + w, 128);
+      if (r == 0) {
+        tma_store_4d(&maps.o, smem_u32(ot), 0, ti[w].t0, ti[w].h, bi);
+        tma_store_4d(&maps.o, smem_u32(ot) + ATOM_BYTES, 64, ti[w].t0, ti[w].h, bi);
+        bulk_commit_group();
+        bulk_wait_group_0();
       }
     }
   }
