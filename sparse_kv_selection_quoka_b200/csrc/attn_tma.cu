@@ -146,9 +146,10 @@ attn_tma_kernel(const __grid_constant__ Maps maps, const AttnArgs a, int nsplit)
   const int ntile_sel = (nsel + N - 1) / N;
   const int ntile_chk = (nchunk + N - 1) / N;
   const int nT = ntile_sel + ntile_chk;
-  // split: rank 0 takes one or two tiles more than rank 1, so that rank 1's
-  // payload transfer overlaps rank 0's last tiles
-  const int n0 = nsplit > 1 ? min(nT, (nT + 3) / 2) : nT;
+  // split: the ranks take halves of the key tiles (each finalises one query
+  // tile and waits for the other's partial of it, so an uneven split would
+  // only make the longer rank longer)
+  const int n0 = nsplit > 1 ? (nT + 1) / 2 : nT;
   const int first = split == 0 ? 0 : n0;
   const int ntiles = split == 0 ? n0 : nT - n0;  // key tiles of this CTA (may be 0)
 
