@@ -82,13 +82,16 @@ __device__ __forceinline__ uint32_t pack_bf16x2(float a, float b) {
   return *reinterpret_cast<uint32_t*>(&h);
 }
 
+// The MMA issue helpers below are called by every lane of the (converged)
+// MMA warp; one elected lane issues.
+
 // S[:, 0:128) = Q K^T for a 128-row Q tile and a 128-key K tile, both in
 // shared memory in the 128-byte-swizzled K-major layout (two 64-column atoms).
 __device__ __forceinline__ void issue_qk(uint32_t tmem_s, uint32_t q_smem, uint32_t k_smem) {
 #pragma unroll
   for (int kk = 0; kk < D / 16; ++kk) {
     const uint32_t koff = (kk >> 2) * ATOM_BYTES + (kk & 3) * 32;
-    umma_bf16_ss(tmem_s, sw128_desc(q_smem + koff, 16, 1024), sw128_desc(k_smem + koff, 16, 1024), IDESC_QK,
+    umma_bf16_ss_warp(tmem_s, sw128_desc(q_smem + koff, 16, 1024), sw128_desc(k_smem + koff, 16, 1024), IDESC_QK,
                  kk > 0 ? 1u : 0u);
   }
 }
@@ -98,8 +101,22 @@ __device__ __forceinline__ void issue_qk(uint32_t tmem_s, uint32_t q_smem, uint3
 __device__ __forceinline__ void issue_pv(uint32_t tmem_o, uint32_t tmem_p, uint32_t v_smem, bool accumulate) {
 #pragma unroll
   for (int kk = 0; kk < N / 16; ++kk)
-    umma_bf16_ts(tmem_o, tmem_p + kk * 8, sw128_desc(v_smem + kk * 2048, ATOM_BYTES, 1024), IDESC_PV,
+    umma_bf16_ts_warp(tmem_o, tmem_p + kk * 8, sw128_desc(v_smem + kk * 2048, ATOM_BYTES, 1024), IDESC_PV,
                  (accumulate || kk > 0) ? 1u : 0u);
+}
+
+// Part `part` of O (+)= P V when the 128 keys are released in PARTS
+// equal parts: the K = 16 steps of keys [part * N / PARTS, (part + 1) * N / PARTS).
+template <int PARTS>
+__device__ __forceinline__ void issue_pv_part(uint32_t tmem_o, uint32_t tmem_p, uint32_t v_smem, int part,
+                                              bool accumulate) {
+  constexpr int KK = N / 16 / PARTS;
+#pragma unroll
+  for (int q = 0; q < KK; ++q) {
+    const int kk = part * KK + q;
+    umma_bf16_ts_warp(tmem_o, tmem_p + kk * 8, sw128_desc(v_smem + kk * 2048, ATOM_BYTES, 1024), IDESC_PV,
+                 (accumulate || kk > 0) ? 1u : 0u);
+  }
 }
 
 // 2^x for two values on the FMA pipe instead of the MUFU: x = n + f with n
@@ -133,14 +150,19 @@ __device__ __forceinline__ void exp2_fma_pair(uint64_t x, float& p0, float& p1) 
 // the row max (3-input max tree), and P = 2^(s * qscale - m) in bf16 over
 // the first 64 S columns (packed two per column), with the products and row
 // sums in paired fp32 arithmetic; of every 8 key pairs, FMA_PAIRS take the
-// FMA-pipe exp2 and the rest the MUFU, so both units share the work. The
-// running max m moves only when it grows by more than RESCALE_THRESHOLD, in
-// which case the O accumulator (complete for the previous tiles) is
-// rescaled in TMEM. Updates m and l. TMEM accesses are warp-collective: no
+// FMA-pipe exp2 and the rest the MUFU. The running max m moves only when it
+// grows by more than RESCALE_THRESHOLD, in which case the O accumulator
+// (complete for the previous tiles) is rescaled in TMEM before any P of the
+// tile is released. P is released to the MMA issuer in PARTS equal key
+// ranges as soon as each is in TMEM: after the part's stores complete, each
+// warp arrives once on p_part[part] (4 arrivals per part), so the P V
+// product of the first keys runs while the later ones are still being
+// exponentiated. Updates m and l. TMEM accesses are warp-collective: no
 // per-row branch surrounds one.
-template <int FMA_PAIRS>
-__device__ __forceinline__ void softmax_tile_1p(uint32_t S, uint32_t O, bool have_o, int base_n, int lim,
-                                                float qscale, float& m, float& l) {
+template <int FMA_PAIRS, int PARTS>
+__device__ __forceinline__ void softmax_tile_split(uint32_t S, uint32_t O, bool have_o, int base_n, int lim,
+                                                   float qscale, float& m, float& l, uint64_t* p_part) {
+  constexpr int CPP = 4 / PARTS;  // 32-key chunks per part
   float v[128];
   __syncwarp();
   tmem_ld64(S, v);
@@ -162,6 +184,18 @@ __device__ __forceinline__ void softmax_tile_1p(uint32_t S, uint32_t O, bool hav
   const float m_new = (m_cand > m + RESCALE_THRESHOLD || m == -INFINITY) ? m_cand : m;
   const float corr = (m_new == m) ? 1.f : ex2(m - m_new);
   const float m_use = m_new == -INFINITY ? 0.f : m_new;
+  // warp-uniform condition: the rescale's TMEM traffic is collective
+  if (have_o && __any_sync(0xffffffffu, corr != 1.f)) {
+#pragma unroll 1
+    for (int c4 = 0; c4 < 4; ++c4) {
+      float o[32];
+      tmem_ld32(O + 32 * c4, o);
+      tmem_wait_ld();
+#pragma unroll
+      for (int u = 0; u < 32; ++u) o[u] *= corr;
+      tmem_st32(O + 32 * c4, o);
+    }
+  }
   const uint64_t qs2 = f2_pack(qscale, qscale), nm2 = f2_pack(-m_use, -m_use);
   uint64_t acc[4] = {0, 0, 0, 0};  // paired row sums (+0.0f halves)
 #pragma unroll
@@ -185,24 +219,19 @@ __device__ __forceinline__ void softmax_tile_1p(uint32_t S, uint32_t O, bool hav
     }
     __syncwarp();
     tmem_st16(S + 16 * c, pk);
+    if (c % CPP == CPP - 1) {
+      // this part's P (and any O rescale) is in TMEM: release it
+      tmem_wait_st();
+      tc_fence_before();
+      __syncwarp();
+      if ((threadIdx.x & 31) == 0) mbar_arrive(&p_part[c / CPP]);
+    }
   }
   float r[8];
 #pragma unroll
   for (int k = 0; k < 4; ++k) f2_unpack(acc[k], r[2 * k], r[2 * k + 1]);
   l = l * corr + (((r[0] + r[1]) + (r[2] + r[3])) + ((r[4] + r[5]) + (r[6] + r[7])));
   m = m_new;
-  // warp-uniform condition: the rescale's TMEM traffic is collective
-  if (have_o && __any_sync(0xffffffffu, corr != 1.f)) {
-#pragma unroll 1
-    for (int c4 = 0; c4 < 4; ++c4) {
-      float o[32];
-      tmem_ld32(O + 32 * c4, o);
-      tmem_wait_ld();
-#pragma unroll
-      for (int u = 0; u < 32; ++u) o[u] *= corr;
-      tmem_st32(O + 32 * c4, o);
-    }
-  }
 }
 
 // One key tile of the online softmax of this thread's query row, on S in

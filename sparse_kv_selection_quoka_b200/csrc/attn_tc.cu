@@ -204,58 +204,61 @@ attn_gather_kernel(const __grid_constant__ AttnMaps maps, const AttnArgs a, int 
     if (bad_index) latch_status(a.status, 6 /* QUOKA_ERR_BOUNDS */);
   } else if (warp == AT_MMA_WARP) {
     // ------------------------------------------------------------ MMA issue
-    if (lane == 0) {
-      const uint32_t q0 = smem_u32(sm.q[0]), q1 = smem_u32(sm.q[1]);
-      const bool v0 = ti[0].valid, v1 = ti[1].valid;
-      auto qk = [&](int w, int s) {
-        issue_qk(tmem + 128u * w, w ? q1 : q0, smem_u32(sm.kv[s][0]));
-        umma_commit(&sm.s_full[w]);
-      };
-      auto pv = [&](int w, int s, bool acc) {
-        issue_pv(tmem + 256u + 128u * w, tmem + 128u * w, smem_u32(sm.kv[s][1]), acc);
-      };
-      int where = 21;
-      bool alive = mbar_wait(&sm.q_full, 0, &sm.abort);
-      for (int it = 0; it < ntiles && alive; ++it) {
-        const int s = it % AT_STAGES;
-        const int sp = (it + AT_STAGES - 1) % AT_STAGES;
-        where = 22;
-        alive = mbar_wait(&sm.kv_full[s], (it / AT_STAGES) & 1, &sm.abort);
-        if (!alive) break;
-        fence_proxy_async_smem();  // the cp.async writes become visible to the tensor core
-        tc_fence_after();
-        if (v0) qk(0, s);
-        if (it > 0) {
-          if (v1) {
-            where = 23;
-            alive = mbar_wait(&sm.p_full[1], (it - 1) & 1, &sm.abort);
-            if (!alive) break;
-            tc_fence_after();
-            pv(1, sp, it - 1 > 0);
-          }
-          umma_commit(&sm.kv_empty[sp]);
-        }
-        if (v1) qk(1, s);
-        if (v0) {
-          where = 24;
-          alive = mbar_wait(&sm.p_full[0], it & 1, &sm.abort);
+    // The whole warp runs this loop in step (waits on every lane, warp-uniform
+    // results); one elected lane issues each MMA and commit.
+    const uint32_t q0 = smem_u32(sm.q[0]), q1 = smem_u32(sm.q[1]);
+    const bool v0 = ti[0].valid, v1 = ti[1].valid;
+    auto qk = [&](int w, int s) {
+      issue_qk(tmem + 128u * w, w ? q1 : q0, smem_u32(sm.kv[s][0]));
+      umma_commit_warp(&sm.s_full[w]);
+    };
+    auto pv = [&](int w, int s, bool acc) {
+      issue_pv(tmem + 256u + 128u * w, tmem + 128u * w, smem_u32(sm.kv[s][1]), acc);
+    };
+    int where = 21;
+    bool alive = mbar_wait_warp(&sm.q_full, 0, &sm.abort);
+    for (int it = 0; it < ntiles && alive; ++it) {
+      const int s = it % AT_STAGES;
+      const int sp = (it + AT_STAGES - 1) % AT_STAGES;
+      where = 22;
+      alive = mbar_wait_warp(&sm.kv_full[s], (it / AT_STAGES) & 1, &sm.abort);
+      if (!alive) break;
+      fence_proxy_async_smem();  // the cp.async writes become visible to the tensor core
+      tc_fence_after();
+      if (v0) qk(0, s);
+      if (it > 0) {
+        if (v1) {
+          where = 23;
+          alive = mbar_wait_warp(&sm.p_full[1], (it - 1) & 1, &sm.abort);
           if (!alive) break;
           tc_fence_after();
-          pv(0, s, it > 0);
+          pv(1, sp, it - 1 > 0);
         }
+        umma_commit_warp(&sm.kv_empty[sp]);
       }
-      if (alive && ntiles > 0 && v1) {
-        where = 25;
-        alive = mbar_wait(&sm.p_full[1], (ntiles - 1) & 1, &sm.abort);
-        if (alive) {
-          tc_fence_after();
-          pv(1, (ntiles - 1) % AT_STAGES, ntiles - 1 > 0);
-        }
+      if (v1) qk(1, s);
+      if (v0) {
+        where = 24;
+        alive = mbar_wait_warp(&sm.p_full[0], it & 1, &sm.abort);
+        if (!alive) break;
+        tc_fence_after();
+        pv(0, s, it > 0);
       }
-      if (!alive) record_abort(sm, a.status, where);
-      umma_commit(&sm.o_final);
-      umma_commit(&sm.mma_done);
-      if (!mbar_drain(&sm.mma_done, 0)) record_abort(sm, a.status, 26);
+    }
+    if (alive && ntiles > 0 && v1) {
+      where = 25;
+      alive = mbar_wait_warp(&sm.p_full[1], (ntiles - 1) & 1, &sm.abort);
+      if (alive) {
+        tc_fence_after();
+        pv(1, (ntiles - 1) % AT_STAGES, ntiles - 1 > 0);
+      }
+    }
+    if (!alive && lane == 0) record_abort(sm, a.status, where);
+    umma_commit_warp(&sm.o_final);
+    umma_commit_warp(&sm.mma_done);
+    const bool drained = __all_sync(0xffffffffu, mbar_drain(&sm.mma_done, 0));
+    if (lane == 0) {
+      if (!drained) record_abort(sm, a.status, 26);
       // rank 0: every MMA is done, so its K/V ring and Q area may now take
       // rank 1's partial results
       if (nsplit > 1 && split == 0) mbar_arrive_remote(mapa_shared(smem_u32(&sm.xfer_free), 1));

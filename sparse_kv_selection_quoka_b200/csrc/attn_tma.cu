@@ -61,6 +61,8 @@ constexpr int VLOAD_WARP = 10;
 // Measured on B200 (Qwen-shaped layer): 0 and 2 run equally fast, more is
 // slower; 0 keeps the kernel free of register spills.
 constexpr int SOFTMAX_FMA_PAIRS = 0;
+// P of a tile is released to the P V product in this many key ranges.
+constexpr int PV_PARTS = 2;
 // split-KV payload of one query tile: partial O (fp32, 128 rows x 128, each
 // row's 16-byte chunks rotated by the row index) followed by (m, l) per row;
 // staged at OUT_OFF of the K/V span, received at IN_OFF
@@ -81,7 +83,7 @@ struct __align__(1024) Smem {
   uint64_t q_full;
   uint64_t k_full[KST], k_empty[KST];
   uint64_t v_full[VST], v_empty[VST];
-  uint64_t s_full[2], p_full[2];
+  uint64_t s_full[2], p_part[2][PV_PARTS];
   uint64_t o_final, mma_done;
   uint64_t xfer_free;  // the peer's landing zone is free (its MMAs are done)
   uint64_t xfer_full;  // the peer's partial of this rank's tile has landed
@@ -165,7 +167,7 @@ attn_tma_kernel(const __grid_constant__ Maps maps, const AttnArgs a, int nsplit)
     }
     for (int w = 0; w < 2; ++w) {
       mbar_init(&sm.s_full[w], 1);
-      mbar_init(&sm.p_full[w], 128);
+      for (int c = 0; c < PV_PARTS; ++c) mbar_init(&sm.p_part[w][c], 4);  // one arrival per warp
     }
     mbar_init(&sm.o_final, 1);
     mbar_init(&sm.mma_done, 1);
@@ -222,55 +224,60 @@ attn_tma_kernel(const __grid_constant__ Maps maps, const AttnArgs a, int nsplit)
     __syncwarp();
   } else if (warp == MMA_WARP) {
     // ------------------------------------------------------------ MMA issue
-    if (lane == 0) {
-      const uint32_t q0 = smem_u32(sm.q[0]), q1 = smem_u32(sm.q[1]);
-      const bool v1 = ti[1].valid;
-      int where = 21;
-      bool alive = mbar_wait(&sm.q_full, 0, &sm.abort);
-      for (int it = 0; it < ntiles && alive; ++it) {
-        const int ks = it % KST, vs = it % VST, vp = (it + VST - 1) % VST;
-        where = 22;
-        alive = mbar_wait(&sm.k_full[ks], (it / KST) & 1, &sm.abort);
-        if (!alive) break;
+    // The whole warp runs this loop in step (waits on every lane, warp-uniform
+    // results); one elected lane issues each MMA and commit.
+    const uint32_t q0 = smem_u32(sm.q[0]), q1 = smem_u32(sm.q[1]);
+    const bool v1 = ti[1].valid;
+    int where = 21;
+    // O_w (+)= P_w V for the tile whose P parts complete phase `ph`, each
+    // part issued as soon as the softmax releases it
+    auto pv = [&](int w, uint32_t v_smem, int ph, bool accumulate) -> bool {
+      for (int c = 0; c < PV_PARTS; ++c) {
+        if (!mbar_wait_warp(&sm.p_part[w][c], ph, &sm.abort)) return false;
         tc_fence_after();
-        issue_qk(tmem, q0, smem_u32(sm.k[ks]));
-        umma_commit(&sm.s_full[0]);
-        if (it > 0) {
-          if (v1) {
-            where = 23;
-            alive = mbar_wait(&sm.p_full[1], (it - 1) & 1, &sm.abort);
-            if (!alive) break;
-            tc_fence_after();
-            issue_pv(tmem + 384u, tmem + 128u, smem_u32(sm.v[vp]), it - 1 > 0);
-          }
-          umma_commit(&sm.v_empty[vp]);
-        }
+        issue_pv_part<PV_PARTS>(tmem + 256u + 128u * w, tmem + 128u * w, v_smem, c, accumulate);
+      }
+      return true;
+    };
+    bool alive = mbar_wait_warp(&sm.q_full, 0, &sm.abort);
+    for (int it = 0; it < ntiles && alive; ++it) {
+      const int ks = it % KST, vs = it % VST, vp = (it + VST - 1) % VST;
+      where = 22;
+      alive = mbar_wait_warp(&sm.k_full[ks], (it / KST) & 1, &sm.abort);
+      if (!alive) break;
+      tc_fence_after();
+      issue_qk(tmem, q0, smem_u32(sm.k[ks]));
+      umma_commit_warp(&sm.s_full[0]);
+      if (it > 0) {
         if (v1) {
-          issue_qk(tmem + 128u, q1, smem_u32(sm.k[ks]));
-          umma_commit(&sm.s_full[1]);
+          where = 23;
+          alive = pv(1, smem_u32(sm.v[vp]), (it - 1) & 1, it - 1 > 0);
+          if (!alive) break;
         }
-        umma_commit(&sm.k_empty[ks]);
-        where = 24;
-        alive = mbar_wait(&sm.v_full[vs], (it / VST) & 1, &sm.abort);
-        if (!alive) break;
-        where = 25;
-        alive = mbar_wait(&sm.p_full[0], it & 1, &sm.abort);
-        if (!alive) break;
-        tc_fence_after();
-        issue_pv(tmem + 256u, tmem, smem_u32(sm.v[vs]), it > 0);
+        umma_commit_warp(&sm.v_empty[vp]);
       }
-      if (alive && ntiles > 0 && v1) {
-        where = 26;
-        alive = mbar_wait(&sm.p_full[1], (ntiles - 1) & 1, &sm.abort);
-        if (alive) {
-          tc_fence_after();
-          issue_pv(tmem + 384u, tmem + 128u, smem_u32(sm.v[(ntiles - 1) % VST]), ntiles - 1 > 0);
-        }
+      if (v1) {
+        issue_qk(tmem + 128u, q1, smem_u32(sm.k[ks]));
+        umma_commit_warp(&sm.s_full[1]);
       }
-      if (!alive) record_abort(sm, a.status, where);
-      umma_commit(&sm.o_final);
-      umma_commit(&sm.mma_done);
-      if (!mbar_drain(&sm.mma_done, 0)) record_abort(sm, a.status, 27);
+      umma_commit_warp(&sm.k_empty[ks]);
+      where = 24;
+      alive = mbar_wait_warp(&sm.v_full[vs], (it / VST) & 1, &sm.abort);
+      if (!alive) break;
+      where = 25;
+      alive = pv(0, smem_u32(sm.v[vs]), it & 1, it > 0);
+      if (!alive) break;
+    }
+    if (alive && ntiles > 0 && v1) {
+      where = 26;
+      alive = pv(1, smem_u32(sm.v[(ntiles - 1) % VST]), (ntiles - 1) & 1, ntiles - 1 > 0);
+    }
+    if (!alive && lane == 0) record_abort(sm, a.status, where);
+    umma_commit_warp(&sm.o_final);
+    umma_commit_warp(&sm.mma_done);
+    const bool drained = __all_sync(0xffffffffu, mbar_drain(&sm.mma_done, 0));
+    if (lane == 0) {
+      if (!drained) record_abort(sm, a.status, 27);
       // every MMA is done (and every load they waited for has landed), so
       // this rank's K/V span may now take the peer's payload
       if (nsplit > 1) mbar_arrive_remote(mapa_shared(smem_u32(&sm.xfer_free), (uint32_t)(split ^ 1)));
@@ -299,10 +306,7 @@ attn_tma_kernel(const __grid_constant__ Maps maps, const AttnArgs a, int nsplit)
       // key at a position p < nchunk with p <= t
       const int base_n = (sel_tile ? gi : gi - ntile_sel) * N;
       const int lim = sel_tile ? nsel : min(nchunk, t + 1);
-      softmax_tile_1p<SOFTMAX_FMA_PAIRS>(S, O, it > 0, base_n, lim, qscale, m, l);
-      tmem_wait_st();
-      tc_fence_before();
-      mbar_arrive(&sm.p_full[w]);
+      softmax_tile_split<SOFTMAX_FMA_PAIRS, PV_PARTS>(S, O, it > 0, base_n, lim, qscale, m, l, sm.p_part[w]);
     }
 
     // ------------------------------------------------ epilogue / combine

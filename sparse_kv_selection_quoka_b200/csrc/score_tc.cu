@@ -180,36 +180,37 @@ score_tc_kernel(const __grid_constant__ CUtensorMap tmap, const ScoreArgs a) {
     // (the producer ran above)
   } else if (warp == 1) {
     // ------------------------------------------------------------ MMA issue
-    if (lane == 0) {
-      const uint32_t idesc = idesc_bf16_f32(SC_KEYS, N, 0, 0);
-      const uint32_t qg = smem_u32(qg_s);
-      bool alive = true;
-      int where = 0;
-      const int NE = a.nepi;
-      for (int it = 0; it < n && alive; ++it) {
-        const int s = it % NS, acc = it % NE;
-        where = 52;
-        alive = mbar_wait(&sb.full[s], (it / NS) & 1, &sb.abort);
-        if (alive && it >= NE) {
-          where = 53;
-          alive = mbar_wait(&sb.tempty[acc], ((it / NE) - 1) & 1, &sb.abort);
-        }
-        if (!alive) break;
-        tc_fence_after();
-        const uint32_t ks = smem_u32(ring + (size_t)s * SC_TILE_BYTES);
-        const uint32_t d = tmem + (uint32_t)(acc * ACC);
-#pragma unroll
-        for (int kk = 0; kk < SC_D / 16; ++kk) {
-          const uint64_t ad = sw128_desc(ks + (kk >> 2) * SC_ATOM + (kk & 3) * 32, 16, 1024);
-          const uint64_t bd = sw128_desc(qg + (kk >> 2) * (N * 128) + (kk & 3) * 32, 16, 1024);
-          umma_bf16_ss(d, ad, bd, idesc, kk > 0 ? 1u : 0u);
-        }
-        umma_commit(&sb.tfull[acc]);
+    // The whole warp runs this loop in step (waits on every lane, warp-uniform
+    // results); one elected lane issues each MMA and commit.
+    const uint32_t idesc = idesc_bf16_f32(SC_KEYS, N, 0, 0);
+    const uint32_t qg = smem_u32(qg_s);
+    bool alive = true;
+    int where = 0;
+    const int NE = a.nepi;
+    for (int it = 0; it < n && alive; ++it) {
+      const int s = it % NS, acc = it % NE;
+      where = 52;
+      alive = mbar_wait_warp(&sb.full[s], (it / NS) & 1, &sb.abort);
+      if (alive && it >= NE) {
+        where = 53;
+        alive = mbar_wait_warp(&sb.tempty[acc], ((it / NE) - 1) & 1, &sb.abort);
       }
-      if (!alive) sc_abort(sb, a.status, where);
-      umma_commit(&sb.done);
-      if (!mbar_drain(&sb.done, 0)) sc_abort(sb, a.status, 54);
+      if (!alive) break;
+      tc_fence_after();
+      const uint32_t ks = smem_u32(ring + (size_t)s * SC_TILE_BYTES);
+      const uint32_t d = tmem + (uint32_t)(acc * ACC);
+#pragma unroll
+      for (int kk = 0; kk < SC_D / 16; ++kk) {
+        const uint64_t ad = sw128_desc(ks + (kk >> 2) * SC_ATOM + (kk & 3) * 32, 16, 1024);
+        const uint64_t bd = sw128_desc(qg + (kk >> 2) * (N * 128) + (kk & 3) * 32, 16, 1024);
+        umma_bf16_ss_warp(d, ad, bd, idesc, kk > 0 ? 1u : 0u);
+      }
+      umma_commit_warp(&sb.tfull[acc]);
     }
+    if (!alive && lane == 0) sc_abort(sb, a.status, where);
+    umma_commit_warp(&sb.done);
+    const bool drained = __all_sync(0xffffffffu, mbar_drain(&sb.done, 0));
+    if (!drained && lane == 0) sc_abort(sb, a.status, 54);
     __syncwarp();
   } else {
     // ------------------------------------------------------------ epilogue
