@@ -5,15 +5,21 @@
 
 A step is one pass of the whole hot path -- (a) mean query and SQ, (b) top-NQ
 queries, (c) normalise + group mean, (d) cosine score + max, (e) top-BSA keys,
-(f)+(g) fused gather + sparse GQA attention -- over one chunk of synthetic
-input resident in HBM. The default workload is the Qwen3-4B-shaped layer at
+(f) gather of the selected rows, (g) sparse GQA attention -- over one chunk
+of synthetic input resident in HBM. The default workload is the Qwen3-4B-shaped layer at
 T = 32768 prior keys (b=1, nq=32, nkv=8, d=128, BCP=512, NQ=32, BSA=4096).
 
 Timing: W warm-up steps, then exactly K timed steps bracketed by a barrier and
 a device synchronisation; before every timed step the L2 is flushed by writing
 a 256 MiB buffer (outside the timed events); each step is timed with CUDA
-events on the launching stream; under torchrun the maximum over ranks is
-reported. Rank 0 prints one JSON line.
+events on the launching stream, placed only at the step's two ends; the step
+is quoka_prefill_chunk (the whole path in one C-ABI call, its kernels
+overlapping at their edges through programmatic dependent launch, as they
+do for a user); under torchrun the maximum over ranks is reported. A second
+pass of K steps runs the same kernels through the three part calls
+(quoka_select | quoka_gather_kv | quoka_sparse_gqa_attn_gathered) with an
+event at every boundary, for the breakdown (ms_select, ms_gather,
+ms_attention) and the rooflines. Rank 0 prints one JSON line.
 
 --impl reference times the CPU oracle (numpy float64) on the host cores
 instead, on a bounded per-step sample of the same workload (one KV head's
@@ -216,9 +222,17 @@ def run_ours(args, rank, world, local_rank):
             evs[1].record(stream)
         q.quoka_sparse_gqa_attn_gathered(Qv, Ks, Vs, cnt, Kcv, Vcv, O=Ob, ws=wsb, stream=stream)
 
+    def whole_chunk(ch):
+        """Steps (a)-(g) as one call, quoka_prefill_chunk: the same kernels as
+        one_chunk, chained on the stream with no event in between."""
+        (Qv, Kv, Vv, Kcv, Vcv), bsa, wsb, Ob, idx, _, _, _ = ch
+        q.quoka_prefill_chunk(Qv, Kv, Vv, Kcv, Vcv, w.NQ, bsa, O=Ob, kv_idx=idx,
+                              ws=wsb, stream=stream)
+
     for _ in range(args.warmup):
         for ch in chunks:
             one_chunk(ch)
+            whole_chunk(ch)
     torch.cuda.synchronize()
     status = q.quoka_get_device_status(chunks[-1][2])
     if status != 0:
@@ -235,8 +249,28 @@ def run_ours(args, rank, world, local_rank):
         torch.distributed.barrier()
     torch.cuda.synchronize()
     n_ev = len(chunks)
-    t_step, t_sel, t_gather, t_attn = 0.0, 0.0, 0.0, 0.0
+    # The step: quoka_prefill_chunk per chunk with events only at the step's
+    # two ends, so the kernels overlap at their edges as they do for a user
+    # (programmatic dependent launch within the call).
+    t_step = 0.0
     per_chunk = [0.0] * n_ev
+    step_evs = []
+    for _ in range(args.steps):
+        flush.fill_(1)
+        e = [torch.cuda.Event(enable_timing=True) for _ in range(2)]
+        e[0].record(stream)
+        for ch in chunks:
+            whole_chunk(ch)
+        e[1].record(stream)
+        step_evs.append(e)
+    torch.cuda.synchronize()
+    for e in step_evs:
+        t_step += e[0].elapsed_time(e[1])
+    # The parts, timed in a second pass with an event at every boundary
+    # (which serialises the parts): select (a)-(e), gather (f), attention (g).
+    if world > 1:
+        torch.distributed.barrier()
+    t_sel, t_gather, t_attn = 0.0, 0.0, 0.0
     evs = []
     for _ in range(args.steps):
         flush.fill_(1)
@@ -257,7 +291,6 @@ def run_ours(args, rank, world, local_rank):
             t_sel += a
             t_gather += g
             t_attn += bms
-            t_step += a + g + bms
             per_chunk[c] += a + g + bms
     clocks = sampler.stop()
 

@@ -88,7 +88,7 @@ gather_kernel(const char* __restrict__ K, int64_t sKb, int64_t sKh, int64_t sKt,
 
 cudaError_t launch_gather(bool is_bf16, int d, Strided K, Strided V, int b, int nkv, int64_t T,
                           const int32_t* kv_idx, const int32_t* kv_count, int bsa, void* Ksel,
-                          void* Vsel, int* status, cudaStream_t stream) {
+                          void* Vsel, int* status, bool pdl, cudaStream_t stream) {
   if (bsa == 0) return cudaSuccess;
   const int es = is_bf16 ? 2 : 4;
   const int row_bytes = d * es;  // 128, 256 or 512
@@ -98,11 +98,21 @@ cudaError_t launch_gather(bool is_bf16, int d, Strided K, Strided V, int b, int 
   const int64_t nitems = (int64_t)bsa << cpr_log2;
   const int64_t per_block = (int64_t)kThreads * kItems;
   dim3 grid((unsigned)((nitems + per_block - 1) / per_block), nkv, b);
-  gather_kernel<<<grid, kThreads, 0, stream>>>(
-      static_cast<const char*>(K.data), K.sb * es, K.sh * es, K.st * es,
-      static_cast<const char*>(V.data), V.sb * es, V.sh * es, V.st * es, T, kv_idx, kv_count, bsa,
-      cpr_log2, static_cast<char*>(Ksel), static_cast<char*>(Vsel), status);
-  return cudaGetLastError();
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = grid;
+  cfg.blockDim = dim3(kThreads);
+  cfg.stream = stream;
+  // the kernel reads nothing before its grid-dependency wait, so it may be
+  // launched while its predecessor finishes
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = pdl ? 1 : 0;
+  return cudaLaunchKernelEx(&cfg, gather_kernel, static_cast<const char*>(K.data), K.sb * es, K.sh * es,
+                            K.st * es, static_cast<const char*>(V.data), V.sb * es, V.sh * es, V.st * es, T,
+                            kv_idx, kv_count, bsa, cpr_log2, static_cast<char*>(Ksel), static_cast<char*>(Vsel),
+                            status);
 }
 
 }  // namespace quoka

@@ -68,7 +68,7 @@ cudaError_t launch_topk(const float* S_agg, int b, int nkv, int64_t T, int bsa,
 // as zeros.
 cudaError_t launch_gather(bool bf16, int d, Strided K, Strided V, int b, int nkv, int64_t T,
                           const int32_t* kv_idx, const int32_t* kv_count, int bsa,
-                          void* Ksel, void* Vsel, int* status, cudaStream_t stream);
+                          void* Ksel, void* Vsel, int* status, bool pdl, cudaStream_t stream);
 
 struct AttnArgs {
   Strided Q, K, V, Kc, Vc;

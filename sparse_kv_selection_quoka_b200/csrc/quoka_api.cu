@@ -279,7 +279,8 @@ quoka_status gather_then_attn(const quoka_tensor* Q, const quoka_tensor* K, cons
     return run_attn(Q, strided(K), strided(V), Kc, Vc, s, s.T, kv_idx, kv_count, bsa_eff, scale, O, lse,
                     status, stream);
   cudaError_t e = quoka::launch_gather(Q->dtype == QUOKA_BF16, (int)s.d, strided(K), strided(V), (int)s.b,
-                                       (int)s.nkv, s.T, kv_idx, kv_count, bsa_eff, ksel, vsel, status, stream);
+                                       (int)s.nkv, s.T, kv_idx, kv_count, bsa_eff, ksel, vsel, status, true,
+                                       stream);
   if (e != cudaSuccess) return cuda_status(e);
   const int64_t sh = (int64_t)bsa_eff * s.d, sb = s.nkv * sh;
   // the attention may launch while the gather finishes (it waits for it)
@@ -351,7 +352,7 @@ quoka_status quoka_gather_kv(const quoka_tensor* K, const quoka_tensor* V, const
   }
   cudaError_t e = quoka::launch_gather(K->dtype == QUOKA_BF16, (int)ks[3], strided(K), strided(V),
                                        (int)ks[0], (int)ks[1], ks[2], kv_idx, kv_count, BSA_eff, Ksel,
-                                       Vsel, status, cs);
+                                       Vsel, status, true, cs);
   return cuda_status(e);
 }
 
@@ -399,7 +400,7 @@ quoka_status quoka_sparse_gqa_attn_gathered(const quoka_tensor* Q, const quoka_t
   if (cudaMemsetAsync(status, 0, 2 * sizeof(int), cs) != cudaSuccess) return QUOKA_ERR_CUDA;
   // the rows of Ksel / Vsel are the selected keys in list order: BSA_eff = T
   return run_attn(Q, strided(Ksel), strided(Vsel), Kc, Vc, s, s.T, nullptr, kv_count, (int)s.T, scale, O,
-                  lse, status, cs);
+                  lse, status, cs, true);
 }
 
 quoka_status quoka_prefill_chunk(const quoka_tensor* Q, const quoka_tensor* K,
