@@ -134,27 +134,15 @@ attn_tma_kernel(const __grid_constant__ Maps maps, const AttnArgs a, int nsplit)
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int j = blockIdx.y, bi = blockIdx.z;
-  pdl_wait();  // the gathered rows and their counts come from the previous kernel
   const int G = a.nq / a.nkv;
   const int split = nsplit > 1 ? (int)cluster_ctarank() : 0;
   const int pair = blockIdx.x / nsplit;
   const int ntt = (a.BCP + 127) / 128;  // row tiles per query head
   TileInfo ti[2];
   pair_tiles(pair, j, G, ntt, ti);      // ti[0] is always valid
-  const int64_t kvrow = (int64_t)bi * a.nkv + j;
-  const int nsel = a.bsa > 0 ? max(0, min(__ldcg(a.kv_count + kvrow), a.bsa)) : 0;
-  const int max_t0 = ti[1].valid ? max(ti[0].t0, ti[1].t0) : ti[0].t0;
-  const int nchunk = min(a.BCP, max_t0 + 128);
-  const int ntile_sel = (nsel + N - 1) / N;
-  const int ntile_chk = (nchunk + N - 1) / N;
-  const int nT = ntile_sel + ntile_chk;
-  // split: the ranks take halves of the key tiles (each finalises one query
-  // tile and waits for the other's partial of it, so an uneven split would
-  // only make the longer rank longer)
-  const int n0 = nsplit > 1 ? (nT + 1) / 2 : nT;
-  const int first = split == 0 ? 0 : n0;
-  const int ntiles = split == 0 ? n0 : nT - n0;  // key tiles of this CTA (may be 0)
 
+  // Setup and the Q loads touch nothing the previous kernel writes: they run
+  // before the grid-dependency wait, overlapping that kernel's tail.
   if (tid == 0) {
     mbar_init(&sm.q_full, 1);
     for (int s = 0; s < KST; ++s) {
@@ -193,21 +181,38 @@ attn_tma_kernel(const __grid_constant__ Maps maps, const AttnArgs a, int nsplit)
   }
   tc_fence_after();
   const uint32_t tmem = sm.tmem_base;
+  if (warp == KLOAD_WARP && lane == 0) {
+    tma_prefetch_desc(&maps.q);
+    tma_prefetch_desc(&maps.ks);
+    tma_prefetch_desc(&maps.kc);
+    tma_prefetch_desc(&maps.o);
+    mbar_arrive_expect_tx(&sm.q_full, (ti[1].valid ? 2 : 1) * TILE_BYTES);
+    for (int w = 0; w < 2; ++w) {
+      if (!ti[w].valid) continue;
+      const uint32_t q_s = smem_u32(sm.q[w]);
+      tma_load_4d(q_s, &maps.q, &sm.q_full, 0, ti[w].t0, ti[w].h, bi);
+      tma_load_4d(q_s + ATOM_BYTES, &maps.q, &sm.q_full, 64, ti[w].t0, ti[w].h, bi);
+    }
+  }
+
+  pdl_wait();  // the gathered rows and their counts come from the previous kernel
+  const int64_t kvrow = (int64_t)bi * a.nkv + j;
+  const int nsel = a.bsa > 0 ? max(0, min(__ldcg(a.kv_count + kvrow), a.bsa)) : 0;
+  const int max_t0 = ti[1].valid ? max(ti[0].t0, ti[1].t0) : ti[0].t0;
+  const int nchunk = min(a.BCP, max_t0 + 128);
+  const int ntile_sel = (nsel + N - 1) / N;
+  const int ntile_chk = (nchunk + N - 1) / N;
+  const int nT = ntile_sel + ntile_chk;
+  // split: the ranks take halves of the key tiles (each finalises one query
+  // tile and waits for the other's partial of it, so an uneven split would
+  // only make the longer rank longer)
+  const int n0 = nsplit > 1 ? (nT + 1) / 2 : nT;
+  const int first = split == 0 ? 0 : n0;
+  const int ntiles = split == 0 ? n0 : nT - n0;  // key tiles of this CTA (may be 0)
 
   if (warp == KLOAD_WARP) {
-    // ------------------------------------------------------------ Q, K loads
+    // ------------------------------------------------------------ K loads
     if (lane == 0) {
-      tma_prefetch_desc(&maps.q);
-      tma_prefetch_desc(&maps.ks);
-      tma_prefetch_desc(&maps.kc);
-      tma_prefetch_desc(&maps.o);
-      mbar_arrive_expect_tx(&sm.q_full, (ti[1].valid ? 2 : 1) * TILE_BYTES);
-      for (int w = 0; w < 2; ++w) {
-        if (!ti[w].valid) continue;
-        const uint32_t q_s = smem_u32(sm.q[w]);
-        tma_load_4d(q_s, &maps.q, &sm.q_full, 0, ti[w].t0, ti[w].h, bi);
-        tma_load_4d(q_s + ATOM_BYTES, &maps.q, &sm.q_full, 64, ti[w].t0, ti[w].h, bi);
-      }
       load_ring<KST>(sm, sm.k, sm.k_full, sm.k_empty, &maps.ks, &maps.kc, first, ntiles, ntile_sel, j, bi,
                      a.status, 11);
       if (!mbar_drain(&sm.q_full, 0)) record_abort(sm, a.status, 13);
