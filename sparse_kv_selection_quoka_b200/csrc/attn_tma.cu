@@ -428,7 +428,7 @@ attn_tma_kernel(const __grid_constant__ Maps maps, const AttnArgs a, int nsplit)
         tma_store_4d(&maps.o, smem_u32(ot), 0, ti[w].t0, ti[w].h, bi);
         tma_store_4d(&maps.o, smem_u32(ot) + ATOM_BYTES, 64, ti[w].t0, ti[w].h, bi);
         bulk_commit_group();
-        bulk_wait_group_0();
+        bulk_wait_group_read_0();  // the staging may go once the copy has read it
       }
     }
   }

@@ -332,8 +332,12 @@ __device__ __forceinline__ void tma_store_4d(const void* tmap, uint32_t src, int
 
 __device__ __forceinline__ void bulk_commit_group() { asm volatile("cp.async.bulk.commit_group;" ::: "memory"); }
 
-// Waits until every committed bulk group of this thread has completed.
-__device__ __forceinline__ void bulk_wait_group_0() { asm volatile("cp.async.bulk.wait_group 0;" ::: "memory"); }
+// Waits until every committed bulk group of this thread has finished reading
+// its shared-memory source (the writes themselves complete with the grid):
+// enough before the CTA exits or the source is reused.
+__device__ __forceinline__ void bulk_wait_group_read_0() {
+  asm volatile("cp.async.bulk.wait_group.read 0;" ::: "memory");
+}
 
 // Bulk copy of `bytes` (a multiple of 16) from this CTA's shared memory to
 // the shared memory of a CTA of the cluster (cluster addresses from mapa);
