@@ -50,8 +50,13 @@ def run_select_and_check(x: inputs.ChunkInputs, dev=None):
         ref = orc.select(x.Q, x.K, x.NQ, x.BSA, override_q_idx=gq)
     T = x.K.shape[2]
     if T > 0:
-        err = np.abs(s_agg.cpu().numpy().astype(np.float64) - ref["S_agg"]).max()
-        assert err <= P.S_TOL, f"S_agg max-abs error {err:.3e}"
+        sg = s_agg.cpu().numpy().astype(np.float64)
+        dif = np.abs(sg - ref["S_agg"])
+        err = dif.max()
+        at = np.unravel_index(int(dif.argmax()), dif.shape)
+        assert err <= P.S_TOL, (f"S_agg max-abs error {err:.3e} at {tuple(int(v) for v in at)}: got "
+                                f"{sg[at]:.6f}, want {ref['S_agg'][at]:.6f}; {int((dif > P.S_TOL).sum())} "
+                                f"entries out of tolerance")
     bsa_eff = min(x.BSA, T)
     gi = kv_idx.cpu().numpy().astype(np.int64)
     gc = kv_count.cpu().numpy()
