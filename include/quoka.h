@@ -108,6 +108,26 @@ quoka_status quoka_select(const quoka_tensor* Q, const quoka_tensor* K, int NQ,
                           int32_t* q_idx, float* s_agg, void* ws,
                           size_t ws_bytes, void* stream);
 
+/* Score variants of quoka_select_ex (bit flags). */
+#define QUOKA_SCORE_DOT_PRODUCT 1u
+
+/* quoka_select with score variants. flags = 0 is quoka_select exactly.
+ * QUOKA_SCORE_DOT_PRODUCT: the ablation the write-up compares the cosine
+ * score against ([QUOKA §2.2], "standard dot-product attention", its Table
+ * 9): the chosen queries are not L2-normalised before the group mean, the
+ * keys are not normalised, and S_agg[j, tau] = max_i Q_group[j, i] . K[tau]
+ * with Q_group the mean over the G heads of the raw chosen queries. The
+ * query choice (steps (a), (b)) is the same. S_agg is then unbounded; the
+ * top-k (same ties and output format) runs without the scoring kernel's
+ * value-bucket histogram.
+ * Other flag bits are rejected with QUOKA_ERR_INVALID_ARG. Arguments
+ * otherwise as quoka_select. */
+quoka_status quoka_select_ex(const quoka_tensor* Q, const quoka_tensor* K,
+                             int NQ, int BSA, int32_t* kv_idx,
+                             int32_t* kv_count, int32_t* q_idx, float* s_agg,
+                             uint32_t flags, void* ws, size_t ws_bytes,
+                             void* stream);
+
 /* Size of the fixed device scratch array behind quoka_select_static. */
 #define QUOKA_STATIC_SCRATCH_BYTES (8u << 20)
 

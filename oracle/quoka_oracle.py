@@ -17,6 +17,9 @@ efficiency" (bqwf.cn, news item 915859), cited below as [QUOKA §x]:
          matmul, take the max over the chosen queries, keep the top-BSA keys
   §4.2   the selected KV is handed to FlashAttention as its input KV with the
          causal mask switched off for it (problem 3)
+  §2.2   also: the cosine score is compared against the standard dot-product
+         score (its Table 9); the dot_product=True variant below drops both
+         L2 normalisations (chosen queries and keys) and keeps everything else
 
 Readings where the article is silent or garbled (each is listed in the design
 notes too):
@@ -121,9 +124,10 @@ def select_queries(SQ, NQ: int) -> np.ndarray:
 # [QUOKA §2.3: Q_norm = Q / norm(Q), Q_group = mean over the group axis]
 # ---------------------------------------------------------------------------
 
-def group_queries(Q, q_idx, nkv: int) -> np.ndarray:
+def group_queries(Q, q_idx, nkv: int, normalize: bool = True) -> np.ndarray:
     """Q_group[b, j, i] = (1/G) sum_g Q[b, jG+g, q_idx[b, jG+g, i]] / |.|
-       -> (b, nkv, NQ, d)."""
+       -> (b, nkv, NQ, d). normalize=False: the raw chosen queries are
+       averaged (the dot-product variant)."""
     Q = _f64(Q)
     b, nq, L, d = Q.shape
     if nq % nkv:
@@ -138,7 +142,7 @@ def group_queries(Q, q_idx, nkv: int) -> np.ndarray:
                 for g in range(G):
                     h = j * G + g
                     q = Q[bi, h, q_idx[bi, h, i]]
-                    acc += q / np.sqrt(np.dot(q, q))
+                    acc += q / np.sqrt(np.dot(q, q)) if normalize else q
                 out[bi, j, i] = acc / G
     return out
 
@@ -148,16 +152,17 @@ def group_queries(Q, q_idx, nkv: int) -> np.ndarray:
 # [QUOKA §2.2 cosine score; §2.3 S = Q_group K_norm^T, S_agg = max over NQ]
 # ---------------------------------------------------------------------------
 
-def key_scores(Q_group, K) -> np.ndarray:
+def key_scores(Q_group, K, normalize: bool = True) -> np.ndarray:
     """S_agg[b, j, tau] = max_i Q_group[b, j, i] . K[b, j, tau] / |K[b, j, tau]|
-       -> (b, nkv, T)."""
+       -> (b, nkv, T). normalize=False: the plain dot product with K (the
+       dot-product variant)."""
     Qg = _f64(Q_group)
     b, nkv, T, d = K.shape
     out = np.empty((b, nkv, T))
     for bi in range(b):
         for j in range(nkv):
             Kh = _f64(K[bi, j])           # one head at a time bounds memory
-            Kn = Kh / np.linalg.norm(Kh, axis=1, keepdims=True)
+            Kn = Kh / np.linalg.norm(Kh, axis=1, keepdims=True) if normalize else Kh
             S = Qg[bi, j] @ Kn.T          # (NQ, T), the library matmul
             out[bi, j] = S.max(axis=0)
     return out
@@ -242,17 +247,20 @@ def sparse_attention(Q, K, V, sel, Kc, Vc, scale: Optional[float] = None):
 # Whole step
 # ---------------------------------------------------------------------------
 
-def select(Q, K, NQ: int, BSA: int, *, override_q_idx=None):
+def select(Q, K, NQ: int, BSA: int, *, override_q_idx=None, dot_product: bool = False):
     """Steps (a)-(e). Returns a dict with SQ, q_idx, Q_group, S_agg, sel.
 
     override_q_idx replaces the top-NQ choice (to check the later steps alone
-    on another implementation's choice of queries)."""
+    on another implementation's choice of queries). dot_product=True scores
+    with the plain dot product: no L2 normalisation of the chosen queries in
+    step (c) nor of the keys in step (d) ([QUOKA §2.2], the comparison of its
+    Table 9); steps (a), (b) and (e) are unchanged."""
     Q = _f64(Q)
     nkv = K.shape[1]
     SQ = query_scores(Q)
     q_idx = select_queries(SQ, NQ) if override_q_idx is None else np.asarray(override_q_idx, dtype=np.int64)
-    Qg = group_queries(Q, q_idx, nkv)
-    S_agg = key_scores(Qg, K)
+    Qg = group_queries(Q, q_idx, nkv, normalize=not dot_product)
+    S_agg = key_scores(Qg, K, normalize=not dot_product)
     sel = select_keys(S_agg, BSA)
     return {"SQ": SQ, "q_idx": q_idx, "Q_group": Qg, "S_agg": S_agg, "sel": sel}
 

@@ -40,6 +40,7 @@ EXPORTS = (
     "quoka_select_workspace_size",
     "quoka_attn_workspace_size",
     "quoka_select",
+    "quoka_select_ex",
     "quoka_gather_kv",
     "quoka_sparse_gqa_attn",
     "quoka_sparse_gqa_attn_gathered",
@@ -95,6 +96,8 @@ def load() -> ctypes.CDLL:
         lib.quoka_attn_workspace_size.argtypes = [_I, _I, _I, _I, _I]
         lib.quoka_select.restype = _I
         lib.quoka_select.argtypes = [_T, _T, _I, _I, _P, _P, _P, _P, _P, _SZ, _P]
+        lib.quoka_select_ex.restype = _I
+        lib.quoka_select_ex.argtypes = [_T, _T, _I, _I, _P, _P, _P, _P, ctypes.c_uint32, _P, _SZ, _P]
         lib.quoka_gather_kv.restype = _I
         lib.quoka_gather_kv.argtypes = [_T, _T, _P, _P, _I, _P, _P, _P, _SZ, _P]
         lib.quoka_sparse_gqa_attn.restype = _I
@@ -175,10 +178,15 @@ def workspace_for(Q: torch.Tensor, K: torch.Tensor, NQ: int, BSA: int) -> torch.
     return torch.empty(n, dtype=torch.uint8, device=Q.device)
 
 
+SCORE_DOT_PRODUCT = 1  # quoka_select_ex flag: plain dot-product score
+
+
 def quoka_select(Q, K, NQ: int, BSA: int, *, kv_idx=None, kv_count=None, q_idx=None,
-                 s_agg=None, want_q_idx=False, want_s_agg=False, ws=None, stream=None):
+                 s_agg=None, want_q_idx=False, want_s_agg=False, ws=None, stream=None,
+                 dot_product=False):
     """Steps (a)-(e). Returns (kv_idx (b,nkv,BSA_eff) int32 ascending,
-    kv_count (b,nkv) int32, q_idx or None, s_agg or None)."""
+    kv_count (b,nkv) int32, q_idx or None, s_agg or None). dot_product=True
+    calls quoka_select_ex with the dot-product score variant."""
     lib = load()
     b, nq, BCP, d = Q.shape
     nkv, T = K.shape[1], K.shape[2]
@@ -195,11 +203,16 @@ def quoka_select(Q, K, NQ: int, BSA: int, *, kv_idx=None, kv_count=None, q_idx=N
     if ws is None:
         ws = workspace_for(Q, K, NQ, BSA)
     qv, kv = tensor_view(Q), tensor_view(K)
-    st = lib.quoka_select(ctypes.byref(qv), ctypes.byref(kv), NQ, BSA,
-                          _ptr(kv_idx) if kv_idx.numel() else None, _ptr(kv_count),
-                          _ptr(q_idx), _ptr(s_agg) if s_agg is not None and s_agg.numel() else None,
-                          _ptr(ws), ws.numel(), _stream(stream))
-    _check(st, "quoka_select")
+    outs = (_ptr(kv_idx) if kv_idx.numel() else None, _ptr(kv_count), _ptr(q_idx),
+            _ptr(s_agg) if s_agg is not None and s_agg.numel() else None)
+    if dot_product:
+        st = lib.quoka_select_ex(ctypes.byref(qv), ctypes.byref(kv), NQ, BSA, *outs, SCORE_DOT_PRODUCT,
+                                 _ptr(ws), ws.numel(), _stream(stream))
+        _check(st, "quoka_select_ex")
+    else:
+        st = lib.quoka_select(ctypes.byref(qv), ctypes.byref(kv), NQ, BSA, *outs, _ptr(ws), ws.numel(),
+                              _stream(stream))
+        _check(st, "quoka_select")
     return kv_idx, kv_count, q_idx, s_agg
 
 

@@ -15,10 +15,11 @@ struct Strided {
 };
 
 // Step (a)+(b)+(c, first half): one CTA per (batch, query head). Writes the
-// chosen chunk positions in rank order and the L2-normalised chosen queries
-// Qhat (b, nq, NQ, d) fp32.
+// chosen chunk positions in rank order and the chosen queries Qhat
+// (b, nq, NQ, d) fp32, L2-normalised when `normalize` (the cosine score;
+// raw for the dot-product score).
 cudaError_t launch_qsel(bool bf16, int d, Strided Q, int b, int nq, int BCP, int NQ,
-                        float* Qhat, int32_t* q_idx, cudaStream_t stream);
+                        float* Qhat, int32_t* q_idx, bool normalize, cudaStream_t stream);
 
 // Step (c, second half): Q_group (b, nkv, NQ, d) fp32 = mean over the G
 // heads of each group of Qhat at the same rank; optionally also the bf16
@@ -32,13 +33,16 @@ cudaError_t launch_qgroup(int d, const float* Qhat, int b, int nq, int nkv, int 
 // Steps (a)-(c) fused (query selection and group mean in one kernel) for
 // bf16, d = 128, BCP <= 512, NQ <= 32, G <= 8: writes q_idx (rank order,
 // when not null), Qg and Qg_hilo as launch_qgroup does, and zeroes `hist`
-// when given. Returns cudaErrorNotSupported for other shapes.
+// when given; `normalize` as for launch_qsel. Returns cudaErrorNotSupported
+// for other shapes.
 cudaError_t launch_qsel_group_fast(Strided Q, int b, int nq, int nkv, int BCP, int NQ, int32_t* q_idx,
-                                   float* Qg, uint16_t* Qg_hilo, uint32_t* hist, cudaStream_t stream);
+                                   float* Qg, uint16_t* Qg_hilo, uint32_t* hist, bool normalize,
+                                   cudaStream_t stream);
 
-// Step (d) on the CUDA cores (fp32 arithmetic; any input dtype).
+// Step (d) on the CUDA cores (fp32 arithmetic; any input dtype). key_norm:
+// divide by |k| (cosine score) or not (dot-product score).
 cudaError_t launch_score_simt(bool bf16, int d, Strided K, int b, int nkv, int64_t T,
-                              const float* Qg, int NQ, float* S_agg, cudaStream_t stream);
+                              const float* Qg, int NQ, float* S_agg, bool key_norm, cudaStream_t stream);
 
 // Step (d) on the tcgen05 tensor cores (bf16 K, Q_group as bf16 hi + lo).
 // Also accumulates, per (batch, KV head), the histogram of the scores'
@@ -46,10 +50,12 @@ cudaError_t launch_score_simt(bool bf16, int d, Strided K, int b, int nkv, int64
 // first digit of the top-k select.
 // Returns cudaErrorNotSupported when the shape has no tensor-core variant.
 // pdl: launch with programmatic stream serialisation (the kernel starts its
-// K stream while the previous kernel in the stream still runs).
+// K stream while the previous kernel in the stream still runs). key_norm:
+// divide by |k| (cosine score) or not (dot-product score; the histogram is
+// then of little use and the caller does not hand it to the top-k).
 cudaError_t launch_score_tc(int d, Strided K, int b, int nkv, int64_t T,
                             const uint16_t* Qg_hilo, int NQ, float* S_agg, uint32_t* hist,
-                            int* status, bool pdl, cudaStream_t stream);
+                            int* status, bool pdl, bool key_norm, cudaStream_t stream);
 
 // Step (e): per (batch, KV head) cluster radix select of the BSA_eff
 // largest scores, ties to the lower index, written in ascending key order.

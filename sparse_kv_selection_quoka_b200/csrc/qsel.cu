@@ -28,7 +28,7 @@ constexpr int QSEL_WARPS = QSEL_THREADS / 32;
 template <typename T, int D>
 __global__ void __launch_bounds__(QSEL_THREADS)
 qsel_kernel(const T* __restrict__ Q, int64_t sQb, int64_t sQh, int64_t sQt, int BCP, int NQ,
-            float* __restrict__ Qhat, int32_t* __restrict__ q_idx) {
+            float* __restrict__ Qhat, int32_t* __restrict__ q_idx, int normalize) {
   extern __shared__ float smem[];
   float* SQ = smem;
   int* sel = reinterpret_cast<int*>(smem + BCP);
@@ -107,7 +107,7 @@ qsel_kernel(const T* __restrict__ Q, int64_t sQb, int64_t sQh, int64_t sQt, int 
       qq += v[k] * v[k];
     }
     qq = warp_sum(qq);
-    const float nrm = fmaxf(sqrtf(qq), 1e-12f);
+    const float nrm = normalize ? fmaxf(sqrtf(qq), 1e-12f) : 1.f;
     float* dst = Qhat + (((int64_t)bi * nq + h) * NQ + i) * D;
 #pragma unroll
     for (int k = 0; k < D / 32; ++k) dst[lane + 32 * k] = v[k] / nrm;
@@ -126,7 +126,7 @@ constexpr size_t QSEL_STAGED_MAX_BYTES = 192 * 1024;
 template <typename T, int D>
 __global__ void __launch_bounds__(QSEL_STAGED_THREADS)
 qsel_staged_kernel(const T* __restrict__ Q, int64_t sQb, int64_t sQh, int64_t sQt, int BCP, int NQ,
-                   float* __restrict__ Qhat, int32_t* __restrict__ q_idx) {
+                   float* __restrict__ Qhat, int32_t* __restrict__ q_idx, int normalize) {
   extern __shared__ __align__(16) uint8_t qs_raw[];
   T* blk = reinterpret_cast<T*>(qs_raw);
   const size_t blk_bytes = ((size_t)BCP * D * sizeof(T) + 15) & ~size_t(15);
@@ -216,7 +216,7 @@ qsel_staged_kernel(const T* __restrict__ Q, int64_t sQb, int64_t sQh, int64_t sQ
       qq += v[k] * v[k];
     }
     qq = warp_sum(qq);
-    const float nrm = fmaxf(sqrtf(qq), 1e-12f);
+    const float nrm = normalize ? fmaxf(sqrtf(qq), 1e-12f) : 1.f;
     float* dst = Qhat + (((int64_t)bi * nq + h) * NQ + i) * D;
 #pragma unroll
     for (int k = 0; k < D / 32; ++k) dst[lane + 32 * k] = v[k] / nrm;
@@ -238,7 +238,7 @@ constexpr int QSEL_CL_MAX = 8;
 template <typename T, int D>
 __global__ void __launch_bounds__(QSEL_CL_THREADS)
 qsel_cluster_kernel(const T* __restrict__ Q, int64_t sQb, int64_t sQh, int64_t sQt, int BCP, int NQ,
-                    int slice, float* __restrict__ Qhat, int32_t* __restrict__ q_idx) {
+                    int slice, float* __restrict__ Qhat, int32_t* __restrict__ q_idx, int normalize) {
   namespace cg = cooperative_groups;
   cg::cluster_group cluster = cg::this_cluster();
   const int C = (int)cluster.num_blocks();
@@ -344,7 +344,7 @@ qsel_cluster_kernel(const T* __restrict__ Q, int64_t sQb, int64_t sQh, int64_t s
     qq += __shfl_xor_sync(0xffffffffu, qq, 1);
     qq += __shfl_xor_sync(0xffffffffu, qq, 2);
     if (keep) {
-      const float nrm = fmaxf(sqrtf(qq), 1e-12f);
+      const float nrm = normalize ? fmaxf(sqrtf(qq), 1e-12f) : 1.f;
       float* dst = Qhat + (((int64_t)bi * nq + h) * NQ + rk) * D;
       for (int k = sub; k < D; k += 4) dst[k] = to_f32(q[k]) / nrm;
       if (sub == 0 && q_idx != nullptr) q_idx[((int64_t)bi * nq + h) * NQ + rk] = t;
@@ -382,7 +382,7 @@ qgroup_kernel(const float* __restrict__ Qhat, int nq, int NQ, float* __restrict_
 
 template <typename T, int D>
 static cudaError_t qsel_typed(Strided Q, int b, int nq, int BCP, int NQ, float* Qhat,
-                              int32_t* q_idx, cudaStream_t stream) {
+                              int32_t* q_idx, bool normalize, cudaStream_t stream) {
   {
     int C = (BCP + 127) / 128;
     if (C > QSEL_CL_MAX) C = QSEL_CL_MAX;
@@ -406,7 +406,7 @@ static cudaError_t qsel_typed(Strided Q, int b, int nq, int BCP, int NQ, float* 
       cfg.attrs = attr;
       cfg.numAttrs = 1;
       return cudaLaunchKernelEx(&cfg, kern, static_cast<const T*>(Q.data), Q.sb, Q.sh, Q.st, BCP, NQ, slice,
-                                Qhat, q_idx);
+                                Qhat, q_idx, (int)normalize);
     }
   }
   const size_t blk_bytes = ((size_t)BCP * D * sizeof(T) + 15) & ~size_t(15);
@@ -416,7 +416,7 @@ static cudaError_t qsel_typed(Strided Q, int b, int nq, int BCP, int NQ, float* 
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)staged);
     if (e != cudaSuccess) return e;
     kern<<<dim3(nq, b), QSEL_STAGED_THREADS, staged, stream>>>(static_cast<const T*>(Q.data), Q.sb, Q.sh, Q.st,
-                                                               BCP, NQ, Qhat, q_idx);
+                                                               BCP, NQ, Qhat, q_idx, (int)normalize);
     return cudaGetLastError();
   }
   const size_t smem = (size_t)BCP * sizeof(float) + (size_t)NQ * sizeof(int);
@@ -426,18 +426,18 @@ static cudaError_t qsel_typed(Strided Q, int b, int nq, int BCP, int NQ, float* 
     if (e != cudaSuccess) return e;
   }
   kern<<<dim3(nq, b), QSEL_THREADS, smem, stream>>>(static_cast<const T*>(Q.data), Q.sb, Q.sh, Q.st,
-                                                    BCP, NQ, Qhat, q_idx);
+                                                    BCP, NQ, Qhat, q_idx, (int)normalize);
   return cudaGetLastError();
 }
 
 cudaError_t launch_qsel(bool is_bf16, int d, Strided Q, int b, int nq, int BCP, int NQ,
-                        float* Qhat, int32_t* q_idx, cudaStream_t stream) {
+                        float* Qhat, int32_t* q_idx, bool normalize, cudaStream_t stream) {
   if (is_bf16) {
-    if (d == 128) return qsel_typed<bf16, 128>(Q, b, nq, BCP, NQ, Qhat, q_idx, stream);
-    if (d == 64) return qsel_typed<bf16, 64>(Q, b, nq, BCP, NQ, Qhat, q_idx, stream);
+    if (d == 128) return qsel_typed<bf16, 128>(Q, b, nq, BCP, NQ, Qhat, q_idx, normalize, stream);
+    if (d == 64) return qsel_typed<bf16, 64>(Q, b, nq, BCP, NQ, Qhat, q_idx, normalize, stream);
   } else {
-    if (d == 128) return qsel_typed<float, 128>(Q, b, nq, BCP, NQ, Qhat, q_idx, stream);
-    if (d == 64) return qsel_typed<float, 64>(Q, b, nq, BCP, NQ, Qhat, q_idx, stream);
+    if (d == 128) return qsel_typed<float, 128>(Q, b, nq, BCP, NQ, Qhat, q_idx, normalize, stream);
+    if (d == 64) return qsel_typed<float, 64>(Q, b, nq, BCP, NQ, Qhat, q_idx, normalize, stream);
   }
   return cudaErrorNotSupported;
 }

@@ -104,7 +104,7 @@ __device__ __forceinline__ void cl_wait() { asm volatile("barrier.cluster.wait.a
 __global__ void __launch_bounds__(QF_THREADS, 1)
 qsel_fast_kernel(const bf16* __restrict__ Q, int64_t sQb, int64_t sQh, int64_t sQt, int nq, int BCP, int NQ,
                  int32_t* __restrict__ q_idx, float* __restrict__ Qg, bf16* __restrict__ Qg_hilo,
-                 uint32_t* __restrict__ hist) {
+                 uint32_t* __restrict__ hist, int normalize) {
   extern __shared__ __align__(16) uint8_t qf_raw[];
   uint8_t* qs = qf_raw;  // [BCP][256 B], chunk c of row t at slot (c ^ (t & 15))
   __shared__ QfShared sh;
@@ -223,7 +223,7 @@ qsel_fast_kernel(const bf16* __restrict__ Q, int64_t sQb, int64_t sQh, int64_t s
       const int t = (int)(~(uint32_t)sh.lists[0][i]);
       const uint4 raw = reinterpret_cast<const uint4*>(qs + (size_t)t * 256)[cc ^ (t & 15)];
       const __nv_bfloat162* h2 = reinterpret_cast<const __nv_bfloat162*>(&raw);
-      const float nrm = sh.nrm[t];
+      const float nrm = normalize ? sh.nrm[t] : 1.f;
 #pragma unroll
       for (int u = 0; u < 4; ++u) {
         const float2 f = __bfloat1622float2(h2[u]);
@@ -292,7 +292,7 @@ qsel_fast_kernel(const bf16* __restrict__ Q, int64_t sQb, int64_t sQh, int64_t s
 }  // namespace
 
 cudaError_t launch_qsel_group_fast(Strided Q, int b, int nq, int nkv, int BCP, int NQ, int32_t* q_idx, float* Qg,
-                                   uint16_t* Qg_hilo, uint32_t* hist, cudaStream_t stream) {
+                                   uint16_t* Qg_hilo, uint32_t* hist, bool normalize, cudaStream_t stream) {
   const int G = nq / nkv;
   if (BCP < 1 || BCP > QF_MAX_BCP || NQ < 1 || NQ > QF_MAX_NQ || NQ > BCP || G < 1 || G > QF_MAX_G)
     return cudaErrorNotSupported;
@@ -314,7 +314,7 @@ cudaError_t launch_qsel_group_fast(Strided Q, int b, int nq, int nkv, int BCP, i
   cfg.attrs = attr;
   cfg.numAttrs = 1;
   return cudaLaunchKernelEx(&cfg, qsel_fast_kernel, static_cast<const bf16*>(Q.data), Q.sb, Q.sh, Q.st, nq, BCP,
-                            NQ, q_idx, Qg, reinterpret_cast<bf16*>(Qg_hilo), hist);
+                            NQ, q_idx, Qg, reinterpret_cast<bf16*>(Qg_hilo), hist, (int)normalize);
 }
 
 }  // namespace quoka

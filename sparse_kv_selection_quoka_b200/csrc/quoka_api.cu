@@ -158,9 +158,12 @@ P* at(void* ws, size_t off) {
 
 // Steps (a)-(e) after validation. kv_idx / kv_count / q_idx / s_agg are the
 // final destinations (workspace regions when the caller passed none).
+// `flags`: QUOKA_SCORE_DOT_PRODUCT selects the plain dot-product score (no
+// L2 normalisation of the chosen queries or of the keys).
 quoka_status run_select(const quoka_tensor* Q, const quoka_tensor* K, const SelectShapes& s, int NQ,
                         int bsa_eff, int32_t* kv_idx, int32_t* kv_count, int32_t* q_idx,
-                        float* s_agg, void* ws, const WsLayout& L, cudaStream_t stream) {
+                        float* s_agg, void* ws, const WsLayout& L, cudaStream_t stream, uint32_t flags = 0u) {
+  const bool cosine = (flags & QUOKA_SCORE_DOT_PRODUCT) == 0u;
   const bool bf = Q->dtype == QUOKA_BF16;
   const int b = (int)s.b, nq = (int)s.nq, nkv = (int)s.nkv, d = (int)s.d, BCP = (int)s.BCP;
   float* qhat = at<float>(ws, L.qhat);
@@ -173,9 +176,9 @@ quoka_status run_select(const quoka_tensor* Q, const quoka_tensor* K, const Sele
 
   cudaError_t e = cudaErrorNotSupported;
   if (bf && d == 128)
-    e = quoka::launch_qsel_group_fast(strided(Q), b, nq, nkv, BCP, NQ, qidx, qg, qhilo, hist, stream);
+    e = quoka::launch_qsel_group_fast(strided(Q), b, nq, nkv, BCP, NQ, qidx, qg, qhilo, hist, cosine, stream);
   if (e == cudaErrorNotSupported) {
-    e = quoka::launch_qsel(bf, d, strided(Q), b, nq, BCP, NQ, qhat, qidx, stream);
+    e = quoka::launch_qsel(bf, d, strided(Q), b, nq, BCP, NQ, qhat, qidx, cosine, stream);
     if (e != cudaSuccess) return cuda_status(e);
     e = quoka::launch_qgroup(d, qhat, b, nq, nkv, NQ, qg, bf ? qhilo : nullptr, bf ? hist : nullptr, stream);
   }
@@ -184,11 +187,13 @@ quoka_status run_select(const quoka_tensor* Q, const quoka_tensor* K, const Sele
   if (s.T > 0) {
     e = cudaErrorNotSupported;
     if (bf) {
-      e = quoka::launch_score_tc(d, strided(K), b, nkv, s.T, qhilo, NQ, sagg, hist, status, true, stream);
-      hist_made = e == cudaSuccess;
+      e = quoka::launch_score_tc(d, strided(K), b, nkv, s.T, qhilo, NQ, sagg, hist, status, true, cosine,
+                                 stream);
+      // the value-bucket histogram spans the cosine range [-1, 1]
+      hist_made = e == cudaSuccess && cosine;
     }
     if (e == cudaErrorNotSupported)
-      e = quoka::launch_score_simt(bf, d, strided(K), b, nkv, s.T, qg, NQ, sagg, stream);
+      e = quoka::launch_score_simt(bf, d, strided(K), b, nkv, s.T, qg, NQ, sagg, cosine, stream);
     if (e != cudaSuccess) return cuda_status(e);
   }
   if (bsa_eff > 0) {
@@ -316,6 +321,13 @@ size_t quoka_attn_workspace_size(int b, int nkv, int d, int BSA_eff, quoka_dtype
 quoka_status quoka_select(const quoka_tensor* Q, const quoka_tensor* K, int NQ, int BSA,
                           int32_t* kv_idx, int32_t* kv_count, int32_t* q_idx, float* s_agg,
                           void* ws, size_t ws_bytes, void* stream) {
+  return quoka_select_ex(Q, K, NQ, BSA, kv_idx, kv_count, q_idx, s_agg, 0u, ws, ws_bytes, stream);
+}
+
+quoka_status quoka_select_ex(const quoka_tensor* Q, const quoka_tensor* K, int NQ, int BSA,
+                             int32_t* kv_idx, int32_t* kv_count, int32_t* q_idx, float* s_agg,
+                             uint32_t flags, void* ws, size_t ws_bytes, void* stream) {
+  if ((flags & ~QUOKA_SCORE_DOT_PRODUCT) != 0u) return QUOKA_ERR_INVALID_ARG;
   SelectShapes s;
   quoka_status st = validate_select(Q, K, NQ, BSA, &s);
   if (st != QUOKA_OK) return st;
@@ -326,7 +338,7 @@ quoka_status quoka_select(const quoka_tensor* Q, const quoka_tensor* K, int NQ, 
   if (st != QUOKA_OK) return st;
   cudaStream_t cs = static_cast<cudaStream_t>(stream);
   if (cudaMemsetAsync(at<int>(ws, L.status), 0, 2 * sizeof(int), cs) != cudaSuccess) return QUOKA_ERR_CUDA;
-  return run_select(Q, K, s, NQ, (int)bsa_eff, kv_idx, kv_count, q_idx, s_agg, ws, L, cs);
+  return run_select(Q, K, s, NQ, (int)bsa_eff, kv_idx, kv_count, q_idx, s_agg, ws, L, cs, flags);
 }
 
 quoka_status quoka_gather_kv(const quoka_tensor* K, const quoka_tensor* V, const int32_t* kv_idx,

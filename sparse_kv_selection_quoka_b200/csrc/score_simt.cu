@@ -18,7 +18,7 @@ constexpr int SCORE_SIMT_THREADS = 128;
 template <typename T, int D>
 __global__ void __launch_bounds__(SCORE_SIMT_THREADS)
 score_simt_kernel(const T* __restrict__ K, int64_t sKb, int64_t sKh, int64_t sKt, int64_t Tlen,
-                  const float* __restrict__ Qg, int NQ, float* __restrict__ S_agg) {
+                  const float* __restrict__ Qg, int NQ, float* __restrict__ S_agg, int key_norm) {
   extern __shared__ float4 qs4[];
   const int j = blockIdx.y, bi = blockIdx.z, nkv = gridDim.y;
   const int64_t row = (int64_t)bi * nkv + j;
@@ -52,12 +52,12 @@ score_simt_kernel(const T* __restrict__ K, int64_t sKb, int64_t sKh, int64_t sKt
     }
     best = fmaxf(best, dot);
   }
-  S_agg[row * Tlen + tau] = best / fmaxf(sqrtf(kk), 1e-12f);
+  S_agg[row * Tlen + tau] = key_norm ? best / fmaxf(sqrtf(kk), 1e-12f) : best;
 }
 
 template <typename T, int D>
 static cudaError_t score_typed(Strided K, int b, int nkv, int64_t T_len, const float* Qg, int NQ,
-                               float* S_agg, cudaStream_t stream) {
+                               float* S_agg, bool key_norm, cudaStream_t stream) {
   const size_t smem = (size_t)NQ * D * sizeof(float);
   auto kern = score_simt_kernel<T, D>;
   if (smem > 48 * 1024) {
@@ -66,19 +66,19 @@ static cudaError_t score_typed(Strided K, int b, int nkv, int64_t T_len, const f
   }
   dim3 grid((unsigned)((T_len + SCORE_SIMT_THREADS - 1) / SCORE_SIMT_THREADS), nkv, b);
   kern<<<grid, SCORE_SIMT_THREADS, smem, stream>>>(static_cast<const T*>(K.data), K.sb, K.sh, K.st,
-                                                   T_len, Qg, NQ, S_agg);
+                                                   T_len, Qg, NQ, S_agg, (int)key_norm);
   return cudaGetLastError();
 }
 
 cudaError_t launch_score_simt(bool is_bf16, int d, Strided K, int b, int nkv, int64_t T_len,
-                              const float* Qg, int NQ, float* S_agg, cudaStream_t stream) {
+                              const float* Qg, int NQ, float* S_agg, bool key_norm, cudaStream_t stream) {
   if (T_len == 0) return cudaSuccess;
   if (is_bf16) {
-    if (d == 128) return score_typed<bf16, 128>(K, b, nkv, T_len, Qg, NQ, S_agg, stream);
-    if (d == 64) return score_typed<bf16, 64>(K, b, nkv, T_len, Qg, NQ, S_agg, stream);
+    if (d == 128) return score_typed<bf16, 128>(K, b, nkv, T_len, Qg, NQ, S_agg, key_norm, stream);
+    if (d == 64) return score_typed<bf16, 64>(K, b, nkv, T_len, Qg, NQ, S_agg, key_norm, stream);
   } else {
-    if (d == 128) return score_typed<float, 128>(K, b, nkv, T_len, Qg, NQ, S_agg, stream);
-    if (d == 64) return score_typed<float, 64>(K, b, nkv, T_len, Qg, NQ, S_agg, stream);
+    if (d == 128) return score_typed<float, 128>(K, b, nkv, T_len, Qg, NQ, S_agg, key_norm, stream);
+    if (d == 64) return score_typed<float, 64>(K, b, nkv, T_len, Qg, NQ, S_agg, key_norm, stream);
   }
   return cudaErrorNotSupported;
 }

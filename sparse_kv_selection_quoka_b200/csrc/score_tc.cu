@@ -72,6 +72,7 @@ struct ScoreArgs {
   int NQ, NQp, nstages, tiles_per_cta, ntiles;
   int nepi;                 // epilogue warpgroups in use (TMEM holds one accumulator each)
   uint32_t tmem_cols;
+  int key_norm;             // 1: divide by |k| (cosine score); 0: plain dot product
 };
 
 __device__ __forceinline__ void sc_abort(ScoreBars& sb, int* status, int where) {
@@ -258,7 +259,7 @@ score_tc_kernel(const __grid_constant__ CUtensorMap tmap, const ScoreArgs a) {
       const float ss = ((ss8[0] + ss8[1]) + (ss8[2] + ss8[3])) + ((ss8[4] + ss8[5]) + (ss8[6] + ss8[7]));
       mbar_arrive(&sb.empty[s]);
       const int64_t key = (int64_t)(t_begin + it) * SC_KEYS + r;
-      const float score = mx / fmaxf(sqrtf(ss), 1e-12f);
+      const float score = a.key_norm ? mx / fmaxf(sqrtf(ss), 1e-12f) : mx;
       if (key < a.T) out[key] = score;
       // first digit of the top-k select: the score's 12-bit value bucket,
       // counted once per distinct bucket within the warp
@@ -290,7 +291,8 @@ score_tc_kernel(const __grid_constant__ CUtensorMap tmap, const ScoreArgs a) {
 }  // namespace
 
 cudaError_t launch_score_tc(int d, Strided K, int b, int nkv, int64_t T, const uint16_t* Qg_hilo, int NQ,
-                            float* S_agg, uint32_t* hist, int* status, bool pdl, cudaStream_t stream) {
+                            float* S_agg, uint32_t* hist, int* status, bool pdl, bool key_norm,
+                            cudaStream_t stream) {
   if (d != SC_D || NQ < 1 || NQ > 128 || T <= 0 || T > (int64_t)INT32_MAX - SC_KEYS) return cudaErrorNotSupported;
   PFN_cuTensorMapEncodeTiled_v12000 encode = tensor_map_encoder();
   if (encode == nullptr) return cudaErrorNotSupported;
@@ -310,6 +312,7 @@ cudaError_t launch_score_tc(int d, Strided K, int b, int nkv, int64_t T, const u
   a.s_agg = S_agg;
   a.hist = hist;
   a.status = status;
+  a.key_norm = key_norm ? 1 : 0;
   a.T = T;
   a.NQ = NQ;
   a.NQp = (NQ + 15) / 16 * 16;  // the epilogue reads 16-column groups

@@ -54,9 +54,11 @@ def check_q_idx(gpu_q_idx: np.ndarray, SQ: np.ndarray, q_idx: np.ndarray) -> boo
 
 
 def check_kv_sets(gpu_idx: np.ndarray, gpu_count: np.ndarray, S_agg: np.ndarray, bsa_eff: int,
-                  sel: np.ndarray) -> int:
+                  sel: np.ndarray, band: float = None) -> int:
     """Checks the CUDA path's selected sets against the oracle's; returns the
-    number of (b, j) rows that differ inside the tie band."""
+    number of (b, j) rows that differ inside the tie band (KV_TIE_BAND, or
+    `band` for scores that are not cosines)."""
+    band = KV_TIE_BAND if band is None else band
     b, nkv, T = S_agg.shape
     assert np.all(gpu_count == bsa_eff), f"counts {np.unique(gpu_count)} != {bsa_eff}"
     n_diff = 0
@@ -72,7 +74,7 @@ def check_kv_sets(gpu_idx: np.ndarray, gpu_count: np.ndarray, S_agg: np.ndarray,
             thr = np.sort(s)[::-1][bsa_eff - 1]
             sym = np.setxor1d(g, sel[bi, j])
             dev = np.abs(s[sym] - thr)
-            assert dev.max() <= KV_TIE_BAND, (
+            assert dev.max() <= band, (
                 f"selected keys differ beyond the tie band at b={bi} j={j}: "
                 f"{len(sym)} keys, max |S - thr| = {dev.max():.3e}")
     return n_diff

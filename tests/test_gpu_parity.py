@@ -334,3 +334,69 @@ def test_out_of_range_index_latched_bf16_tensor_core_path(path):
     O, _ = q().quoka_sparse_gqa_attn(Q, K, V, idx, cnt, Kc, Vc, ws=ws)
     assert q().quoka_get_device_status(ws) == 6
     assert torch.isfinite(O.float()).all()
+
+
+def test_index_reuse_across_layers():
+    """A later layer attends over the key set an earlier layer selected
+    (steps (a)-(e) skipped on that layer): quoka_select on layer A, then
+    quoka_sparse_gqa_attn on layer B's Q, K, V with layer A's kv_idx, for
+    both attention paths (gathered copy, and gathered while loading)."""
+    xa = inputs.make_chunk(1, 8, 2, 128, 3000, 200, 8, 600, dtype="bf16", structure="llama", seed=61)
+    xb = inputs.make_chunk(1, 8, 2, 128, 3000, 200, 8, 600, dtype="bf16", structure="llama", seed=62)
+    _, gi, gc = run_select_and_check(xa)
+    Q, K, V, Kc, Vc = (P.to_dev(a, xb.dtype) for a in (xb.Q, xb.K, xb.V, xb.Kc, xb.Vc))
+    idx = torch.from_numpy(gi.astype(np.int32)).cuda()
+    cnt = torch.from_numpy(gc.astype(np.int32)).cuda()
+    O_ref, L_ref = orc.sparse_attention(xb.Q, xb.K, xb.V, gi, xb.Kc, xb.Vc)
+    for ws in (None, torch.zeros(256, dtype=torch.uint8, device="cuda")):
+        O, lse = q().quoka_sparse_gqa_attn(Q, K, V, idx, cnt, Kc, Vc, want_lse=True, ws=ws)
+        torch.cuda.synchronize()
+        err = np.abs(O.float().cpu().numpy().astype(np.float64) - O_ref).max()
+        lerr = np.abs(lse.cpu().numpy().astype(np.float64) - L_ref).max()
+        assert err <= P.o_tol(xb.dtype), f"O max-abs error {err:.3e}"
+        assert lerr <= max(P.LSE_TOL, P.o_tol(xb.dtype)), f"lse max-abs error {lerr:.3e}"
+
+
+@pytest.mark.parametrize("shape", [
+    # b, nq, nkv, d, T, BCP, NQ, BSA, dtype, structure: the fused tensor-core
+    # path (bf16, d = 128), the general query select with the tensor-core
+    # score, and the fp32 path on the CUDA cores
+    (1, 8, 2, 128, 3000, 200, 8, 600, "bf16", "llama"),
+    (2, 6, 3, 64, 900, 70, 5, 200, "bf16", "iid"),
+    (1, 4, 2, 64, 700, 40, 4, 100, "f32", "llama"),
+], ids=["bf16_d128", "bf16_d64", "f32_d64"])
+def test_dot_product_score_variant(shape):
+    """quoka_select_ex with QUOKA_SCORE_DOT_PRODUCT vs the oracle's
+    dot_product=True. The scores are unbounded, so the S_agg tolerance and
+    the top-BSA tie band scale with the largest score."""
+    b, nq, nkv, d, T, BCP, NQ, BSA, dt, st = shape
+    x = inputs.make_chunk(b, nq, nkv, d, T, BCP, NQ, BSA, dtype=dt, structure=st, seed=71)
+    Q, K = P.to_dev(x.Q, dt), P.to_dev(x.K, dt)
+    kv_idx, kv_count, q_idx, s_agg = q().quoka_select(Q, K, NQ, BSA, want_q_idx=True, want_s_agg=True,
+                                                      dot_product=True)
+    torch.cuda.synchronize()
+    ref = orc.select(x.Q, x.K, NQ, BSA, dot_product=True)
+    gq = q_idx.cpu().numpy().astype(np.int64)
+    if not P.check_q_idx(gq, ref["SQ"], ref["q_idx"]):
+        ref = orc.select(x.Q, x.K, NQ, BSA, override_q_idx=gq, dot_product=True)
+    scale = max(1.0, float(np.abs(ref["S_agg"]).max()))
+    err = np.abs(s_agg.cpu().numpy().astype(np.float64) - ref["S_agg"]).max()
+    assert err <= P.S_TOL * scale, f"S_agg max-abs error {err:.3e} (scores up to {scale:.1f})"
+    P.check_kv_sets(kv_idx.cpu().numpy().astype(np.int64), kv_count.cpu().numpy(), ref["S_agg"],
+                    min(BSA, T), ref["sel"], band=P.KV_TIE_BAND * scale)
+    # flags 0 through quoka_select_ex is quoka_select
+    lib = q().load()
+    from sparse_kv_selection_quoka_b200._lib import tensor_view, _ptr, _stream
+    ws = q().workspace_for(Q, K, NQ, BSA)
+    i0 = torch.empty_like(kv_idx)
+    c0 = torch.empty_like(kv_count)
+    qv, kv = tensor_view(Q), tensor_view(K)
+    import ctypes
+    st0 = lib.quoka_select_ex(ctypes.byref(qv), ctypes.byref(kv), NQ, BSA, _ptr(i0), _ptr(c0), None, None, 0,
+                              _ptr(ws), ws.numel(), _stream(None))
+    assert st0 == 0
+    i1, _, _, _ = q().quoka_select(Q, K, NQ, BSA)
+    torch.cuda.synchronize()
+    assert torch.equal(i0, i1)
+    assert lib.quoka_select_ex(ctypes.byref(qv), ctypes.byref(kv), NQ, BSA, _ptr(i0), _ptr(c0), None, None, 2,
+                               _ptr(ws), ws.numel(), _stream(None)) != 0

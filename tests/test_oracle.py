@@ -423,3 +423,66 @@ def test_attention_rows_match_sdpa_dense():
     for n, (bi, h, t) in enumerate(rows):
         np.testing.assert_allclose(O_rows[n], O_ref[bi, h, t], atol=1e-12)
         assert abs(lse_rows[n] - lse_ref[bi, h, t]) < 1e-12
+
+
+# ------------------------------------------------ dot-product score variant
+# [QUOKA §2.2] compares its cosine score with the standard dot-product score;
+# the oracle's dot_product=True drops the L2 normalisation of the chosen
+# queries and of the keys and keeps everything else.
+
+def _unit_rows(x):
+    return x / np.linalg.norm(x, axis=-1, keepdims=True)
+
+
+def test_dot_product_equals_cosine_on_unit_vectors():
+    """With every query and key of unit norm the two scores coincide, so
+    the whole selection does too."""
+    r = rng(21)
+    Q = _unit_rows(r.standard_normal((2, 6, 12, 8)))
+    K = _unit_rows(r.standard_normal((2, 3, 40, 8)))
+    cos = orc.select(Q, K, NQ=4, BSA=9)
+    dot = orc.select(Q, K, NQ=4, BSA=9, dot_product=True)
+    np.testing.assert_array_equal(dot["q_idx"], cos["q_idx"])
+    np.testing.assert_allclose(dot["S_agg"], cos["S_agg"], atol=1e-14)
+    np.testing.assert_array_equal(dot["sel"], cos["sel"])
+
+
+def test_dot_product_scales_with_the_keys_and_not_with_their_norm():
+    """Scaling all keys by c > 0 scales the dot-product score by c and keeps
+    the selection; scaling one key changes its score by that factor only
+    (the cosine score ignores both)."""
+    r = rng(22)
+    Q = r.standard_normal((1, 4, 10, 6))
+    K = r.standard_normal((1, 2, 25, 6))
+    base = orc.select(Q, K, NQ=3, BSA=7, dot_product=True)
+    scaled = orc.select(Q, 3.5 * K, NQ=3, BSA=7, dot_product=True)
+    np.testing.assert_allclose(scaled["S_agg"], 3.5 * base["S_agg"], rtol=1e-13)
+    np.testing.assert_array_equal(scaled["sel"], base["sel"])
+    K2 = K.copy()
+    K2[0, 1, 5] *= 0.25
+    one = orc.select(Q, K2, NQ=3, BSA=7, dot_product=True)
+    expect = base["S_agg"].copy()
+    expect[0, 1, 5] = 0.25 * base["S_agg"][0, 1, 5]
+    np.testing.assert_allclose(one["S_agg"], expect, rtol=1e-13, atol=1e-15)
+    cos1 = orc.select(Q, K, NQ=3, BSA=7)
+    cos2 = orc.select(Q, K2, NQ=3, BSA=7)
+    np.testing.assert_allclose(cos2["S_agg"], cos1["S_agg"], atol=1e-13)
+
+
+def test_dot_product_is_mean_of_per_head_raw_dots():
+    """By linearity, the max over chosen queries of (mean of the group's raw
+    chosen queries) . k equals the max of the mean of the per-head raw dot
+    products, computed here pair by pair with numpy.einsum."""
+    r = rng(23)
+    b, nq, nkv, L, T, d, NQ = 2, 6, 2, 9, 15, 5, 4
+    G = nq // nkv
+    Q = r.standard_normal((b, nq, L, d))
+    K = r.standard_normal((b, nkv, T, d))
+    res = orc.select(Q, K, NQ=NQ, BSA=3, dot_product=True)
+    q_idx = res["q_idx"]
+    chosen = np.take_along_axis(Q, q_idx[..., None], axis=2)          # (b, nq, NQ, d)
+    per_head = np.einsum("bhid,bhtd->bhit", chosen, np.repeat(K, G, axis=1))
+    expect = per_head.reshape(b, nkv, G, NQ, T).mean(axis=2).max(axis=2)
+    np.testing.assert_allclose(res["S_agg"], expect, atol=1e-12)
+    # and the query choice is the cosine variant's (steps (a), (b) unchanged)
+    np.testing.assert_array_equal(q_idx, orc.select(Q, K, NQ=NQ, BSA=3)["q_idx"])
