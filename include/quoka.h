@@ -193,6 +193,26 @@ quoka_status quoka_sparse_gqa_attn(const quoka_tensor* Q, const quoka_tensor* K,
                                    float scale, void* O, float* lse, void* ws,
                                    size_t ws_bytes, void* stream);
 
+/* Options of quoka_sparse_gqa_attn_ex (bit flags). */
+#define QUOKA_ATTN_NO_CHUNK_KEYS 1u
+
+/* quoka_sparse_gqa_attn with options; flags = 0 is quoka_sparse_gqa_attn
+ * exactly. QUOKA_ATTN_NO_CHUNK_KEYS leaves the chunk's own keys (Kc, Vc) out:
+ * the softmax runs over the selected keys only. This is one rank's partial
+ * attention when the prior keys are split over ranks (only one rank adds the
+ * chunk's keys); rows with no visible key give O = 0 and lse = -inf, and
+ * quoka_combine_partials merges the ranks' (O, lse). Kc and Vc must still
+ * be valid tensors of their usual shape (they are not read). Other flag
+ * bits are rejected with QUOKA_ERR_INVALID_ARG. */
+quoka_status quoka_sparse_gqa_attn_ex(const quoka_tensor* Q, const quoka_tensor* K,
+                                      const quoka_tensor* V,
+                                      const int32_t* kv_idx,
+                                      const int32_t* kv_count, int BSA_eff,
+                                      const quoka_tensor* Kc,
+                                      const quoka_tensor* Vc, float scale,
+                                      void* O, float* lse, uint32_t flags,
+                                      void* ws, size_t ws_bytes, void* stream);
+
 /* Step (g) on a selected KV that is already gathered, [QUOKA §4.2 problem 3]:
  * the attention of quoka_sparse_gqa_attn with key n of KV head j being row
  * n of Ksel[b, j] / Vsel[b, j] (n < kv_count[b, j]) instead of an indexed
@@ -224,6 +244,82 @@ quoka_status quoka_prefill_chunk(const quoka_tensor* Q, const quoka_tensor* K,
                                  float scale, void* O, float* lse,
                                  int32_t* kv_idx_out, void* ws, size_t ws_bytes,
                                  void* stream);
+
+/* ---- Prior keys split over ranks (context parallelism) -----------------
+ * The T prior keys of every (batch, KV head) are split into contiguous
+ * shards, shard r on rank r in ascending order. Each rank runs
+ * quoka_select (or quoka_select_ex) on its shard with the global BSA, then:
+ *   1. quoka_shard_candidate_scores: its candidates (key indices) and their
+ *      scores, padded to C = min(BSA, T_max) (T_max the largest shard;
+ *      padding: index -1, score -inf);
+ *   2. the ranks exchange the scores (an all-gather: (N, b, nkv, C) floats)
+ *      and quoka_shard_interleave lays them out rank-major per row;
+ *   3. quoka_topk over the concatenated lists ((b, nkv, N * C) scores) with
+ *      BSA_eff = min(BSA, T_total): positions into that list;
+ *   4. quoka_shard_take: this rank's share of the selection as key indices
+ *      of its shard (ascending) and their count;
+ *   5. quoka_sparse_gqa_attn_ex over them (rank 0 alone without
+ *      QUOKA_ATTN_NO_CHUNK_KEYS, so the chunk's own keys count once) with
+ *      lse;
+ *   6. the ranks exchange (O, lse) and quoka_combine_partials merges them.
+ * The selection equals the single-device one: every key of the global
+ * top-BSA is among its shard's top-BSA, and ties at the BSA-th score go to
+ * the lower global index as on one device. The package module
+ * sparse_kv_selection_quoka_b200.sharded runs these steps with
+ * torch.distributed. */
+
+/* This rank's candidate list padded to length C >= Cl: for
+ * n < kv_count[b, j] (clamped to Cl) cand_idx[b, j, n] = kv_idx[b, j, n] and
+ * scores[b, j, n] = s_agg[b, j, that index]; for the rest of [0, C)
+ * cand_idx = -1 and scores = -inf. s_agg (b, nkv, T) float; kv_idx
+ * (b, nkv, Cl) int32 (quoka_select's output); outs (b, nkv, C); all
+ * contiguous. An index outside [0, T) is not read (-inf, -1) and latches
+ * QUOKA_ERR_BOUNDS in ws (may be NULL). */
+quoka_status quoka_shard_candidate_scores(const float* s_agg, int b, int nkv,
+                                          int64_t T, const int32_t* kv_idx,
+                                          const int32_t* kv_count, int Cl, int C,
+                                          float* scores, int32_t* cand_idx,
+                                          void* ws, size_t ws_bytes,
+                                          void* stream);
+
+/* out[row, r, :] = in[r, row, :] for 32-bit elements: in (N, rows, C) (an
+ * all-gather's output), out (rows, N * C), both contiguous and 4-byte
+ * aligned. */
+quoka_status quoka_shard_interleave(const void* in, int N, int64_t rows,
+                                    int64_t C, void* out, void* stream);
+
+/* Step (e) alone, [QUOKA §2.3]: the min(BSA, T) largest of scores (b, nkv, T)
+ * float (contiguous) per row, ties to the lower index, ascending, into
+ * kv_idx (b, nkv, BSA_eff) and kv_count (b, nkv). ws (may be NULL): the
+ * status word. T <= the top-k's limit (QUOKA_ERR_UNSUPPORTED beyond). */
+quoka_status quoka_topk(const float* scores, int b, int nkv, int64_t T, int BSA,
+                        int32_t* kv_idx, int32_t* kv_count, void* ws,
+                        size_t ws_bytes, void* stream);
+
+/* This rank's share of a selection over the ranks' concatenated candidate
+ * lists: sel_pos (b, nkv, S) int32 ascending positions in [0, N * C),
+ * sel_count (b, nkv) entries valid; cand_idx (b, nkv, C) int32 this rank's
+ * candidate key indices (its list is positions [rank * C, (rank + 1) * C)).
+ * Out: kv_idx (b, nkv, C) int32, ascending key indices of this rank's
+ * picks (entries past the count left as written), kv_count (b, nkv). A pick
+ * whose candidate index is negative latches QUOKA_ERR_BOUNDS in ws (may be
+ * NULL). */
+quoka_status quoka_shard_take(const int32_t* sel_pos, const int32_t* sel_count,
+                              int b, int nkv, int S, const int32_t* cand_idx,
+                              int C, int rank, int32_t* kv_idx,
+                              int32_t* kv_count, void* ws, size_t ws_bytes,
+                              void* stream);
+
+/* Merge of N partial attentions over disjoint key sets:
+ * O = sum_r exp(lse_r - LSE) O_r, LSE = log sum_r exp(lse_r) per row.
+ * O_parts (N, b, nq, BCP, d) of dtype, lse_parts (N, b, nq, BCP) float,
+ * O out (b, nq, BCP, d) of dtype, lse out (b, nq, BCP) float or NULL; all
+ * contiguous, O_parts and O 16-byte aligned, d in {64, 128}. Rows that every
+ * rank saw empty give O = 0, LSE = -inf. */
+quoka_status quoka_combine_partials(const void* O_parts, const float* lse_parts,
+                                    int N, int b, int nq, int BCP, int d,
+                                    quoka_dtype dtype, void* O, float* lse,
+                                    void* stream);
 
 /* Synchronises `stream`, then reads the device status word of `ws` into
  * *device_status (a quoka_status value; QUOKA_OK if the latest call that

@@ -207,12 +207,16 @@ def gather_kv(K, V, sel):
 #  it; the chunk's own keys causally]
 # ---------------------------------------------------------------------------
 
-def sparse_attention(Q, K, V, sel, Kc, Vc, scale: Optional[float] = None):
+def sparse_attention(Q, K, V, sel, Kc, Vc, scale: Optional[float] = None, include_chunk: bool = True):
     """O[b, h, t] = sum_k softmax_k(scale * Q[b,h,t] . k) v over
     k in {K[b, j, sel[b, j]]} U {Kc[b, j, s] : s <= t}, j = floor(h / G).
 
     Returns (O (b, nq, BCP, d), LSE (b, nq, BCP)) with
-    LSE = log sum_k exp(scale * q . k)."""
+    LSE = log sum_k exp(scale * q . k).
+
+    include_chunk=False leaves the chunk's own keys out (one rank's part
+    when the prior keys are split over ranks); a row with no key left gets
+    O = 0 and LSE = -inf."""
     Q = _f64(Q)
     Kc = _f64(Kc)
     Vc = _f64(Vc)
@@ -235,6 +239,22 @@ def sparse_attention(Q, K, V, sel, Kc, Vc, scale: Optional[float] = None):
             s_idx = np.arange(L)
             hidden = s_idx[None, :] > s_idx[:, None]
             logits[:, n_sel:][hidden] = -np.inf
+            if not include_chunk:
+                logits[:, n_sel:] = -np.inf
+            if logits.shape[1] == 0 or not np.isfinite(logits).any(axis=1).all():
+                # rows with no key at all: O = 0, LSE = -inf
+                empty = ~np.isfinite(logits).any(axis=1) if logits.shape[1] else np.ones(L, dtype=bool)
+                O[bi, h] = 0.0
+                LSE[bi, h] = -np.inf
+                live = ~empty
+                if live.any():
+                    lg = logits[live]
+                    m = lg.max(axis=1, keepdims=True)
+                    p = np.exp(lg - m)
+                    denom = p.sum(axis=1, keepdims=True)
+                    O[bi, h][live] = (p @ vals) / denom
+                    LSE[bi, h][live] = (m + np.log(denom))[:, 0]
+                continue
             m = logits.max(axis=1, keepdims=True)
             p = np.exp(logits - m)
             denom = p.sum(axis=1, keepdims=True)

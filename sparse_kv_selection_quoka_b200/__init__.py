@@ -22,6 +22,11 @@ __all__ = [
     "quoka_status_string",
     "QuokaError",
     "quoka_select_static",
+    "quoka_shard_candidate_scores",
+    "quoka_shard_interleave",
+    "quoka_topk",
+    "quoka_shard_take",
+    "quoka_combine_partials",
 ]
 
 

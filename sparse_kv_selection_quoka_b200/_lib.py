@@ -48,6 +48,12 @@ EXPORTS = (
     "quoka_get_device_status",
     "quoka_status_string",
     "quoka_select_static",
+    "quoka_sparse_gqa_attn_ex",
+    "quoka_shard_candidate_scores",
+    "quoka_shard_interleave",
+    "quoka_topk",
+    "quoka_shard_take",
+    "quoka_combine_partials",
 )
 
 
@@ -112,6 +118,19 @@ def load() -> ctypes.CDLL:
         lib.quoka_status_string.argtypes = [_I]
         lib.quoka_select_static.restype = _I
         lib.quoka_select_static.argtypes = [_T, _T, _I, _I, _P, _P, _P, _P, _P]
+        lib.quoka_sparse_gqa_attn_ex.restype = _I
+        lib.quoka_sparse_gqa_attn_ex.argtypes = [_T, _T, _T, _P, _P, _I, _T, _T, _F, _P, _P, ctypes.c_uint32,
+                                                 _P, _SZ, _P]
+        lib.quoka_shard_candidate_scores.restype = _I
+        lib.quoka_shard_candidate_scores.argtypes = [_P, _I, _I, _I64, _P, _P, _I, _I, _P, _P, _P, _SZ, _P]
+        lib.quoka_shard_interleave.restype = _I
+        lib.quoka_shard_interleave.argtypes = [_P, _I, _I64, _I64, _P, _P]
+        lib.quoka_topk.restype = _I
+        lib.quoka_topk.argtypes = [_P, _I, _I, _I64, _I, _P, _P, _P, _SZ, _P]
+        lib.quoka_shard_take.restype = _I
+        lib.quoka_shard_take.argtypes = [_P, _P, _I, _I, _I, _P, _I, _I, _P, _P, _P, _SZ, _P]
+        lib.quoka_combine_partials.restype = _I
+        lib.quoka_combine_partials.argtypes = [_P, _P, _I, _I, _I, _I, _I, _I, _P, _P, _P]
         _lib = lib
         return lib
 
@@ -234,8 +253,11 @@ def quoka_gather_kv(K, V, kv_idx, kv_count, *, Ksel=None, Vsel=None, ws=None, st
     return Ksel, Vsel
 
 
+ATTN_NO_CHUNK_KEYS = 1  # quoka_sparse_gqa_attn_ex flag: the chunk's own keys left out
+
+
 def quoka_sparse_gqa_attn(Q, K, V, kv_idx, kv_count, Kc, Vc, scale=None, *, O=None, lse=None,
-                          want_lse=False, ws=None, stream=None):
+                          want_lse=False, ws=None, stream=None, no_chunk=False):
     """Steps (f)+(g). Returns (O (b,nq,BCP,d), lse or None). Without `ws`
     a workspace of quoka_attn_workspace_size bytes is allocated (the path
     that gathers the selected rows first); a 256-byte `ws` selects the path
@@ -252,12 +274,15 @@ def quoka_sparse_gqa_attn(Q, K, V, kv_idx, kv_count, Kc, Vc, scale=None, *, O=No
         n = quoka_attn_workspace_size(b, K.shape[1], d, kv_idx.shape[2], Q.dtype)
         ws = torch.empty(max(n, 256), dtype=torch.uint8, device=Q.device)
     views = [tensor_view(x) for x in (Q, K, V, Kc, Vc)]
-    st = lib.quoka_sparse_gqa_attn(ctypes.byref(views[0]), ctypes.byref(views[1]), ctypes.byref(views[2]),
-                                   _ptr(kv_idx) if kv_idx.numel() else None, _ptr(kv_count),
-                                   kv_idx.shape[2], ctypes.byref(views[3]), ctypes.byref(views[4]),
-                                   float(scale), _ptr(O), _ptr(lse), _ptr(ws), ws.numel(),
-                                   _stream(stream))
-    _check(st, "quoka_sparse_gqa_attn")
+    args = ([ctypes.byref(views[0]), ctypes.byref(views[1]), ctypes.byref(views[2]),
+             _ptr(kv_idx) if kv_idx.numel() else None, _ptr(kv_count), kv_idx.shape[2],
+             ctypes.byref(views[3]), ctypes.byref(views[4]), float(scale), _ptr(O), _ptr(lse)])
+    if no_chunk:
+        st = lib.quoka_sparse_gqa_attn_ex(*args, ATTN_NO_CHUNK_KEYS, _ptr(ws), ws.numel(), _stream(stream))
+        _check(st, "quoka_sparse_gqa_attn_ex")
+    else:
+        st = lib.quoka_sparse_gqa_attn(*args, _ptr(ws), ws.numel(), _stream(stream))
+        _check(st, "quoka_sparse_gqa_attn")
     return O, lse
 
 
@@ -351,3 +376,83 @@ def quoka_select_static(Q, K, NQ: int, BSA: int, *, kv_idx=None, kv_count=None, 
                                  _stream(stream))
     _check(st, "quoka_select_static")
     return kv_idx, kv_count, q_idx, s_agg
+
+
+# ---------------------------------------------------------------- prior keys split over ranks
+
+def quoka_shard_candidate_scores(s_agg, kv_idx, kv_count, C, *, scores=None, cand_idx=None, ws=None,
+                                 stream=None):
+    """This rank's candidates padded to length C: returns (scores (b,nkv,C)
+    float, cand_idx (b,nkv,C) int32), padding -inf / -1."""
+    lib = load()
+    b, nkv, T = s_agg.shape
+    Cl = kv_idx.shape[2]
+    if scores is None:
+        scores = torch.empty((b, nkv, C), dtype=torch.float32, device=s_agg.device)
+    if cand_idx is None:
+        cand_idx = torch.empty((b, nkv, C), dtype=torch.int32, device=s_agg.device)
+    st = lib.quoka_shard_candidate_scores(_ptr(s_agg), b, nkv, T, _ptr(kv_idx) if kv_idx.numel() else None,
+                                          _ptr(kv_count), Cl, C, _ptr(scores), _ptr(cand_idx), _ptr(ws),
+                                          0 if ws is None else ws.numel(), _stream(stream))
+    _check(st, "quoka_shard_candidate_scores")
+    return scores, cand_idx
+
+
+def quoka_shard_interleave(gathered, *, out=None, stream=None):
+    """(N, b, nkv, C) 32-bit -> (b, nkv, N * C), rank-major within a row."""
+    lib = load()
+    N, b, nkv, C = gathered.shape
+    if out is None:
+        out = torch.empty((b, nkv, N * C), dtype=gathered.dtype, device=gathered.device)
+    st = lib.quoka_shard_interleave(_ptr(gathered), N, b * nkv, C, _ptr(out), _stream(stream))
+    _check(st, "quoka_shard_interleave")
+    return out
+
+
+def quoka_topk(scores, BSA, *, kv_idx=None, kv_count=None, ws=None, stream=None):
+    """Step (e) alone on scores (b, nkv, T): (kv_idx (b,nkv,min(BSA,T)) int32
+    ascending, kv_count (b,nkv))."""
+    lib = load()
+    b, nkv, T = scores.shape
+    n = min(BSA, T)
+    if kv_idx is None:
+        kv_idx = torch.empty((b, nkv, n), dtype=torch.int32, device=scores.device)
+    if kv_count is None:
+        kv_count = torch.empty((b, nkv), dtype=torch.int32, device=scores.device)
+    st = lib.quoka_topk(_ptr(scores), b, nkv, T, BSA, _ptr(kv_idx) if kv_idx.numel() else None,
+                        _ptr(kv_count), _ptr(ws), 0 if ws is None else ws.numel(), _stream(stream))
+    _check(st, "quoka_topk")
+    return kv_idx, kv_count
+
+
+def quoka_shard_take(sel_pos, sel_count, cand_idx, rank, *, kv_idx=None, kv_count=None, ws=None, stream=None):
+    """This rank's share of a selection over the concatenated candidate
+    lists: (kv_idx (b,nkv,C) int32 ascending, kv_count (b,nkv))."""
+    lib = load()
+    b, nkv, S = sel_pos.shape
+    C = cand_idx.shape[2]
+    if kv_idx is None:
+        kv_idx = torch.zeros((b, nkv, C), dtype=torch.int32, device=cand_idx.device)
+    if kv_count is None:
+        kv_count = torch.empty((b, nkv), dtype=torch.int32, device=cand_idx.device)
+    st = lib.quoka_shard_take(_ptr(sel_pos) if sel_pos.numel() else None, _ptr(sel_count), b, nkv, S,
+                              _ptr(cand_idx) if cand_idx.numel() else None, C, rank,
+                              _ptr(kv_idx) if kv_idx.numel() else None, _ptr(kv_count), _ptr(ws),
+                              0 if ws is None else ws.numel(), _stream(stream))
+    _check(st, "quoka_shard_take")
+    return kv_idx, kv_count
+
+
+def quoka_combine_partials(O_parts, lse_parts, *, O=None, lse=None, stream=None):
+    """Merge (N, b, nq, BCP, d) partial outputs by their (N, b, nq, BCP)
+    log-sum-exps: returns (O (b,nq,BCP,d), lse (b,nq,BCP))."""
+    lib = load()
+    N, b, nq, BCP, d = O_parts.shape
+    if O is None:
+        O = torch.empty((b, nq, BCP, d), dtype=O_parts.dtype, device=O_parts.device)
+    if lse is None:
+        lse = torch.empty((b, nq, BCP), dtype=torch.float32, device=O_parts.device)
+    st = lib.quoka_combine_partials(_ptr(O_parts), _ptr(lse_parts), N, b, nq, BCP, d, _dtype_code(O_parts),
+                                    _ptr(O), _ptr(lse), _stream(stream))
+    _check(st, "quoka_combine_partials")
+    return O, lse

@@ -35,7 +35,7 @@ attn_simt_kernel(AttnArgs a) {
   const bool row_ok = t < a.BCP;
   const int64_t kvrow = (int64_t)bi * a.nkv + j;
   const int nsel = a.bsa > 0 ? max(0, min(a.kv_count[kvrow], a.bsa)) : 0;
-  const int nchunk = min(a.BCP, t0 + AS_ROWS);
+  const int nchunk = a.no_chunk ? 0 : min(a.BCP, t0 + AS_ROWS);
   const int total = nsel + nchunk;
 
   const float qscale = a.scale * 1.4426950408889634f;  // log2(e)
@@ -113,7 +113,7 @@ attn_simt_kernel(AttnArgs a) {
     }
   }
   if (!row_ok) return;
-  const float inv = 1.f / l;
+  const float inv = l > 0.f ? 1.f / l : 0.f;  // no visible key: O = 0, lse = -inf
   T* op = static_cast<T*>(a.O) + (((int64_t)bi * a.nq + h) * a.BCP + t) * D + part * DP;
 #pragma unroll
   for (int k = 0; k < DP; ++k) op[k] = from_f32<T>(o[k] * inv);

@@ -401,7 +401,7 @@ attn_gather_kernel(const __grid_constant__ AttnMaps maps, const AttnArgs a, int 
 }  // namespace
 
 cudaError_t launch_attn_tc_gather(const AttnArgs& a, cudaStream_t stream) {
-  if (a.d != D) return cudaErrorNotSupported;
+  if (a.d != D || a.no_chunk) return cudaErrorNotSupported;
   AttnMaps maps;
   if (!encode_bf16_4d(&maps.q, a.Q.data, D, a.BCP, a.nq, a.b, a.Q.st, a.Q.sh, a.Q.sb, 128))
     return cudaErrorNotSupported;

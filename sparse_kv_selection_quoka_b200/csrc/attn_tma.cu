@@ -185,9 +185,9 @@ attn_tma_kernel(const __grid_constant__ Maps maps, const AttnArgs a) {
   pdl_wait();  // the gathered rows and their counts come from the previous kernel
   const int64_t kvrow = (int64_t)bi * a.nkv + j;
   const int nsel = a.bsa > 0 ? max(0, min(__ldcg(a.kv_count + kvrow), a.bsa)) : 0;
-  const int nchunk = min(a.BCP, t0 + 128);
+  const int nchunk = a.no_chunk ? 0 : min(a.BCP, t0 + 128);
   const int ntile_sel = (nsel + N - 1) / N;
-  const int nT = ntile_sel + (nchunk + N - 1) / N;  // key tiles (>= 1)
+  const int nT = ntile_sel + (nchunk + N - 1) / N;  // key tiles (0 only without the chunk's keys)
   const int npair = (nT + 1) / 2;
 
   if (warp == LOAD_WARP) {
@@ -244,7 +244,7 @@ attn_tma_kernel(const __grid_constant__ Maps maps, const AttnArgs a) {
       alive = pv(0, kt0, i);
     }
     // the last odd tile's product
-    if (alive && (nT & 1) == 0) {
+    if (alive && nT > 0 && (nT & 1) == 0) {
       where = 26;
       alive = pv(1, nT - 1, npair - 1);
     }
@@ -293,12 +293,12 @@ attn_tma_kernel(const __grid_constant__ Maps maps, const AttnArgs a) {
     named_barrier_sync(1, 256);
     const float m0 = ml[r * 2], l0 = ml[r * 2 + 1];
     const float m1 = ml[(128 + r) * 2], l1 = ml[(128 + r) * 2 + 1];
-    const bool have1 = nT > 1;  // uniform: warpgroup 1 accumulated into O1
+    const bool have0 = nT > 0, have1 = nT > 1;  // uniform: warpgroup w accumulated into O_w
     const float M = fmaxf(m0, m1);
     const float f0 = m0 == -INFINITY ? 0.f : ex2(m0 - M);
     const float f1 = m1 == -INFINITY ? 0.f : ex2(m1 - M);
     const float L = f0 * l0 + f1 * l1;
-    const float inv = 1.f / L;
+    const float inv = L > 0.f ? 1.f / L : 0.f;  // no visible key: O = 0, lse = -inf
     // warpgroup w combines, normalises and stages output columns
     // [64w, 64w + 64) of its rows, bf16, in the 128-byte-swizzled layout the
     // TMA store reads (the Q area: every MMA is done)
@@ -307,9 +307,13 @@ attn_tma_kernel(const __grid_constant__ Maps maps, const AttnArgs a) {
 #pragma unroll 1
     for (int c2 = 0; c2 < 2; ++c2) {
       float o[32], p[32];
-      tmem_ld32(O0 + 32 * c2, o);
+      if (have0) tmem_ld32(O0 + 32 * c2, o);
       if (have1) tmem_ld32(O1 + 32 * c2, p);
       tmem_wait_ld();
+      if (!have0) {
+#pragma unroll
+        for (int u = 0; u < 32; ++u) o[u] = 0.f;
+      }
       if (!have1) {
 #pragma unroll
         for (int u = 0; u < 32; ++u) p[u] = 0.f;

@@ -87,6 +87,8 @@ struct AttnArgs {
   void* O;                  // (b, nq, BCP, d) contiguous, dtype of Q
   float* lse;               // (b, nq, BCP) or null
   int* status;
+  int no_chunk = 0;         // 1: the chunk's own keys are left out (a shard's partial attention);
+                            // rows with no visible key then give O = 0 and lse = -inf
 };
 
 // Steps (f)+(g) in fp32 on the CUDA cores (any input dtype).

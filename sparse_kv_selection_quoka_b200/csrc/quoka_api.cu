@@ -246,8 +246,9 @@ quoka_status validate_attn(const quoka_tensor* Q, const quoka_tensor* K, const q
 quoka_status run_attn(const quoka_tensor* Q, Strided K, Strided V, const quoka_tensor* Kc,
                       const quoka_tensor* Vc, const AttnShapes& s, int64_t T, const int32_t* kv_idx,
                       const int32_t* kv_count, int bsa_eff, float scale, void* O, float* lse,
-                      int* status, cudaStream_t stream, bool pdl = false) {
+                      int* status, cudaStream_t stream, bool pdl = false, bool no_chunk = false) {
   quoka::AttnArgs a;
+  a.no_chunk = no_chunk ? 1 : 0;
   a.Q = strided(Q);
   a.K = K;
   a.V = V;
@@ -279,10 +280,10 @@ quoka_status gather_then_attn(const quoka_tensor* Q, const quoka_tensor* K, cons
                               const quoka_tensor* Kc, const quoka_tensor* Vc, const AttnShapes& s,
                               const int32_t* kv_idx, const int32_t* kv_count, int bsa_eff, float scale,
                               void* O, float* lse, void* ksel, void* vsel, int* status,
-                              cudaStream_t stream) {
+                              cudaStream_t stream, bool no_chunk = false) {
   if (ksel == nullptr || vsel == nullptr || bsa_eff == 0)
     return run_attn(Q, strided(K), strided(V), Kc, Vc, s, s.T, kv_idx, kv_count, bsa_eff, scale, O, lse,
-                    status, stream);
+                    status, stream, false, no_chunk);
   cudaError_t e = quoka::launch_gather(Q->dtype == QUOKA_BF16, (int)s.d, strided(K), strided(V), (int)s.b,
                                        (int)s.nkv, s.T, kv_idx, kv_count, bsa_eff, ksel, vsel, status, true,
                                        stream);
@@ -290,7 +291,7 @@ quoka_status gather_then_attn(const quoka_tensor* Q, const quoka_tensor* K, cons
   const int64_t sh = (int64_t)bsa_eff * s.d, sb = s.nkv * sh;
   // the attention may launch while the gather finishes (it waits for it)
   return run_attn(Q, Strided{ksel, sb, sh, s.d}, Strided{vsel, sb, sh, s.d}, Kc, Vc, s, bsa_eff, nullptr,
-                  kv_count, bsa_eff, scale, O, lse, status, stream, true);
+                  kv_count, bsa_eff, scale, O, lse, status, stream, true, no_chunk);
 }
 
 }  // namespace
@@ -373,6 +374,17 @@ quoka_status quoka_sparse_gqa_attn(const quoka_tensor* Q, const quoka_tensor* K,
                                    const int32_t* kv_count, int BSA_eff, const quoka_tensor* Kc,
                                    const quoka_tensor* Vc, float scale, void* O, float* lse,
                                    void* ws, size_t ws_bytes, void* stream) {
+  return quoka_sparse_gqa_attn_ex(Q, K, V, kv_idx, kv_count, BSA_eff, Kc, Vc, scale, O, lse, 0u, ws, ws_bytes,
+                                  stream);
+}
+
+quoka_status quoka_sparse_gqa_attn_ex(const quoka_tensor* Q, const quoka_tensor* K,
+                                      const quoka_tensor* V, const int32_t* kv_idx,
+                                      const int32_t* kv_count, int BSA_eff, const quoka_tensor* Kc,
+                                      const quoka_tensor* Vc, float scale, void* O, float* lse,
+                                      uint32_t flags, void* ws, size_t ws_bytes, void* stream) {
+  if ((flags & ~QUOKA_ATTN_NO_CHUNK_KEYS) != 0u) return QUOKA_ERR_INVALID_ARG;
+  const bool no_chunk = (flags & QUOKA_ATTN_NO_CHUNK_KEYS) != 0u;
   AttnShapes s;
   quoka_status st = validate_attn(Q, K, V, Kc, Vc, &s);
   if (st != QUOKA_OK) return st;
@@ -392,7 +404,7 @@ quoka_status quoka_sparse_gqa_attn(const quoka_tensor* Q, const quoka_tensor* K,
     vsel = static_cast<char*>(ksel) + align_up((size_t)(s.b * s.nkv * BSA_eff * s.d) * 2);
   }
   return gather_then_attn(Q, K, V, Kc, Vc, s, kv_idx, kv_count, BSA_eff, scale, O, lse, ksel, vsel, status,
-                          cs);
+                          cs, no_chunk);
 }
 
 quoka_status quoka_sparse_gqa_attn_gathered(const quoka_tensor* Q, const quoka_tensor* Ksel,

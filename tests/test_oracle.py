@@ -486,3 +486,94 @@ def test_dot_product_is_mean_of_per_head_raw_dots():
     np.testing.assert_allclose(res["S_agg"], expect, atol=1e-12)
     # and the query choice is the cosine variant's (steps (a), (b) unchanged)
     np.testing.assert_array_equal(q_idx, orc.select(Q, K, NQ=NQ, BSA=3)["q_idx"])
+
+
+# ------------------------------------------- prior keys split over ranks
+# The sharded step (sparse_kv_selection_quoka_b200.sharded) rests on two
+# facts pinned here on the oracle: the union of every shard's top-BSA holds
+# the global top-BSA, and softmax partials over disjoint key sets merge by
+# their log-sum-exp.
+
+def test_attention_without_chunk_keys():
+    """include_chunk=False over every prior key is dense non-causal attention
+    over K (torch's library attention); with no selected key the rows are
+    empty (O = 0, LSE = -inf)."""
+    r = rng(31)
+    b, nq, nkv, d, T, L = 1, 4, 2, 8, 9, 5
+    Q = r.standard_normal((b, nq, L, d))
+    K = r.standard_normal((b, nkv, T, d))
+    V = r.standard_normal((b, nkv, T, d))
+    Kc = r.standard_normal((b, nkv, L, d))
+    Vc = r.standard_normal((b, nkv, L, d))
+    sel = np.broadcast_to(np.arange(T), (b, nkv, T))
+    O, lse = orc.sparse_attention(Q, K, V, sel, Kc, Vc, include_chunk=False)
+    G = nq // nkv
+    Kr = torch.from_numpy(np.repeat(K, G, axis=1))
+    Vr = torch.from_numpy(np.repeat(V, G, axis=1))
+    ref = torch.nn.functional.scaled_dot_product_attention(torch.from_numpy(Q), Kr, Vr).numpy()
+    np.testing.assert_allclose(O, ref, atol=1e-12)
+    O0, lse0 = orc.sparse_attention(Q, K, V, np.zeros((b, nkv, 0), dtype=np.int64), Kc, Vc,
+                                    include_chunk=False)
+    assert np.all(O0 == 0.0) and np.all(np.isneginf(lse0))
+
+
+def _merge_shard_selection(S_agg, T_shards, BSA):
+    """Global top-BSA from the shards' own top-BSA candidates, ranked over
+    their concatenation (shard order, ascending positions) with ties to the
+    earlier entry."""
+    offs = np.cumsum([0] + list(T_shards))
+    b, nkv, _ = S_agg.shape
+    n = min(BSA, offs[-1])
+    out = np.empty((b, nkv, n), dtype=np.int64)
+    for bi in range(b):
+        for j in range(nkv):
+            cand = []
+            for r, Tr in enumerate(T_shards):
+                local = orc.select_keys(S_agg[bi:bi + 1, j:j + 1, offs[r]:offs[r + 1]], BSA)[0, 0]
+                cand.extend(int(offs[r] + t) for t in local)
+            cand = np.array(cand, dtype=np.int64)
+            sc = S_agg[bi, j, cand]
+            order = np.lexsort((np.arange(len(cand)), -sc))
+            out[bi, j] = np.sort(cand[order[:n]])
+    return out
+
+
+@pytest.mark.parametrize("T_shards", [(40, 40), (30, 11, 0, 25), (5, 70)])
+def test_shard_candidates_hold_the_global_selection(T_shards):
+    """Merging the shards' top-BSA gives exactly the one-device top-BSA,
+    ties included (scores drawn on a coarse grid, so many tie)."""
+    r = rng(32)
+    T = sum(T_shards)
+    S = np.round(r.standard_normal((2, 3, T)) * 4) / 4     # many exact ties
+    for BSA in (1, 7, 20, T):
+        np.testing.assert_array_equal(_merge_shard_selection(S, T_shards, BSA), orc.select_keys(S, BSA))
+
+
+def test_lse_merge_of_shard_partials_is_the_whole_attention():
+    """The softmax over a key set split into shards (chunk keys on the first
+    one only) is the log-sum-exp merge of the per-shard softmaxes."""
+    r = rng(33)
+    b, nq, nkv, d, L = 1, 4, 2, 8, 6
+    T_shards = (7, 0, 5)
+    T = sum(T_shards)
+    offs = np.cumsum([0] + list(T_shards))
+    Q = r.standard_normal((b, nq, L, d))
+    K = r.standard_normal((b, nkv, T, d))
+    V = r.standard_normal((b, nkv, T, d))
+    Kc = r.standard_normal((b, nkv, L, d))
+    Vc = r.standard_normal((b, nkv, L, d))
+    sel = np.sort(r.permutation(T)[:8])
+    full, full_lse = orc.sparse_attention(Q, K, V, np.broadcast_to(sel, (b, nkv, 8)), Kc, Vc)
+    Os, ls = [], []
+    for rk in range(len(T_shards)):
+        mine = sel[(sel >= offs[rk]) & (sel < offs[rk + 1])] - offs[rk]
+        Ks, Vs = K[:, :, offs[rk]:offs[rk + 1]], V[:, :, offs[rk]:offs[rk + 1]]
+        O_r, l_r = orc.sparse_attention(Q, Ks, Vs, np.broadcast_to(mine, (b, nkv, len(mine))), Kc, Vc,
+                                        include_chunk=(rk == 0))
+        Os.append(O_r)
+        ls.append(l_r)
+    lse = np.logaddexp.reduce(np.stack(ls), axis=0)
+    w = np.exp(np.stack(ls) - lse)
+    O = (w[..., None] * np.stack(Os)).sum(axis=0)
+    np.testing.assert_allclose(O, full, atol=1e-12)
+    np.testing.assert_allclose(lse, full_lse, atol=1e-12)
