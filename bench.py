@@ -141,6 +141,22 @@ class ClockSampler:
 
 # ---------------------------------------------------------------- workload
 
+def max_over_ranks(values, world: int, device="cpu"):
+    """Per-rank timings -> their maximum over the ranks of the default
+    process group, on every rank (the values themselves at world 1)."""
+    t = torch.tensor([float(v) for v in values], dtype=torch.float64, device=device)
+    if world > 1:
+        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+    return [float(v) for v in t.cpu()]
+
+
+def job_throughput(world: int, units_per_rank: float, ms_step: float) -> float:
+    """Whole-job units per second: every rank processes units_per_rank per
+    step (weak scaling, replicas), the step taking ms_step (the slowest
+    rank's time)."""
+    return world * units_per_rank / (ms_step / 1e3)
+
+
 def make_inputs(name: str, rank: int):
     from sparse_kv_selection_quoka_b200 import inputs
     w = inputs._lookup(name)
@@ -295,15 +311,13 @@ def run_ours(args, rank, world, local_rank):
     clocks = sampler.stop()
 
     K_ = args.steps
-    times = torch.tensor([t_step / K_, t_sel / K_, t_gather / K_, t_attn / K_], dtype=torch.float64, device=dev)
-    if world > 1:
-        torch.distributed.all_reduce(times, op=torch.distributed.ReduceOp.MAX)
-    ms_step, ms_sel, ms_gather, ms_attn = (float(v) for v in times.cpu())
+    ms_step, ms_sel, ms_gather, ms_attn = max_over_ranks(
+        [t_step / K_, t_sel / K_, t_gather / K_, t_attn / K_], world, dev)
 
     tokens_per_step = w.b * (w.T if sweep else w.BCP)
     if sweep:
         tokens_per_step = w.b * x.n_chunks * x.BCP
-    value = world * tokens_per_step / (ms_step / 1e3)
+    value = job_throughput(world, tokens_per_step, ms_step)
 
     hbm, tf_burst, tf_sus, peak_src = _peaks()
     if sweep:
@@ -416,12 +430,10 @@ def run_e2e(args, w, x, chunks, q, dev, stream, tokens_per_step, world, sweep):
         step()
     e1.record(stream)
     torch.cuda.synchronize()
-    ms = torch.tensor([e0.elapsed_time(e1) / n], dtype=torch.float64, device=dev)
     if world > 1:
         torch.distributed.barrier()
-        torch.distributed.all_reduce(ms, op=torch.distributed.ReduceOp.MAX)
-    ms = float(ms.item())
-    return {"value": world * tokens_per_step / (ms / 1e3), "unit": UNIT, "ms_per_step": ms,
+    ms = max_over_ranks([e0.elapsed_time(e1) / n], world, dev)[0]
+    return {"value": job_throughput(world, tokens_per_step, ms), "unit": UNIT, "ms_per_step": ms,
             "steps": n, "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
             "call": "quoka_prefill_chunk (C ABI) with pinned-host inputs copied in and O copied out every step"}
 
