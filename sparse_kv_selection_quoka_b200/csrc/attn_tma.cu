@@ -22,7 +22,7 @@
 // softmax. After the last tile the two partial results of every row are in
 // the same SM's TMEM and are combined there.
 //
-// Warp roles (320 threads):
+// Warp roles (352 threads):
 //   warps 0-7   softmax: warpgroup w = warp / 4, one query row per thread
 //               (row = TMEM lane); then the combine of the two partials,
 //               normalisation, and the bf16 output tile stored with TMA.
@@ -32,8 +32,9 @@
 //               the first half of its keys as soon as that half of P is in
 //               TMEM.
 //   warp 9      TMA loads of Q, then of each key tile's K (3-stage ring, a
-//               stage released by its QK^T) and V (3-stage ring, released
-//               by its PV).
+//               stage released by its QK^T).
+//   warp 10     TMA loads of each key tile's V (3-stage ring, a stage
+//               released by its PV).
 // TMEM: S0 | S1 | O0 | O1, 128 columns each (512).
 // Every wait is bounded: a wait that gives up records QUOKA_ERR_TIMEOUT and
 // the CTA unwinds (waits for in-flight copies and MMAs, frees TMEM).
@@ -52,9 +53,10 @@ namespace {
 
 constexpr int KST = 3;  // K ring depth
 constexpr int VST = 3;  // V ring depth
-constexpr int THREADS = 320;
+constexpr int THREADS = 352;
 constexpr int MMA_WARP = 8;
-constexpr int LOAD_WARP = 9;
+constexpr int LOAD_WARP = 9;    // Q and K
+constexpr int VLOAD_WARP = 10;  // V
 // Of every 8 key pairs, how many take the FMA-pipe exp2 in the softmax.
 // Measured on B200 (Qwen-shaped layer): 0 and 2 run equally fast, more is
 // slower; 0 keeps the kernel free of register spills.
@@ -97,36 +99,34 @@ __device__ __forceinline__ void drain_ring(Smem& sm, uint64_t* full, int nload, 
   }
 }
 
-// One thread: K and V of key tiles 0 .. nT - 1 (selected tiles from the
-// gathered maps, then chunk tiles), each into the next stage of its ring
-// once that stage is released. The stages tile kt needs are released by
-// the QK^T and the PV of tile kt - 3; the MMA order (QK0(2i), PV1(2i-1),
+// One thread per ring (K or V): the tiles 0 .. nT - 1 (selected tiles from
+// the gathered maps, then chunk tiles), each into the next stage of its ring
+// once that stage is released. The stages tile kt needs are released by the
+// QK^T (K) and the PV (V) of tile kt - 3; the MMA order (QK0(2i), PV1(2i-1),
 // QK1(2i+1), PV0(2i)) issues the PV of a tile right after the QK^T of the
 // next one, so both come before the QK^T of tile kt - 1: the loads never
-// wait on a product that waits on a later load.
+// wait on a product that waits on a later load. With a thread per ring, a K
+// load never queues behind a V stage that is released later.
+template <bool IS_V>
 __device__ __forceinline__ void load_kv(Smem& sm, const Maps& maps, int nT, int ntile_sel, int j, int bi,
                                         int* status) {
-  int nk = 0, nv = 0;
+  constexpr int ST = IS_V ? VST : KST;
+  uint64_t* const full = IS_V ? sm.v_full : sm.k_full;
+  uint64_t* const empty = IS_V ? sm.v_empty : sm.k_empty;
+  int nl = 0;
   for (int kt = 0; kt < nT; ++kt) {
     const bool sel_tile = kt < ntile_sel;
-    const int y = (sel_tile ? kt : kt - ntile_sel) * N;
-    const int ks = kt % KST, vs = kt % VST;
-    if (kt >= KST && !mbar_wait(&sm.k_empty[ks], ((kt / KST) - 1) & 1, &sm.abort)) {
-      record_abort(sm, status, 11);
+    const int s = kt % ST;
+    if (kt >= ST && !mbar_wait(&empty[s], ((kt / ST) - 1) & 1, &sm.abort)) {
+      record_abort(sm, status, IS_V ? 14 : 11);
       break;
     }
-    load_tile(smem_u32(sm.k[ks]), sel_tile ? &maps.ks : &maps.kc, &sm.k_full[ks], y, j, bi);
-    nk = kt + 1;
-    if (kt >= VST && !mbar_wait(&sm.v_empty[vs], ((kt / VST) - 1) & 1, &sm.abort)) {
-      record_abort(sm, status, 14);
-      break;
-    }
-    load_tile(smem_u32(sm.v[vs]), sel_tile ? &maps.vs : &maps.vc, &sm.v_full[vs], y, j, bi);
-    nv = kt + 1;
+    const CUtensorMap* m = IS_V ? (sel_tile ? &maps.vs : &maps.vc) : (sel_tile ? &maps.ks : &maps.kc);
+    load_tile(smem_u32(IS_V ? sm.v[s] : sm.k[s]), m, &full[s], (sel_tile ? kt : kt - ntile_sel) * N, j, bi);
+    nl = kt + 1;
   }
-  drain_ring<KST>(sm, sm.k_full, nk, status, 12);
-  drain_ring<VST>(sm, sm.v_full, nv, status, 15);
-  if (!mbar_drain(&sm.q_full, 0)) record_abort(sm, status, 13);
+  drain_ring<ST>(sm, full, nl, status, IS_V ? 15 : 12);
+  if (!IS_V && !mbar_drain(&sm.q_full, 0)) record_abort(sm, status, 13);
 }
 
 __global__ void __launch_bounds__(THREADS, 1)
@@ -192,7 +192,10 @@ attn_tma_kernel(const __grid_constant__ Maps maps, const AttnArgs a) {
 
   if (warp == LOAD_WARP) {
     // ------------------------------------------------------------ TMA loads
-    if (lane == 0) load_kv(sm, maps, nT, ntile_sel, j, bi, a.status);
+    if (lane == 0) load_kv<false>(sm, maps, nT, ntile_sel, j, bi, a.status);
+    __syncwarp();
+  } else if (warp == VLOAD_WARP) {
+    if (lane == 0) load_kv<true>(sm, maps, nT, ntile_sel, j, bi, a.status);
     __syncwarp();
   } else if (warp == MMA_WARP) {
     // ------------------------------------------------------------ MMA issue
