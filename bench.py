@@ -19,7 +19,11 @@ do for a user); under torchrun the maximum over ranks is reported. A second
 pass of K steps runs the same kernels through the three part calls
 (quoka_select | quoka_gather_kv | quoka_sparse_gqa_attn_gathered) with an
 event at every boundary, for the breakdown (ms_select, ms_gather,
-ms_attention) and the rooflines. Rank 0 prints one JSON line.
+ms_attention) and the rooflines. For a single-chunk workload, `decode`
+reports a decode step (BCP = 1, NQ = 1) on the same cache: the whole step
+through quoka_prefill_chunk (which takes the short-chunk attention) and, on
+its selection, that attention alone against the prefill attention kernels.
+Rank 0 prints one JSON line.
 
 --impl reference times the CPU oracle (numpy float64) on the host cores
 instead, on a bounded per-step sample of the same workload (one KV head's
@@ -373,10 +377,68 @@ def run_ours(args, rank, world, local_rank):
     }
     if sweep:
         out["per_chunk_ms"] = [p / K_ for p in per_chunk]
+    else:
+        out["decode"] = measure_decode(q, w, dev, stream, flush, Q, K, V, Kc, Vc, min(K_, 50))
     if not args.no_e2e:
         out["e2e"] = run_e2e(args, w, x, chunks, q, dev, stream, tokens_per_step, world, sweep)
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         out["cpu_baseline"] = cpu_baseline(w, x, sweep)
+    return out
+
+
+def measure_decode(q, w, dev, stream, flush, Q, K, V, Kc, Vc, steps):
+    """A decode step on the workload's cache: BCP = 1 (the chunk's first
+    token), NQ = 1, the same T and BSA, through quoka_prefill_chunk (which
+    takes the short-chunk attention), L2 flushed before every timed call;
+    then, on that step's selection, the short-chunk attention alone
+    (quoka_decode_attn) and the prefill attention kernels on the same
+    selection (quoka_sparse_gqa_attn: gather, then 128-row tiles)."""
+    Q1, Kc1, Vc1 = (a[:, :, :1].contiguous() for a in (Q, Kc, Vc))
+    bsa_eff = min(w.BSA, w.T)
+    ws = q.workspace_for(Q1, K, 1, w.BSA)
+    O1 = torch.empty_like(Q1)
+    idx = torch.empty((w.b, w.nkv, bsa_eff), dtype=torch.int32, device=dev)
+    cnt = torch.full((w.b, w.nkv), bsa_eff, dtype=torch.int32, device=dev)
+    wsa = torch.empty(max(256, q.quoka_attn_workspace_size(w.b, w.nkv, w.d, bsa_eff, Q1.dtype)),
+                      dtype=torch.uint8, device=dev)
+    wsd = torch.empty(q.quoka_decode_workspace_size(w.b, w.nq, w.nkv, w.d, 1, bsa_eff, Q1.dtype),
+                      dtype=torch.uint8, device=dev)
+    calls = {
+        "ms_step": lambda: q.quoka_prefill_chunk(Q1, K, V, Kc1, Vc1, 1, w.BSA, O=O1, kv_idx=idx, ws=ws,
+                                                 stream=stream),
+        "ms_attention": lambda: q.quoka_decode_attn(Q1, K, V, idx, cnt, Kc1, Vc1, O=O1, ws=wsd, stream=stream),
+        "ms_attention_prefill_kernels": lambda: q.quoka_sparse_gqa_attn(Q1, K, V, idx, cnt, Kc1, Vc1, O=O1,
+                                                                        ws=wsa, stream=stream),
+    }
+    out = {"BCP": 1, "NQ": 1, "steps": steps}
+    for name, f in calls.items():
+        for _ in range(3):
+            f()
+        evs = []
+        for _ in range(steps):
+            flush.fill_(1)
+            # a short device-side wait after the flush: these calls take less
+            # GPU time than their host-side argument marshalling, and the
+            # wait lets the host enqueue the whole call before the timed
+            # region starts, so the events see the device's time only
+            torch.cuda._sleep(200000)
+            e = [torch.cuda.Event(enable_timing=True) for _ in range(2)]
+            e[0].record(stream)
+            f()
+            e[1].record(stream)
+            evs.append(e)
+        torch.cuda.synchronize()
+        out[name] = sum(a.elapsed_time(b) for a, b in evs) / steps
+    for wsx in (ws, wsd):
+        if q.quoka_get_device_status(wsx) != 0:
+            raise RuntimeError("device status after the decode measurement")
+    es = 2 if Q1.dtype == torch.bfloat16 else 4
+    nbytes = (2 * w.b * w.nkv * bsa_eff * w.d + 2 * w.b * w.nq * w.d + 2 * w.b * w.nkv * w.d) * es
+    gbs = nbytes / (out["ms_attention"] / 1e3) / 1e9
+    hbm = _peaks()[0]
+    out["attention_bytes"] = nbytes
+    out["attention_gbs"] = gbs
+    out["attention_frac_hbm"] = gbs / hbm
     return out
 
 

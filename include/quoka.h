@@ -233,6 +233,29 @@ quoka_status quoka_sparse_gqa_attn_gathered(const quoka_tensor* Q,
                                             void* O, float* lse, void* ws,
                                             size_t ws_bytes, void* stream);
 
+/* Steps (f)+(g) for a short chunk: a decode step (BCP = 1) or a short block
+ * of speculative tokens, [QUOKA §4.2 problem 3] and its generation-speed use
+ * in §4. The same attention as quoka_sparse_gqa_attn (same arguments and
+ * layouts; results equal up to rounding), computed for chunks whose G * BCP
+ * query rows per KV head are at most 64 (G = nq / nkv), d = 64 or 128: the
+ * keys of each KV head (its kv_count selected rows, then its BCP chunk keys)
+ * are cut into slices of 64, each slice read by index straight from the
+ * cache and attended by all G * BCP query rows of the head in fp32 (bf16 or
+ * fp32 inputs), and the slices' partial outputs are merged by their
+ * log-sum-exps. quoka_prefill_chunk takes this path by itself for such
+ * chunks.
+ *   ws  at least quoka_decode_workspace_size() bytes, 256-byte aligned: the
+ *       status words, then the fp32 partials.
+ * Returns QUOKA_ERR_UNSUPPORTED when G * BCP > 64 or d is not 64 / 128. */
+size_t quoka_decode_workspace_size(int b, int nq, int nkv, int d, int BCP,
+                                   int BSA_eff, quoka_dtype dtype);
+quoka_status quoka_decode_attn(const quoka_tensor* Q, const quoka_tensor* K,
+                               const quoka_tensor* V, const int32_t* kv_idx,
+                               const int32_t* kv_count, int BSA_eff,
+                               const quoka_tensor* Kc, const quoka_tensor* Vc,
+                               float scale, void* O, float* lse, void* ws,
+                               size_t ws_bytes, void* stream);
+
 /* The whole step (a)-(g): quoka_select followed by quoka_sparse_gqa_attn on
  * one stream, with no host synchronisation in between. ws must hold
  * quoka_workspace_size() bytes.

@@ -13,6 +13,8 @@ __all__ = [
     "quoka_workspace_size",
     "quoka_select_workspace_size",
     "quoka_attn_workspace_size",
+    "quoka_decode_workspace_size",
+    "quoka_decode_attn",
     "quoka_select",
     "quoka_gather_kv",
     "quoka_sparse_gqa_attn",

@@ -54,6 +54,8 @@ EXPORTS = (
     "quoka_topk",
     "quoka_shard_take",
     "quoka_combine_partials",
+    "quoka_decode_workspace_size",
+    "quoka_decode_attn",
 )
 
 
@@ -129,6 +131,10 @@ def load() -> ctypes.CDLL:
         lib.quoka_topk.argtypes = [_P, _I, _I, _I64, _I, _P, _P, _P, _SZ, _P]
         lib.quoka_shard_take.restype = _I
         lib.quoka_shard_take.argtypes = [_P, _P, _I, _I, _I, _P, _I, _I, _P, _P, _P, _SZ, _P]
+        lib.quoka_decode_workspace_size.restype = _SZ
+        lib.quoka_decode_workspace_size.argtypes = [_I, _I, _I, _I, _I, _I, _I]
+        lib.quoka_decode_attn.restype = _I
+        lib.quoka_decode_attn.argtypes = [_T, _T, _T, _P, _P, _I, _T, _T, _F, _P, _P, _P, _SZ, _P]
         lib.quoka_combine_partials.restype = _I
         lib.quoka_combine_partials.argtypes = [_P, _P, _I, _I, _I, _I, _I, _I, _P, _P, _P]
         _lib = lib
@@ -185,6 +191,36 @@ def quoka_select_workspace_size(b, nq, nkv, d, T, BCP, NQ, BSA, dtype) -> int:
 
 def quoka_attn_workspace_size(b, nkv, d, BSA_eff, dtype) -> int:
     return int(load().quoka_attn_workspace_size(b, nkv, d, BSA_eff, _code(dtype)))
+
+
+def quoka_decode_workspace_size(b, nq, nkv, d, BCP, BSA_eff, dtype) -> int:
+    return int(load().quoka_decode_workspace_size(b, nq, nkv, d, BCP, BSA_eff, _code(dtype)))
+
+
+def quoka_decode_attn(Q, K, V, kv_idx, kv_count, Kc, Vc, scale=None, *, O=None, lse=None, want_lse=False,
+                      ws=None, stream=None):
+    """Steps (f)+(g) for a short chunk (G * BCP <= 64 query rows per KV head):
+    the attention of quoka_sparse_gqa_attn, by key slices read straight from
+    the cache. Returns (O (b,nq,BCP,d), lse or None); `ws` defaults to a new
+    workspace of quoka_decode_workspace_size bytes."""
+    lib = load()
+    b, nq, BCP, d = Q.shape
+    if scale is None:
+        scale = d ** -0.5
+    if O is None:
+        O = torch.empty((b, nq, BCP, d), dtype=Q.dtype, device=Q.device)
+    if lse is None and want_lse:
+        lse = torch.empty((b, nq, BCP), dtype=torch.float32, device=Q.device)
+    if ws is None:
+        n = quoka_decode_workspace_size(b, nq, K.shape[1], d, BCP, kv_idx.shape[2], Q.dtype)
+        ws = torch.empty(max(n, 256), dtype=torch.uint8, device=Q.device)
+    views = [tensor_view(x) for x in (Q, K, V, Kc, Vc)]
+    st = lib.quoka_decode_attn(ctypes.byref(views[0]), ctypes.byref(views[1]), ctypes.byref(views[2]),
+                               _ptr(kv_idx) if kv_idx.numel() else None, _ptr(kv_count), kv_idx.shape[2],
+                               ctypes.byref(views[3]), ctypes.byref(views[4]), float(scale), _ptr(O), _ptr(lse),
+                               _ptr(ws), ws.numel(), _stream(stream))
+    _check(st, "quoka_decode_attn")
+    return O, lse
 
 
 def workspace_for(Q: torch.Tensor, K: torch.Tensor, NQ: int, BSA: int) -> torch.Tensor:

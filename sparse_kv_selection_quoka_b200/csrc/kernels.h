@@ -103,4 +103,28 @@ cudaError_t launch_attn_simt(bool bf16, const AttnArgs& a, cudaStream_t stream);
 cudaError_t launch_attn_tc(const AttnArgs& a, bool pdl, cudaStream_t stream);
 cudaError_t launch_attn_tc_gather(const AttnArgs& a, cudaStream_t stream);
 
+// Steps (f)+(g) for short chunks (decode steps, short speculative blocks):
+// the G * BCP query rows of a KV head together, its keys in slices of 64 (one
+// CTA each, rows read by index from the cache), fp32 partial outputs and
+// log-sum-exps merged by a second kernel (decode_attn.cu).
+constexpr int kDecodeMaxRows = 64;  // G * BCP
+struct DecodeArgs {
+  Strided Q, K, V, Kc, Vc;  // K, V: the full cache (b, nkv, T, d)
+  int b, nq, nkv, d, BCP;
+  int64_t T;
+  const int32_t* kv_idx;    // (b, nkv, bsa)
+  const int32_t* kv_count;  // (b, nkv)
+  int bsa;
+  float scale;
+  float* O_parts;           // (nsplit, b, nq, BCP, d) fp32
+  float* lse_parts;         // (nsplit, b, nq, BCP) fp32
+  int nsplit;               // decode_splits(bsa, BCP)
+  void* O;                  // (b, nq, BCP, d) contiguous, dtype of Q
+  float* lse;               // (b, nq, BCP) or null
+  int* status;
+};
+int decode_splits(int bsa, int BCP);
+size_t decode_smem_bytes(bool bf16, int R, int d);
+cudaError_t launch_decode_attn(bool bf16, const DecodeArgs& a, bool pdl, cudaStream_t stream);
+
 }  // namespace quoka

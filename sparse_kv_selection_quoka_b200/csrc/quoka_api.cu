@@ -32,8 +32,16 @@ struct WsLayout {
   size_t select_total = 0;  // end of what quoka_select needs
   size_t ksel = 0;      // (b, nkv, BSA_eff, d) bf16: gathered selected K (tensor-core attention)
   size_t vsel = 0;      // (b, nkv, BSA_eff, d) bf16: gathered selected V
+  size_t dparts = 0;    // short chunks: (nsplit, b, nq, BCP, d) fp32 partial outputs
+  size_t dlse = 0;      // short chunks: (nsplit, b, nq, BCP) fp32 partial log-sum-exps
   size_t total = 0;
 };
+
+// Chunks whose G * BCP query rows per KV head fit one CTA of the decode
+// attention take it (its fp32 partials live in the workspace).
+bool short_chunk(int64_t nq, int64_t nkv, int64_t BCP, int64_t d) {
+  return nkv > 0 && nq % nkv == 0 && (nq / nkv) * BCP <= quoka::kDecodeMaxRows && (d == 64 || d == 128);
+}
 
 // The tensor-core attention (bf16, d = 128) streams the selected rows from a
 // contiguous gathered copy when the workspace holds one.
@@ -42,7 +50,7 @@ bool uses_gather_buffers(quoka_dtype dtype, int64_t d, int64_t bsa_eff) {
 }
 
 WsLayout ws_layout(int64_t b, int64_t nq, int64_t nkv, int64_t d, int64_t T, int64_t NQ,
-                   int64_t bsa_eff, bool gather_buffers) {
+                   int64_t bsa_eff, bool gather_buffers, int64_t BCP = 0, bool decode = false) {
   WsLayout L;
   size_t off = 0;
   auto take = [&](size_t bytes) {
@@ -64,8 +72,19 @@ WsLayout ws_layout(int64_t b, int64_t nq, int64_t nkv, int64_t d, int64_t T, int
     L.ksel = take((size_t)(b * nkv * bsa_eff * d) * 2);
     L.vsel = take((size_t)(b * nkv * bsa_eff * d) * 2);
   }
+  if (decode) {
+    const int64_t rows = (int64_t)quoka::decode_splits((int)bsa_eff, (int)BCP) * b * nq * BCP;
+    L.dparts = take((size_t)(rows * d) * 4);
+    L.dlse = take((size_t)rows * 4);
+  }
   L.total = off;
   return L;
+}
+
+// Workspace of quoka_decode_attn: the status words, then the partials.
+size_t decode_ws_bytes(int64_t b, int64_t nq, int64_t d, int64_t BCP, int64_t bsa_eff) {
+  const int64_t rows = (int64_t)quoka::decode_splits((int)bsa_eff, (int)BCP) * b * nq * BCP;
+  return kAlign + align_up((size_t)(rows * d) * 4) + align_up((size_t)rows * 4);
 }
 
 // Workspace of quoka_sparse_gqa_attn alone: the status words, then (when
@@ -294,6 +313,38 @@ quoka_status gather_then_attn(const quoka_tensor* Q, const quoka_tensor* K, cons
                   kv_count, bsa_eff, scale, O, lse, status, stream, true, no_chunk);
 }
 
+// Steps (f)+(g) for a short chunk (short_chunk()): the slice kernel reads the
+// selected rows by index from the cache, then the merge kernel.
+quoka_status run_decode(const quoka_tensor* Q, const quoka_tensor* K, const quoka_tensor* V,
+                        const quoka_tensor* Kc, const quoka_tensor* Vc, const AttnShapes& s,
+                        const int32_t* kv_idx, const int32_t* kv_count, int bsa_eff, float scale, void* O,
+                        float* lse, float* O_parts, float* lse_parts, int* status, cudaStream_t stream,
+                        bool pdl) {
+  quoka::DecodeArgs a;
+  a.Q = strided(Q);
+  a.K = strided(K);
+  a.V = strided(V);
+  a.Kc = strided(Kc);
+  a.Vc = strided(Vc);
+  a.b = (int)s.b;
+  a.nq = (int)s.nq;
+  a.nkv = (int)s.nkv;
+  a.d = (int)s.d;
+  a.BCP = (int)s.BCP;
+  a.T = s.T;
+  a.kv_idx = kv_idx;
+  a.kv_count = kv_count;
+  a.bsa = bsa_eff;
+  a.scale = scale;
+  a.O_parts = O_parts;
+  a.lse_parts = lse_parts;
+  a.nsplit = quoka::decode_splits(bsa_eff, (int)s.BCP);
+  a.O = O;
+  a.lse = lse;
+  a.status = status;
+  return cuda_status(quoka::launch_decode_attn(Q->dtype == QUOKA_BF16, a, pdl, stream));
+}
+
 }  // namespace
 
 extern "C" {
@@ -303,7 +354,10 @@ size_t quoka_workspace_size(int b, int nq, int nkv, int d, int64_t T, int BCP, i
   if (b < 1 || nq < 1 || nkv < 1 || d < 1 || T < 0 || BCP < 1 || NQ < 1 || BSA < 0) return 0;
   if (nq % nkv != 0 || (dtype != QUOKA_F32 && dtype != QUOKA_BF16)) return 0;
   const int64_t bsa_eff = std::min<int64_t>(BSA, T);
-  return ws_layout(b, nq, nkv, d, T, NQ, bsa_eff, uses_gather_buffers(dtype, d, bsa_eff)).total;
+  const bool dec = short_chunk(nq, nkv, BCP, d);
+  // (a short chunk's layout keeps the gather buffers too: the same workspace
+  // then also gives quoka_sparse_gqa_attn its fastest path)
+  return ws_layout(b, nq, nkv, d, T, NQ, bsa_eff, uses_gather_buffers(dtype, d, bsa_eff), BCP, dec).total;
 }
 
 size_t quoka_select_workspace_size(int b, int nq, int nkv, int d, int64_t T, int BCP, int NQ, int BSA,
@@ -427,6 +481,36 @@ quoka_status quoka_sparse_gqa_attn_gathered(const quoka_tensor* Q, const quoka_t
                   lse, status, cs, true);
 }
 
+size_t quoka_decode_workspace_size(int b, int nq, int nkv, int d, int BCP, int BSA_eff, quoka_dtype dtype) {
+  if (b < 1 || nq < 1 || nkv < 1 || BCP < 1 || BSA_eff < 0) return 0;
+  if (dtype != QUOKA_F32 && dtype != QUOKA_BF16) return 0;
+  if (!short_chunk(nq, nkv, BCP, d)) return 0;
+  return decode_ws_bytes(b, nq, d, BCP, BSA_eff);
+}
+
+quoka_status quoka_decode_attn(const quoka_tensor* Q, const quoka_tensor* K, const quoka_tensor* V,
+                               const int32_t* kv_idx, const int32_t* kv_count, int BSA_eff,
+                               const quoka_tensor* Kc, const quoka_tensor* Vc, float scale, void* O,
+                               float* lse, void* ws, size_t ws_bytes, void* stream) {
+  AttnShapes s;
+  quoka_status st = validate_attn(Q, K, V, Kc, Vc, &s);
+  if (st != QUOKA_OK) return st;
+  if (!short_chunk(s.nq, s.nkv, s.BCP, s.d)) return QUOKA_ERR_UNSUPPORTED;
+  if (BSA_eff < 0 || kv_count == nullptr || (BSA_eff > 0 && kv_idx == nullptr)) return QUOKA_ERR_INVALID_ARG;
+  if (O == nullptr || !aligned16(O)) return QUOKA_ERR_INVALID_ARG;
+  if (!(scale > 0.f) || scale != scale) return QUOKA_ERR_INVALID_ARG;
+  const size_t need = decode_ws_bytes(s.b, s.nq, s.d, s.BCP, BSA_eff);
+  if (ws == nullptr || ((uintptr_t)ws % kAlign) != 0 || ws_bytes < need) return QUOKA_ERR_WORKSPACE;
+  cudaStream_t cs = static_cast<cudaStream_t>(stream);
+  int* status = static_cast<int*>(ws);
+  if (cudaMemsetAsync(status, 0, 2 * sizeof(int), cs) != cudaSuccess) return QUOKA_ERR_CUDA;
+  const int64_t rows = (int64_t)quoka::decode_splits(BSA_eff, (int)s.BCP) * s.b * s.nq * s.BCP;
+  float* O_parts = reinterpret_cast<float*>(static_cast<char*>(ws) + kAlign);
+  float* lse_parts = reinterpret_cast<float*>(reinterpret_cast<char*>(O_parts) + align_up((size_t)(rows * s.d) * 4));
+  return run_decode(Q, K, V, Kc, Vc, s, kv_idx, kv_count, BSA_eff, scale, O, lse, O_parts, lse_parts, status, cs,
+                    false);
+}
+
 quoka_status quoka_prefill_chunk(const quoka_tensor* Q, const quoka_tensor* K,
                                  const quoka_tensor* V, const quoka_tensor* Kc,
                                  const quoka_tensor* Vc, int NQ, int BSA, float scale, void* O,
@@ -441,8 +525,9 @@ quoka_status quoka_prefill_chunk(const quoka_tensor* Q, const quoka_tensor* K,
   if (O == nullptr || !aligned16(O)) return QUOKA_ERR_INVALID_ARG;
   if (!(scale > 0.f) || scale != scale) return QUOKA_ERR_INVALID_ARG;
   const int64_t bsa_eff = std::min<int64_t>(BSA, s.T);
+  const bool dec = short_chunk(s.nq, s.nkv, s.BCP, s.d);
   const bool gb = uses_gather_buffers(Q->dtype, s.d, bsa_eff);
-  const WsLayout L = ws_layout(s.b, s.nq, s.nkv, s.d, s.T, NQ, bsa_eff, gb);
+  const WsLayout L = ws_layout(s.b, s.nq, s.nkv, s.d, s.T, NQ, bsa_eff, gb, s.BCP, dec);
   st = check_ws(ws, ws_bytes, L.total);
   if (st != QUOKA_OK) return st;
   cudaStream_t cs = static_cast<cudaStream_t>(stream);
@@ -452,6 +537,9 @@ quoka_status quoka_prefill_chunk(const quoka_tensor* Q, const quoka_tensor* K,
   int32_t* kv_count = at<int32_t>(ws, L.kvcount);
   st = run_select(Q, K, s, NQ, (int)bsa_eff, kv_idx, kv_count, nullptr, nullptr, ws, L, cs);
   if (st != QUOKA_OK) return st;
+  if (dec)  // a short chunk: the decode attention (waits for the selection's last kernel)
+    return run_decode(Q, K, V, Kc, Vc, as, kv_idx, kv_count, (int)bsa_eff, scale, O, lse, at<float>(ws, L.dparts),
+                      at<float>(ws, L.dlse), status, cs, true);
   return gather_then_attn(Q, K, V, Kc, Vc, as, kv_idx, kv_count, (int)bsa_eff, scale, O, lse,
                           gb ? at<void>(ws, L.ksel) : nullptr, gb ? at<void>(ws, L.vsel) : nullptr, status, cs);
 }

@@ -33,6 +33,16 @@ def to_dev(x: np.ndarray, dtype: str) -> torch.Tensor:
     return t.cuda()
 
 
+def to_dev_view(x: np.ndarray, dtype: str, pad: int = 64) -> torch.Tensor:
+    """x (b, h, T, d) as the leading T rows of a longer (b, h, T + pad, d)
+    device buffer: a strided view (heads T + pad rows apart), as a slice of a
+    larger cache would be."""
+    b, h, T, d = x.shape
+    big = np.zeros((b, h, T + pad, d), dtype=np.float32)
+    big[:, :, :T] = x
+    return to_dev(big, dtype)[:, :, :T]
+
+
 def check_q_idx(gpu_q_idx: np.ndarray, SQ: np.ndarray, q_idx: np.ndarray) -> bool:
     """Returns True when identical; False when they differ only inside the
     near-tie band (asserts otherwise)."""

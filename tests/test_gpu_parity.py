@@ -90,6 +90,15 @@ def run_prefill_and_check(x: inputs.ChunkInputs, ref, gi, rows=None, dev=None):
         lerr = np.abs(Ls - L_ref).max()
     assert err <= tol, f"O max-abs error {err:.3e} > {tol}"
     assert lerr <= max(P.LSE_TOL, tol), f"LSE max-abs error {lerr:.3e}"
+    # quoka_prefill_chunk takes the decode attention for short chunks: the
+    # prefill attention kernels must agree on the same selection too
+    gi_t = torch.from_numpy(gi.astype(np.int32)).cuda()
+    cnt = torch.full(gi.shape[:2], gi.shape[2], dtype=torch.int32, device="cuda")
+    O2, _ = q().quoka_sparse_gqa_attn(Q, K, V, gi_t, cnt, Kc, Vc)
+    torch.cuda.synchronize()
+    O2g = O2.float().cpu().numpy().astype(np.float64)
+    err2 = np.abs(O2g - O_ref).max() if rows is None else np.abs(np.stack([O2g[r] for r in rows]) - O_ref).max()
+    assert err2 <= tol, f"quoka_sparse_gqa_attn O max-abs error {err2:.3e} > {tol}"
     return O
 
 

@@ -137,6 +137,27 @@ def test_attention_rejects_bad_arguments_on_host(lib):
     assert g(B(Q), B(K), B(K), B(Kc), B(Kc), 0, 10, 0.1, buf, None, None, ws, 1 << 30, None) == 1
 
 
+def test_decode_attention_rejects_bad_arguments_on_host(lib):
+    f = lib.quoka_decode_attn
+    B = ctypes.byref
+    buf = ctypes.c_void_p(0x200000)
+    ws = ctypes.c_void_p(0x100000)
+    K = _view((1, 2, 500, 128))
+    # G * BCP = 4 * 17 = 68 query rows per KV head: not a short chunk
+    Q, Kc = _view((1, 8, 17, 128)), _view((1, 2, 17, 128))
+    assert f(B(Q), B(K), B(K), buf, buf, 10, B(Kc), B(Kc), 0.1, buf, None, ws, 1 << 30, None) == 2
+    # G * BCP = 64: accepted shapes, but a workspace one byte short, or misaligned
+    Q, Kc = _view((1, 8, 16, 128)), _view((1, 2, 16, 128))
+    need = lib.quoka_decode_workspace_size(1, 8, 2, 128, 16, 10, 0)
+    assert need > 256
+    assert f(B(Q), B(K), B(K), buf, buf, 10, B(Kc), B(Kc), 0.1, buf, None, ws, need - 1, None) == 3
+    assert f(B(Q), B(K), B(K), buf, buf, 10, B(Kc), B(Kc), 0.1, buf, None, ctypes.c_void_p(0x100010), need,
+             None) == 3
+    assert f(B(Q), B(K), B(K), buf, buf, 10, B(Kc), B(Kc), -1.0, buf, None, ws, need, None) == 1
+    assert f(B(Q), B(K), B(K), None, buf, 10, B(Kc), B(Kc), 0.1, buf, None, ws, need, None) == 1
+    assert lib.quoka_decode_workspace_size(1, 8, 2, 96, 1, 10, 0) == 0  # d = 96
+
+
 def test_binding_fails_loudly_without_library(tmp_path, monkeypatch):
     from sparse_kv_selection_quoka_b200 import _lib
     monkeypatch.setattr(_lib, "LIB_PATH", str(tmp_path / "missing.so"))
