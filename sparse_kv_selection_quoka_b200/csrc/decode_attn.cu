@@ -72,9 +72,6 @@ struct SliceSmem {
   __host__ __device__ static constexpr size_t bytes(int R) { return ml_off(R) + (size_t)R * 2 * 4; }
 };
 
-template <typename T>
-__device__ __forceinline__ float elt_f32(const T* p) { return to_f32(*p); }
-
 // grid (nsplit, nkv, b). Slice s covers key numbers [64 s, 64 s + 64) of the
 // head's list (selected keys 0 .. nsel - 1, then chunk keys).
 template <typename T, int D>
@@ -159,39 +156,46 @@ __global__ void __launch_bounds__(kThreads) decode_slice_kernel(const DecodeArgs
   }
   __syncthreads();
 
-  // scores: thread (k, parity) for rows parity, parity + 2, ..., 8 rows at a
-  // time; key n0 + k is visible to row r when it is a selected key, or a
-  // chunk key at a position not after the row's
+  // scores: two threads per key (lanes 2k, 2k + 1 of the key's pair), each
+  // over half of d, 4 query rows at a time in independent accumulators, the
+  // halves summed by one shuffle; key n0 + k is visible to row r when it is
+  // a selected key, or a chunk key at a position not after the row's
   {
-    const int k = tid & (KS - 1), r0 = tid / KS;
+    static_assert(KS * 2 == kThreads, "two threads per key");
+    constexpr int HALF = CPR / 2;  // 16-byte chunks per half row
+    const int k = tid >> 1, half = tid & 1;
     const int n = n0 + k;
-    const uint4* krow = reinterpret_cast<const uint4*>(Ksb + k * L::KROW);
-    for (int q0 = r0; q0 < R; q0 += 16) {
-      float acc[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
+    const uint4* krow = reinterpret_cast<const uint4*>(Ksb + k * L::KROW) + half * HALF;
+    for (int r0 = 0; r0 < R; r0 += 4) {
+      float acc[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll 2
-      for (int c = 0; c < CPR; ++c) {
+      for (int c = 0; c < HALF; ++c) {
         float kf[EPC];
         to_f32x<T>(krow[c], kf);
 #pragma unroll
-        for (int u = 0; u < 8; ++u) {
-          const int r = q0 + 2 * u;
-          if (r < R) {
-            const float4* qr = reinterpret_cast<const float4*>(Qs + r * D + c * EPC);
+        for (int i = 0; i < 4; ++i) {
+          const int r = min(r0 + i, R - 1);  // (rows past R: computed, not stored)
+          const float4* qr = reinterpret_cast<const float4*>(Qs + r * D + (half * HALF + c) * EPC);
 #pragma unroll
-            for (int i = 0; i < EPC / 4; ++i) {
-              const float4 qq = qr[i];
-              acc[u] = fmaf(qq.x, kf[4 * i], fmaf(qq.y, kf[4 * i + 1],
-                                                  fmaf(qq.z, kf[4 * i + 2], fmaf(qq.w, kf[4 * i + 3], acc[u]))));
-            }
+          for (int e4 = 0; e4 < EPC / 4; ++e4) {
+            const float4 qq = qr[e4];
+            acc[i] = fmaf(qq.x, kf[4 * e4], acc[i]);
+            acc[i] = fmaf(qq.y, kf[4 * e4 + 1], acc[i]);
+            acc[i] = fmaf(qq.z, kf[4 * e4 + 2], acc[i]);
+            acc[i] = fmaf(qq.w, kf[4 * e4 + 3], acc[i]);
           }
         }
       }
 #pragma unroll
-      for (int u = 0; u < 8; ++u) {
-        const int r = q0 + 2 * u;
-        if (r < R) {
-          const bool vis = k < nk && (n < nsel || n - nsel <= r % a.BCP);
-          Ps[r * KS + k] = vis ? acc[u] : -INFINITY;
+      for (int i = 0; i < 4; ++i) acc[i] += __shfl_xor_sync(0xffffffffu, acc[i], 1);
+      if (half == 0) {
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+          const int r = r0 + i;
+          if (r < R) {
+            const bool vis = k < nk && (n < nsel || n - nsel <= r % a.BCP);
+            Ps[r * KS + k] = vis ? acc[i] : -INFINITY;
+          }
         }
       }
     }
@@ -317,25 +321,38 @@ decode_merge_kernel(const float* __restrict__ O_parts, const float* __restrict__
   const int cg = tid % ncg, sl = tid / ncg;
   float m = -INFINITY, l = 0.f;
   float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
-#pragma unroll 4
-  for (int s = sl; s < nsplit; s += nsl) {
-    const float ls = __ldcg(lse_parts + (int64_t)s * rows + row);
-    const float4 x = __ldcg(reinterpret_cast<const float4*>(O_parts + ((int64_t)s * rows + row) * d) + cg);
-    if (ls > m) {
-      const float f = m == -INFINITY ? 0.f : expf(m - ls);
-      acc.x *= f;
-      acc.y *= f;
-      acc.z *= f;
-      acc.w *= f;
-      l *= f;
-      m = ls;
+  constexpr int BATCH = 8;  // slices whose loads are in flight together
+  for (int s0 = sl; s0 < nsplit; s0 += BATCH * nsl) {
+    float ls[BATCH];
+    float4 x[BATCH];
+#pragma unroll
+    for (int i = 0; i < BATCH; ++i) {
+      const int s = s0 + i * nsl;
+      ls[i] = -INFINITY;
+      x[i] = make_float4(0.f, 0.f, 0.f, 0.f);
+      if (s < nsplit) {
+        ls[i] = __ldcg(lse_parts + (int64_t)s * rows + row);
+        x[i] = __ldcg(reinterpret_cast<const float4*>(O_parts + ((int64_t)s * rows + row) * d) + cg);
+      }
     }
-    const float w = ls == -INFINITY ? 0.f : expf(ls - m);
-    acc.x = fmaf(w, x.x, acc.x);
-    acc.y = fmaf(w, x.y, acc.y);
-    acc.z = fmaf(w, x.z, acc.z);
-    acc.w = fmaf(w, x.w, acc.w);
-    l += w;
+#pragma unroll
+    for (int i = 0; i < BATCH; ++i) {
+      if (ls[i] > m) {
+        const float f = m == -INFINITY ? 0.f : expf(m - ls[i]);
+        acc.x *= f;
+        acc.y *= f;
+        acc.z *= f;
+        acc.w *= f;
+        l *= f;
+        m = ls[i];
+      }
+      const float w = ls[i] == -INFINITY ? 0.f : expf(ls[i] - m);
+      acc.x = fmaf(w, x[i].x, acc.x);
+      acc.y = fmaf(w, x[i].y, acc.y);
+      acc.z = fmaf(w, x[i].z, acc.z);
+      acc.w = fmaf(w, x[i].w, acc.w);
+      l += w;
+    }
   }
   part[tid] = acc;
   pm[tid] = m;
@@ -400,11 +417,6 @@ cudaError_t launch_typed(const DecodeArgs& a, bool pdl, cudaStream_t stream) {
 }  // namespace
 
 int decode_splits(int bsa, int BCP) { return (bsa + BCP + KS - 1) / KS; }
-
-size_t decode_smem_bytes(bool bf16, int R, int d) {
-  if (d == 128) return bf16 ? SliceSmem<__nv_bfloat16, 128>::bytes(R) : SliceSmem<float, 128>::bytes(R);
-  return bf16 ? SliceSmem<__nv_bfloat16, 64>::bytes(R) : SliceSmem<float, 64>::bytes(R);
-}
 
 cudaError_t launch_decode_attn(bool bf16, const DecodeArgs& a, bool pdl, cudaStream_t stream) {
   const int R = (a.nq / a.nkv) * a.BCP;

@@ -124,7 +124,6 @@ struct DecodeArgs {
   int* status;
 };
 int decode_splits(int bsa, int BCP);
-size_t decode_smem_bytes(bool bf16, int R, int d);
 cudaError_t launch_decode_attn(bool bf16, const DecodeArgs& a, bool pdl, cudaStream_t stream);
 
 }  // namespace quoka
