@@ -257,8 +257,9 @@ quoka_status quoka_decode_attn(const quoka_tensor* Q, const quoka_tensor* K,
                                size_t ws_bytes, void* stream);
 
 /* The whole step (a)-(g): quoka_select followed by quoka_sparse_gqa_attn on
- * one stream, with no host synchronisation in between. ws must hold
- * quoka_workspace_size() bytes.
+ * one stream, with no host synchronisation in between; for a short chunk
+ * (G * BCP <= 64 query rows per KV head, d = 64 or 128) the attention is
+ * quoka_decode_attn's. ws must hold quoka_workspace_size() bytes.
  *   kv_idx_out (b, nkv, BSA_eff) int32 or NULL: the selected set (else kept
  *   in ws). lse may be NULL. */
 quoka_status quoka_prefill_chunk(const quoka_tensor* Q, const quoka_tensor* K,
