@@ -112,7 +112,9 @@ score_tc_kernel(const __grid_constant__ CUtensorMap tmap, const ScoreArgs a) {
   if (tid == 0) {
     for (int s = 0; s < NS; ++s) {
       mbar_init(&sb.full[s], 1);
-      mbar_init(&sb.empty[s], 128);  // released by the epilogue warpgroup that read |k|
+      // released once the tile's MMAs are done (one commit) and the epilogue
+      // warpgroup has read |k| from it (128 arrivals)
+      mbar_init(&sb.empty[s], 129);
     }
     for (int q = 0; q < SC_EPI; ++q) {
       mbar_init(&sb.tfull[q], 1);
@@ -207,6 +209,7 @@ score_tc_kernel(const __grid_constant__ CUtensorMap tmap, const ScoreArgs a) {
         umma_bf16_ss_warp(d, ad, bd, idesc, kk > 0 ? 1u : 0u);
       }
       umma_commit_warp(&sb.tfull[acc]);
+      umma_commit_warp(&sb.empty[s]);  // the stage's share of its release
     }
     if (!alive && lane == 0) sc_abort(sb, a.status, where);
     umma_commit_warp(&sb.done);
@@ -223,24 +226,9 @@ score_tc_kernel(const __grid_constant__ CUtensorMap tmap, const ScoreArgs a) {
     const int NE = a.nepi;  // warpgroups g >= NE stay idle
     for (int it = g; it < n && g < NE; it += NE) {
       const int s = it % NS, acc = g;
-      if (!sc_warp_wait(&sb.tfull[acc], (it / NE) & 1, sb, a.status, 55)) break;
-      tc_fence_after();
-      float mx4[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
-      const uint32_t tbase = tmem + lane_off + (uint32_t)(acc * ACC);
-      for (int c0 = 0; c0 < a.NQp; c0 += 16) {
-        float hi[16], lo[16];
-        tmem_ld16(tbase + c0, hi);
-        tmem_ld16(tbase + a.NQp + c0, lo);
-        tmem_wait_ld();
-#pragma unroll
-        for (int u = 0; u < 16; ++u)
-          if (c0 + u < a.NQ) mx4[u & 3] = fmaxf(mx4[u & 3], hi[u] + lo[u]);
-      }
-      const float mx = fmaxf(fmaxf(mx4[0], mx4[1]), fmaxf(mx4[2], mx4[3]));
-      tc_fence_before();
-      mbar_arrive(&sb.tempty[acc]);
-      // |k| from the tile in shared memory (the TMA writes are visible to
-      // threads that observe the stage's barrier)
+      // |k| first, straight from the landed tile (the TMA writes are visible
+      // to threads that observe the stage's barrier), so that the stage is
+      // released without waiting for this tile's MMA result
       if (!sc_warp_wait(&sb.full[s], (it / NS) & 1, sb, a.status, 56)) break;
       const uint8_t* tile = ring + (size_t)s * SC_TILE_BYTES;
       // eight independent partial sums keep the FMA chain short
@@ -258,6 +246,23 @@ score_tc_kernel(const __grid_constant__ CUtensorMap tmap, const ScoreArgs a) {
       }
       const float ss = ((ss8[0] + ss8[1]) + (ss8[2] + ss8[3])) + ((ss8[4] + ss8[5]) + (ss8[6] + ss8[7]));
       mbar_arrive(&sb.empty[s]);
+      // then the tile's scores against the group means, from TMEM
+      if (!sc_warp_wait(&sb.tfull[acc], (it / NE) & 1, sb, a.status, 55)) break;
+      tc_fence_after();
+      float mx4[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
+      const uint32_t tbase = tmem + lane_off + (uint32_t)(acc * ACC);
+      for (int c0 = 0; c0 < a.NQp; c0 += 16) {
+        float hi[16], lo[16];
+        tmem_ld16(tbase + c0, hi);
+        tmem_ld16(tbase + a.NQp + c0, lo);
+        tmem_wait_ld();
+#pragma unroll
+        for (int u = 0; u < 16; ++u)
+          if (c0 + u < a.NQ) mx4[u & 3] = fmaxf(mx4[u & 3], hi[u] + lo[u]);
+      }
+      const float mx = fmaxf(fmaxf(mx4[0], mx4[1]), fmaxf(mx4[2], mx4[3]));
+      tc_fence_before();
+      mbar_arrive(&sb.tempty[acc]);
       const int64_t key = (int64_t)(t_begin + it) * SC_KEYS + r;
       const float score = a.key_norm ? mx / fmaxf(sqrtf(ss), 1e-12f) : mx;
       if (key < a.T) out[key] = score;
