@@ -97,6 +97,33 @@ def _view(shape, dtype=1, data=0x10000, stride=None):
     return v
 
 
+def test_workspace_size_covers_every_call_host_only(lib):
+    """quoka_workspace_size is the select part, plus the gathered copy (bf16,
+    d = 128), plus, for a short chunk (G * BCP <= 64), the decode attention's
+    partials: so one workspace serves quoka_select, quoka_sparse_gqa_attn at
+    its fastest, quoka_decode_attn and quoka_prefill_chunk."""
+    al = lambda n: (n + 255) // 256 * 256
+    cases = [  # b, nq, nkv, d, T, BCP, NQ, BSA, dtype (1 = bf16)
+        (1, 32, 8, 128, 32768, 512, 32, 4096, 1),
+        (1, 32, 8, 128, 32768, 1, 1, 4096, 1),
+        (2, 16, 2, 128, 3000, 8, 8, 700, 1),
+        (1, 6, 3, 64, 900, 3, 3, 200, 0),
+        (1, 8, 2, 128, 0, 1, 1, 0, 1),
+    ]
+    for b, nq, nkv, d, T, BCP, NQ, BSA, dt in cases:
+        full = lib.quoka_workspace_size(b, nq, nkv, d, T, BCP, NQ, BSA, dt)
+        sel = lib.quoka_select_workspace_size(b, nq, nkv, d, T, BCP, NQ, BSA, dt)
+        bsa = min(BSA, T)
+        att = lib.quoka_attn_workspace_size(b, nkv, d, bsa, dt)
+        dec = lib.quoka_decode_workspace_size(b, nq, nkv, d, BCP, bsa, dt)
+        gathered = 2 * al(b * nkv * bsa * d * 2) if (dt == 1 and d == 128 and bsa > 0) else 0
+        short = (nq // nkv) * BCP <= 64
+        assert (dec > 0) == short
+        assert att == 256 + gathered
+        assert full == sel + gathered + (dec - 256 if short else 0)
+        assert full >= max(sel, att, dec)
+
+
 def test_select_rejects_bad_arguments_on_host(lib):
     Q = _view((1, 8, 64, 128))
     K = _view((1, 2, 500, 128))
