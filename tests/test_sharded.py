@@ -101,16 +101,17 @@ def _free_port() -> int:
         return s.getsockname()[1]
 
 
-def _case(T_shards, seed):
+def _case(T_shards, seed, BCP=24):
     T = sum(T_shards)
-    x = inputs.make_chunk(1, 4, 2, 32, T, 24, 5, 20, dtype="f32", structure="llama", seed=seed)
+    NQ = min(5, BCP)
+    x = inputs.make_chunk(1, 4, 2, 32, T, BCP, NQ, 20, dtype="f32", structure="llama", seed=seed)
     return x
 
 
-def _gloo_rank(rank, world, port, T_shards, seed, out_dir):
+def _gloo_rank(rank, world, port, T_shards, seed, out_dir, BCP=24):
     dist.init_process_group("gloo", init_method=f"tcp://127.0.0.1:{port}", rank=rank, world_size=world)
     try:
-        x = _case(T_shards, seed)
+        x = _case(T_shards, seed, BCP)
         offs = np.cumsum([0] + list(T_shards))
         sl = slice(offs[rank], offs[rank + 1])
         t = lambda a: torch.from_numpy(np.ascontiguousarray(a, dtype=np.float64))
@@ -126,13 +127,14 @@ def _gloo_rank(rank, world, port, T_shards, seed, out_dir):
         dist.destroy_process_group()
 
 
-@pytest.mark.parametrize("T_shards", [(90, 60), (50, 0, 77)], ids=["two_ranks", "three_ranks_one_empty"])
-def test_sharded_exchange_gloo(T_shards, tmp_path):
+@pytest.mark.parametrize("T_shards,BCP", [((90, 60), 24), ((50, 0, 77), 24), ((70, 45), 1)],
+                         ids=["two_ranks", "three_ranks_one_empty", "two_ranks_decode_step"])
+def test_sharded_exchange_gloo(T_shards, BCP, tmp_path):
     world = len(T_shards)
     port = _free_port()
-    mp.start_processes(_gloo_rank, args=(world, port, T_shards, 81, str(tmp_path)), nprocs=world, join=True,
+    mp.start_processes(_gloo_rank, args=(world, port, T_shards, 81, str(tmp_path), BCP), nprocs=world, join=True,
                        start_method="spawn")
-    x = _case(T_shards, 81)
+    x = _case(T_shards, 81, BCP)
     ref = orc.prefill_chunk(x.Q, x.K, x.V, x.Kc, x.Vc, x.NQ, x.BSA)
     sel = [[set() for _ in range(x.K.shape[1])] for _ in range(x.K.shape[0])]
     for r in range(world):
