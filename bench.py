@@ -23,7 +23,10 @@ ms_attention) and the rooflines. For a single-chunk workload, `decode`
 reports a decode step (BCP = 1, NQ = 1) on the same cache: the whole step
 through quoka_prefill_chunk (which takes the short-chunk attention) and, on
 its selection, that attention alone against the prefill attention kernels.
-Rank 0 prints one JSON line.
+With the default workload, `per_workload` repeats the measurement (without
+the e2e, decode and oracle legs) on the Llama-shaped layer at T = 8192, the
+chunked-prefill sweep (b = 8, 64 chunks of 256, with its per-chunk time
+curve) and the 128K-key layer. Rank 0 prints one JSON line.
 
 --impl reference times the CPU oracle (numpy float64) on the host cores
 instead, on a bounded per-step sample of the same workload (one KV head's
@@ -50,10 +53,9 @@ import torch  # noqa: E402
 METRIC = "prefill chunk-tokens/sec at T=32K (keys-scored/sec, % HBM and tensor-pipe peak alongside)"
 UNIT = "chunk-tokens/s"
 FLUSH_BYTES = 256 << 20
-def kernels_per_chunk(T, bsa_eff):
-    """Our kernel launches in one chunk's step: query select, group mean,
-    scoring (T > 0), top-k and gather (BSA_eff > 0), attention."""
-    return 2 + (1 if T > 0 else 0) + (2 if bsa_eff > 0 else 0) + 1
+DEFAULT_WORKLOAD = "qwen3-4b_T32k"
+# measured beside the default workload in every default run
+OTHER_WORKLOADS = ("llama3.2-3b_T8k", "sweep_b8_S16k", "long_T128k_G8")
 
 
 def _peaks():
@@ -187,202 +189,291 @@ def gather_bytes(b, nkv, d, bsa_eff, es):
 
 # ---------------------------------------------------------------- our arm
 
+def kernels_per_chunk(w, T, bsa_eff):
+    """Our kernel launches in one quoka_prefill_chunk call on a bf16, d = 128
+    workload: query select + group mean (one fused kernel for BCP <= 512,
+    NQ <= 32, G <= 8, else two), the scoring (T > 0), the top-k and the
+    gather (BSA_eff > 0), and the attention (a short chunk's takes two)."""
+    G = w.nq // w.nkv
+    fused = w.dtype == "bf16" and w.d == 128 and w.BCP <= 512 and w.NQ <= 32 and G <= 8
+    short = G * w.BCP <= 64
+    n = (1 if fused else 2) + (1 if T > 0 else 0)
+    if bsa_eff > 0:
+        n += 1 if short else 2
+    return n + (2 if short else 1)
+
+
+class WorkloadRun:
+    """Device buffers of one workload on this rank: a list of chunks (one,
+    or the sweep's 64), each with its strided input views, its workspace and
+    its outputs, all resident in HBM before any timing."""
+
+    def __init__(self, q, name, rank, dev):
+        self.w, self.x = make_inputs(name, rank)
+        w, x = self.w, self.x
+        self.sweep = w.name.startswith("sweep")
+        self.tdt = torch.bfloat16 if w.dtype == "bf16" else torch.float32
+        self.es = 2 if w.dtype == "bf16" else 4
+        tdt = self.tdt
+
+        def to_dev(a):
+            return torch.from_numpy(np.ascontiguousarray(a, dtype=np.float32)).to(tdt).to(dev)
+
+        self.chunks = []
+        if self.sweep:
+            self.Qs, self.Ks, self.Vs = (to_dev(a) for a in (x.Qs, x.Ks, x.Vs))
+            L = x.BCP
+            for c in range(x.n_chunks):
+                T = c * L
+                views = (self.Qs[:, :, T:T + L], self.Ks[:, :, :T], self.Vs[:, :, :T],
+                         self.Ks[:, :, T:T + L], self.Vs[:, :, T:T + L])
+                self.chunks.append(self._chunk(q, views, x.budget(T), T, L, dev))
+            self.BCP = L
+        else:
+            self.dev_inputs = [to_dev(a) for a in (x.Q, x.K, x.V, x.Kc, x.Vc)]
+            self.chunks.append(self._chunk(q, tuple(self.dev_inputs), w.BSA, w.T, w.BCP, dev))
+            self.BCP = w.BCP
+
+    def _chunk(self, q, views, bsa, T, L, dev):
+        w = self.w
+        be = min(bsa, T)
+        return {
+            "views": views, "bsa": bsa, "T": T, "bsa_eff": be,
+            "ws": q.workspace_for(views[0], views[1], w.NQ, bsa),
+            "O": torch.empty((w.b, w.nq, L, w.d), dtype=self.tdt, device=dev),
+            "kv_idx": torch.empty((w.b, w.nkv, be), dtype=torch.int32, device=dev),
+            "kv_count": torch.empty((w.b, w.nkv), dtype=torch.int32, device=dev),
+            "sel": tuple(torch.empty((w.b, w.nkv, be, w.d), dtype=self.tdt, device=dev) for _ in range(2)),
+        }
+
+    # the work of one step, in both forms
+    def whole(self, q, ch, stream):
+        """Steps (a)-(g) as one call, quoka_prefill_chunk."""
+        Qv, Kv, Vv, Kcv, Vcv = ch["views"]
+        q.quoka_prefill_chunk(Qv, Kv, Vv, Kcv, Vcv, self.w.NQ, ch["bsa"], O=ch["O"], kv_idx=ch["kv_idx"],
+                              ws=ch["ws"], stream=stream)
+
+    def parts(self, q, ch, stream, evs=None):
+        """Steps (a)-(e) | (f) | (g) through the three part calls; with `evs`
+        (two events) each boundary is recorded, so every part is timed on
+        its own."""
+        Qv, Kv, Vv, Kcv, Vcv = ch["views"]
+        Ks, Vs = ch["sel"]
+        q.quoka_select(Qv, Kv, self.w.NQ, ch["bsa"], kv_idx=ch["kv_idx"], kv_count=ch["kv_count"], ws=ch["ws"],
+                       stream=stream)
+        if evs is not None:
+            evs[0].record(stream)
+        q.quoka_gather_kv(Kv, Vv, ch["kv_idx"], ch["kv_count"], Ksel=Ks, Vsel=Vs, ws=ch["ws"], stream=stream)
+        if evs is not None:
+            evs[1].record(stream)
+        q.quoka_sparse_gqa_attn_gathered(Qv, Ks, Vs, ch["kv_count"], Kcv, Vcv, O=ch["O"], ws=ch["ws"],
+                                         stream=stream)
+
+    # algorithmic work of one step
+    def flops(self):
+        w = self.w
+        return sum(attn_flops(w.b, w.nq, w.d, self.BCP, ch["bsa_eff"]) for ch in self.chunks)
+
+    def select_bytes(self):
+        w = self.w
+        return sum(select_bytes(w.b, w.nq, w.nkv, w.d, ch["T"], self.BCP, ch["bsa_eff"], self.es)
+                   for ch in self.chunks)
+
+    def gather_bytes(self):
+        w = self.w
+        return sum(gather_bytes(w.b, w.nkv, w.d, ch["bsa_eff"], self.es) for ch in self.chunks)
+
+    def keys(self):
+        return sum(self.w.b * self.w.nkv * ch["T"] for ch in self.chunks)
+
+    def tokens(self):
+        return self.w.b * self.BCP * len(self.chunks)
+
+    def launches(self):
+        return sum(kernels_per_chunk(self.w, ch["T"], ch["bsa_eff"]) for ch in self.chunks)
+
+    def status_ok(self, q):
+        return all(q.quoka_get_device_status(ch["ws"]) == 0 for ch in self.chunks)
+
+
+def time_run(q, run, steps, warmup, flush, stream, world, dev, sampler=None):
+    """W warm-up steps, then K timed steps of quoka_prefill_chunk (events at
+    the step's two ends only, L2 flushed before each step, outside the
+    events), then K steps of the part calls with an event at every
+    boundary. Timings are maxima over the ranks."""
+    for _ in range(warmup):
+        for ch in run.chunks:
+            run.parts(q, ch, stream)
+            run.whole(q, ch, stream)
+    torch.cuda.synchronize()
+    if not run.status_ok(q):
+        raise RuntimeError(f"device status after the warm-up of {run.w.name}")
+    if sampler is not None:
+        sampler.start()
+        time.sleep(0.3)
+        # a short untimed burst so the sampler sees the GPU under load
+        for _ in range(max(3, warmup)):
+            for ch in run.chunks:
+                run.whole(q, ch, stream)
+    if world > 1:
+        torch.distributed.barrier()
+    torch.cuda.synchronize()
+    step_evs = []
+    for _ in range(steps):
+        flush.fill_(1)
+        e = [torch.cuda.Event(enable_timing=True) for _ in range(2)]
+        e[0].record(stream)
+        for ch in run.chunks:
+            run.whole(q, ch, stream)
+        e[1].record(stream)
+        step_evs.append(e)
+    torch.cuda.synchronize()
+    t_step = sum(a.elapsed_time(b) for a, b in step_evs)
+    if world > 1:
+        torch.distributed.barrier()
+    n = len(run.chunks)
+    per_chunk = [0.0] * n
+    t_sel = t_gather = t_attn = 0.0
+    evs = []
+    for _ in range(steps):
+        flush.fill_(1)
+        one = []
+        for ch in run.chunks:
+            e = [torch.cuda.Event(enable_timing=True) for _ in range(4)]
+            e[0].record(stream)
+            run.parts(q, ch, stream, evs=e[1:3])
+            e[3].record(stream)
+            one.append(e)
+        evs.append(one)
+    torch.cuda.synchronize()
+    for one in evs:
+        for c, e in enumerate(one):
+            a, g, at = e[0].elapsed_time(e[1]), e[1].elapsed_time(e[2]), e[2].elapsed_time(e[3])
+            t_sel += a
+            t_gather += g
+            t_attn += at
+            per_chunk[c] += a + g + at
+    clocks = sampler.stop() if sampler is not None else None
+    if world > 1:
+        torch.distributed.barrier()
+    if not run.status_ok(q):
+        raise RuntimeError(f"device status after timing {run.w.name}")
+    vals = max_over_ranks([t_step / steps, t_sel / steps, t_gather / steps, t_attn / steps]
+                          + [p / steps for p in per_chunk], world, dev)
+    return {"ms_step": vals[0], "ms_select": vals[1], "ms_gather": vals[2], "ms_attention": vals[3],
+            "per_chunk_ms": vals[4:], "clocks": clocks}
+
+
+def rooflines(run, t, world):
+    """Throughput and roofline figures of a timed run (see time_run)."""
+    hbm, tf_burst, _, peak_src = _peaks()
+    w = run.w
+    flops, sbytes, gbytes = run.flops(), run.select_bytes(), run.gather_bytes()
+    attn_tflops = flops / (t["ms_attention"] / 1e3) / 1e12
+    sel_gbs = sbytes / (t["ms_select"] / 1e3) / 1e9
+    g_gbs = gbytes / (t["ms_gather"] / 1e3) / 1e9
+    return {
+        "value": job_throughput(world, run.tokens(), t["ms_step"]),
+        "keys_scored_per_s": world * run.keys() / (t["ms_select"] / 1e3),
+        "keys_scored_per_s_query_heads": world * run.keys() * (w.nq // w.nkv) / (t["ms_select"] / 1e3),
+        "roofline": {"kernel": ("sparse GQA attention (tcgen05)" if w.dtype == "bf16"
+                                else "sparse GQA attention (fp32 CUDA cores)"),
+                     "bound": "tensor", "achieved": attn_tflops, "peak": tf_burst, "unit": "TFLOP/s",
+                     "frac": attn_tflops / tf_burst, "traffic": None,
+                     "peak_kind": f"bf16 dense, burst, {peak_src}",
+                     "algorithmic_flops_per_launch": flops / max(1, len(run.chunks))},
+        "roofline_select": {"steps": "(a)-(e)", "bound": "hbm", "achieved": sel_gbs, "peak": hbm, "unit": "GB/s",
+                            "frac": sel_gbs / hbm, "frac_of_8TBs": sel_gbs / 8000.0,
+                            "algorithmic_bytes_per_step": sbytes},
+        "roofline_gather": {"steps": "(f)", "bound": "hbm", "achieved": g_gbs, "peak": hbm, "unit": "GB/s",
+                            "frac": g_gbs / hbm, "algorithmic_bytes_per_step": gbytes},
+    }
+
+
 def run_ours(args, rank, world, local_rank):
     import sparse_kv_selection_quoka_b200 as q
-    from sparse_kv_selection_quoka_b200 import inputs
 
     q.load()
     dev = torch.device("cuda", local_rank)
     torch.cuda.set_device(dev)
-    w, x = make_inputs(args.workload, rank)
-    tdt = torch.bfloat16 if w.dtype == "bf16" else torch.float32
-    es = 2 if w.dtype == "bf16" else 4
     flush = torch.empty(FLUSH_BYTES, dtype=torch.uint8, device=dev)
     stream = torch.cuda.current_stream()
-
-    def to_dev(a):
-        return torch.from_numpy(np.ascontiguousarray(a, dtype=np.float32)).to(tdt).to(dev)
-
-    sweep = w.name.startswith("sweep")
-    if sweep:
-        Qs, Ks, Vs = (to_dev(a) for a in (x.Qs, x.Ks, x.Vs))
-        L = x.BCP
-        chunks = []
-        for c in range(x.n_chunks):
-            T = c * L
-            bsa = x.budget(T)
-            views = (Qs[:, :, T:T + L], Ks[:, :, :T], Vs[:, :, :T], Ks[:, :, T:T + L], Vs[:, :, T:T + L])
-            ws = q.workspace_for(views[0], views[1], x.NQ, bsa)
-            O = torch.empty((w.b, w.nq, L, w.d), dtype=tdt, device=dev)
-            kv_idx = torch.empty((w.b, w.nkv, min(bsa, T)), dtype=torch.int32, device=dev)
-            kv_count = torch.empty((w.b, w.nkv), dtype=torch.int32, device=dev)
-            sel_kv = tuple(torch.empty((w.b, w.nkv, min(bsa, T), w.d), dtype=tdt, device=dev) for _ in range(2))
-            chunks.append((views, bsa, ws, O, kv_idx, kv_count, T, sel_kv))
-    else:
-        Q, K, V, Kc, Vc = (to_dev(a) for a in (x.Q, x.K, x.V, x.Kc, x.Vc))
-        bsa_eff = min(w.BSA, w.T)
-        ws = q.workspace_for(Q, K, w.NQ, w.BSA)
-        O = torch.empty((w.b, w.nq, w.BCP, w.d), dtype=tdt, device=dev)
-        kv_idx = torch.empty((w.b, w.nkv, bsa_eff), dtype=torch.int32, device=dev)
-        kv_count = torch.empty((w.b, w.nkv), dtype=torch.int32, device=dev)
-        sel_kv = tuple(torch.empty((w.b, w.nkv, bsa_eff, w.d), dtype=tdt, device=dev) for _ in range(2))
-        chunks = [((Q, K, V, Kc, Vc), w.BSA, ws, O, kv_idx, kv_count, w.T, sel_kv)]
-
-    def one_chunk(ch, evs=None):
-        """Steps (a)-(e) | (f) | (g) through the public calls; with `evs`
-        (three events) each boundary is recorded, so every part is timed on
-        its own: quoka_sparse_gqa_attn with a full workspace runs exactly
-        the gather and attention kernels below."""
-        (Qv, Kv, Vv, Kcv, Vcv), bsa, wsb, Ob, idx, cnt, _, (Ks, Vs) = ch
-        q.quoka_select(Qv, Kv, w.NQ, bsa, kv_idx=idx, kv_count=cnt, ws=wsb, stream=stream)
-        if evs is not None:
-            evs[0].record(stream)
-        q.quoka_gather_kv(Kv, Vv, idx, cnt, Ksel=Ks, Vsel=Vs, ws=wsb, stream=stream)
-        if evs is not None:
-            evs[1].record(stream)
-        q.quoka_sparse_gqa_attn_gathered(Qv, Ks, Vs, cnt, Kcv, Vcv, O=Ob, ws=wsb, stream=stream)
-
-    def whole_chunk(ch):
-        """Steps (a)-(g) as one call, quoka_prefill_chunk: the same kernels as
-        one_chunk, chained on the stream with no event in between."""
-        (Qv, Kv, Vv, Kcv, Vcv), bsa, wsb, Ob, idx, _, _, _ = ch
-        q.quoka_prefill_chunk(Qv, Kv, Vv, Kcv, Vcv, w.NQ, bsa, O=Ob, kv_idx=idx,
-                              ws=wsb, stream=stream)
-
-    for _ in range(args.warmup):
-        for ch in chunks:
-            one_chunk(ch)
-            whole_chunk(ch)
-    torch.cuda.synchronize()
-    status = q.quoka_get_device_status(chunks[-1][2])
-    if status != 0:
-        raise RuntimeError(f"device status {status} after warm-up")
-
+    run = WorkloadRun(q, args.workload, rank, dev)
+    w = run.w
     sampler = ClockSampler(local_rank)
-    sampler.start()
-    time.sleep(0.3)
-    # a short untimed burst so the sampler sees the GPU under load
-    for _ in range(max(3, args.warmup)):
-        for ch in chunks:
-            one_chunk(ch)
-    if world > 1:
-        torch.distributed.barrier()
-    torch.cuda.synchronize()
-    n_ev = len(chunks)
-    # The step: quoka_prefill_chunk per chunk with events only at the step's
-    # two ends, so the kernels overlap at their edges as they do for a user
-    # (programmatic dependent launch within the call).
-    t_step = 0.0
-    per_chunk = [0.0] * n_ev
-    step_evs = []
-    for _ in range(args.steps):
-        flush.fill_(1)
-        e = [torch.cuda.Event(enable_timing=True) for _ in range(2)]
-        e[0].record(stream)
-        for ch in chunks:
-            whole_chunk(ch)
-        e[1].record(stream)
-        step_evs.append(e)
-    torch.cuda.synchronize()
-    for e in step_evs:
-        t_step += e[0].elapsed_time(e[1])
-    # The parts, timed in a second pass with an event at every boundary
-    # (which serialises the parts): select (a)-(e), gather (f), attention (g).
-    if world > 1:
-        torch.distributed.barrier()
-    t_sel, t_gather, t_attn = 0.0, 0.0, 0.0
-    evs = []
-    for _ in range(args.steps):
-        flush.fill_(1)
-        step_evs = []
-        for ch in chunks:
-            e = [torch.cuda.Event(enable_timing=True) for _ in range(5)]
-            e[0].record(stream)
-            one_chunk(ch, evs=e[1:4])
-            e[4].record(stream)
-            step_evs.append(e)
-        evs.append(step_evs)
-    torch.cuda.synchronize()
-    if world > 1:
-        torch.distributed.barrier()
-    for step_evs in evs:
-        for c, e in enumerate(step_evs):
-            a, g, bms = e[0].elapsed_time(e[1]), e[1].elapsed_time(e[2]), e[2].elapsed_time(e[4])
-            t_sel += a
-            t_gather += g
-            t_attn += bms
-            per_chunk[c] += a + g + bms
-    clocks = sampler.stop()
-
+    t = time_run(q, run, args.steps, args.warmup, flush, stream, world, dev, sampler=sampler)
+    rf = rooflines(run, t, world)
     K_ = args.steps
-    ms_step, ms_sel, ms_gather, ms_attn = max_over_ranks(
-        [t_step / K_, t_sel / K_, t_gather / K_, t_attn / K_], world, dev)
-
-    tokens_per_step = w.b * (w.T if sweep else w.BCP)
-    if sweep:
-        tokens_per_step = w.b * x.n_chunks * x.BCP
-    value = job_throughput(world, tokens_per_step, ms_step)
-
-    hbm, tf_burst, tf_sus, peak_src = _peaks()
-    if sweep:
-        flops = sum(attn_flops(w.b, w.nq, w.d, x.BCP, min(ch[1], ch[6])) for ch in chunks)
-        sbytes = sum(select_bytes(w.b, w.nq, w.nkv, w.d, ch[6], x.BCP, min(ch[1], ch[6]), es) for ch in chunks)
-        gbytes = sum(gather_bytes(w.b, w.nkv, w.d, min(ch[1], ch[6]), es) for ch in chunks)
-        keys = sum(w.b * w.nkv * ch[6] for ch in chunks)
-    else:
-        flops = attn_flops(w.b, w.nq, w.d, w.BCP, min(w.BSA, w.T))
-        sbytes = select_bytes(w.b, w.nq, w.nkv, w.d, w.T, w.BCP, min(w.BSA, w.T), es)
-        gbytes = gather_bytes(w.b, w.nkv, w.d, min(w.BSA, w.T), es)
-        keys = w.b * w.nkv * w.T
-    attn_tflops = flops / (ms_attn / 1e3) / 1e12
-    sel_gbs = sbytes / (ms_sel / 1e3) / 1e9
     out = {
         "metric": METRIC,
-        "value": value,
+        "value": rf["value"],
         "unit": UNIT,
         "n_gpus": world,
         "steps": K_,
         "warmup": args.warmup,
-        "ms_per_step": ms_step,
+        "ms_per_step": t["ms_step"],
         "higher_is_better": True,
         "scaling": "weak",
         "vs_baseline": None,
         "dtype": w.dtype,
-        "data": "synthetic (seeded; shapes and value structure of the workload, see DESIGN.md)",
+        "data": "synthetic (seeded; the workload's shapes and planted value structure)",
         "config": {"workload": w.name, "b": w.b, "nq": w.nq, "nkv": w.nkv, "d": w.d,
                    "T": w.T, "BCP": w.BCP, "NQ": w.NQ, "BSA": w.BSA, "parallelism": f"replicas{world}",
                    "l2": "flushed before every timed step (256 MiB write, untimed)"},
-        "keys_scored_per_s": world * keys / (ms_sel / 1e3),
-        "keys_scored_per_s_query_heads": world * keys * (w.nq // w.nkv) / (ms_sel / 1e3),
-        "ms_select": ms_sel,
-        "ms_gather": ms_gather,
-        "ms_attention": ms_attn,
-        "roofline": {"kernel": "sparse GQA attention (tcgen05)" if w.dtype == "bf16" else "sparse GQA attention (fp32 CUDA cores)",
-                     "bound": "tensor", "achieved": attn_tflops, "peak": tf_burst,
-                     "unit": "TFLOP/s", "frac": attn_tflops / tf_burst,
-                     "traffic": (_profiled_traffic("attn_tma_qwen3-4b_T32k.md",
-                                                   "sparse_kv_selection_quoka_b200/csrc/attn_tma.cu",
-                                                   "sparse_kv_selection_quoka_b200/csrc/attn_common.cuh")
-                                 if w.name == "qwen3-4b_T32k" and w.dtype == "bf16" else None),
-                     "peak_kind": f"bf16 dense, burst, {peak_src}",
-                     "algorithmic_flops_per_launch": flops / max(1, len(chunks))},
-        "roofline_select": {"steps": "(a)-(e)", "bound": "hbm", "achieved": sel_gbs, "peak": hbm,
-                            "unit": "GB/s", "frac": sel_gbs / hbm, "frac_of_8TBs": sel_gbs / 8000.0,
-                            "algorithmic_bytes_per_step": sbytes},
-        "roofline_gather": {"steps": "(f)", "bound": "hbm", "achieved": gbytes / (ms_gather / 1e3) / 1e9,
-                            "peak": hbm, "unit": "GB/s", "frac": gbytes / (ms_gather / 1e3) / 1e9 / hbm,
-                            "algorithmic_bytes_per_step": gbytes},
-        "clocks": clocks,
-        "gpu_launches": sum(kernels_per_chunk(ch[6], min(ch[1], ch[6])) for ch in chunks) * K_,
+        "keys_scored_per_s": rf["keys_scored_per_s"],
+        "keys_scored_per_s_query_heads": rf["keys_scored_per_s_query_heads"],
+        "ms_select": t["ms_select"],
+        "ms_gather": t["ms_gather"],
+        "ms_attention": t["ms_attention"],
+        "roofline": rf["roofline"],
+        "roofline_select": rf["roofline_select"],
+        "roofline_gather": rf["roofline_gather"],
+        "clocks": t["clocks"],
+        "gpu_launches": run.launches() * K_,
     }
-    if sweep:
-        out["per_chunk_ms"] = [p / K_ for p in per_chunk]
+    if w.name == "qwen3-4b_T32k" and w.dtype == "bf16":
+        out["roofline"]["traffic_from_committed_profile"] = _profiled_traffic(
+            "attn_tma_qwen3-4b_T32k.md", "sparse_kv_selection_quoka_b200/csrc/attn_tma.cu",
+            "sparse_kv_selection_quoka_b200/csrc/attn_common.cuh")
+    if run.sweep:
+        out["per_chunk_ms"] = t["per_chunk_ms"]
     else:
+        Q, K, V, Kc, Vc = run.dev_inputs
         out["decode"] = measure_decode(q, w, dev, stream, flush, Q, K, V, Kc, Vc, min(K_, 50))
     if not args.no_e2e:
-        out["e2e"] = run_e2e(args, w, x, chunks, q, dev, stream, tokens_per_step, world, sweep)
+        out["e2e"] = run_e2e(args, run, q, dev, stream, world)
+    if not args.no_other_workloads and args.workload == DEFAULT_WORKLOAD:
+        out["per_workload"] = other_workloads(q, args, rank, world, dev, stream, flush, exclude=w.name)
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
-        out["cpu_baseline"] = cpu_baseline(w, x, sweep)
+        out["cpu_baseline"] = cpu_baseline(run.w, run.x, run.sweep)
+    return out
+
+
+def other_workloads(q, args, rank, world, dev, stream, flush, exclude):
+    """The same measurement (no e2e, decode or oracle legs) on the other
+    bf16 workloads: the Llama-shaped layer, the chunked-prefill sweep (with
+    its per-chunk time curve) and the 128K-key layer."""
+    out = {}
+    for name in OTHER_WORKLOADS:
+        if name == exclude:
+            continue
+        run = WorkloadRun(q, name, rank, dev)
+        steps = max(3, min(args.steps, 50 if not run.sweep else 10))
+        t = time_run(q, run, steps, 3, flush, stream, world, dev)
+        rf = rooflines(run, t, world)
+        w = run.w
+        entry = {"config": {"b": w.b, "nq": w.nq, "nkv": w.nkv, "d": w.d, "T": w.T, "BCP": w.BCP, "NQ": w.NQ,
+                            "BSA": w.BSA if not run.sweep else "25% of T (min 256)"},
+                 "steps": steps, "ms_per_step": t["ms_step"], "value": rf["value"], "unit": UNIT,
+                 "keys_scored_per_s": rf["keys_scored_per_s"], "ms_select": t["ms_select"],
+                 "ms_gather": t["ms_gather"], "ms_attention": t["ms_attention"], "roofline": rf["roofline"],
+                 "roofline_select": rf["roofline_select"], "roofline_gather": rf["roofline_gather"],
+                 "gpu_launches": run.launches() * steps}
+        if run.sweep:
+            entry["per_chunk_ms"] = t["per_chunk_ms"]
+        out[name] = entry
+        del run
+        torch.cuda.empty_cache()
     return out
 
 
@@ -442,43 +533,34 @@ def measure_decode(q, w, dev, stream, flush, Q, K, V, Kc, Vc, steps):
     return out
 
 
-def run_e2e(args, w, x, chunks, q, dev, stream, tokens_per_step, world, sweep):
+def run_e2e(args, run, q, dev, stream, world):
     """The same metric through the public whole-step call with host buffers:
     every step copies that step's inputs from pinned host memory to the
     device, runs quoka_prefill_chunk, and copies the output back."""
-    tdt = chunks[0][3].dtype
-    hosts, devs, outs = [], [], []
-    h2d = d2h = 0
-    if sweep:
-        # the whole sequence's inputs are uploaded once per step
-        host = [torch.from_numpy(np.ascontiguousarray(a, dtype=np.float32)).to(tdt).pin_memory()
-                for a in (x.Qs, x.Ks, x.Vs)]
-        dbuf = [torch.empty_like(h, device=dev) for h in host]
-        h2d = sum(h.numel() * h.element_size() for h in host)
-    else:
-        host = [torch.from_numpy(np.ascontiguousarray(a, dtype=np.float32)).to(tdt).pin_memory()
-                for a in (x.Q, x.K, x.V, x.Kc, x.Vc)]
-        dbuf = [torch.empty_like(h, device=dev) for h in host]
-        h2d = sum(h.numel() * h.element_size() for h in host)
-    O_host = [torch.empty(ch[3].shape, dtype=tdt).pin_memory() for ch in chunks]
+    x, w, tdt = run.x, run.w, run.tdt
+    arrays = (x.Qs, x.Ks, x.Vs) if run.sweep else (x.Q, x.K, x.V, x.Kc, x.Vc)
+    host = [torch.from_numpy(np.ascontiguousarray(a, dtype=np.float32)).to(tdt).pin_memory() for a in arrays]
+    dbuf = [torch.empty_like(h, device=dev) for h in host]
+    h2d = sum(h.numel() * h.element_size() for h in host)
+    O_host = [torch.empty(ch["O"].shape, dtype=tdt).pin_memory() for ch in run.chunks]
     d2h = sum(o.numel() * o.element_size() for o in O_host)
 
     def step():
         for h, d_ in zip(host, dbuf):
             d_.copy_(h, non_blocking=True)
-        if sweep:
+        if run.sweep:
             Qs, Ks, Vs = dbuf
-            for c, ch in enumerate(chunks):
-                T = ch[6]
-                L = x.BCP
+            L = run.BCP
+            for c, ch in enumerate(run.chunks):
+                T = ch["T"]
                 q.quoka_prefill_chunk(Qs[:, :, T:T + L], Ks[:, :, :T], Vs[:, :, :T], Ks[:, :, T:T + L],
-                                      Vs[:, :, T:T + L], w.NQ, ch[1], O=ch[3], ws=ch[2], stream=stream)
-                O_host[c].copy_(ch[3], non_blocking=True)
+                                      Vs[:, :, T:T + L], w.NQ, ch["bsa"], O=ch["O"], ws=ch["ws"], stream=stream)
+                O_host[c].copy_(ch["O"], non_blocking=True)
         else:
             Q, K, V, Kc, Vc = dbuf
-            ch = chunks[0]
-            q.quoka_prefill_chunk(Q, K, V, Kc, Vc, w.NQ, w.BSA, O=ch[3], ws=ch[2], stream=stream)
-            O_host[0].copy_(ch[3], non_blocking=True)
+            ch = run.chunks[0]
+            q.quoka_prefill_chunk(Q, K, V, Kc, Vc, w.NQ, w.BSA, O=ch["O"], ws=ch["ws"], stream=stream)
+            O_host[0].copy_(ch["O"], non_blocking=True)
 
     for _ in range(max(1, args.warmup // 2)):
         step()
@@ -495,9 +577,21 @@ def run_e2e(args, w, x, chunks, q, dev, stream, tokens_per_step, world, sweep):
     if world > 1:
         torch.distributed.barrier()
     ms = max_over_ranks([e0.elapsed_time(e1) / n], world, dev)[0]
-    return {"value": job_throughput(world, tokens_per_step, ms), "unit": UNIT, "ms_per_step": ms,
+    # what bounds it: the host-to-device copy of the inputs, alone
+    e2, e3 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e2.record(stream)
+    for _ in range(n):
+        for h, d_ in zip(host, dbuf):
+            d_.copy_(h, non_blocking=True)
+    e3.record(stream)
+    torch.cuda.synchronize()
+    ms_h2d = max_over_ranks([e2.elapsed_time(e3) / n], world, dev)[0]
+    return {"value": job_throughput(world, run.tokens(), ms), "unit": UNIT, "ms_per_step": ms,
             "steps": n, "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
-            "call": "quoka_prefill_chunk (C ABI) with pinned-host inputs copied in and O copied out every step"}
+            "h2d_gbs_in_step": h2d / (ms / 1e3) / 1e9,
+            "ms_h2d_copies_alone": ms_h2d, "h2d_gbs_alone": h2d / (ms_h2d / 1e3) / 1e9,
+            "call": "quoka_prefill_chunk (C ABI) with pinned-host inputs copied in and O copied out every step; "
+                    "the input copy bounds it"}
 
 
 # ---------------------------------------------------------------- CPU oracle
@@ -521,29 +615,48 @@ def _oracle_head_step(x, j):
     return orc.prefill_chunk(Qj, x.K[:, sl], x.V[:, sl], x.Kc[:, sl], x.Vc[:, sl], x.NQ, x.BSA)
 
 
-def cpu_baseline(w, x, sweep, budget_s=12.0):
-    """The oracle as it stands on the host cores, on a bounded sample of the
-    workload: whole KV-head groups (1/nkv of a step each) until ~budget_s."""
-    if sweep:
-        x = x.chunk(x.n_chunks // 2)
+def _time_oracle_groups(x, nkv, budget_s, max_groups):
+    """Times whole KV-head groups of the oracle until budget_s or
+    max_groups; returns (groups, seconds)."""
     t0 = time.perf_counter()
     n = 0
     while True:
-        _oracle_head_step(x, n % w.nkv)
+        _oracle_head_step(x, n % nkv)
         n += 1
-        if time.perf_counter() - t0 >= budget_s or n >= 4 * w.nkv:
+        if time.perf_counter() - t0 >= budget_s or n >= max_groups:
             break
-    dt = time.perf_counter() - t0
-    tokens = x.Q.shape[0] * x.Q.shape[2] * n / w.nkv
-    return {"value": tokens / dt, "unit": UNIT, "cores": _blas_threads(), "kind": "oracle",
-            "sample": f"{n} KV-head groups ({n}/{w.nkv} of a step) of workload {w.name}"
-                      + (" (chunk 32 of the sweep)" if sweep else "") + f", {dt:.1f} s",
-            "host_cpu_count": os.cpu_count()}
+    return n, time.perf_counter() - t0
+
+
+def cpu_baseline(w, x, sweep, budget_s=10.0):
+    """The oracle as it stands on the host cores, on a bounded sample of the
+    workload: whole KV-head groups (1/nkv of a step each), timed with the
+    BLAS pool at its default size (all cores) and again with one thread."""
+    if sweep:
+        x = x.chunk(x.n_chunks // 2)
+    tokens_per_group = x.Q.shape[0] * x.Q.shape[2] / w.nkv
+    n, dt = _time_oracle_groups(x, w.nkv, budget_s, 2 * w.nkv)
+    out = {"value": tokens_per_group * n / dt, "unit": UNIT, "cores": _blas_threads(), "kind": "oracle",
+           "sample": f"{n} KV-head groups (each 1/{w.nkv} of a step) of workload {w.name}"
+                     + (" (chunk 32 of the sweep)" if sweep else "") + f", {dt:.1f} s",
+           "host_cpu_count": os.cpu_count()}
+    try:
+        import threadpoolctl
+        with threadpoolctl.threadpool_limits(1):
+            n1, dt1 = _time_oracle_groups(x, w.nkv, budget_s, w.nkv)
+        out["one_thread"] = {"value": tokens_per_group * n1 / dt1, "unit": UNIT, "cores": 1,
+                             "sample": f"{n1} KV-head groups, {dt1:.1f} s"}
+    except ImportError:
+        out["one_thread"] = None
+    return out
 
 
 def run_reference(args, rank, world):
-    """The CPU oracle as the reference arm: each step is one KV-head group of
-    the workload (1/nkv of the work), on the host cores."""
+    """The CPU oracle as the reference arm. Its step is a bounded sample of
+    the workload: one KV-head group (the G query heads of one KV head over
+    the whole chunk, 1/nkv of the work, heads being independent through
+    every step). ms_per_step is the measured time of that sample, and the
+    metric counts the chunk tokens it stands for (BCP * b / nkv)."""
     if rank != 0:
         return None
     from sparse_kv_selection_quoka_b200 import inputs
@@ -556,19 +669,19 @@ def run_reference(args, rank, world):
     for s in range(args.steps):
         _oracle_head_step(x, s % w.nkv)
     dt = time.perf_counter() - t0
-    ms_sample = dt / args.steps * 1e3
-    ms_step = ms_sample * w.nkv
-    tokens = x.Q.shape[0] * x.Q.shape[2]
+    ms_step = dt / args.steps * 1e3
+    tokens = x.Q.shape[0] * x.Q.shape[2] / w.nkv
     value = tokens / (ms_step / 1e3)
     cores = _blas_threads()
+    sample = f"one KV-head group per step (1/{w.nkv} of a step of {w.name}: {tokens:g} chunk-tokens' worth)"
     return {"impl": "reference", "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world,
             "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms_step,
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
             "data": "synthetic (seeded)",
             "config": {"workload": w.name, "b": w.b, "nq": w.nq, "nkv": w.nkv, "d": w.d, "T": w.T,
-                       "BCP": w.BCP, "NQ": w.NQ, "BSA": w.BSA, "parallelism": "host cores"},
-            "cpu_baseline": {"value": value, "unit": UNIT, "cores": cores, "kind": "oracle",
-                             "sample": f"one KV-head group (1/{w.nkv} of the step) per timed step"},
+                       "BCP": w.BCP, "NQ": w.NQ, "BSA": w.BSA, "parallelism": "host cores",
+                       "sample": sample, "sampled_fraction_of_step": 1.0 / w.nkv},
+            "cpu_baseline": {"value": value, "unit": UNIT, "cores": cores, "kind": "oracle", "sample": sample},
             "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
             "gpu_launches": 0}
 
@@ -578,10 +691,12 @@ def main():
     ap.add_argument("--gpus", type=int, default=1)
     ap.add_argument("--steps", type=int, default=200)
     ap.add_argument("--warmup", type=int, default=20)
-    ap.add_argument("--workload", default="qwen3-4b_T32k")
+    ap.add_argument("--workload", default=DEFAULT_WORKLOAD)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-other-workloads", action="store_true",
+                    help="skip the per_workload block (the other bf16 workloads)")
     args = ap.parse_args()
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")

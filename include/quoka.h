@@ -9,9 +9,10 @@
  *   §2.2              cosine score S_ij = Q_i.K_j / (|Q_i| |K_j|)
  *   §2.3              GQA-aware aggregation: L2-normalise the chosen queries
  *                     and the keys, mean the queries over each KV head's
- *                     query-head group, S = Q_group K_norm^T (b,nkv,NQ,T),
- *                     S_agg = max over the NQ queries (b,nkv,T),
- *                     indices = topk(S_agg, BSA)
+ *                     query-head group, score every key against those group
+ *                     means (b,nkv,NQ,T), keep each key's largest score over
+ *                     the NQ queries (b,nkv,T), and select the BSA keys with
+ *                     the highest such score per KV head
  *   §4.2 problem 3    the selected KV is the attention's input KV, with the
  *                     causal mask off for it
  *
@@ -25,7 +26,8 @@
  *     the caller owns all memory. The library never allocates or frees
  *     device memory; scratch space is the caller's workspace `ws`
  *     (device pointer, at least quoka_workspace_size() bytes, 256-byte
- *     aligned).
+ *     aligned). The one exception is quoka_select_static, whose scratch is a
+ *     fixed device array inside the library (see its declaration).
  *   - `stream` is a cudaStream_t passed as void* (NULL = legacy default
  *     stream). Every call only enqueues work on it and returns; nothing
  *     synchronises with the host.
@@ -256,7 +258,8 @@ quoka_status quoka_decode_attn(const quoka_tensor* Q, const quoka_tensor* K,
                                float scale, void* O, float* lse, void* ws,
                                size_t ws_bytes, void* stream);
 
-/* The whole step (a)-(g): quoka_select followed by quoka_sparse_gqa_attn on
+/* The whole step (a)-(g), [QUOKA §2.1 Algorithm 1, §2.2, §2.3, §4.2 problem
+ * 3]: quoka_select followed by quoka_sparse_gqa_attn on
  * one stream, with no host synchronisation in between; for a short chunk
  * (G * BCP <= 64 query rows per KV head, d = 64 or 128) the attention is
  * quoka_decode_attn's. ws must hold quoka_workspace_size() bytes.
@@ -351,6 +354,38 @@ quoka_status quoka_combine_partials(const void* O_parts, const float* lse_parts,
  * the synchronisation failed, QUOKA_ERR_INVALID_ARG for NULL pointers. */
 quoka_status quoka_get_device_status(const void* ws, void* stream,
                                      int32_t* device_status);
+
+/* Synchronises `stream`, then reads the fault-site word of `ws` (the word
+ * after the status word) into *site: 0 when the latest call that used ws
+ * latched no device fault, else a small code naming the kernel and the wait
+ * or check where the first fault happened (diagnostic only; the codes of
+ * the scoring kernel are 51-57, those of the attention 11-15, 21-27 and
+ * 31-33). Returns as quoka_get_device_status. */
+quoka_status quoka_get_device_fault_site(const void* ws, void* stream,
+                                         int32_t* site);
+
+/* Test hooks of the tensor-core scoring and attention kernels (bf16,
+ * d = 128). The QUOKA write-up has no counterpart: they exist so that a test
+ * can run the timeout path of those kernels without hanging the GPU.
+ *   wait_limit_ns  bound of every wait inside those kernels for the launches
+ *                  that follow (0 restores the default of 2 s).
+ *   inject         QUOKA_DEBUG_INJECT_NONE, or one barrier made to expect
+ *                  one arrival more than it ever receives in every launch
+ *                  that follows: QUOKA_DEBUG_INJECT_SCORE (the scoring
+ *                  kernel's release of its first TMEM accumulator) or
+ *                  QUOKA_DEBUG_INJECT_ATTN (the attention's first release
+ *                  of P to the P V product). The waiting warp gives up after
+ *                  wait_limit_ns, latches QUOKA_ERR_TIMEOUT and a fault site
+ *                  in ws, and the kernel unwinds (in-flight copies and
+ *                  products drained, TMEM freed); the outputs of that call
+ *                  are unspecified.
+ * Process-wide and read at launch time: set them only while no other
+ * thread launches this library's kernels, and reset them with (0, NONE).
+ * Returns QUOKA_ERR_INVALID_ARG for an unknown `inject`. */
+#define QUOKA_DEBUG_INJECT_NONE 0u
+#define QUOKA_DEBUG_INJECT_SCORE 1u
+#define QUOKA_DEBUG_INJECT_ATTN 2u
+quoka_status quoka_debug_set_wait_hooks(uint64_t wait_limit_ns, uint32_t inject);
 
 /* A static, human-readable name of a status code. */
 const char* quoka_status_string(quoka_status status);

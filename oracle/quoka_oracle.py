@@ -121,7 +121,8 @@ def select_queries(SQ, NQ: int) -> np.ndarray:
 
 # ---------------------------------------------------------------------------
 # Step (c): normalise the chosen queries, mean over each GQA group
-# [QUOKA §2.3: Q_norm = Q / norm(Q), Q_group = mean over the group axis]
+# [QUOKA §2.3: each chosen query divided by its L2 norm, then averaged over
+#  the query heads of its KV head's group]
 # ---------------------------------------------------------------------------
 
 def group_queries(Q, q_idx, nkv: int, normalize: bool = True) -> np.ndarray:
@@ -169,7 +170,8 @@ def key_scores(Q_group, K, normalize: bool = True) -> np.ndarray:
 
 
 # ---------------------------------------------------------------------------
-# Step (e): top-BSA keys per KV head   [QUOKA §2.3: indices = topk(S_agg, BSA)]
+# Step (e): top-BSA keys per KV head   [QUOKA §2.3: the BSA keys with the
+# highest aggregated score are kept]
 # ---------------------------------------------------------------------------
 
 def select_keys(S_agg, BSA: int) -> np.ndarray:

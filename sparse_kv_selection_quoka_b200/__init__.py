@@ -21,6 +21,8 @@ __all__ = [
     "quoka_sparse_gqa_attn_gathered",
     "quoka_prefill_chunk",
     "quoka_get_device_status",
+    "quoka_get_device_fault_site",
+    "quoka_debug_set_wait_hooks",
     "quoka_status_string",
     "QuokaError",
     "quoka_select_static",

@@ -56,6 +56,8 @@ EXPORTS = (
     "quoka_combine_partials",
     "quoka_decode_workspace_size",
     "quoka_decode_attn",
+    "quoka_get_device_fault_site",
+    "quoka_debug_set_wait_hooks",
 )
 
 
@@ -135,6 +137,10 @@ def load() -> ctypes.CDLL:
         lib.quoka_decode_workspace_size.argtypes = [_I, _I, _I, _I, _I, _I, _I]
         lib.quoka_decode_attn.restype = _I
         lib.quoka_decode_attn.argtypes = [_T, _T, _T, _P, _P, _I, _T, _T, _F, _P, _P, _P, _SZ, _P]
+        lib.quoka_get_device_fault_site.restype = _I
+        lib.quoka_get_device_fault_site.argtypes = [_P, _P, ctypes.POINTER(ctypes.c_int32)]
+        lib.quoka_debug_set_wait_hooks.restype = _I
+        lib.quoka_debug_set_wait_hooks.argtypes = [ctypes.c_uint64, ctypes.c_uint32]
         lib.quoka_combine_partials.restype = _I
         lib.quoka_combine_partials.argtypes = [_P, _P, _I, _I, _I, _I, _I, _I, _P, _P, _P]
         _lib = lib
@@ -376,6 +382,28 @@ def quoka_get_device_status(ws, stream=None) -> int:
     st = lib.quoka_get_device_status(_ptr(ws), _stream(stream), ctypes.byref(out))
     _check(st, "quoka_get_device_status")
     return int(out.value)
+
+
+def quoka_get_device_fault_site(ws, stream=None) -> int:
+    """Synchronise the stream and return the fault-site word of ws (0: no
+    device fault in the latest call that used ws)."""
+    lib = load()
+    out = ctypes.c_int32(0)
+    st = lib.quoka_get_device_fault_site(_ptr(ws), _stream(stream), ctypes.byref(out))
+    _check(st, "quoka_get_device_fault_site")
+    return int(out.value)
+
+
+DEBUG_INJECT_NONE = 0
+DEBUG_INJECT_SCORE = 1
+DEBUG_INJECT_ATTN = 2
+
+
+def quoka_debug_set_wait_hooks(wait_limit_ns: int = 0, inject: int = DEBUG_INJECT_NONE) -> None:
+    """Test hooks of the tensor-core kernels: the bound of every wait (0 =
+    the default 2 s) and an injected barrier that never completes (see
+    include/quoka.h). Process-wide; reset with no arguments."""
+    _check(load().quoka_debug_set_wait_hooks(int(wait_limit_ns), int(inject)), "quoka_debug_set_wait_hooks")
 
 
 def quoka_status_string(status: int) -> str:

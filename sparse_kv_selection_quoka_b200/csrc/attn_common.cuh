@@ -51,10 +51,11 @@ __device__ __forceinline__ void record_abort(Smem& sm, int* status, int where) {
   latch_where(status, where);
 }
 
-// Warp-uniform bounded wait (every lane polls; all lanes agree on the result).
+// Warp-uniform bounded wait (every lane polls; all lanes agree on the
+// result), bounded by the kernel's wait limit sm.wait_ns.
 template <class Smem>
 __device__ __forceinline__ bool warp_wait(uint64_t* bar, uint32_t parity, Smem& sm, int* status, int where) {
-  const bool ok = mbar_wait(bar, parity, &sm.abort);
+  const bool ok = mbar_wait(bar, parity, &sm.abort, sm.wait_ns);
   const bool all_ok = __all_sync(0xffffffffu, ok);
   if (!all_ok && (threadIdx.x & 31) == 0) record_abort(sm, status, where);
   return all_ok;
@@ -119,38 +120,12 @@ __device__ __forceinline__ void issue_pv_part(uint32_t tmem_o, uint32_t tmem_p, 
   }
 }
 
-// 2^x for two values on the FMA pipe instead of the MUFU: x = n + f with n
-// the nearest integer (adding 1.5 * 2^23 rounds to it) and f in [-1/2, 1/2];
-// 2^f from a cubic fitted to it by least squares on Chebyshev nodes of
-// [-1/2, 1/2] (relative error below 8e-5, far under bf16 resolution); 2^n
-// added straight into the exponent field. x is clamped at -126, where the
-// result (about 1e-38) is as good as the MUFU's flushed zero for a softmax.
-__device__ __forceinline__ void exp2_fma_pair(uint64_t x, float& p0, float& p1) {
-  constexpr float kRound = 12582912.f;  // 1.5 * 2^23
-  float x0, x1;
-  f2_unpack(x, x0, x1);
-  const uint64_t xc = f2_pack(fmaxf(x0, -126.f), fmaxf(x1, -126.f));
-  const uint64_t j = f2_add(xc, f2_pack(kRound, kRound));          // n in the low mantissa bits
-  const uint64_t n = f2_add(j, f2_pack(-kRound, -kRound));
-  const uint64_t f = f2_fma(n, f2_pack(-1.f, -1.f), xc);          // x - n, exact
-  uint64_t q = f2_fma(f2_pack(0.055088683807510905f, 0.055088683807510905f), f,
-                      f2_pack(0.24260405145947916f, 0.24260405145947916f));
-  q = f2_fma(q, f, f2_pack(0.6932762416819607f, 0.6932762416819607f));
-  q = f2_fma(q, f, f2_pack(0.9999289403695112f, 0.9999289403695112f));
-  float q0, q1, j0, j1;
-  f2_unpack(q, q0, q1);
-  f2_unpack(j, j0, j1);
-  p0 = __uint_as_float(__float_as_uint(q0) + (__float_as_uint(j0) << 23));
-  p1 = __uint_as_float(__float_as_uint(q1) + (__float_as_uint(j1) << 23));
-}
-
 // One key tile of the online softmax of this thread's query row, single
 // pass: the row's 128 scores are read from TMEM once into registers. Key c
 // of the tile (key number base_n + c) is visible when base_n + c < lim. Then
 // the row max (3-input max tree), and P = 2^(s * qscale - m) in bf16 over
 // the first 64 S columns (packed two per column), with the products and row
-// sums in paired fp32 arithmetic; of every 8 key pairs, FMA_PAIRS take the
-// FMA-pipe exp2 and the rest the MUFU. The running max m moves only when it
+// sums in paired fp32 arithmetic and the exp2 on the MUFU. The running max m moves only when it
 // grows by more than RESCALE_THRESHOLD, in which case the O accumulator
 // (complete for the previous tiles) is rescaled in TMEM before any P of the
 // tile is released. P is released to the MMA issuer in PARTS equal key
@@ -159,7 +134,7 @@ __device__ __forceinline__ void exp2_fma_pair(uint64_t x, float& p0, float& p1) 
 // product of the first keys runs while the later ones are still being
 // exponentiated. Updates m and l. TMEM accesses are warp-collective: no
 // per-row branch surrounds one.
-template <int FMA_PAIRS, int PARTS>
+template <int PARTS>
 __device__ __forceinline__ void softmax_tile_split(uint32_t S, uint32_t O, bool have_o, int base_n, int lim,
                                                    float qscale, float& m, float& l, uint64_t* p_part) {
   constexpr int CPP = 4 / PARTS;  // 32-key chunks per part
@@ -205,15 +180,9 @@ __device__ __forceinline__ void softmax_tile_split(uint32_t S, uint32_t O, bool 
     for (int u = 0; u < 32; u += 2) {
       const int e = 32 * c + u;
       const uint64_t x = f2_fma(f2_pack(v[e], v[e + 1]), qs2, nm2);
-      float p0, p1;
-      if (((e >> 1) & 7) < FMA_PAIRS) {
-        exp2_fma_pair(x, p0, p1);
-      } else {
-        float x0, x1;
-        f2_unpack(x, x0, x1);
-        p0 = ex2(x0);
-        p1 = ex2(x1);
-      }
+      float x0, x1;
+      f2_unpack(x, x0, x1);
+      const float p0 = ex2(x0), p1 = ex2(x1);
       acc[(u >> 1) & 3] = f2_add(acc[(u >> 1) & 3], f2_pack(p0, p1));
       pk[u >> 1] = pack_bf16x2(p0, p1);
     }

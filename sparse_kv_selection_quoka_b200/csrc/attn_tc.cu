@@ -76,6 +76,7 @@ struct __align__(1024) AttnSmem {
   uint64_t xfer_full;   // (rank 0) rank 1's partial results have landed
   uint32_t tmem_base;
   int abort;
+  uint64_t wait_ns;     // bound of every wait
 };
 // The split-KV landing zone in rank 0 reuses the K/V ring (partial O, fp32,
 // [tile][row][128] with a per-row chunk rotation) and the Q area (m, l).
@@ -120,6 +121,7 @@ attn_gather_kernel(const __grid_constant__ AttnMaps maps, const AttnArgs a, int 
     mbar_init(&sm.xfer_free, 1);
     mbar_init(&sm.xfer_full, SOFTMAX_THREADS);
     sm.abort = 0;
+    sm.wait_ns = kWaitLimitNs;
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
   }
   if (warp == AT_MMA_WARP) {

@@ -36,8 +36,10 @@
 //   warp 10     TMA loads of each key tile's V (3-stage ring, a stage
 //               released by its PV).
 // TMEM: S0 | S1 | O0 | O1, 128 columns each (512).
-// Every wait is bounded: a wait that gives up records QUOKA_ERR_TIMEOUT and
-// the CTA unwinds (waits for in-flight copies and MMAs, frees TMEM).
+// Every wait is bounded (by the launch's wait limit, 2 s unless a test sets
+// another): a wait that gives up records QUOKA_ERR_TIMEOUT and a fault-site
+// code, and the CTA unwinds (waits for in-flight copies and MMAs, frees
+// TMEM, stores no output tile).
 #include <stddef.h>
 
 #include "attn_common.cuh"
@@ -57,10 +59,6 @@ constexpr int THREADS = 352;
 constexpr int MMA_WARP = 8;
 constexpr int LOAD_WARP = 9;    // Q and K
 constexpr int VLOAD_WARP = 10;  // V
-// Of every 8 key pairs, how many take the FMA-pipe exp2 in the softmax.
-// Measured on B200 (Qwen-shaped layer): 0 and 2 run equally fast, more is
-// slower; 0 keeps the kernel free of register spills.
-constexpr int SOFTMAX_FMA_PAIRS = 0;
 // P of a tile is released to the P V product in this many key ranges.
 constexpr int PV_PARTS = 2;
 
@@ -79,6 +77,7 @@ struct __align__(1024) Smem {
   uint64_t o_final, mma_done;
   uint32_t tmem_base;
   int abort;
+  uint64_t wait_ns;  // bound of every wait
 };
 
 // TMA boxes of one 128-row tile (two 64-column atoms).
@@ -95,7 +94,7 @@ template <int STAGES>
 __device__ __forceinline__ void drain_ring(Smem& sm, uint64_t* full, int nload, int* status, int where) {
   for (int s = 0; s < STAGES; ++s) {
     const int nf = nload > s ? (nload - s + STAGES - 1) / STAGES : 0;
-    if (nf > 0 && !mbar_drain(&full[s], (nf - 1) & 1)) record_abort(sm, status, where);
+    if (nf > 0 && !mbar_drain(&full[s], (nf - 1) & 1, sm.wait_ns)) record_abort(sm, status, where);
   }
 }
 
@@ -117,7 +116,7 @@ __device__ __forceinline__ void load_kv(Smem& sm, const Maps& maps, int nT, int 
   for (int kt = 0; kt < nT; ++kt) {
     const bool sel_tile = kt < ntile_sel;
     const int s = kt % ST;
-    if (kt >= ST && !mbar_wait(&empty[s], ((kt / ST) - 1) & 1, &sm.abort)) {
+    if (kt >= ST && !mbar_wait(&empty[s], ((kt / ST) - 1) & 1, &sm.abort, sm.wait_ns)) {
       record_abort(sm, status, IS_V ? 14 : 11);
       break;
     }
@@ -126,7 +125,7 @@ __device__ __forceinline__ void load_kv(Smem& sm, const Maps& maps, int nT, int 
     nl = kt + 1;
   }
   drain_ring<ST>(sm, full, nl, status, IS_V ? 15 : 12);
-  if (!IS_V && !mbar_drain(&sm.q_full, 0)) record_abort(sm, status, 13);
+  if (!IS_V && !mbar_drain(&sm.q_full, 0, sm.wait_ns)) record_abort(sm, status, 13);
 }
 
 __global__ void __launch_bounds__(THREADS, 1)
@@ -155,11 +154,14 @@ attn_tma_kernel(const __grid_constant__ Maps maps, const AttnArgs a) {
     }
     for (int w = 0; w < 2; ++w) {
       mbar_init(&sm.s_full[w], 1);
-      for (int c = 0; c < PV_PARTS; ++c) mbar_init(&sm.p_part[w][c], 4);  // one arrival per warp
+      // one arrival per warp (the test hook makes the first part of
+      // warpgroup 0 wait for an arrival that never comes)
+      for (int c = 0; c < PV_PARTS; ++c) mbar_init(&sm.p_part[w][c], (a.inject && w == 0 && c == 0) ? 5 : 4);
     }
     mbar_init(&sm.o_final, 1);
     mbar_init(&sm.mma_done, 1);
     sm.abort = 0;
+    sm.wait_ns = a.wait_ns;
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
   }
   if (warp == MMA_WARP) {
@@ -206,7 +208,7 @@ attn_tma_kernel(const __grid_constant__ Maps maps, const AttnArgs a) {
     // S_w = Q K(kt)^T, the K stage released once the product is done
     auto qk = [&](int w, int kt) -> bool {
       const int ks = kt % KST;
-      if (!mbar_wait_warp(&sm.k_full[ks], (kt / KST) & 1, &sm.abort)) return false;
+      if (!mbar_wait_warp(&sm.k_full[ks], (kt / KST) & 1, &sm.abort, sm.wait_ns)) return false;
       tc_fence_after();
       issue_qk(tmem + 128u * w, q0, smem_u32(sm.k[ks]));
       umma_commit_warp(&sm.s_full[w]);
@@ -218,16 +220,16 @@ attn_tma_kernel(const __grid_constant__ Maps maps, const AttnArgs a) {
     // once the product is done
     auto pv = [&](int w, int kt, int i) -> bool {
       const int vs = kt % VST;
-      if (!mbar_wait_warp(&sm.v_full[vs], (kt / VST) & 1, &sm.abort)) return false;
+      if (!mbar_wait_warp(&sm.v_full[vs], (kt / VST) & 1, &sm.abort, sm.wait_ns)) return false;
       for (int c = 0; c < PV_PARTS; ++c) {
-        if (!mbar_wait_warp(&sm.p_part[w][c], i & 1, &sm.abort)) return false;
+        if (!mbar_wait_warp(&sm.p_part[w][c], i & 1, &sm.abort, sm.wait_ns)) return false;
         tc_fence_after();
         issue_pv_part<PV_PARTS>(tmem + 256u + 128u * w, tmem + 128u * w, smem_u32(sm.v[vs]), c, i > 0);
       }
       umma_commit_warp(&sm.v_empty[vs]);
       return true;
     };
-    bool alive = mbar_wait_warp(&sm.q_full, 0, &sm.abort);
+    bool alive = mbar_wait_warp(&sm.q_full, 0, &sm.abort, sm.wait_ns);
     for (int i = 0; i < npair && alive; ++i) {
       const int kt0 = 2 * i, kt1 = 2 * i + 1;
       where = 22;
@@ -254,7 +256,7 @@ attn_tma_kernel(const __grid_constant__ Maps maps, const AttnArgs a) {
     if (!alive && lane == 0) record_abort(sm, a.status, where);
     umma_commit_warp(&sm.o_final);
     umma_commit_warp(&sm.mma_done);
-    const bool drained = __all_sync(0xffffffffu, mbar_drain(&sm.mma_done, 0));
+    const bool drained = __all_sync(0xffffffffu, mbar_drain(&sm.mma_done, 0, sm.wait_ns));
     if (!drained && lane == 0) record_abort(sm, a.status, 27);
     __syncwarp();
   } else {
@@ -279,7 +281,7 @@ attn_tma_kernel(const __grid_constant__ Maps maps, const AttnArgs a) {
       // key at a position p < nchunk with p <= t
       const int base_n = (sel_tile ? kt : kt - ntile_sel) * N;
       const int lim = sel_tile ? nsel : min(nchunk, t + 1);
-      softmax_tile_split<SOFTMAX_FMA_PAIRS, PV_PARTS>(S, tmem + lane_off + 256u + 128u * w, i > 0, base_n, lim,
+      softmax_tile_split<PV_PARTS>(S, tmem + lane_off + 256u + 128u * w, i > 0, base_n, lim,
                                                      qscale, m, l, sm.p_part[w]);
     }
 
@@ -336,7 +338,8 @@ attn_tma_kernel(const __grid_constant__ Maps maps, const AttnArgs a) {
     // rows past the chunk are clipped by the store
     fence_proxy_async_smem();
     named_barrier_sync(1, 256);
-    if (tid == 0) {
+    // (after a timeout the tile is not stored: the status word reports it)
+    if (tid == 0 && !*reinterpret_cast<volatile int*>(&sm.abort)) {
       tma_store_4d(&maps.o, smem_u32(sm.q), 0, t0, h, bi);
       tma_store_4d(&maps.o, smem_u32(sm.q) + ATOM_BYTES, 64, t0, h, bi);
       bulk_commit_group();
@@ -354,10 +357,14 @@ attn_tma_kernel(const __grid_constant__ Maps maps, const AttnArgs a) {
 
 }  // namespace
 
-cudaError_t launch_attn_tc(const AttnArgs& a, bool pdl, cudaStream_t stream) {
-  if (a.d != D) return cudaErrorNotSupported;
+cudaError_t launch_attn_tc(const AttnArgs& args, bool pdl, cudaStream_t stream) {
+  if (args.d != D) return cudaErrorNotSupported;
   // rows gathered by index while loading: the other kernel
-  if (a.kv_idx != nullptr && a.bsa > 0) return launch_attn_tc_gather(a, stream);
+  if (args.kv_idx != nullptr && args.bsa > 0) return launch_attn_tc_gather(args, stream);
+  AttnArgs a = args;
+  const WaitHooks hooks = wait_hooks();
+  a.wait_ns = hooks.wait_ns;
+  a.inject = hooks.inject == INJECT_ATTN_TMA ? 1 : 0;
   Maps maps;
   const int64_t oh = (int64_t)a.BCP * D, ob = (int64_t)a.nq * oh;  // O is contiguous
   if (!encode_bf16_4d(&maps.q, a.Q.data, D, a.BCP, a.nq, a.b, a.Q.st, a.Q.sh, a.Q.sb, 128) ||

@@ -8,6 +8,19 @@
 
 namespace quoka {
 
+// Test hooks, set through quoka_debug_set_wait_hooks and read by the
+// launchers of the tensor-core scoring and attention kernels: the bound of
+// every wait in those kernels (2 s by default), and an optional fault
+// injection that makes one barrier expect one arrival more than it ever
+// receives, so that the timeout path (give up, latch QUOKA_ERR_TIMEOUT and a
+// fault site, drain, free TMEM, exit) runs without hanging the GPU.
+enum : uint32_t { INJECT_NONE = 0u, INJECT_SCORE_TC = 1u, INJECT_ATTN_TMA = 2u };
+struct WaitHooks {
+  uint64_t wait_ns;
+  uint32_t inject;
+};
+WaitHooks wait_hooks();
+
 // Element-stride description of a (b, heads, rows, d) tensor.
 struct Strided {
   const void* data;
@@ -89,6 +102,8 @@ struct AttnArgs {
   int* status;
   int no_chunk = 0;         // 1: the chunk's own keys are left out (a shard's partial attention);
                             // rows with no visible key then give O = 0 and lse = -inf
+  uint64_t wait_ns = 0;     // bound of every wait (set by the launcher from wait_hooks())
+  int inject = 0;           // test hook (set by the launcher from wait_hooks())
 };
 
 // Steps (f)+(g) in fp32 on the CUDA cores (any input dtype).

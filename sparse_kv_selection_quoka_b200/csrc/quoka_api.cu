@@ -6,9 +6,25 @@
 #include <string.h>
 
 #include <algorithm>
+#include <atomic>
 
 #include "kernels.h"
 #include "quoka.h"
+
+namespace quoka {
+
+namespace {
+// Test hooks of quoka_debug_set_wait_hooks (process-wide).
+std::atomic<uint64_t> g_wait_ns{0};
+std::atomic<uint32_t> g_inject{INJECT_NONE};
+}  // namespace
+
+WaitHooks wait_hooks() {
+  const uint64_t ns = g_wait_ns.load(std::memory_order_relaxed);
+  return WaitHooks{ns == 0 ? 2000000000ull : ns, g_inject.load(std::memory_order_relaxed)};
+}
+
+}  // namespace quoka
 
 namespace {
 
@@ -552,6 +568,25 @@ quoka_status quoka_get_device_status(const void* ws, void* stream, int32_t* devi
     return QUOKA_ERR_CUDA;
   if (cudaStreamSynchronize(cs) != cudaSuccess) return QUOKA_ERR_CUDA;
   *device_status = v;
+  return QUOKA_OK;
+}
+
+quoka_status quoka_get_device_fault_site(const void* ws, void* stream, int32_t* site) {
+  if (ws == nullptr || site == nullptr) return QUOKA_ERR_INVALID_ARG;
+  cudaStream_t cs = static_cast<cudaStream_t>(stream);
+  int32_t v = 0;
+  if (cudaMemcpyAsync(&v, static_cast<const int32_t*>(ws) + 1, sizeof(int32_t), cudaMemcpyDeviceToHost, cs) !=
+      cudaSuccess)
+    return QUOKA_ERR_CUDA;
+  if (cudaStreamSynchronize(cs) != cudaSuccess) return QUOKA_ERR_CUDA;
+  *site = v;
+  return QUOKA_OK;
+}
+
+quoka_status quoka_debug_set_wait_hooks(uint64_t wait_limit_ns, uint32_t inject) {
+  if (inject > QUOKA_DEBUG_INJECT_ATTN) return QUOKA_ERR_INVALID_ARG;
+  quoka::g_wait_ns.store(wait_limit_ns, std::memory_order_relaxed);
+  quoka::g_inject.store(inject, std::memory_order_relaxed);
   return QUOKA_OK;
 }
 

@@ -32,8 +32,10 @@
 // Measured on B200 (Qwen-shaped layer): computing |k|^2 on the tensor core
 // instead (the diagonal of a K K^T product) costs more MMA time per tile
 // than it saves.
-// Every wait is bounded (see sm100.cuh); a wait that gives up records
-// QUOKA_ERR_TIMEOUT and the CTA unwinds.
+// Every wait is bounded (by the launch's wait limit, 2 s unless a test sets
+// another); a wait that gives up records QUOKA_ERR_TIMEOUT and a fault-site
+// code, and the CTA unwinds: the producer waits for the tile loads it issued
+// to land, the MMA warp for its products, TMEM is freed, and the CTA exits.
 #include "common.cuh"
 #include "kernels.h"
 #include "sm100.cuh"
@@ -73,6 +75,8 @@ struct ScoreArgs {
   int nepi;                 // epilogue warpgroups in use (TMEM holds one accumulator each)
   uint32_t tmem_cols;
   int key_norm;             // 1: divide by |k| (cosine score); 0: plain dot product
+  uint64_t wait_ns;         // bound of every wait
+  int inject;               // test hook: accumulator 0's release expects one arrival more than it gets
 };
 
 __device__ __forceinline__ void sc_abort(ScoreBars& sb, int* status, int where) {
@@ -82,8 +86,8 @@ __device__ __forceinline__ void sc_abort(ScoreBars& sb, int* status, int where) 
 }
 
 __device__ __forceinline__ bool sc_warp_wait(uint64_t* bar, uint32_t parity, ScoreBars& sb, int* status,
-                                             int where) {
-  const bool ok = mbar_wait(bar, parity, &sb.abort);
+                                             int where, uint64_t limit_ns) {
+  const bool ok = mbar_wait(bar, parity, &sb.abort, limit_ns);
   const bool all_ok = __all_sync(0xffffffffu, ok);
   if (!all_ok && (threadIdx.x & 31) == 0) sc_abort(sb, status, where);
   return all_ok;
@@ -118,7 +122,8 @@ score_tc_kernel(const __grid_constant__ CUtensorMap tmap, const ScoreArgs a) {
     }
     for (int q = 0; q < SC_EPI; ++q) {
       mbar_init(&sb.tfull[q], 1);
-      mbar_init(&sb.tempty[q], 128);
+      // (the test hook makes accumulator 0 wait for an arrival that never comes)
+      mbar_init(&sb.tempty[q], (q == 0 && a.inject) ? 129 : 128);
     }
     mbar_init(&sb.done, 1);
     sb.abort = 0;
@@ -138,9 +143,10 @@ score_tc_kernel(const __grid_constant__ CUtensorMap tmap, const ScoreArgs a) {
     // ------------------------------------------------------------ TMA producer
     // (starts at once: the K stream does not depend on the query groups)
     if (lane == 0) {
+      int issued = 0;
       for (int it = 0; it < n; ++it) {
         const int s = it % NS;
-        if (it >= NS && !mbar_wait(&sb.empty[s], ((it / NS) - 1) & 1, &sb.abort)) {
+        if (it >= NS && !mbar_wait(&sb.empty[s], ((it / NS) - 1) & 1, &sb.abort, a.wait_ns)) {
           sc_abort(sb, a.status, 51);
           break;
         }
@@ -149,6 +155,15 @@ score_tc_kernel(const __grid_constant__ CUtensorMap tmap, const ScoreArgs a) {
         const int y = (t_begin + it) * SC_KEYS;
         tma_load_4d(dst, &tmap, &sb.full[s], 0, y, j, bi);
         tma_load_4d(dst + SC_ATOM, &tmap, &sb.full[s], 64, y, j, bi);
+        issued = it + 1;
+      }
+      // Wait (bounded) until the last load into each stage has landed, so that
+      // no copy is still writing this CTA's shared memory when it exits, even
+      // if a consumer gave up before reading it. In a normal run every load
+      // has been consumed already and these return at once.
+      for (int s = 0; s < NS; ++s) {
+        const int nf = issued > s ? (issued - s + NS - 1) / NS : 0;  // loads into stage s
+        if (nf > 0 && !mbar_drain(&sb.full[s], (nf - 1) & 1, a.wait_ns)) sc_abort(sb, a.status, 57);
       }
     }
     __syncwarp();
@@ -193,10 +208,10 @@ score_tc_kernel(const __grid_constant__ CUtensorMap tmap, const ScoreArgs a) {
     for (int it = 0; it < n && alive; ++it) {
       const int s = it % NS, acc = it % NE;
       where = 52;
-      alive = mbar_wait_warp(&sb.full[s], (it / NS) & 1, &sb.abort);
+      alive = mbar_wait_warp(&sb.full[s], (it / NS) & 1, &sb.abort, a.wait_ns);
       if (alive && it >= NE) {
         where = 53;
-        alive = mbar_wait_warp(&sb.tempty[acc], ((it / NE) - 1) & 1, &sb.abort);
+        alive = mbar_wait_warp(&sb.tempty[acc], ((it / NE) - 1) & 1, &sb.abort, a.wait_ns);
       }
       if (!alive) break;
       tc_fence_after();
@@ -213,7 +228,7 @@ score_tc_kernel(const __grid_constant__ CUtensorMap tmap, const ScoreArgs a) {
     }
     if (!alive && lane == 0) sc_abort(sb, a.status, where);
     umma_commit_warp(&sb.done);
-    const bool drained = __all_sync(0xffffffffu, mbar_drain(&sb.done, 0));
+    const bool drained = __all_sync(0xffffffffu, mbar_drain(&sb.done, 0, a.wait_ns));
     if (!drained && lane == 0) sc_abort(sb, a.status, 54);
     __syncwarp();
   } else {
@@ -229,7 +244,7 @@ score_tc_kernel(const __grid_constant__ CUtensorMap tmap, const ScoreArgs a) {
       // |k| first, straight from the landed tile (the TMA writes are visible
       // to threads that observe the stage's barrier), so that the stage is
       // released without waiting for this tile's MMA result
-      if (!sc_warp_wait(&sb.full[s], (it / NS) & 1, sb, a.status, 56)) break;
+      if (!sc_warp_wait(&sb.full[s], (it / NS) & 1, sb, a.status, 56, a.wait_ns)) break;
       const uint8_t* tile = ring + (size_t)s * SC_TILE_BYTES;
       // eight independent partial sums keep the FMA chain short
       float ss8[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
@@ -247,7 +262,7 @@ score_tc_kernel(const __grid_constant__ CUtensorMap tmap, const ScoreArgs a) {
       const float ss = ((ss8[0] + ss8[1]) + (ss8[2] + ss8[3])) + ((ss8[4] + ss8[5]) + (ss8[6] + ss8[7]));
       mbar_arrive(&sb.empty[s]);
       // then the tile's scores against the group means, from TMEM
-      if (!sc_warp_wait(&sb.tfull[acc], (it / NE) & 1, sb, a.status, 55)) break;
+      if (!sc_warp_wait(&sb.tfull[acc], (it / NE) & 1, sb, a.status, 55, a.wait_ns)) break;
       tc_fence_after();
       float mx4[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
       const uint32_t tbase = tmem + lane_off + (uint32_t)(acc * ACC);
@@ -318,6 +333,9 @@ cudaError_t launch_score_tc(int d, Strided K, int b, int nkv, int64_t T, const u
   a.hist = hist;
   a.status = status;
   a.key_norm = key_norm ? 1 : 0;
+  const WaitHooks hooks = wait_hooks();
+  a.wait_ns = hooks.wait_ns;
+  a.inject = hooks.inject == INJECT_SCORE_TC ? 1 : 0;
   a.T = T;
   a.NQ = NQ;
   a.NQp = (NQ + 15) / 16 * 16;  // the epilogue reads 16-column groups

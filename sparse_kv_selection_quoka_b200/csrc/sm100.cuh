@@ -44,32 +44,34 @@ __device__ __forceinline__ uint64_t globaltimer_ns() {
   return t;
 }
 
-// Upper bound of any single wait in the kernels (a legitimate wait lasts
-// microseconds).
+// Default upper bound of any single wait in the kernels (a legitimate wait
+// lasts microseconds). Kernels that take their bound from the host pass it
+// as `limit_ns`.
 constexpr uint64_t kWaitLimitNs = 2000000000ull;
 
 // Waits for the phase with the given parity to complete. Gives up after
-// kWaitLimitNs (or as soon as the abort flag is set) and returns false; the
+// limit_ns (or as soon as the abort flag is set) and returns false; the
 // caller then records a timeout and unwinds.
-__device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, volatile int* abort_flag) {
+__device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, volatile int* abort_flag,
+                                          uint64_t limit_ns = kWaitLimitNs) {
   if (mbar_try_wait(bar, parity)) return true;
   const uint64_t t0 = globaltimer_ns();
   for (uint32_t it = 1;; ++it) {
     if (mbar_try_wait(bar, parity)) return true;
     if ((it & 15u) == 0u) {
       if (*abort_flag) return false;
-      if (globaltimer_ns() - t0 > kWaitLimitNs) return false;
+      if (globaltimer_ns() - t0 > limit_ns) return false;
     }
   }
 }
 
 // Bounded wait that ignores the abort flag: used to drain work already
-// issued (e.g. in-flight MMAs) before resources are released.
-__device__ __forceinline__ bool mbar_drain(uint64_t* bar, uint32_t parity) {
+// issued (e.g. in-flight MMAs or copies) before resources are released.
+__device__ __forceinline__ bool mbar_drain(uint64_t* bar, uint32_t parity, uint64_t limit_ns = kWaitLimitNs) {
   const uint64_t t0 = globaltimer_ns();
   for (uint32_t it = 0;; ++it) {
     if (mbar_try_wait(bar, parity)) return true;
-    if ((it & 15u) == 15u && globaltimer_ns() - t0 > kWaitLimitNs) return false;
+    if ((it & 15u) == 15u && globaltimer_ns() - t0 > limit_ns) return false;
   }
 }
 
@@ -207,8 +209,9 @@ __device__ __forceinline__ void umma_commit_warp(uint64_t* bar) {
 
 // Bounded wait made by every lane of a warp; the result is the same on all
 // lanes, which are converged again on return.
-__device__ __forceinline__ bool mbar_wait_warp(uint64_t* bar, uint32_t parity, volatile int* abort_flag) {
-  return __all_sync(0xffffffffu, mbar_wait(bar, parity, abort_flag));
+__device__ __forceinline__ bool mbar_wait_warp(uint64_t* bar, uint32_t parity, volatile int* abort_flag,
+                                               uint64_t limit_ns = kWaitLimitNs) {
+  return __all_sync(0xffffffffu, mbar_wait(bar, parity, abort_flag, limit_ns));
 }
 
 // D[tmem] (+)= A[tmem] x B[smem desc]; A (M x 16 bf16 for one MMA) lives in
@@ -337,16 +340,6 @@ __device__ __forceinline__ void bulk_commit_group() { asm volatile("cp.async.bul
 // enough before the CTA exits or the source is reused.
 __device__ __forceinline__ void bulk_wait_group_read_0() {
   asm volatile("cp.async.bulk.wait_group.read 0;" ::: "memory");
-}
-
-// Bulk copy of `bytes` (a multiple of 16) from this CTA's shared memory to
-// the shared memory of a CTA of the cluster (cluster addresses from mapa);
-// the destination's mbarrier receives the transferred bytes.
-__device__ __forceinline__ void bulk_copy_to_cluster(uint32_t dst, uint32_t src, uint32_t bytes, uint32_t mbar) {
-  asm volatile("cp.async.bulk.shared::cluster.shared::cta.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(
-                   dst),
-               "r"(src), "r"(bytes), "r"(mbar)
-               : "memory");
 }
 
 // Barrier over `count` threads (a multiple of 32) of the CTA, id 1..15.

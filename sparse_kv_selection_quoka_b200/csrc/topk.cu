@@ -1,6 +1,7 @@
 // Top-BSA key selection per (batch, KV head).
 //
-// [QUOKA §2.3] indices = topk(S_agg, BSA). Ties at the BSA-th score go to the
+// [QUOKA §2.3] the BSA keys of each KV head with the highest aggregated
+// score S_agg are kept. Ties at the BSA-th score go to the
 // lower key index, and the chosen indices are written in ascending key order
 // (the sorted format the attention kernels read). (QUOKA = the technical
 // write-up "QUOKA: how it reshapes LLM prefill efficiency", bqwf.cn news item
@@ -121,7 +122,7 @@ __device__ __forceinline__ void cluster_wait() { asm volatile("barrier.cluster.w
 template <bool CLUSTER>
 __global__ void __launch_bounds__(TOPK_THREADS)
 topk_kernel(const float* __restrict__ S, int64_t T, int bsa, int slice, const uint32_t* __restrict__ ghist,
-            int32_t* __restrict__ kv_idx, int32_t* __restrict__ kv_count) {
+            int32_t* __restrict__ kv_idx, int32_t* __restrict__ kv_count, const int* __restrict__ status) {
   extern __shared__ uint32_t smem_dyn[];
   uint32_t* keys = smem_dyn;          // [slice]: this CTA's keys
   uint32_t* glist = smem_dyn + slice;  // [TOPK_LIST_MAX]: all ranks' candidates, in rank order
@@ -159,6 +160,14 @@ topk_kernel(const float* __restrict__ S, int64_t T, int bsa, int slice, const ui
   // still run until this wait returns: they are read with L2-coherent loads
   // (never the read-only path, which assumes data fixed for the kernel's life).
   pdl_wait();
+  // A device fault latched earlier in the call (a scoring kernel that gave
+  // up) leaves the scores and their histogram incomplete: select nothing.
+  // Every CTA of the cluster reads the same word (nothing writes it while
+  // this kernel runs), so they all leave here together.
+  if (status != nullptr && __ldcg(status) != 0) {
+    if (c == 0 && tid == 0) kv_count[row] = 0;
+    return;
+  }
   if (ghist != nullptr) {
     const uint32_t* Hg = ghist + row * TOPK_BINS;
     constexpr int q0 = TOPK_BINS / TOPK_THREADS;
@@ -320,7 +329,7 @@ topk_kernel(const float* __restrict__ S, int64_t T, int bsa, int slice, const ui
         if (lane == 0) base = atomicAdd(&sh.ncand, (uint32_t)__popc(cb));
         base = __shfl_sync(0xffffffffu, base, 0);
         const uint32_t pos = base + (uint32_t)__popc(cb & ((1u << lane) - 1u));
-        if (cand) clist[pos] = k;  // pos < cnt0 <= TOPK_LIST_MAX
+        if (cand && pos < (uint32_t)TOPK_LIST_MAX) clist[pos] = k;  // pos < cnt0 <= TOPK_LIST_MAX
       }
     }
     gt = __reduce_add_sync(0xffffffffu, gt);
@@ -354,12 +363,15 @@ topk_kernel(const float* __restrict__ S, int64_t T, int bsa, int slice, const ui
       if (lane == C - 1) sh.rank_base[C] = incl;
     }
     __syncthreads();
-    const int nl = (int)sh.rank_base[C];  // == cnt0
+    // == cnt0 (the bounds below only guard the shared-memory lists should
+    // a histogram ever disagree with the scores)
+    const int nl = min((int)sh.rank_base[C], TOPK_LIST_MAX);
     for (int g = tid; g < nl; g += TOPK_THREADS) {
       int r = 0;
       while (r + 1 < C && (uint32_t)g >= sh.rank_base[r + 1]) ++r;
       const uint32_t* cl = CLUSTER ? cluster.map_shared_rank(clist, r) : clist;
-      glist[g] = cl[g - sh.rank_base[r]];
+      const uint32_t at = (uint32_t)g - sh.rank_base[r];
+      glist[g] = at < (uint32_t)TOPK_LIST_MAX ? cl[at] : 0u;
       sh.grank[g] = (uint8_t)r;
     }
     // done reading the other CTAs' shared memory (their wait at the end
@@ -565,7 +577,8 @@ int64_t topk_max_T() { return (int64_t)TOPK_MAX_CLUSTER * TOPK_MAX_SLICE; }
 
 cudaError_t launch_topk(const float* S_agg, int b, int nkv, int64_t T, int bsa, const uint32_t* hist,
                         int32_t* kv_idx, int32_t* kv_count, int* status, bool pdl, cudaStream_t stream) {
-  (void)status;  // every wait in the kernel is a hardware barrier phase that all threads reach
+  // (every wait in the kernel is a hardware barrier phase that all threads
+  // reach; `status` is only read, to skip the select after an earlier fault)
   if (bsa <= 0 || T <= 0 || bsa > T || T > topk_max_T()) return cudaErrorInvalidValue;
   int C = (int)((T + TOPK_SLICE_TARGET - 1) / TOPK_SLICE_TARGET);
   if (C > TOPK_MAX_CLUSTER) C = TOPK_MAX_CLUSTER;
@@ -597,7 +610,8 @@ cudaError_t launch_topk(const float* S_agg, int b, int nkv, int64_t T, int bsa, 
   }
   cfg.attrs = attr;
   cfg.numAttrs = na;
-  return cudaLaunchKernelEx(&cfg, kern, S_agg, T, bsa, slice, hist, kv_idx, kv_count);
+  return cudaLaunchKernelEx(&cfg, kern, S_agg, T, bsa, slice, hist, kv_idx, kv_count,
+                            static_cast<const int*>(status));
 }
 
 }  // namespace quoka

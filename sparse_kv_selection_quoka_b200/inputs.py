@@ -7,11 +7,12 @@ both the CUDA path and the CPU oracle may take their inputs from here.
 Every tensor is drawn in float32 from numpy's PCG64 with a fixed seed and a
 fixed draw order (noise for Q, K, V, Kc, Vc first, then the planted
 structure), and is rounded once to bfloat16 (round-to-nearest-even) for the
-bf16 workloads. The value structure follows the workload descriptions of the
-QUOKA write-up's long-context evaluation (Llama3-3B / Qwen3-4B shaped layers,
-"Long-context evaluation", section 3.1): queries share a per-group mean
-direction, a fraction of them are outliers with no mean component, and a set
-of "heavy" keys is aligned with the outlier directions.
+bf16 workloads. The shapes are those of the Llama3-3B / Qwen3-4B layers the
+QUOKA write-up evaluates on; its evaluation runs on real model activations,
+which are not available here, so the value structure is a synthetic stand-in
+defined with these workloads: queries share a per-group mean direction, a
+fraction of them are outliers with no mean component, and a set of "heavy"
+keys is aligned with the outlier directions.
 
 Layouts (row-major, contiguous):
   Q  (b, nq,  BCP, d)   the chunk's queries

@@ -149,7 +149,16 @@ def test_long_workload_T128k():
     nq, L = x.Q.shape[1], x.Q.shape[2]
     rows = [(0, int(h), int(t)) for h, t in zip(r.integers(0, nq, 48), r.integers(0, L, 48))]
     rows += [(0, 0, 0), (0, nq - 1, L - 1), (0, 5, 127), (0, 63, 128)]
-    run_prefill_and_check(x, ref, gi, rows=rows)
+    O = run_prefill_and_check(x, ref, gi, rows=rows)
+    # every row of one whole KV head (its G query heads x the chunk: every
+    # query tile and every chunk-key tail), against the oracle in full
+    j = 3
+    G = nq // x.K.shape[1]
+    hs = slice(j * G, (j + 1) * G)
+    js = slice(j, j + 1)
+    O_ref, _ = orc.sparse_attention(x.Q[:, hs], x.K[:, js], x.V[:, js], gi[:, js], x.Kc[:, js], x.Vc[:, js])
+    err = np.abs(O[:, hs].float().cpu().numpy().astype(np.float64) - O_ref).max()
+    assert err <= P.O_TOL_BF16, f"KV head {j}: O max-abs error {err:.3e}"
 
 
 @pytest.fixture(scope="module")
