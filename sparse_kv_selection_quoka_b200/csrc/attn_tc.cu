@@ -85,7 +85,7 @@ static_assert(sizeof(float) * 2 * 128 * D <= AT_STAGES * 2 * TILE_BYTES, "landin
 __global__ void __launch_bounds__(AT_THREADS, 1)
 attn_gather_kernel(const __grid_constant__ AttnMaps maps, const AttnArgs a, int nsplit) {
   extern __shared__ uint8_t smem_raw[];
-  AttnSmem& sm = *reinterpret_cast<AttnSmem*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  AttnSmem& sm = *reinterpret_cast<AttnSmem*>(align_smem_1024(smem_raw));
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int j = blockIdx.y, bi = blockIdx.z;

@@ -131,7 +131,7 @@ __device__ __forceinline__ void load_kv(Smem& sm, const Maps& maps, int nT, int 
 __global__ void __launch_bounds__(THREADS, 1)
 attn_tma_kernel(const __grid_constant__ Maps maps, const AttnArgs a) {
   extern __shared__ uint8_t smem_raw[];
-  Smem& sm = *reinterpret_cast<Smem*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  Smem& sm = *reinterpret_cast<Smem*>(align_smem_1024(smem_raw));
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int j = blockIdx.y, bi = blockIdx.z;

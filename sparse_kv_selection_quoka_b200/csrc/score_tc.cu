@@ -96,7 +96,7 @@ __device__ __forceinline__ bool sc_warp_wait(uint64_t* bar, uint32_t parity, Sco
 __global__ void __launch_bounds__(SC_THREADS, 1)
 score_tc_kernel(const __grid_constant__ CUtensorMap tmap, const ScoreArgs a) {
   extern __shared__ uint8_t smem_raw[];
-  uint8_t* base = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  uint8_t* base = align_smem_1024(smem_raw);
   const int N = 2 * a.NQp;                         // MMA N: hi rows then lo rows
   const int ACC = N;                               // columns of one accumulator
   uint8_t* qg_s = base;                            // [2 atoms][N rows][128 B]

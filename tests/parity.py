@@ -88,3 +88,9 @@ def check_kv_sets(gpu_idx: np.ndarray, gpu_count: np.ndarray, S_agg: np.ndarray,
                 f"selected keys differ beyond the tie band at b={bi} j={j}: "
                 f"{len(sym)} keys, max |S - thr| = {dev.max():.3e}")
     return n_diff
+
+
+def bf16_round(x: np.ndarray) -> np.ndarray:
+    """float -> bfloat16 (round to nearest even) -> float32, on the host."""
+    t = torch.from_numpy(np.ascontiguousarray(x, dtype=np.float32))
+    return t.to(torch.bfloat16).to(torch.float32).numpy()

@@ -418,3 +418,62 @@ def test_dot_product_score_variant(shape):
     assert torch.equal(i0, i1)
     assert lib.quoka_select_ex(ctypes.byref(qv), ctypes.byref(kv), NQ, BSA, _ptr(i0), _ptr(c0), None, None, 2,
                                _ptr(ws), ws.numel(), _stream(None)) != 0
+
+
+def _crowded_bucket_inputs(n_crowd, n_levels, seed, gap=2e-5):
+    """Keys whose threshold value bucket (width 1/2048 of the cosine range)
+    holds n_crowd keys: n_levels distinct bf16 key vectors near the first
+    group mean's direction, all scoring inside one bucket, at least `gap`
+    apart (far above the fp32 scores' rounding), each repeated at random
+    positions (exact ties). BSA cuts through the crowd. The levels are
+    picked with the oracle's scores, so the expected selection is exact:
+    order between levels and ties (lower index) alike."""
+    T, BSA = 8192, n_crowd // 2 + 7
+    x = inputs.make_chunk(1, 8, 2, 128, T, 128, 8, BSA, dtype="bf16", structure="iid", seed=seed)
+    rng = np.random.default_rng(seed)
+    Qg = orc.select(x.Q, x.K, x.NQ, BSA)["Q_group"]
+    for j in range(2):
+        u = Qg[0, j, 0] / np.linalg.norm(Qg[0, j, 0])
+        cand = P.bf16_round(11.0 * u[None, :] + 0.05 * rng.standard_normal((800, 128)))
+        sc = orc.key_scores(Qg[:, j:j + 1], cand[None, None])[0, 0]
+        b = np.floor((sc + 1.0) * 2048.0)
+        vals, cnts = np.unique(b, return_counts=True)
+        idx = np.where(b == vals[np.argmax(cnts)])[0]
+        order = idx[np.argsort(sc[idx])]
+        pick = [order[0]]
+        for i in order[1:]:
+            if sc[i] - sc[pick[-1]] >= gap:
+                pick.append(i)
+        assert len(pick) >= n_levels, "not enough separated levels in one bucket"
+        pick = rng.permutation(pick)[:n_levels]
+        pos = rng.choice(T, n_crowd, replace=False)
+        x.K[0, j, pos] = cand[np.asarray(pick)[np.arange(n_crowd) % n_levels]]
+    return x
+
+
+@pytest.mark.parametrize("n_crowd", [1000, 5000], ids=["list_radix", "row_radix"])
+def test_crowded_threshold_bucket(n_crowd):
+    """The BSA-th score's value bucket holds 1000 keys (the candidate list
+    is resolved by radix passes) or 5000 (more than the list holds: radix
+    passes over the row), with exact ties: the selection must equal the
+    oracle's exactly, both from quoka_select and from quoka_topk on the
+    scores quoka_select returned."""
+    x = _crowded_bucket_inputs(n_crowd, 10, 90 + n_crowd)
+    ref = orc.select(x.Q, x.K, x.NQ, x.BSA)
+    for j in range(2):  # the case is what it claims to be
+        s = ref["S_agg"][0, j]
+        thr = np.sort(s)[::-1][x.BSA - 1]
+        bins = np.floor((s + 1.0) * 2048.0)
+        assert (bins == np.floor((thr + 1.0) * 2048.0)).sum() >= n_crowd
+    Q, K = P.to_dev(x.Q, x.dtype), P.to_dev(x.K, x.dtype)
+    kv_idx, kv_count, q_idx, s_agg = q().quoka_select(Q, K, x.NQ, x.BSA, want_q_idx=True, want_s_agg=True)
+    torch.cuda.synchronize()
+    gq = q_idx.cpu().numpy().astype(np.int64)
+    if not P.check_q_idx(gq, ref["SQ"], ref["q_idx"]):
+        ref = orc.select(x.Q, x.K, x.NQ, x.BSA, override_q_idx=gq)
+    assert np.abs(s_agg.cpu().numpy().astype(np.float64) - ref["S_agg"]).max() <= P.S_TOL
+    np.testing.assert_array_equal(kv_idx.cpu().numpy(), ref["sel"])
+    assert np.all(kv_count.cpu().numpy() == x.BSA)
+    i2, c2 = q().quoka_topk(s_agg, x.BSA)
+    torch.cuda.synchronize()
+    np.testing.assert_array_equal(i2.cpu().numpy(), ref["sel"])
