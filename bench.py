@@ -53,6 +53,11 @@ import torch  # noqa: E402
 METRIC = "prefill chunk-tokens/sec at T=32K (keys-scored/sec, % HBM and tensor-pipe peak alongside)"
 UNIT = "chunk-tokens/s"
 FLUSH_BYTES = 256 << 20
+# device-side wait (clock cycles, ~100 µs) enqueued after each flush, outside
+# the timed events: the host's argument marshalling for a call can take
+# longer than the call's device time, and the wait lets the host enqueue the
+# whole timed region before the device reaches it
+HOST_LEAD_CYCLES = 200000
 DEFAULT_WORKLOAD = "qwen3-4b_T32k"
 # measured beside the default workload in every default run
 OTHER_WORKLOADS = ("llama3.2-3b_T8k", "sweep_b8_S16k", "long_T128k_G8")
@@ -321,6 +326,10 @@ def time_run(q, run, steps, warmup, flush, stream, world, dev, sampler=None):
     step_evs = []
     for _ in range(steps):
         flush.fill_(1)
+        # a device-side wait after the flush (outside the events) keeps the
+        # host's enqueueing ahead of the device, so that no host-side gap
+        # falls inside a timed region
+        torch.cuda._sleep(HOST_LEAD_CYCLES * len(run.chunks))
         e = [torch.cuda.Event(enable_timing=True) for _ in range(2)]
         e[0].record(stream)
         for ch in run.chunks:
@@ -339,6 +348,7 @@ def time_run(q, run, steps, warmup, flush, stream, world, dev, sampler=None):
         flush.fill_(1)
         one = []
         for ch in run.chunks:
+            torch.cuda._sleep(HOST_LEAD_CYCLES)
             e = [torch.cuda.Event(enable_timing=True) for _ in range(4)]
             e[0].record(stream)
             run.parts(q, ch, stream, evs=e[1:3])
@@ -512,7 +522,7 @@ def measure_decode(q, w, dev, stream, flush, Q, K, V, Kc, Vc, steps):
             # GPU time than their host-side argument marshalling, and the
             # wait lets the host enqueue the whole call before the timed
             # region starts, so the events see the device's time only
-            torch.cuda._sleep(200000)
+            torch.cuda._sleep(HOST_LEAD_CYCLES)
             e = [torch.cuda.Event(enable_timing=True) for _ in range(2)]
             e[0].record(stream)
             f()

@@ -36,8 +36,11 @@
  *   - Faults that only the device can see (a key index outside [0, T), a
  *     bounded wait that gave up) are latched into a status word at the start
  *     of `ws` and read back with quoka_get_device_status(). Every call that
- *     takes `ws` first clears that word (an asynchronous 4-byte memset on
- *     `stream`), so the word reports the faults of the latest call.
+ *     takes `ws` clears that word (and the fault-site word after it) on
+ *     `stream` before any of its kernels can latch a fault: quoka_select,
+ *     quoka_select_ex and quoka_prefill_chunk in their first kernel (whose
+ *     successors latch only after waiting for it), the other calls with an
+ *     8-byte memset. The word reports the faults of the latest call.
  *   - Calls on different streams with different workspaces may run
  *     concurrently. Two calls sharing one workspace must be ordered.
  */
@@ -146,15 +149,16 @@ quoka_status quoka_select_ex(const quoka_tensor* Q, const quoka_tensor* K,
  *   quoka_select_workspace_size() exceeds it are rejected with QUOKA_ERR_WORKSPACE before anything is
  *   enqueued. Nothing is allocated (no cudaMalloc or cudaFree, no allocating
  *   library call).
- *   The first call on each device looks up the array's device address (with
- *   that device current) and caches it; make that first call before any
- *   stream capture begins.
+ *   Every call looks up the array's device address in the context current
+ *   at the call (cudaGetSymbolAddress), so nothing goes stale after a
+ *   cudaDeviceReset or under another context.
  *   All calls on a device share the array and it keeps the last call's
- *   contents (each call clears its status word first; everything else is
+ *   contents (each call clears its status words first; everything else is
  *   rewritten before it is read). Calls that overlap on the GPU race on the
  *   array: order them (one stream, or events between streams).
- *   quoka_get_device_status() cannot reach this array; device faults of
- *   these calls are not reported. */
+ *   The device faults of the latest call are read with
+ *   quoka_get_device_status(NULL, ...) / quoka_get_device_fault_site(NULL,
+ *   ...). */
 quoka_status quoka_select_static(const quoka_tensor* Q, const quoka_tensor* K, int NQ,
                                  int BSA, int32_t* kv_idx, int32_t* kv_count,
                                  int32_t* q_idx, float* s_agg, void* stream);
@@ -350,8 +354,10 @@ quoka_status quoka_combine_partials(const void* O_parts, const float* lse_parts,
 
 /* Synchronises `stream`, then reads the device status word of `ws` into
  * *device_status (a quoka_status value; QUOKA_OK if the latest call that
- * used ws latched no device fault). Returns QUOKA_ERR_CUDA if the copy or
- * the synchronisation failed, QUOKA_ERR_INVALID_ARG for NULL pointers. */
+ * used ws latched no device fault). ws = NULL reads the status word of
+ * quoka_select_static's fixed scratch on the current device. Returns
+ * QUOKA_ERR_CUDA if the copy or the synchronisation failed,
+ * QUOKA_ERR_INVALID_ARG if device_status is NULL. */
 quoka_status quoka_get_device_status(const void* ws, void* stream,
                                      int32_t* device_status);
 
@@ -360,7 +366,8 @@ quoka_status quoka_get_device_status(const void* ws, void* stream,
  * latched no device fault, else a small code naming the kernel and the wait
  * or check where the first fault happened (diagnostic only; the codes of
  * the scoring kernel are 51-57, those of the attention 11-15, 21-27 and
- * 31-33). Returns as quoka_get_device_status. */
+ * 31-33). ws = NULL as for quoka_get_device_status. Returns as
+ * quoka_get_device_status. */
 quoka_status quoka_get_device_fault_site(const void* ws, void* stream,
                                          int32_t* site);
 

@@ -376,7 +376,8 @@ def quoka_prefill_chunk(Q, K, V, Kc, Vc, NQ: int, BSA: int, scale=None, *, O=Non
 
 
 def quoka_get_device_status(ws, stream=None) -> int:
-    """Synchronise the stream and return the device status word of ws."""
+    """Synchronise the stream and return the device status word of ws
+    (ws = None: that of quoka_select_static's fixed scratch)."""
     lib = load()
     out = ctypes.c_int32(0)
     st = lib.quoka_get_device_status(_ptr(ws), _stream(stream), ctypes.byref(out))
@@ -386,7 +387,8 @@ def quoka_get_device_status(ws, stream=None) -> int:
 
 def quoka_get_device_fault_site(ws, stream=None) -> int:
     """Synchronise the stream and return the fault-site word of ws (0: no
-    device fault in the latest call that used ws)."""
+    device fault in the latest call that used ws; ws = None: quoka_select_static's
+    fixed scratch)."""
     lib = load()
     out = ctypes.c_int32(0)
     st = lib.quoka_get_device_fault_site(_ptr(ws), _stream(stream), ctypes.byref(out))

@@ -16,18 +16,6 @@ template <typename T> __device__ __forceinline__ T from_f32(float x);
 template <> __device__ __forceinline__ float from_f32<float>(float x) { return x; }
 template <> __device__ __forceinline__ bf16 from_f32<bf16>(float x) { return __float2bfloat16_rn(x); }
 
-// Latch the first device-side fault of a call into the workspace status
-// word (0 = no fault). Later faults keep the first code.
-__device__ __forceinline__ void latch_status(int* status, int code) {
-  if (status != nullptr) atomicCAS(status, 0, code);
-}
-
-// Record where the first device-side fault of a call happened (the word
-// after the status word; diagnostic only).
-__device__ __forceinline__ void latch_where(int* status, int where) {
-  if (status != nullptr) atomicCAS(status + 1, 0, where);
-}
-
 __device__ __forceinline__ float warp_sum(float v) {
 #pragma unroll
   for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
@@ -70,6 +58,37 @@ __device__ __forceinline__ uint32_t score_key(float f) {
 // CTA of this grid has called it or exited.
 __device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
 __device__ __forceinline__ void pdl_trigger() { asm volatile("griddepcontrol.launch_dependents;" ::: "memory"); }
+
+// Latch the first device-side fault of a call into the workspace status
+// word (0 = no fault). Later faults keep the first code. The calls whose
+// first kernel clears the status words (instead of a memset before the
+// kernels) rely on this: the latch first waits for the predecessor grid
+// (pdl_wait, a no-op without programmatic launch), and each kernel of such
+// a call executes that wait before it completes, so every latch is ordered
+// after the clearing. A latch happens only on a fault, so the wait costs
+// nothing in a normal run.
+__device__ __forceinline__ void latch_status(int* status, int code) {
+  if (status == nullptr) return;
+  pdl_wait();
+  atomicCAS(status, 0, code);
+}
+
+// Record where the first device-side fault of a call happened (the word
+// after the status word; diagnostic only). Ordered like latch_status.
+__device__ __forceinline__ void latch_where(int* status, int where) {
+  if (status == nullptr) return;
+  pdl_wait();
+  atomicCAS(status + 1, 0, where);
+}
+
+// Clear the two status words at the start of a call's first kernel (block
+// 0, thread 0); see latch_status.
+__device__ __forceinline__ void clear_status(int* status) {
+  if (status != nullptr && blockIdx.x == 0 && blockIdx.y == 0 && blockIdx.z == 0 && threadIdx.x == 0) {
+    status[0] = 0;
+    status[1] = 0;
+  }
+}
 
 // 12-bit bucket of a score, linear over [-1, 1] (cosine-type scores lie
 // there): floor((s + 1) * 2048) clamped to [0, 4095]. Non-decreasing in the

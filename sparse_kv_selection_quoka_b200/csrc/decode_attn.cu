@@ -301,6 +301,230 @@ __global__ void __launch_bounds__(kThreads) decode_slice_kernel(const DecodeArgs
   }
 }
 
+// ---------------------------------------------------------------------------
+// bf16 inputs: the same slice on the tensor cores (mma.sync m16n8k16, bf16 x
+// bf16 -> fp32). With only R = G * BCP <= 64 query rows the slice is bound
+// by its loads, not by arithmetic; what the tensor cores remove is the
+// instruction stream of the CUDA-core dot products (thousands of shared
+// memory reads and FMAs per thread), which kept the SMs issuing long after
+// the slice's rows had arrived. The query rows are padded to Rp, a multiple
+// of 16 (padding rows are zero and their results unused).
+//   S (Rp x 64) = Q K^T: warp w takes keys [16 w, 16 w + 16);
+//   softmax per row in fp32 (one warp per row), P rounded to bf16;
+//   O (Rp x D) = P V: warp w takes columns [w D / 4, (w + 1) D / 4).
+// Q, K and V rows sit in shared memory with a 16-byte pad each, P rows with
+// one too, so that every 8-row ldmatrix phase hits 32 distinct banks.
+
+__device__ __forceinline__ void ldsm_x4(uint32_t addr, uint32_t* r) {
+  asm volatile("ldmatrix.sync.aligned.m8n8.x4.shared.b16 {%0, %1, %2, %3}, [%4];"
+               : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3])
+               : "r"(addr));
+}
+__device__ __forceinline__ void ldsm_x4_trans(uint32_t addr, uint32_t* r) {
+  asm volatile("ldmatrix.sync.aligned.m8n8.x4.trans.shared.b16 {%0, %1, %2, %3}, [%4];"
+               : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3])
+               : "r"(addr));
+}
+// c (16 x 8, fp32) += a (16 x 16, bf16, row-major) * b (16 x 8, bf16, column-major)
+__device__ __forceinline__ void mma_bf16_16816(float* c, const uint32_t* a, uint32_t b0, uint32_t b1) {
+  asm volatile(
+      "mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 {%0, %1, %2, %3}, {%4, %5, %6, %7}, {%8, %9}, "
+      "{%0, %1, %2, %3};"
+      : "+f"(c[0]), "+f"(c[1]), "+f"(c[2]), "+f"(c[3])
+      : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
+}
+
+// Shared memory of a tensor-core slice, in this order: Q rows [Rp], K rows
+// [KS], V rows [KS] (bf16, ROWB bytes each), scores [R][KS] fp32, P rows [Rp]
+// (bf16, PROWB bytes each), (m, l) per row [R][2] fp32.
+template <int D>
+struct MmaSliceSmem {
+  static constexpr int ROWB = D * 2 + 16;
+  static constexpr int PROWB = KS * 2 + 16;
+  __host__ __device__ static constexpr size_t k_off(int Rp) { return (size_t)Rp * ROWB; }
+  __host__ __device__ static constexpr size_t v_off(int Rp) { return k_off(Rp) + (size_t)KS * ROWB; }
+  __host__ __device__ static constexpr size_t s_off(int Rp) { return v_off(Rp) + (size_t)KS * ROWB; }
+  __host__ __device__ static constexpr size_t p_off(int Rp) { return s_off(Rp) + (size_t)Rp * KS * 4; }
+  __host__ __device__ static constexpr size_t ml_off(int Rp) { return p_off(Rp) + (size_t)Rp * PROWB; }
+  __host__ __device__ static constexpr size_t bytes(int Rp) { return ml_off(Rp) + (size_t)Rp * 2 * 4; }
+};
+
+template <int D>
+__global__ void __launch_bounds__(kThreads) decode_slice_mma_kernel(const DecodeArgs a) {
+  using L = MmaSliceSmem<D>;
+  using T = __nv_bfloat16;
+  constexpr int CPR = D / 8;  // 16-byte chunks per row
+  static_assert(KS == 64 && kThreads == 128, "four warps of 16 keys");
+  extern __shared__ __align__(16) uint8_t dsm[];
+  __shared__ const T* kp[KS];
+  __shared__ const T* vp[KS];
+  __shared__ int nsel_s;
+  const int G = a.nq / a.nkv, R = G * a.BCP, Rp = (R + 15) & ~15;
+  const uint32_t qbase = sm100::smem_u32(dsm), kbase = qbase + (uint32_t)L::k_off(Rp);
+  const uint32_t vbase = qbase + (uint32_t)L::v_off(Rp), pbase = qbase + (uint32_t)L::p_off(Rp);
+  float* Ss = reinterpret_cast<float*>(dsm + L::s_off(Rp));
+  float* ml = reinterpret_cast<float*>(dsm + L::ml_off(Rp));
+  const int s = blockIdx.x, j = blockIdx.y, bi = blockIdx.z, tid = threadIdx.x;
+  const int warp = tid >> 5, lane = tid & 31, grp = lane >> 2, tig = lane & 3;
+  const float qscale = a.scale * 1.4426950408889634f;  // scores in log2 units
+  const T* Q = static_cast<const T*>(a.Q.data);
+
+  pdl_trigger();
+  // the query rows (not written by any earlier kernel of the step): row r is
+  // head j * G + r / BCP, chunk position r % BCP; padding rows are zeroed
+  for (int e = tid; e < Rp * CPR; e += kThreads) {
+    const int r = e / CPR, c = e % CPR;
+    const T* src = Q;
+    uint32_t n = 0u;
+    if (r < R) {
+      src = Q + bi * a.Q.sb + (j * G + r / a.BCP) * a.Q.sh + (r % a.BCP) * a.Q.st + c * 8;
+      n = 16u;
+    }
+    sm100::cp_async_16(qbase + r * L::ROWB + c * 16, src, n);
+  }
+  sm100::cp_async_commit();
+
+  pdl_wait();  // the indices and counts may come from the previous kernel
+  const int64_t kvrow = (int64_t)bi * a.nkv + j;
+  const int n0 = s * KS;
+  if (tid < KS) {
+    const int n = n0 + tid;
+    const int cnt = a.bsa > 0 ? __ldcg(a.kv_count + kvrow) : 0;
+    const int32_t tau = n < a.bsa ? __ldcg(a.kv_idx + kvrow * a.bsa + n) : -1;
+    const int nsel = max(0, min(cnt, a.bsa));
+    const T* kr = nullptr;
+    const T* vr = nullptr;
+    if (n < nsel) {
+      if (tau >= 0 && (int64_t)tau < a.T) {
+        kr = static_cast<const T*>(a.K.data) + bi * a.K.sb + j * a.K.sh + tau * a.K.st;
+        vr = static_cast<const T*>(a.V.data) + bi * a.V.sb + j * a.V.sh + tau * a.V.st;
+      } else if (a.status != nullptr) {
+        latch_status(a.status, 6 /* QUOKA_ERR_BOUNDS */);  // the key reads as zeros
+      }
+    } else if (n - nsel < a.BCP) {
+      const int c = n - nsel;
+      kr = static_cast<const T*>(a.Kc.data) + bi * a.Kc.sb + j * a.Kc.sh + c * a.Kc.st;
+      vr = static_cast<const T*>(a.Vc.data) + bi * a.Vc.sb + j * a.Vc.sh + c * a.Vc.st;
+    }
+    kp[tid] = kr;
+    vp[tid] = vr;
+    if (tid == 0) nsel_s = nsel;
+  }
+  __syncthreads();
+  const int nsel = nsel_s;
+  const int nk = max(0, min(KS, nsel + a.BCP - n0));  // keys of this slice
+  for (int e = tid; e < KS * CPR; e += kThreads) {
+    const int k = e / CPR, c = e % CPR;
+    const T* kr = kp[k];
+    const T* vr = vp[k];
+    sm100::cp_async_16(kbase + k * L::ROWB + c * 16, kr ? kr + c * 8 : Q, kr ? 16u : 0u);
+    sm100::cp_async_16(vbase + k * L::ROWB + c * 16, vr ? vr + c * 8 : Q, vr ? 16u : 0u);
+  }
+  sm100::cp_async_commit();
+  sm100::cp_async_wait<0>();
+  __syncthreads();
+
+  // S = Q K^T for keys [16 warp, 16 warp + 16), scaled, masked, into Ss
+  for (int mt = 0; mt < Rp / 16; ++mt) {
+    float c[2][4] = {{0.f, 0.f, 0.f, 0.f}, {0.f, 0.f, 0.f, 0.f}};
+    const int arow = mt * 16 + (lane & 7) + 8 * ((lane >> 3) & 1);
+#pragma unroll
+    for (int k0 = 0; k0 < D; k0 += 32) {
+      uint32_t a0[4], a1[4];
+      ldsm_x4(qbase + arow * L::ROWB + (k0 + 8 * (lane >> 4)) * 2, a0);
+      ldsm_x4(qbase + arow * L::ROWB + (k0 + 16 + 8 * (lane >> 4)) * 2, a1);
+#pragma unroll
+      for (int nt = 0; nt < 2; ++nt) {
+        uint32_t b[4];
+        const int key = 16 * warp + 8 * nt + (lane & 7);
+        ldsm_x4(kbase + key * L::ROWB + (k0 + 8 * (lane >> 3)) * 2, b);
+        mma_bf16_16816(c[nt], a0, b[0], b[1]);
+        mma_bf16_16816(c[nt], a1, b[2], b[3]);
+      }
+    }
+#pragma unroll
+    for (int nt = 0; nt < 2; ++nt) {
+#pragma unroll
+      for (int hf = 0; hf < 2; ++hf) {
+        const int r = mt * 16 + grp + 8 * hf;
+        if (r >= R) continue;
+        const int k = 16 * warp + 8 * nt + 2 * tig;
+        float v[2];
+#pragma unroll
+        for (int u = 0; u < 2; ++u) {
+          const int n = n0 + k + u;
+          const bool vis = k + u < nk && (n < nsel || n - nsel <= r % a.BCP);
+          v[u] = vis ? c[nt][2 * hf + u] * qscale : -INFINITY;
+        }
+        *reinterpret_cast<float2*>(Ss + r * KS + k) = make_float2(v[0], v[1]);
+      }
+    }
+  }
+  __syncthreads();
+
+  // per row: max, probabilities 2^(s - m) (bf16 into P), their sum, and the
+  // slice's log-sum-exp (one warp per row)
+  const int64_t rows = (int64_t)a.b * a.nq * a.BCP;
+  for (int r = warp; r < R; r += kThreads / 32) {
+    const float s0 = Ss[r * KS + lane], s1 = Ss[r * KS + lane + 32];
+    float m = fmaxf(s0, s1);
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
+    const float p0 = m == -INFINITY ? 0.f : exp2f(s0 - m);
+    const float p1 = m == -INFINITY ? 0.f : exp2f(s1 - m);
+    T* pr = reinterpret_cast<T*>(dsm + L::p_off(Rp) + (size_t)r * L::PROWB);
+    pr[lane] = __float2bfloat16_rn(p0);
+    pr[lane + 32] = __float2bfloat16_rn(p1);
+    float l = p0 + p1;
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) l += __shfl_xor_sync(0xffffffffu, l, o);
+    if (lane == 0) {
+      ml[2 * r] = m;
+      ml[2 * r + 1] = l;
+      const int h = j * G + r / a.BCP, t = r % a.BCP;
+      const int64_t row = ((int64_t)bi * a.nq + h) * a.BCP + t;
+      a.lse_parts[(int64_t)s * rows + row] = l > 0.f ? (m + log2f(l)) * 0.6931471805599453f : -INFINITY;
+    }
+  }
+  __syncthreads();
+
+  // O = P V for columns [warp D / 4, (warp + 1) D / 4), normalised by l
+  constexpr int NTO = D / 32;  // 8-column tiles per warp
+  for (int mt = 0; mt < Rp / 16; ++mt) {
+    float o[NTO][4];
+#pragma unroll
+    for (int nt = 0; nt < NTO; ++nt) o[nt][0] = o[nt][1] = o[nt][2] = o[nt][3] = 0.f;
+    const int arow = mt * 16 + (lane & 7) + 8 * ((lane >> 3) & 1);
+#pragma unroll
+    for (int k0 = 0; k0 < KS; k0 += 16) {
+      uint32_t pa[4];
+      ldsm_x4(pbase + arow * L::PROWB + (k0 + 8 * (lane >> 4)) * 2, pa);
+      const int key = k0 + (lane & 7) + 8 * ((lane >> 3) & 1);
+#pragma unroll
+      for (int nt = 0; nt < NTO; nt += 2) {
+        uint32_t b[4];
+        const int col = warp * (D / 4) + 8 * nt + 8 * (lane >> 4);
+        ldsm_x4_trans(vbase + key * L::ROWB + col * 2, b);
+        mma_bf16_16816(o[nt], pa, b[0], b[1]);
+        mma_bf16_16816(o[nt + 1], pa, b[2], b[3]);
+      }
+    }
+#pragma unroll
+    for (int hf = 0; hf < 2; ++hf) {
+      const int r = mt * 16 + grp + 8 * hf;
+      if (r >= R) continue;
+      const float l = ml[2 * r + 1];
+      const float inv = l > 0.f ? 1.f / l : 0.f;
+      const int h = j * G + r / a.BCP, t = r % a.BCP;
+      const int64_t row = ((int64_t)bi * a.nq + h) * a.BCP + t;
+      float* dst = a.O_parts + ((int64_t)s * rows + row) * D + warp * (D / 4) + 2 * tig;
+#pragma unroll
+      for (int nt = 0; nt < NTO; ++nt)
+        *reinterpret_cast<float2*>(dst + 8 * nt) = make_float2(o[nt][2 * hf] * inv, o[nt][2 * hf + 1] * inv);
+    }
+  }
+}
+
 // O = sum_s w_s O_s, w_s = exp(lse_s - LSE), LSE = log sum_s exp(lse_s) over
 // the slices of a query row; rows without a visible key (all lse = -inf)
 // give O = 0, LSE = -inf. One CTA per query row: the slices are spread over
@@ -386,9 +610,10 @@ decode_merge_kernel(const float* __restrict__ O_parts, const float* __restrict__
 template <typename T, int D>
 cudaError_t launch_typed(const DecodeArgs& a, bool pdl, cudaStream_t stream) {
   const int R = (a.nq / a.nkv) * a.BCP;
-  const size_t smem = SliceSmem<T, D>::bytes(R);
-  cudaError_t e = cudaFuncSetAttribute(decode_slice_kernel<T, D>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                       (int)smem);
+  constexpr bool kMma = sizeof(T) == 2;
+  auto* kern = kMma ? decode_slice_mma_kernel<D> : decode_slice_kernel<T, D>;
+  const size_t smem = kMma ? MmaSliceSmem<D>::bytes((R + 15) & ~15) : SliceSmem<T, D>::bytes(R);
+  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (e != cudaSuccess) return e;
   cudaLaunchAttribute attr[1];
   attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
@@ -400,7 +625,7 @@ cudaError_t launch_typed(const DecodeArgs& a, bool pdl, cudaStream_t stream) {
   cfg.stream = stream;
   cfg.attrs = attr;
   cfg.numAttrs = pdl ? 1 : 0;
-  e = cudaLaunchKernelEx(&cfg, decode_slice_kernel<T, D>, a);
+  e = cudaLaunchKernelEx(&cfg, kern, a);
   if (e != cudaSuccess) return e;
   const int64_t rows = (int64_t)a.b * a.nq * a.BCP;
   cudaLaunchConfig_t mc = {};

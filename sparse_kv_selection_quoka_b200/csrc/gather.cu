@@ -42,12 +42,21 @@ gather_kernel(const char* __restrict__ K, int64_t sKb, int64_t sKh, int64_t sKt,
   const int64_t row = (int64_t)bi * nkv + j;
   pdl_trigger();  // the attention may launch once every CTA has started
   pdl_wait();     // the indices may come from the previous kernel
-  // (indices possibly written by the previous kernel: L2-coherent loads)
-  const int cnt = max(0, min(__ldcg(kv_count + row), bsa));
   const int64_t nitems = (int64_t)bsa << cpr_log2;
   const int64_t i0 = (int64_t)blockIdx.x * (kThreads * kItems) + threadIdx.x;
   const int cmask = (1 << cpr_log2) - 1;
   const int row_bytes = 16 << cpr_log2;
+  // The count and every item's index are loaded together (L2-coherent
+  // loads: possibly written by the previous kernel); an index past the
+  // count is read (the list has bsa entries per row) but not used.
+  const int cnt_raw = __ldcg(kv_count + row);
+  int32_t tau_u[kItems];
+#pragma unroll
+  for (int u = 0; u < kItems; ++u) {
+    const int64_t i = i0 + u * kThreads;
+    tau_u[u] = i < nitems ? __ldcg(kv_idx + row * bsa + (int)(i >> cpr_log2)) : -1;
+  }
+  const int cnt = max(0, min(cnt_raw, bsa));
   const char* Kb = K + bi * sKb + j * sKh;
   const char* Vb = V + bi * sVb + j * sVh;
   char* Kd = Ksel + row * bsa * row_bytes;
@@ -63,7 +72,7 @@ gather_kernel(const char* __restrict__ K, int64_t sKb, int64_t sKh, int64_t sKt,
     vv[u] = kv[u];
     if (i >= nitems) continue;
     if (n < cnt) {
-      const int32_t tau = __ldcg(kv_idx + row * bsa + n);
+      const int32_t tau = tau_u[u];
       if (tau >= 0 && (int64_t)tau < T) {
         kv[u] = ld_stream(reinterpret_cast<const uint4*>(Kb + tau * sKt) + c);
         vv[u] = ld_stream(reinterpret_cast<const uint4*>(Vb + tau * sVt) + c);

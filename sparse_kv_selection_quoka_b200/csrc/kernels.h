@@ -38,18 +38,21 @@ cudaError_t launch_qsel(bool bf16, int d, Strided Q, int b, int nq, int BCP, int
 // heads of each group of Qhat at the same rank; optionally also the bf16
 // hi/lo split (b, nkv, 2*NQ, d): rows [0, NQ) hi, rows [NQ, 2NQ) lo.
 // When `hist` is given, also zeroes the (b * nkv, TOPK_HIST_BINS) score
-// histogram that the tensor-core scoring kernel fills.
+// histogram that the tensor-core scoring kernel fills. When `status` is
+// given, clears the call's two status words (the first kernel of a call
+// that may latch nothing runs before it).
 constexpr int TOPK_HIST_BINS = 4096;
 cudaError_t launch_qgroup(int d, const float* Qhat, int b, int nq, int nkv, int NQ,
-                          float* Qg, uint16_t* Qg_hilo, uint32_t* hist, cudaStream_t stream);
+                          float* Qg, uint16_t* Qg_hilo, uint32_t* hist, int* status, cudaStream_t stream);
 
 // Steps (a)-(c) fused (query selection and group mean in one kernel) for
-// bf16, d = 128, BCP <= 512, NQ <= 32, G <= 8: writes q_idx (rank order,
-// when not null), Qg and Qg_hilo as launch_qgroup does, and zeroes `hist`
-// when given; `normalize` as for launch_qsel. Returns cudaErrorNotSupported
-// for other shapes.
+// bf16, d = 128, BCP <= 512, NQ <= 32, G <= 8, or a one-query chunk
+// (BCP = 1, G <= 32): writes q_idx (rank order, when not null), Qg and
+// Qg_hilo as launch_qgroup does, zeroes `hist` and clears the status words
+// when given; `normalize` as for launch_qsel. Returns
+// cudaErrorNotSupported for other shapes.
 cudaError_t launch_qsel_group_fast(Strided Q, int b, int nq, int nkv, int BCP, int NQ, int32_t* q_idx,
-                                   float* Qg, uint16_t* Qg_hilo, uint32_t* hist, bool normalize,
+                                   float* Qg, uint16_t* Qg_hilo, uint32_t* hist, int* status, bool normalize,
                                    cudaStream_t stream);
 
 // Step (d) on the CUDA cores (fp32 arithmetic; any input dtype). key_norm:

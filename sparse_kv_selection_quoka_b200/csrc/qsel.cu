@@ -358,8 +358,9 @@ qsel_cluster_kernel(const T* __restrict__ Q, int64_t sQb, int64_t sQh, int64_t s
 template <int D>
 __global__ void __launch_bounds__(D)
 qgroup_kernel(const float* __restrict__ Qhat, int nq, int NQ, float* __restrict__ Qg,
-              bf16* __restrict__ Qg_hilo, uint32_t* __restrict__ hist) {
+              bf16* __restrict__ Qg_hilo, uint32_t* __restrict__ hist, int* __restrict__ status) {
   const int i = blockIdx.x, j = blockIdx.y, bi = blockIdx.z, nkv = gridDim.y;
+  clear_status(status);  // (the query select before it latches nothing)
   const int G = nq / nkv;
   const int k = threadIdx.x;
   float acc = 0.f;
@@ -443,11 +444,11 @@ cudaError_t launch_qsel(bool is_bf16, int d, Strided Q, int b, int nq, int BCP, 
 }
 
 cudaError_t launch_qgroup(int d, const float* Qhat, int b, int nq, int nkv, int NQ, float* Qg,
-                          uint16_t* Qg_hilo, uint32_t* hist, cudaStream_t stream) {
+                          uint16_t* Qg_hilo, uint32_t* hist, int* status, cudaStream_t stream) {
   dim3 grid(NQ, nkv, b);
   bf16* hl = reinterpret_cast<bf16*>(Qg_hilo);
-  if (d == 128) qgroup_kernel<128><<<grid, 128, 0, stream>>>(Qhat, nq, NQ, Qg, hl, hist);
-  else if (d == 64) qgroup_kernel<64><<<grid, 64, 0, stream>>>(Qhat, nq, NQ, Qg, hl, hist);
+  if (d == 128) qgroup_kernel<128><<<grid, 128, 0, stream>>>(Qhat, nq, NQ, Qg, hl, hist, status);
+  else if (d == 64) qgroup_kernel<64><<<grid, 64, 0, stream>>>(Qhat, nq, NQ, Qg, hl, hist, status);
   else return cudaErrorNotSupported;
   return cudaGetLastError();
 }

@@ -104,7 +104,7 @@ __device__ __forceinline__ void cl_wait() { asm volatile("barrier.cluster.wait.a
 __global__ void __launch_bounds__(QF_THREADS, 1)
 qsel_fast_kernel(const bf16* __restrict__ Q, int64_t sQb, int64_t sQh, int64_t sQt, int nq, int BCP, int NQ,
                  int32_t* __restrict__ q_idx, float* __restrict__ Qg, bf16* __restrict__ Qg_hilo,
-                 uint32_t* __restrict__ hist, int normalize) {
+                 uint32_t* __restrict__ hist, int* __restrict__ status, int normalize) {
   extern __shared__ __align__(16) uint8_t qf_raw[];
   uint8_t* qs = qf_raw;  // [BCP][256 B], chunk c of row t at slot (c ^ (t & 15))
   __shared__ QfShared sh;
@@ -115,6 +115,7 @@ qsel_fast_kernel(const bf16* __restrict__ Q, int64_t sQb, int64_t sQh, int64_t s
   const int h = j * G + g;
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const bf16* Qh = Q + bi * sQb + h * sQh;
+  clear_status(status);  // the call's first kernel
   pdl_trigger();  // the scoring kernel may launch and start streaming K
 
   // 1. stage the rows; thread (rg, cc) handles chunk cc of rows rg, rg + 32, ...
@@ -289,11 +290,63 @@ qsel_fast_kernel(const bf16* __restrict__ Q, int64_t sQb, int64_t sQh, int64_t s
   cl_wait();
 }
 
+// A chunk of one query (BCP = 1, a decode step): Algorithm 1 has a single
+// candidate, so every head keeps position 0 (NQ = 1) and steps (a)-(b)
+// leave nothing to compute. What remains of step (c): each of the G heads'
+// query is L2-normalised and the G are averaged (in head order) as above.
+// One CTA (4 warps) per (batch, KV head): a warp takes one head at a time,
+// lane l holding columns 4l .. 4l + 3.
+constexpr int Q1_THREADS = 128;
+constexpr int Q1_MAX_G = 32;
+
+__global__ void __launch_bounds__(Q1_THREADS)
+qsel_one_kernel(const bf16* __restrict__ Q, int64_t sQb, int64_t sQh, int nq, int G, int32_t* __restrict__ q_idx,
+                float* __restrict__ Qg, bf16* __restrict__ Qg_hilo, uint32_t* __restrict__ hist,
+                int* __restrict__ status, int normalize) {
+  __shared__ __align__(16) float qhat[Q1_MAX_G][QF_D];
+  const int j = blockIdx.x, bi = blockIdx.y, nkv = gridDim.x;
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  clear_status(status);  // the call's first kernel
+  pdl_trigger();  // the scoring kernel may launch and start streaming K
+  for (int g = warp; g < G; g += Q1_THREADS / 32) {
+    const int h = j * G + g;
+    const uint2 raw = __ldg(reinterpret_cast<const uint2*>(Q + bi * sQb + h * sQh) + lane);
+    const float f[4] = {__uint_as_float(raw.x << 16), __uint_as_float(raw.x & 0xFFFF0000u),
+                        __uint_as_float(raw.y << 16), __uint_as_float(raw.y & 0xFFFF0000u)};
+    const float qq = warp_sum((f[0] * f[0] + f[1] * f[1]) + (f[2] * f[2] + f[3] * f[3]));
+    const float nrm = normalize ? fmaxf(sqrtf(qq), 1e-12f) : 1.f;
+    reinterpret_cast<float4*>(qhat[g])[lane] = make_float4(f[0] / nrm, f[1] / nrm, f[2] / nrm, f[3] / nrm);
+    if (lane == 0 && q_idx != nullptr) q_idx[(int64_t)bi * nq + h] = 0;
+  }
+  __syncthreads();
+  const int64_t row = (int64_t)bi * nkv + j;
+  float acc = 0.f;
+  for (int g = 0; g < G; ++g) acc += qhat[g][tid];
+  const float o = acc * (1.f / (float)G);
+  Qg[row * QF_D + tid] = o;
+  if (Qg_hilo != nullptr) {
+    const bf16 hi = __float2bfloat16_rn(o);
+    Qg_hilo[row * 2 * QF_D + tid] = hi;
+    Qg_hilo[(row * 2 + 1) * QF_D + tid] = __float2bfloat16_rn(o - __bfloat162float(hi));
+  }
+  if (hist != nullptr) {
+    uint4* hr = reinterpret_cast<uint4*>(hist + row * TOPK_HIST_BINS);
+    for (int z = tid; z < TOPK_HIST_BINS / 4; z += Q1_THREADS) hr[z] = make_uint4(0u, 0u, 0u, 0u);
+  }
+}
+
 }  // namespace
 
 cudaError_t launch_qsel_group_fast(Strided Q, int b, int nq, int nkv, int BCP, int NQ, int32_t* q_idx, float* Qg,
-                                   uint16_t* Qg_hilo, uint32_t* hist, bool normalize, cudaStream_t stream) {
+                                   uint16_t* Qg_hilo, uint32_t* hist, int* status, bool normalize,
+                                   cudaStream_t stream) {
   const int G = nq / nkv;
+  if (BCP == 1 && NQ == 1 && G >= 1 && G <= Q1_MAX_G && b <= 65535) {
+    qsel_one_kernel<<<dim3(nkv, b), Q1_THREADS, 0, stream>>>(static_cast<const bf16*>(Q.data), Q.sb, Q.sh, nq, G,
+                                                             q_idx, Qg, reinterpret_cast<bf16*>(Qg_hilo), hist,
+                                                             status, (int)normalize);
+    return cudaGetLastError();
+  }
   if (BCP < 1 || BCP > QF_MAX_BCP || NQ < 1 || NQ > QF_MAX_NQ || NQ > BCP || G < 1 || G > QF_MAX_G)
     return cudaErrorNotSupported;
   if (nkv > 65535 || b > 65535) return cudaErrorNotSupported;
@@ -314,7 +367,7 @@ cudaError_t launch_qsel_group_fast(Strided Q, int b, int nq, int nkv, int BCP, i
   cfg.attrs = attr;
   cfg.numAttrs = 1;
   return cudaLaunchKernelEx(&cfg, qsel_fast_kernel, static_cast<const bf16*>(Q.data), Q.sb, Q.sh, Q.st, nq, BCP,
-                            NQ, q_idx, Qg, reinterpret_cast<bf16*>(Qg_hilo), hist, (int)normalize);
+                            NQ, q_idx, Qg, reinterpret_cast<bf16*>(Qg_hilo), hist, status, (int)normalize);
 }
 
 }  // namespace quoka

@@ -24,6 +24,9 @@ WaitHooks wait_hooks() {
   return WaitHooks{ns == 0 ? 2000000000ull : ns, g_inject.load(std::memory_order_relaxed)};
 }
 
+// Device address of quoka_select_static's fixed scratch (select_static.cu).
+quoka_status static_scratch_address(void** out);
+
 }  // namespace quoka
 
 namespace {
@@ -211,11 +214,13 @@ quoka_status run_select(const quoka_tensor* Q, const quoka_tensor* K, const Sele
 
   cudaError_t e = cudaErrorNotSupported;
   if (bf && d == 128)
-    e = quoka::launch_qsel_group_fast(strided(Q), b, nq, nkv, BCP, NQ, qidx, qg, qhilo, hist, cosine, stream);
+    e = quoka::launch_qsel_group_fast(strided(Q), b, nq, nkv, BCP, NQ, qidx, qg, qhilo, hist, status, cosine,
+                                      stream);
   if (e == cudaErrorNotSupported) {
     e = quoka::launch_qsel(bf, d, strided(Q), b, nq, BCP, NQ, qhat, qidx, cosine, stream);
     if (e != cudaSuccess) return cuda_status(e);
-    e = quoka::launch_qgroup(d, qhat, b, nq, nkv, NQ, qg, bf ? qhilo : nullptr, bf ? hist : nullptr, stream);
+    e = quoka::launch_qgroup(d, qhat, b, nq, nkv, NQ, qg, bf ? qhilo : nullptr, bf ? hist : nullptr, status,
+                             stream);
   }
   if (e != cudaSuccess) return cuda_status(e);
   bool hist_made = false;
@@ -408,7 +413,7 @@ quoka_status quoka_select_ex(const quoka_tensor* Q, const quoka_tensor* K, int N
   st = check_ws(ws, ws_bytes, L.select_total);
   if (st != QUOKA_OK) return st;
   cudaStream_t cs = static_cast<cudaStream_t>(stream);
-  if (cudaMemsetAsync(at<int>(ws, L.status), 0, 2 * sizeof(int), cs) != cudaSuccess) return QUOKA_ERR_CUDA;
+  // (the status words are cleared by the first kernel)
   return run_select(Q, K, s, NQ, (int)bsa_eff, kv_idx, kv_count, q_idx, s_agg, ws, L, cs, flags);
 }
 
@@ -547,8 +552,7 @@ quoka_status quoka_prefill_chunk(const quoka_tensor* Q, const quoka_tensor* K,
   st = check_ws(ws, ws_bytes, L.total);
   if (st != QUOKA_OK) return st;
   cudaStream_t cs = static_cast<cudaStream_t>(stream);
-  int* status = at<int>(ws, L.status);
-  if (cudaMemsetAsync(status, 0, 2 * sizeof(int), cs) != cudaSuccess) return QUOKA_ERR_CUDA;
+  int* status = at<int>(ws, L.status);  // cleared by the selection's first kernel
   int32_t* kv_idx = kv_idx_out != nullptr ? kv_idx_out : at<int32_t>(ws, L.kvidx);
   int32_t* kv_count = at<int32_t>(ws, L.kvcount);
   st = run_select(Q, K, s, NQ, (int)bsa_eff, kv_idx, kv_count, nullptr, nullptr, ws, L, cs);
@@ -561,7 +565,13 @@ quoka_status quoka_prefill_chunk(const quoka_tensor* Q, const quoka_tensor* K,
 }
 
 quoka_status quoka_get_device_status(const void* ws, void* stream, int32_t* device_status) {
-  if (ws == nullptr || device_status == nullptr) return QUOKA_ERR_INVALID_ARG;
+  if (device_status == nullptr) return QUOKA_ERR_INVALID_ARG;
+  if (ws == nullptr) {  // the fixed scratch of quoka_select_static
+    void* p = nullptr;
+    const quoka_status st = quoka::static_scratch_address(&p);
+    if (st != QUOKA_OK) return st;
+    ws = p;
+  }
   cudaStream_t cs = static_cast<cudaStream_t>(stream);
   int32_t v = 0;
   if (cudaMemcpyAsync(&v, ws, sizeof(int32_t), cudaMemcpyDeviceToHost, cs) != cudaSuccess)
@@ -572,7 +582,13 @@ quoka_status quoka_get_device_status(const void* ws, void* stream, int32_t* devi
 }
 
 quoka_status quoka_get_device_fault_site(const void* ws, void* stream, int32_t* site) {
-  if (ws == nullptr || site == nullptr) return QUOKA_ERR_INVALID_ARG;
+  if (site == nullptr) return QUOKA_ERR_INVALID_ARG;
+  if (ws == nullptr) {  // the fixed scratch of quoka_select_static
+    void* p = nullptr;
+    const quoka_status st = quoka::static_scratch_address(&p);
+    if (st != QUOKA_OK) return st;
+    ws = p;
+  }
   cudaStream_t cs = static_cast<cudaStream_t>(stream);
   int32_t v = 0;
   if (cudaMemcpyAsync(&v, static_cast<const int32_t*>(ws) + 1, sizeof(int32_t), cudaMemcpyDeviceToHost, cs) !=

@@ -15,36 +15,29 @@
 // ordering between them) race on it; callers must order them.
 #include <cuda_runtime.h>
 
-#include <mutex>
-
 #include "quoka.h"
 
 namespace {
 
 __device__ __align__(256) unsigned char g_select_scratch[QUOKA_STATIC_SCRATCH_BYTES];
 
-constexpr int kMaxDevices = 64;
-std::mutex g_setup_mutex;
-void* g_scratch_addr[kMaxDevices] = {};
+}  // namespace
 
-// Device address of g_select_scratch on the current device. In host code
-// the symbol name is only a host-side stand-in, so the address is looked up
-// once per device (with that device current) and cached.
-quoka_status scratch_for_current_device(void** out) {
-  int dev = -1;
-  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0) return QUOKA_ERR_CUDA;
-  if (dev >= kMaxDevices) return QUOKA_ERR_UNSUPPORTED;
-  std::lock_guard<std::mutex> lock(g_setup_mutex);
-  if (g_scratch_addr[dev] == nullptr) {
-    void* p = nullptr;
-    if (cudaGetSymbolAddress(&p, g_select_scratch) != cudaSuccess || p == nullptr) return QUOKA_ERR_CUDA;
-    g_scratch_addr[dev] = p;
-  }
-  *out = g_scratch_addr[dev];
+namespace quoka {
+
+// Device address of g_select_scratch in the current context. In host code
+// the symbol name is only a host-side stand-in; the runtime resolves it for
+// the context current at the call, so the address is looked up on every
+// call rather than cached (a cached address would go stale after
+// cudaDeviceReset or under another context on the same device).
+quoka_status static_scratch_address(void** out) {
+  void* p = nullptr;
+  if (cudaGetSymbolAddress(&p, g_select_scratch) != cudaSuccess || p == nullptr) return QUOKA_ERR_CUDA;
+  *out = p;
   return QUOKA_OK;
 }
 
-}  // namespace
+}  // namespace quoka
 
 extern "C" quoka_status quoka_select_static(const quoka_tensor* Q, const quoka_tensor* K, int NQ,
                                             int BSA, int32_t* kv_idx, int32_t* kv_count,
@@ -56,11 +49,11 @@ extern "C" quoka_status quoka_select_static(const quoka_tensor* Q, const quoka_t
   if (need == 0) return QUOKA_ERR_INVALID_ARG;
   if (need > (size_t)QUOKA_STATIC_SCRATCH_BYTES) return QUOKA_ERR_WORKSPACE;
   void* scratch = nullptr;
-  const quoka_status st = scratch_for_current_device(&scratch);
+  const quoka_status st = quoka::static_scratch_address(&scratch);
   if (st != QUOKA_OK) return st;
-  // quoka_select clears the scratch's status word on `stream` before its
-  // kernels run; every other scratch region is fully written before it is
-  // read, so the previous call's contents never leak into this one.
+  // quoka_select's first kernel clears the scratch's status words; every
+  // other scratch region is fully written before it is read, so the previous
+  // call's contents never leak into this one.
   return quoka_select(Q, K, NQ, BSA, kv_idx, kv_count, q_idx, s_agg, scratch,
                       (size_t)QUOKA_STATIC_SCRATCH_BYTES, stream);
 }

@@ -45,6 +45,7 @@ CASES = [
     (1, 6, 3, 64, 900, 3, 200, "f32", [[200, 0, 17]], False),      # fp32, d = 64, a head with chunk keys only
     (1, 4, 4, 128, 129, 2, 128, "bf16", "full", False),            # G = 1, BSA_eff = T
     (1, 8, 2, 128, 0, 1, 0, "bf16", "full", False),                # T = 0: the chunk's own key only
+    (2, 12, 2, 64, 1500, 5, 400, "bf16", [[400, 3], [0, 399]], True),  # d = 64, 30 rows (two 16-row tiles)
 ]
 
 
@@ -107,6 +108,37 @@ def test_decode_step_through_prefill_chunk(BCP):
     from tests.test_gpu_parity import run_prefill_and_check, run_select_and_check
     ref, gi, _ = run_select_and_check(x)
     run_prefill_and_check(x, ref, gi)
+
+
+ONE_TOKEN = [
+    # b, nq, nkv, T, BSA, strided Q, dot-product score
+    (2, 48, 3, 5000, 900, True, False),   # G = 16 query heads per KV head
+    (1, 32, 1, 3000, 3000, False, False),  # G = 32, BSA_eff = T
+    (1, 8, 8, 1000, 100, False, True),     # G = 1, the dot-product score
+]
+
+
+@pytest.mark.gpu
+@pytest.mark.parametrize("k", range(len(ONE_TOKEN)), ids=[f"b{c[0]}_nq{c[1]}_nkv{c[2]}_T{c[3]}" for c in ONE_TOKEN])
+def test_one_token_selection(k):
+    """A one-query chunk: every head keeps its only query (q_idx = 0, the one
+    candidate of Algorithm 1), and S_agg / the selected keys follow from the
+    group mean of the G normalised (or raw) queries. Against the oracle."""
+    b, nq, nkv, T, BSA, strided, dot = ONE_TOKEN[k]
+    x = inputs.make_chunk(b, nq, nkv, 128, T, 1, 1, BSA, dtype="bf16", structure="llama", seed=330 + k)
+    Q = P.to_dev_view(x.Q, "bf16") if strided else P.to_dev(x.Q, "bf16")
+    K = P.to_dev(x.K, "bf16")
+    kv_idx, kv_count, q_idx, s_agg = q().quoka_select(Q, K, 1, BSA, want_q_idx=True, want_s_agg=True,
+                                                      dot_product=dot)
+    torch.cuda.synchronize()
+    assert torch.equal(q_idx.cpu(), torch.zeros((b, nq, 1), dtype=torch.int32))
+    ref = orc.select(x.Q, x.K, 1, BSA, dot_product=dot)
+    assert np.array_equal(ref["q_idx"], np.zeros((b, nq, 1)))
+    scale = max(1.0, float(np.abs(ref["S_agg"]).max())) if dot else 1.0
+    err = np.abs(s_agg.cpu().numpy().astype(np.float64) - ref["S_agg"]).max()
+    assert err <= P.S_TOL * scale, f"S_agg max-abs error {err:.3e}"
+    P.check_kv_sets(kv_idx.cpu().numpy().astype(np.int64), kv_count.cpu().numpy(), ref["S_agg"], min(BSA, T),
+                    ref["sel"], band=P.KV_TIE_BAND * scale)
 
 
 # ---------------------------------------------------------------- host side

@@ -48,8 +48,12 @@ def test_static_scratch_select_matches_workspace_select_twice():
         pytest.skip("no CUDA device")
     first = inputs.make_chunk(1, 24, 8, 128, 8192, 256, 16, 2048, dtype="bf16", structure="llama", seed=41)
     second = inputs.make_chunk(2, 8, 2, 128, 3000, 100, 7, 500, dtype="bf16", structure="qwen", seed=42)
+    import sparse_kv_selection_quoka_b200 as q
     for x in (first, second):
         _compare(*_both(x))
+        # the fixed scratch's status words (ws = NULL): no device fault
+        assert q.quoka_get_device_status(None) == 0
+        assert q.quoka_get_device_fault_site(None) == 0
 
 
 def test_static_scratch_rejects_oversized_shapes():
