@@ -197,14 +197,21 @@ def gather_bytes(b, nkv, d, bsa_eff, es):
 def kernels_per_chunk(w, T, bsa_eff):
     """Our kernel launches in one quoka_prefill_chunk call on a bf16, d = 128
     workload: query select + group mean (one fused kernel for BCP <= 512,
-    NQ <= 32, G <= 8, else two), the scoring (T > 0), the top-k and the
-    gather (BSA_eff > 0), and the attention (a short chunk's takes two)."""
+    NQ <= 32, G <= 8 or for one query, else two), the scoring (T > 0), the
+    top-k and the gather (BSA_eff > 0), and the attention (a short chunk's
+    takes two; so do split key ranges, with their merge)."""
     G = w.nq // w.nkv
-    fused = w.dtype == "bf16" and w.d == 128 and w.BCP <= 512 and w.NQ <= 32 and G <= 8
+    fused = w.dtype == "bf16" and w.d == 128 and ((w.BCP <= 512 and w.NQ <= 32 and G <= 8)
+                                                   or (w.BCP == 1 and G <= 32))
     short = G * w.BCP <= 64
     n = (1 if fused else 2) + (1 if T > 0 else 0)
     if bsa_eff > 0:
         n += 1 if short else 2
+        # the merge of the attention's split key ranges (few query tiles)
+        tiles = w.b * w.nq * ((w.BCP + 127) // 128)
+        if not short and w.dtype == "bf16" and w.d == 128 and 2 * tiles <= 148:
+            if min(4, 148 // tiles, ((bsa_eff + 127) // 128 + 1) // 2) >= 2:
+                n += 1
     return n + (2 if short else 1)
 
 

@@ -22,6 +22,15 @@
 // softmax. After the last tile the two partial results of every row are in
 // the same SM's TMEM and are combined there.
 //
+// Split key ranges: when the query tiles alone leave most SMs idle (short
+// chunks, few heads), each query tile's key tiles are cut into nsplit
+// contiguous ranges and the grid runs one CTA per (tile, range). Such a CTA
+// stores its range's output, normalised by the range's own softmax sum, as
+// a bf16 tile (the same TMA store, into a partial buffer) with the range's
+// log-sum-exp in fp32; a merge kernel then combines the
+// ranges of every row: O = sum_s exp(lse_s - LSE) O_s, LSE = log sum_s
+// exp(lse_s).
+//
 // Warp roles (352 threads):
 //   warps 0-7   softmax: warpgroup w = warp / 4, one query row per thread
 //               (row = TMEM lane); then the combine of the two partials,
@@ -41,6 +50,8 @@
 // code, and the CTA unwinds (waits for in-flight copies and MMAs, frees
 // TMEM, stores no output tile).
 #include <stddef.h>
+
+#include <algorithm>
 
 #include "attn_common.cuh"
 #include "kernels.h"
@@ -64,6 +75,7 @@ constexpr int PV_PARTS = 2;
 
 struct Maps {
   CUtensorMap q, ks, vs, kc, vc, o;
+  CUtensorMap op;  // split key ranges: the partial outputs, (nsplit * b, nq, BCP, d)
 };
 
 struct __align__(1024) Smem {
@@ -107,21 +119,22 @@ __device__ __forceinline__ void drain_ring(Smem& sm, uint64_t* full, int nload, 
 // wait on a product that waits on a later load. With a thread per ring, a K
 // load never queues behind a V stage that is released later.
 template <bool IS_V>
-__device__ __forceinline__ void load_kv(Smem& sm, const Maps& maps, int nT, int ntile_sel, int j, int bi,
-                                        int* status) {
+__device__ __forceinline__ void load_kv(Smem& sm, const Maps& maps, int nT, int kt_base, int ntile_sel, int j,
+                                        int bi, int* status) {
   constexpr int ST = IS_V ? VST : KST;
   uint64_t* const full = IS_V ? sm.v_full : sm.k_full;
   uint64_t* const empty = IS_V ? sm.v_empty : sm.k_empty;
   int nl = 0;
   for (int kt = 0; kt < nT; ++kt) {
-    const bool sel_tile = kt < ntile_sel;
+    const bool sel_tile = kt_base + kt < ntile_sel;
     const int s = kt % ST;
     if (kt >= ST && !mbar_wait(&empty[s], ((kt / ST) - 1) & 1, &sm.abort, sm.wait_ns)) {
       record_abort(sm, status, IS_V ? 14 : 11);
       break;
     }
     const CUtensorMap* m = IS_V ? (sel_tile ? &maps.vs : &maps.vc) : (sel_tile ? &maps.ks : &maps.kc);
-    load_tile(smem_u32(IS_V ? sm.v[s] : sm.k[s]), m, &full[s], (sel_tile ? kt : kt - ntile_sel) * N, j, bi);
+    load_tile(smem_u32(IS_V ? sm.v[s] : sm.k[s]), m, &full[s],
+              (sel_tile ? kt_base + kt : kt_base + kt - ntile_sel) * N, j, bi);
     nl = kt + 1;
   }
   drain_ring<ST>(sm, full, nl, status, IS_V ? 15 : 12);
@@ -137,8 +150,9 @@ attn_tma_kernel(const __grid_constant__ Maps maps, const AttnArgs a) {
   const int j = blockIdx.y, bi = blockIdx.z;
   const int G = a.nq / a.nkv;
   const int ntt = (a.BCP + 127) / 128;  // row tiles per query head
-  const int h = j * G + (int)blockIdx.x / ntt;
-  const int t0 = ((int)blockIdx.x % ntt) * 128;
+  const int qt = (int)blockIdx.x % (G * ntt), split = (int)blockIdx.x / (G * ntt);
+  const int h = j * G + qt / ntt;
+  const int t0 = (qt % ntt) * 128;
 
   // Setup and the Q load touch nothing the previous kernel writes: they run
   // before the grid-dependency wait, overlapping that kernel's tail.
@@ -189,15 +203,18 @@ attn_tma_kernel(const __grid_constant__ Maps maps, const AttnArgs a) {
   const int nsel = a.bsa > 0 ? max(0, min(__ldcg(a.kv_count + kvrow), a.bsa)) : 0;
   const int nchunk = a.no_chunk ? 0 : min(a.BCP, t0 + 128);
   const int ntile_sel = (nsel + N - 1) / N;
-  const int nT = ntile_sel + (nchunk + N - 1) / N;  // key tiles (0 only without the chunk's keys)
+  const int nT_all = ntile_sel + (nchunk + N - 1) / N;  // key tiles (0 only without the chunk's keys)
+  // this CTA's key tiles: range `split` of nsplit (all of them when 1)
+  const int kt_base = (int)((int64_t)nT_all * split / a.nsplit);
+  const int nT = (int)((int64_t)nT_all * (split + 1) / a.nsplit) - kt_base;
   const int npair = (nT + 1) / 2;
 
   if (warp == LOAD_WARP) {
     // ------------------------------------------------------------ TMA loads
-    if (lane == 0) load_kv<false>(sm, maps, nT, ntile_sel, j, bi, a.status);
+    if (lane == 0) load_kv<false>(sm, maps, nT, kt_base, ntile_sel, j, bi, a.status);
     __syncwarp();
   } else if (warp == VLOAD_WARP) {
-    if (lane == 0) load_kv<true>(sm, maps, nT, ntile_sel, j, bi, a.status);
+    if (lane == 0) load_kv<true>(sm, maps, nT, kt_base, ntile_sel, j, bi, a.status);
     __syncwarp();
   } else if (warp == MMA_WARP) {
     // ------------------------------------------------------------ MMA issue
@@ -270,17 +287,22 @@ attn_tma_kernel(const __grid_constant__ Maps maps, const AttnArgs a) {
     float m = -INFINITY, l = 0.f;
     bool alive = true;
     const int nmine = (nT - w + 1) / 2;  // key tiles of this warpgroup (warpgroup-uniform)
+    // the range's selected tiles come first (none when it starts past them);
+    // selected key numbers relative to the range's first key
+    const int sel_rel = ntile_sel - kt_base;
+    const int nsel_rel = nsel - kt_base * N;
     for (int i = 0; i < nmine && alive; ++i) {
       alive = warp_wait(&sm.s_full[w], i & 1, sm, a.status, 31 + w);
       if (!alive) break;
       tc_fence_after();
-      const int kt = 2 * i + w;
-      const bool sel_tile = kt < ntile_sel;
-      // key c of the tile is key number base_n + c of its list; it is
-      // visible to row t when it is a selected key below nsel, or a chunk
-      // key at a position p < nchunk with p <= t
-      const int base_n = (sel_tile ? kt : kt - ntile_sel) * N;
-      const int lim = sel_tile ? nsel : min(nchunk, t + 1);
+      const int kt = 2 * i + w;  // (within this CTA's key range)
+      const bool sel_tile = kt < sel_rel;
+      // key c of the tile is key number base_n + c of its list (selected
+      // keys counted from the range's first one); it is visible to row t
+      // when it is a selected key below nsel, or a chunk key at a position
+      // p < nchunk with p <= t
+      const int base_n = (sel_tile ? kt : kt - sel_rel) * N;
+      const int lim = sel_tile ? nsel_rel : min(nchunk, t + 1);
       softmax_tile_split<PV_PARTS>(S, tmem + lane_off + 256u + 128u * w, i > 0, base_n, lim,
                                                      qscale, m, l, sm.p_part[w]);
     }
@@ -306,9 +328,11 @@ attn_tma_kernel(const __grid_constant__ Maps maps, const AttnArgs a) {
     const float inv = L > 0.f ? 1.f / L : 0.f;  // no visible key: O = 0, lse = -inf
     // warpgroup w combines, normalises and stages output columns
     // [64w, 64w + 64) of its rows, bf16, in the 128-byte-swizzled layout the
-    // TMA store reads (the Q area: every MMA is done)
+    // TMA store reads (the Q area: every MMA is done); a key range of a split
+    // tile stores them to its partial output instead
     const uint32_t O0 = tmem + lane_off + 256u + 64u * w;
     const uint32_t O1 = tmem + lane_off + 384u + 64u * w;
+    const bool part = a.nsplit > 1;
 #pragma unroll 1
     for (int c2 = 0; c2 < 2; ++c2) {
       float o[32], p[32];
@@ -333,15 +357,23 @@ attn_tma_kernel(const __grid_constant__ Maps maps, const AttnArgs a) {
         *reinterpret_cast<uint4*>(sm.q + sw128_offset(r, (64 * w + 32 * c2 + u) >> 3, 128)) = pk;
       }
     }
-    if (w == 0 && t < a.BCP && a.lse != nullptr)
-      a.lse[((int64_t)bi * a.nq + h) * a.BCP + t] = (M + __log2f(L)) * 0.6931471805599453f;
+    if (w == 0 && t < a.BCP) {
+      const int64_t orow = ((int64_t)bi * a.nq + h) * a.BCP + t;
+      if (part)
+        a.lse_parts[(int64_t)split * a.b * a.nq * a.BCP + orow] =
+            L > 0.f ? (M + __log2f(L)) * 0.6931471805599453f : -INFINITY;
+      else if (a.lse != nullptr)
+        a.lse[orow] = (M + __log2f(L)) * 0.6931471805599453f;
+    }
     // rows past the chunk are clipped by the store
     fence_proxy_async_smem();
     named_barrier_sync(1, 256);
     // (after a timeout the tile is not stored: the status word reports it)
     if (tid == 0 && !*reinterpret_cast<volatile int*>(&sm.abort)) {
-      tma_store_4d(&maps.o, smem_u32(sm.q), 0, t0, h, bi);
-      tma_store_4d(&maps.o, smem_u32(sm.q) + ATOM_BYTES, 64, t0, h, bi);
+      const CUtensorMap* om = part ? &maps.op : &maps.o;
+      const int zb = part ? split * a.b + bi : bi;
+      tma_store_4d(om, smem_u32(sm.q), 0, t0, h, zb);
+      tma_store_4d(om, smem_u32(sm.q) + ATOM_BYTES, 64, t0, h, zb);
       bulk_commit_group();
       bulk_wait_group_read_0();  // the staging may go once the copy has read it
     }
@@ -355,13 +387,67 @@ attn_tma_kernel(const __grid_constant__ Maps maps, const AttnArgs a) {
   }
 }
 
+// The merge of the key ranges of split tiles: one thread per 8 output
+// elements of a row. Ranges that saw no visible key (lse = -inf) weigh 0; a
+// row with none gives O = 0, lse = -inf.
+constexpr int kMergeThreads = 256;
+
+__global__ void __launch_bounds__(kMergeThreads)
+attn_split_merge_kernel(const bf16* __restrict__ O_parts, const float* __restrict__ lse_parts, int nsplit,
+                        int64_t rows, bf16* __restrict__ O, float* __restrict__ lse) {
+  pdl_wait();  // the partials come from the attention kernel
+  const int64_t g = (int64_t)blockIdx.x * kMergeThreads + threadIdx.x;
+  if (g >= rows * (D / 8)) return;
+  const int64_t row = g / (D / 8);
+  const int c0 = (int)(g % (D / 8)) * 8;
+  float ls[4];
+  float M = -INFINITY;
+#pragma unroll
+  for (int s = 0; s < 4; ++s) {
+    ls[s] = s < nsplit ? __ldcg(lse_parts + (int64_t)s * rows + row) : -INFINITY;
+    M = fmaxf(M, ls[s]);
+  }
+  float acc[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
+  float L = 0.f;
+#pragma unroll
+  for (int s = 0; s < 4; ++s) {
+    if (ls[s] == -INFINITY) continue;
+    const float wgt = __expf(ls[s] - M);
+    L += wgt;
+    const uint4 raw = __ldcg(reinterpret_cast<const uint4*>(O_parts + ((int64_t)s * rows + row) * D + c0));
+    const uint32_t wd[4] = {raw.x, raw.y, raw.z, raw.w};
+#pragma unroll
+    for (int u = 0; u < 4; ++u) {
+      acc[2 * u] = fmaf(wgt, __uint_as_float(wd[u] << 16), acc[2 * u]);
+      acc[2 * u + 1] = fmaf(wgt, __uint_as_float(wd[u] & 0xFFFF0000u), acc[2 * u + 1]);
+    }
+  }
+  const float inv = L > 0.f ? 1.f / L : 0.f;
+  uint4 pk;
+  pk.x = pack_bf16x2(acc[0] * inv, acc[1] * inv);
+  pk.y = pack_bf16x2(acc[2] * inv, acc[3] * inv);
+  pk.z = pack_bf16x2(acc[4] * inv, acc[5] * inv);
+  pk.w = pack_bf16x2(acc[6] * inv, acc[7] * inv);
+  *reinterpret_cast<uint4*>(O + row * D + c0) = pk;
+  if (c0 == 0 && lse != nullptr) lse[row] = L > 0.f ? M + __logf(L) : -INFINITY;
+}
+
 }  // namespace
+
+int attn_splits(int64_t tiles, int nt) {
+  if (tiles < 1 || 2 * tiles > kAttnWaveCTAs) return 1;
+  int s = (int)std::min<int64_t>(4, kAttnWaveCTAs / tiles);
+  s = std::min(s, nt / 2);
+  return s < 2 ? 1 : s;
+}
 
 cudaError_t launch_attn_tc(const AttnArgs& args, bool pdl, cudaStream_t stream) {
   if (args.d != D) return cudaErrorNotSupported;
   // rows gathered by index while loading: the other kernel
   if (args.kv_idx != nullptr && args.bsa > 0) return launch_attn_tc_gather(args, stream);
   AttnArgs a = args;
+  if (a.nsplit < 1 || a.nsplit > 4 || (a.nsplit > 1 && (a.O_parts == nullptr || a.lse_parts == nullptr)))
+    return cudaErrorInvalidValue;
   const WaitHooks hooks = wait_hooks();
   a.wait_ns = hooks.wait_ns;
   a.inject = hooks.inject == INJECT_ATTN_TMA ? 1 : 0;
@@ -372,6 +458,12 @@ cudaError_t launch_attn_tc(const AttnArgs& args, bool pdl, cudaStream_t stream) 
       !encode_bf16_4d(&maps.vc, a.Vc.data, D, a.BCP, a.nkv, a.b, a.Vc.st, a.Vc.sh, a.Vc.sb, 128) ||
       !encode_bf16_4d(&maps.o, a.O, D, a.BCP, a.nq, a.b, D, oh, ob, 128))
     return cudaErrorNotSupported;
+  if (a.nsplit > 1) {
+    if (!encode_bf16_4d(&maps.op, a.O_parts, D, a.BCP, a.nq, (uint64_t)a.nsplit * a.b, D, oh, ob, 128))
+      return cudaErrorNotSupported;
+  } else {
+    maps.op = maps.o;  // never written
+  }
   if (a.bsa > 0) {
     // the gathered selected rows (b, nkv, bsa, d)
     if (!encode_bf16_4d(&maps.ks, a.K.data, D, a.bsa, a.nkv, a.b, a.K.st, a.K.sh, a.K.sb, 128) ||
@@ -386,7 +478,7 @@ cudaError_t launch_attn_tc(const AttnArgs& args, bool pdl, cudaStream_t stream) 
   if (e != cudaSuccess) return e;
   const int G = a.nq / a.nkv;
   cudaLaunchConfig_t cfg = {};
-  cfg.gridDim = dim3(G * ((a.BCP + 127) / 128), a.nkv, a.b);  // one query tile per CTA
+  cfg.gridDim = dim3(G * ((a.BCP + 127) / 128) * a.nsplit, a.nkv, a.b);  // one query tile (range) per CTA
   cfg.blockDim = dim3(THREADS);
   cfg.dynamicSmemBytes = smem;
   cfg.stream = stream;
@@ -395,7 +487,18 @@ cudaError_t launch_attn_tc(const AttnArgs& args, bool pdl, cudaStream_t stream) 
   attr[0].val.programmaticStreamSerializationAllowed = 1;
   cfg.attrs = attr;
   cfg.numAttrs = pdl ? 1 : 0;
-  return cudaLaunchKernelEx(&cfg, attn_tma_kernel, maps, a);
+  e = cudaLaunchKernelEx(&cfg, attn_tma_kernel, maps, a);
+  if (e != cudaSuccess || a.nsplit == 1) return e;
+  const int64_t rows = (int64_t)a.b * a.nq * a.BCP;
+  cudaLaunchConfig_t mc = {};
+  mc.gridDim = dim3((unsigned)((rows * (D / 8) + kMergeThreads - 1) / kMergeThreads));
+  mc.blockDim = dim3(kMergeThreads);
+  mc.stream = stream;
+  mc.attrs = attr;
+  mc.numAttrs = 1;  // waits for the attention inside
+  return cudaLaunchKernelEx(&mc, attn_split_merge_kernel, static_cast<const bf16*>(a.O_parts),
+                            static_cast<const float*>(a.lse_parts), a.nsplit, rows, static_cast<bf16*>(a.O),
+                            a.lse);
 }
 
 }  // namespace quoka

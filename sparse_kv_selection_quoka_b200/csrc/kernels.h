@@ -107,7 +107,21 @@ struct AttnArgs {
                             // rows with no visible key then give O = 0 and lse = -inf
   uint64_t wait_ns = 0;     // bound of every wait (set by the launcher from wait_hooks())
   int inject = 0;           // test hook (set by the launcher from wait_hooks())
+  // Split key ranges (tensor-core attention over gathered rows only): with
+  // nsplit > 1 every query tile's key tiles are cut into nsplit contiguous
+  // ranges, one CTA each; a CTA writes its range's normalised partial output
+  // and log-sum-exp, and a merge kernel combines them into O / lse.
+  int nsplit = 1;
+  void* O_parts = nullptr;     // (nsplit * b, nq, BCP, d) bf16, contiguous
+  float* lse_parts = nullptr;  // (nsplit, b, nq, BCP) fp32
 };
+
+// Key-range splits of the tensor-core attention for a launch of `tiles`
+// 128-row query tiles with at most `nt` key tiles each: 1 when the tiles
+// already fill the GPU, else as many ranges (<= 4, each of >= 2 key tiles)
+// as keep the CTAs within one wave of kAttnWaveCTAs.
+constexpr int kAttnWaveCTAs = 148;  // SMs of a B200: one attention CTA per SM
+int attn_splits(int64_t tiles, int nt);
 
 // Steps (f)+(g) in fp32 on the CUDA cores (any input dtype).
 cudaError_t launch_attn_simt(bool bf16, const AttnArgs& a, cudaStream_t stream);

@@ -51,10 +51,30 @@ struct WsLayout {
   size_t select_total = 0;  // end of what quoka_select needs
   size_t ksel = 0;      // (b, nkv, BSA_eff, d) bf16: gathered selected K (tensor-core attention)
   size_t vsel = 0;      // (b, nkv, BSA_eff, d) bf16: gathered selected V
+  size_t aparts = 0;    // split key ranges of the tensor-core attention: partials
+  size_t aparts_bytes = 0;
   size_t dparts = 0;    // short chunks: (nsplit, b, nq, BCP, d) fp32 partial outputs
   size_t dlse = 0;      // short chunks: (nsplit, b, nq, BCP) fp32 partial log-sum-exps
   size_t total = 0;
 };
+
+// Key-range splits of the tensor-core attention over the gathered rows
+// (bf16, d = 128) for a chunk of b * nq * ceil(BCP / 128) query tiles and
+// BSA_eff selected keys (with the chunk's own keys unless no_chunk).
+int attn_nsplit(int64_t b, int64_t nq, int64_t BCP, int64_t d, int64_t bsa_eff, bool bf16, bool no_chunk) {
+  if (!bf16 || d != 128) return 1;
+  const int64_t tiles = b * nq * ((BCP + 127) / 128);
+  const int64_t nt = (bsa_eff + 127) / 128 + (no_chunk ? 0 : 1);
+  return quoka::attn_splits(tiles, (int)std::min<int64_t>(nt, 1 << 20));
+}
+
+// Bytes of the partials of `nsplit` key ranges: (nsplit * b, nq, BCP, d)
+// bf16 outputs, then (nsplit, b, nq, BCP) fp32 log-sum-exps.
+size_t attn_parts_bytes(int64_t b, int64_t nq, int64_t BCP, int64_t d, int nsplit) {
+  if (nsplit <= 1) return 0;
+  const int64_t rows = (int64_t)nsplit * b * nq * BCP;
+  return align_up((size_t)(rows * d) * 2) + align_up((size_t)rows * 4);
+}
 
 // Chunks whose G * BCP query rows per KV head fit one CTA of the decode
 // attention take it (its fp32 partials live in the workspace).
@@ -70,6 +90,7 @@ bool uses_gather_buffers(quoka_dtype dtype, int64_t d, int64_t bsa_eff) {
 
 WsLayout ws_layout(int64_t b, int64_t nq, int64_t nkv, int64_t d, int64_t T, int64_t NQ,
                    int64_t bsa_eff, bool gather_buffers, int64_t BCP = 0, bool decode = false) {
+  // (gather_buffers implies bf16, d = 128)
   WsLayout L;
   size_t off = 0;
   auto take = [&](size_t bytes) {
@@ -90,6 +111,10 @@ WsLayout ws_layout(int64_t b, int64_t nq, int64_t nkv, int64_t d, int64_t T, int
   if (gather_buffers) {
     L.ksel = take((size_t)(b * nkv * bsa_eff * d) * 2);
     L.vsel = take((size_t)(b * nkv * bsa_eff * d) * 2);
+    if (BCP > 0) {
+      L.aparts_bytes = attn_parts_bytes(b, nq, BCP, d, attn_nsplit(b, nq, BCP, d, bsa_eff, true, false));
+      if (L.aparts_bytes > 0) L.aparts = take(L.aparts_bytes);
+    }
   }
   if (decode) {
     const int64_t rows = (int64_t)quoka::decode_splits((int)bsa_eff, (int)BCP) * b * nq * BCP;
@@ -286,7 +311,8 @@ quoka_status validate_attn(const quoka_tensor* Q, const quoka_tensor* K, const q
 quoka_status run_attn(const quoka_tensor* Q, Strided K, Strided V, const quoka_tensor* Kc,
                       const quoka_tensor* Vc, const AttnShapes& s, int64_t T, const int32_t* kv_idx,
                       const int32_t* kv_count, int bsa_eff, float scale, void* O, float* lse,
-                      int* status, cudaStream_t stream, bool pdl = false, bool no_chunk = false) {
+                      int* status, cudaStream_t stream, bool pdl = false, bool no_chunk = false,
+                      void* parts = nullptr, size_t parts_bytes = 0) {
   quoka::AttnArgs a;
   a.no_chunk = no_chunk ? 1 : 0;
   a.Q = strided(Q);
@@ -307,6 +333,17 @@ quoka_status run_attn(const quoka_tensor* Q, Strided K, Strided V, const quoka_t
   a.O = O;
   a.lse = lse;
   a.status = status;
+  if (kv_idx == nullptr && parts != nullptr) {
+    // split key ranges when the query tiles leave most SMs idle and the
+    // workspace holds the partials
+    const int ns = attn_nsplit(s.b, s.nq, s.BCP, s.d, bsa_eff, Q->dtype == QUOKA_BF16, no_chunk);
+    if (ns > 1 && parts_bytes >= attn_parts_bytes(s.b, s.nq, s.BCP, s.d, ns)) {
+      const int64_t rows = (int64_t)ns * s.b * s.nq * s.BCP;
+      a.nsplit = ns;
+      a.O_parts = parts;
+      a.lse_parts = reinterpret_cast<float*>(static_cast<char*>(parts) + align_up((size_t)(rows * s.d) * 2));
+    }
+  }
   cudaError_t e = cudaErrorNotSupported;
   if (Q->dtype == QUOKA_BF16) e = quoka::launch_attn_tc(a, pdl, stream);
   if (e == cudaErrorNotSupported) e = quoka::launch_attn_simt(Q->dtype == QUOKA_BF16, a, stream);
@@ -320,7 +357,8 @@ quoka_status gather_then_attn(const quoka_tensor* Q, const quoka_tensor* K, cons
                               const quoka_tensor* Kc, const quoka_tensor* Vc, const AttnShapes& s,
                               const int32_t* kv_idx, const int32_t* kv_count, int bsa_eff, float scale,
                               void* O, float* lse, void* ksel, void* vsel, int* status,
-                              cudaStream_t stream, bool no_chunk = false) {
+                              cudaStream_t stream, bool no_chunk = false, void* parts = nullptr,
+                              size_t parts_bytes = 0) {
   if (ksel == nullptr || vsel == nullptr || bsa_eff == 0)
     return run_attn(Q, strided(K), strided(V), Kc, Vc, s, s.T, kv_idx, kv_count, bsa_eff, scale, O, lse,
                     status, stream, false, no_chunk);
@@ -331,7 +369,7 @@ quoka_status gather_then_attn(const quoka_tensor* Q, const quoka_tensor* K, cons
   const int64_t sh = (int64_t)bsa_eff * s.d, sb = s.nkv * sh;
   // the attention may launch while the gather finishes (it waits for it)
   return run_attn(Q, Strided{ksel, sb, sh, s.d}, Strided{vsel, sb, sh, s.d}, Kc, Vc, s, bsa_eff, nullptr,
-                  kv_count, bsa_eff, scale, O, lse, status, stream, true, no_chunk);
+                  kv_count, bsa_eff, scale, O, lse, status, stream, true, no_chunk, parts, parts_bytes);
 }
 
 // Steps (f)+(g) for a short chunk (short_chunk()): the slice kernel reads the
@@ -473,13 +511,19 @@ quoka_status quoka_sparse_gqa_attn_ex(const quoka_tensor* Q, const quoka_tensor*
   // with room for the gathered copy, the selected rows are gathered first
   void* ksel = nullptr;
   void* vsel = nullptr;
+  void* parts = nullptr;
+  size_t parts_bytes = 0;
   const bool gb = uses_gather_buffers(Q->dtype, s.d, BSA_eff);
-  if (gb && ws_bytes >= attn_ws_bytes(s.b, s.nkv, s.d, BSA_eff, true)) {
+  const size_t gb_end = attn_ws_bytes(s.b, s.nkv, s.d, BSA_eff, true);
+  if (gb && ws_bytes >= gb_end) {
     ksel = static_cast<char*>(ws) + kAlign;
     vsel = static_cast<char*>(ksel) + align_up((size_t)(s.b * s.nkv * BSA_eff * s.d) * 2);
+    // (room past the gathered copy takes the split ranges' partials)
+    parts = static_cast<char*>(ws) + gb_end;
+    parts_bytes = ws_bytes - gb_end;
   }
   return gather_then_attn(Q, K, V, Kc, Vc, s, kv_idx, kv_count, BSA_eff, scale, O, lse, ksel, vsel, status,
-                          cs, no_chunk);
+                          cs, no_chunk, parts, parts_bytes);
 }
 
 quoka_status quoka_sparse_gqa_attn_gathered(const quoka_tensor* Q, const quoka_tensor* Ksel,
@@ -498,8 +542,9 @@ quoka_status quoka_sparse_gqa_attn_gathered(const quoka_tensor* Q, const quoka_t
   int* status = static_cast<int*>(ws);
   if (cudaMemsetAsync(status, 0, 2 * sizeof(int), cs) != cudaSuccess) return QUOKA_ERR_CUDA;
   // the rows of Ksel / Vsel are the selected keys in list order: BSA_eff = T
+  // (room past the status words takes the split ranges' partials)
   return run_attn(Q, strided(Ksel), strided(Vsel), Kc, Vc, s, s.T, nullptr, kv_count, (int)s.T, scale, O,
-                  lse, status, cs, true);
+                  lse, status, cs, true, false, static_cast<char*>(ws) + kAlign, ws_bytes - kAlign);
 }
 
 size_t quoka_decode_workspace_size(int b, int nq, int nkv, int d, int BCP, int BSA_eff, quoka_dtype dtype) {
@@ -561,7 +606,8 @@ quoka_status quoka_prefill_chunk(const quoka_tensor* Q, const quoka_tensor* K,
     return run_decode(Q, K, V, Kc, Vc, as, kv_idx, kv_count, (int)bsa_eff, scale, O, lse, at<float>(ws, L.dparts),
                       at<float>(ws, L.dlse), status, cs, true);
   return gather_then_attn(Q, K, V, Kc, Vc, as, kv_idx, kv_count, (int)bsa_eff, scale, O, lse,
-                          gb ? at<void>(ws, L.ksel) : nullptr, gb ? at<void>(ws, L.vsel) : nullptr, status, cs);
+                          gb ? at<void>(ws, L.ksel) : nullptr, gb ? at<void>(ws, L.vsel) : nullptr, status, cs,
+                          false, L.aparts_bytes > 0 ? at<void>(ws, L.aparts) : nullptr, L.aparts_bytes);
 }
 
 quoka_status quoka_get_device_status(const void* ws, void* stream, int32_t* device_status) {

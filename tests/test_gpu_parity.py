@@ -266,6 +266,33 @@ def test_partial_count_bf16_tensor_core_path(path):
         assert np.abs(got - O_ref).max() <= P.O_TOL_BF16
 
 
+@pytest.mark.parametrize("ws_kind", ["split", "whole"])
+def test_split_key_ranges(ws_kind):
+    """bf16, d = 128 over gathered rows with few query tiles (8: most SMs
+    idle), so that, given room in the workspace, every query tile's key
+    tiles are cut into ranges whose partials a merge kernel combines; with a
+    256-byte workspace the same call runs unsplit. Both against the oracle.
+    The second KV head keeps 5 selected keys, so some of its ranges hold no
+    key tile at all (lse = -inf partials). The workspace starts as all-ones
+    bytes: partials must be written before they are read."""
+    from tests.test_decode import oracle_attention
+    x = inputs.make_chunk(1, 4, 2, 128, 3000, 200, 8, 600, dtype="bf16", structure="llama", seed=18)
+    rng = np.random.default_rng(18)
+    sel = np.stack([[np.sort(rng.choice(3000, 600, replace=False)) for _ in range(2)]])
+    counts = np.array([[600, 5]], dtype=np.int32)
+    Q, K, V, Kc, Vc = (P.to_dev(a, "bf16") for a in (x.Q, x.K, x.V, x.Kc, x.Vc))
+    idx = torch.from_numpy(sel.astype(np.int32)).cuda()
+    cnt = torch.from_numpy(counts).cuda()
+    Ks, Vs = q().quoka_gather_kv(K, V, idx, cnt)
+    n = (16 << 20) if ws_kind == "split" else 256
+    ws = torch.full((n,), 255, dtype=torch.uint8, device="cuda")
+    O, lse = q().quoka_sparse_gqa_attn_gathered(Q, Ks, Vs, cnt, Kc, Vc, want_lse=True, ws=ws)
+    assert q().quoka_get_device_status(ws) == 0
+    O_ref, L_ref = oracle_attention(x, sel, counts)
+    assert np.abs(O.float().cpu().numpy() - O_ref).max() <= P.O_TOL_BF16
+    assert np.abs(lse.cpu().numpy() - L_ref).max() <= P.O_TOL_BF16
+
+
 def test_gathered_attention_fp32_and_partial_counts():
     """quoka_gather_kv + quoka_sparse_gqa_attn_gathered in fp32 (CUDA-core
     path), with counts below the row length: the gather writes zeros past the

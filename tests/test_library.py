@@ -99,16 +99,28 @@ def _view(shape, dtype=1, data=0x10000, stride=None):
 
 def test_workspace_size_covers_every_call_host_only(lib):
     """quoka_workspace_size is the select part, plus the gathered copy (bf16,
-    d = 128), plus, for a short chunk (G * BCP <= 64), the decode attention's
-    partials: so one workspace serves quoka_select, quoka_sparse_gqa_attn at
-    its fastest, quoka_decode_attn and quoka_prefill_chunk."""
+    d = 128), plus the partials of the attention's split key ranges when the
+    query tiles fill less than half of the GPU, plus, for a short chunk
+    (G * BCP <= 64), the decode attention's partials: so one workspace serves
+    quoka_select, quoka_sparse_gqa_attn at its fastest, quoka_decode_attn and
+    quoka_prefill_chunk."""
     al = lambda n: (n + 255) // 256 * 256
+
+    def splits(b, nq, BCP, bsa):
+        # key-range splits of the tensor-core attention: one wave of 148 CTAs
+        tiles = b * nq * ((BCP + 127) // 128)
+        if 2 * tiles > 148:
+            return 1
+        s = min(4, 148 // tiles, ((bsa + 127) // 128 + 1) // 2)
+        return s if s >= 2 else 1
+
     cases = [  # b, nq, nkv, d, T, BCP, NQ, BSA, dtype (1 = bf16)
         (1, 32, 8, 128, 32768, 512, 32, 4096, 1),
         (1, 32, 8, 128, 32768, 1, 1, 4096, 1),
         (2, 16, 2, 128, 3000, 8, 8, 700, 1),
         (1, 6, 3, 64, 900, 3, 3, 200, 0),
         (1, 8, 2, 128, 0, 1, 1, 0, 1),
+        (1, 24, 8, 128, 8192, 256, 16, 2048, 1),  # 48 query tiles: split key ranges
     ]
     for b, nq, nkv, d, T, BCP, NQ, BSA, dt in cases:
         full = lib.quoka_workspace_size(b, nq, nkv, d, T, BCP, NQ, BSA, dt)
@@ -117,10 +129,13 @@ def test_workspace_size_covers_every_call_host_only(lib):
         att = lib.quoka_attn_workspace_size(b, nkv, d, bsa, dt)
         dec = lib.quoka_decode_workspace_size(b, nq, nkv, d, BCP, bsa, dt)
         gathered = 2 * al(b * nkv * bsa * d * 2) if (dt == 1 and d == 128 and bsa > 0) else 0
+        ns = splits(b, nq, BCP, bsa) if gathered else 1
+        rows = ns * b * nq * BCP
+        parts = al(rows * d * 2) + al(rows * 4) if ns > 1 else 0
         short = (nq // nkv) * BCP <= 64
         assert (dec > 0) == short
         assert att == 256 + gathered
-        assert full == sel + gathered + (dec - 256 if short else 0)
+        assert full == sel + gathered + parts + (dec - 256 if short else 0)
         assert full >= max(sel, att, dec)
 
 
