@@ -160,14 +160,9 @@ topk_kernel(const float* __restrict__ S, int64_t T, int bsa, int slice, const ui
   // still run until this wait returns: they are read with L2-coherent loads
   // (never the read-only path, which assumes data fixed for the kernel's life).
   pdl_wait();
-  // A device fault latched earlier in the call (a scoring kernel that gave
-  // up) leaves the scores and their histogram incomplete: select nothing.
-  // Every CTA of the cluster reads the same word (nothing writes it while
-  // this kernel runs), so they all leave here together.
-  if (status != nullptr && __ldcg(status) != 0) {
-    if (c == 0 && tid == 0) kv_count[row] = 0;
-    return;
-  }
+  // (the status word is loaded with the histogram and the scores, and
+  // tested once they are staged)
+  const int fault = status != nullptr ? __ldcg(status) : 0;
   if (ghist != nullptr) {
     const uint32_t* Hg = ghist + row * TOPK_BINS;
     constexpr int q0 = TOPK_BINS / TOPK_THREADS;
@@ -186,6 +181,15 @@ topk_kernel(const float* __restrict__ S, int64_t T, int bsa, int slice, const ui
     for (int e = 4 * n4 + tid; e < n; e += TOPK_THREADS) keys[e] = score_key(__ldcg(Sr + lo + e));
   } else {
     for (int e = tid; e < n; e += TOPK_THREADS) keys[e] = score_key(__ldcg(Sr + lo + e));
+  }
+  // A device fault latched earlier in the call (a scoring kernel that gave
+  // up) leaves the scores and their histogram incomplete: select nothing.
+  // Every CTA of the cluster read the same word (nothing writes it while
+  // this kernel runs) before any cluster barrier, so they all leave here
+  // together.
+  if (fault != 0) {
+    if (c == 0 && tid == 0) kv_count[row] = 0;
+    return;
   }
 
   // From a histogram over `nbins` bins (this CTA's H, optionally summed over
@@ -520,48 +524,54 @@ topk_kernel(const float* __restrict__ S, int64_t T, int bsa, int slice, const ui
     __syncthreads();
   }
 
-  // 3. Warp w owns the contiguous segment [w*seg, (w+1)*seg) of the slice:
-  // it counts its keys > u* and == u* (lane-strided reads: no bank
-  // conflicts), one block scan places the warps, and each writes its picks
-  // in index order.
-  const int seg = (n + TOPK_WARPS - 1) / TOPK_WARPS;
-  const int s0 = min(n, warp * seg), s1 = min(n, s0 + seg);
-  uint32_t g = 0u, q_eq = 0u;
-  for (int e = s0 + lane; e < s1; e += 32) {
-    const uint32_t k = keys[e];
-    g += (k > ustar);
-    q_eq += (k == ustar);
-  }
-  // both counts in one scan: (gt << 16) | eq (per-CTA counts < 65536)
-  uint32_t packed = (g << 16) | q_eq;
-  packed = __reduce_add_sync(0xffffffffu, packed);
-  uint32_t cta_total;
-  const uint32_t wincl = block_scan_incl(lane == 0 ? packed : 0u, sh, &cta_total);
-  const uint32_t wex = wincl - (lane == 0 ? packed : 0u);  // valid in lane 0
-  const uint32_t w_gt_before = __shfl_sync(0xffffffffu, wex >> 16, 0);
-  const uint32_t w_eq_before = __shfl_sync(0xffffffffu, wex & 0xFFFFu, 0);
-  const uint32_t w_eq = packed & 0xFFFFu;  // warp sums are replicated in every lane
-  // this warp's share of the tied keys, and its first output position
+  // 3. The picks in index order, in rounds of 4 * TOPK_THREADS keys: in a
+  // round thread t owns the 4 consecutive keys from 4 * TOPK_THREADS * r +
+  // 4 t (one 16-byte shared-memory read), counts its keys > u* and == u*,
+  // and one block scan of both counts places every thread: it writes its
+  // keys > u* and the ties that still fall within this CTA's share, in
+  // order.
   const uint32_t take_cta = sh.take_eq;
-  const uint32_t w_take = take_cta > w_eq_before ? min(w_eq, take_cta - w_eq_before) : 0u;
-  uint32_t out = sh.sel_base + w_gt_before + min(w_eq_before, take_cta);
-  uint32_t eq_used = 0u;
+  uint32_t out_base = sh.sel_base;  // output position of this round's first pick
+  uint32_t eq_base = 0u;            // ties of this slice in earlier rounds
   int32_t* dst = kv_idx + row * bsa;
-  for (int base = s0; base < s1; base += 32) {
-    const int e = base + lane;
-    const uint32_t k = e < s1 ? keys[e] : 0u;
-    const bool is_gt = e < s1 && k > ustar;
-    const bool is_eq = e < s1 && k == ustar;
-    const uint32_t below = (1u << lane) - 1u;
-    const uint32_t eqb = __ballot_sync(0xffffffffu, is_eq);
-    const bool take_it = is_gt || (is_eq && eq_used + (uint32_t)__popc(eqb & below) < w_take);
-    const uint32_t selb = __ballot_sync(0xffffffffu, take_it);
-    if (take_it) {
-      const uint32_t pos = out + (uint32_t)__popc(selb & below);
-      if (pos < (uint32_t)bsa) dst[pos] = (int32_t)(lo + e);
+  for (int r0 = 0; r0 < n; r0 += 4 * TOPK_THREADS) {
+    const int e0 = r0 + 4 * tid;
+    uint32_t k[4];
+    if (e0 + 3 < n) {
+      const uint4 v = *reinterpret_cast<const uint4*>(keys + e0);
+      k[0] = v.x;
+      k[1] = v.y;
+      k[2] = v.z;
+      k[3] = v.w;
+    } else {
+#pragma unroll
+      for (int u = 0; u < 4; ++u) k[u] = e0 + u < n ? keys[e0 + u] : 0u;
     }
-    out += (uint32_t)__popc(selb);
-    eq_used += (uint32_t)__popc(eqb);
+    uint32_t g = 0u, q_eq = 0u;
+#pragma unroll
+    for (int u = 0; u < 4; ++u) {
+      const bool valid = e0 + u < n;
+      g += valid && k[u] > ustar;
+      q_eq += valid && k[u] == ustar;
+    }
+    // both counts in one scan: (gt << 16) | eq (per-round counts <= 4096)
+    const uint32_t packed = (g << 16) | q_eq;
+    uint32_t tot;
+    const uint32_t ex = block_scan_incl(packed, sh, &tot) - packed;
+    uint32_t eq_seen = eq_base + (ex & 0xFFFFu);  // ties of this slice before this thread's keys
+    uint32_t pos = out_base + (ex >> 16) + min(eq_seen, take_cta) - min(eq_base, take_cta);
+#pragma unroll
+    for (int u = 0; u < 4; ++u) {
+      if (e0 + u >= n) continue;
+      bool take = k[u] > ustar;
+      if (k[u] == ustar) take = eq_seen++ < take_cta;
+      if (take) {
+        if (pos < (uint32_t)bsa) dst[pos] = (int32_t)(lo + e0 + u);
+        ++pos;
+      }
+    }
+    out_base += (tot >> 16) + min(eq_base + (tot & 0xFFFFu), take_cta) - min(eq_base, take_cta);
+    eq_base += tot & 0xFFFFu;
   }
   if (c == 0 && tid == 0) kv_count[row] = bsa;
   // every CTA stays until the others are done reading its shared memory
