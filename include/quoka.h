@@ -38,9 +38,11 @@
  *     of `ws` and read back with quoka_get_device_status(). Every call that
  *     takes `ws` clears that word (and the fault-site word after it) on
  *     `stream` before any of its kernels can latch a fault: quoka_select,
- *     quoka_select_ex and quoka_prefill_chunk in their first kernel (whose
- *     successors latch only after waiting for it), the other calls with an
- *     8-byte memset. The word reports the faults of the latest call.
+ *     quoka_select_ex and quoka_prefill_chunk in their first kernel,
+ *     quoka_gather_kv and quoka_decode_attn in a one-thread kernel of their
+ *     own, the other calls with an 8-byte memset; a kernel latches only
+ *     after the kernel before it in the call has completed. The word
+ *     reports the faults of the latest call.
  *   - Calls on different streams with different workspaces may run
  *     concurrently. Two calls sharing one workspace must be ordered.
  */
