@@ -96,6 +96,10 @@ def test_decode_out_of_range_index_is_latched_not_read():
     O, _ = q().quoka_decode_attn(Q, K, V, idx, cnt, Kc, Vc, ws=ws)
     assert q().quoka_get_device_status(ws) == 6
     assert torch.isfinite(O.float()).all()
+    # the next valid call on the same workspace clears the status first
+    good = torch.tensor([[[1, 5, 99, 250, 299]]], dtype=torch.int32, device="cuda")
+    q().quoka_decode_attn(Q, K, V, good, cnt, Kc, Vc, ws=ws)
+    assert q().quoka_get_device_status(ws) == 0
 
 
 @pytest.mark.gpu

@@ -366,6 +366,15 @@ def test_out_of_range_index_is_latched_not_read():
     torch.cuda.synchronize()
     # the in-range rows were still gathered
     np.testing.assert_array_equal(Ks[0, 0, :3].cpu().numpy(), x.K[0, 0, [1, 5, 99]])
+    # each call clears the status words first: valid calls on the same
+    # workspace read 0 again (the gather's clear runs in a kernel of its own)
+    good = torch.tensor([[[1, 5, 99, 7, 8]]], dtype=torch.int32, device="cuda")
+    q().quoka_gather_kv(K, V, good, cnt, ws=ws)
+    assert q().quoka_get_device_status(ws) == 0 and q().quoka_get_device_fault_site(ws) == 0
+    q().quoka_gather_kv(K, V, idx, cnt, ws=ws)
+    assert q().quoka_get_device_status(ws) == 6
+    q().quoka_sparse_gqa_attn(Q, K, V, good, cnt, Kc, Vc, ws=ws)
+    assert q().quoka_get_device_status(ws) == 0
 
 
 @pytest.mark.parametrize("path", ["gathered", "fused"])
