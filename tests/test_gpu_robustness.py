@@ -159,3 +159,33 @@ def test_headline_step_repeats_bit_identical():
     O_ref, _ = orc.sparse_attention_rows(x.Q, x.K, x.V, gi, x.Kc, x.Vc, rows)
     got = np.stack([O0[rw] for rw in rows])
     assert np.abs(got - O_ref).max() <= P.O_TOL_BF16
+
+
+@pytest.mark.parametrize("BCP", [512, 1])
+def test_step_replays_from_a_cuda_graph(BCP):
+    """quoka_prefill_chunk enqueues only kernels and a memset on its stream
+    (no allocation, no synchronisation), so a CUDA graph can capture the
+    whole step; replaying the graph gives the eager call's outputs bit for
+    bit (Qwen-shaped layer at T = 8192, a full chunk and a decode token)."""
+    x = inputs.make_chunk(1, 32, 8, 128, 8192, BCP, min(32, BCP), 2048, dtype="bf16", structure="qwen", seed=83)
+    Q, K, V, Kc, Vc = (P.to_dev(a, x.dtype) for a in (x.Q, x.K, x.V, x.Kc, x.Vc))
+    ws = q().workspace_for(Q, K, x.NQ, x.BSA)
+    O = torch.empty_like(Q)
+    kv_idx = torch.empty((1, 8, 2048), dtype=torch.int32, device="cuda")
+    s = torch.cuda.Stream()
+    with torch.cuda.stream(s):
+        q().quoka_prefill_chunk(Q, K, V, Kc, Vc, x.NQ, x.BSA, O=O, kv_idx=kv_idx, ws=ws, stream=s)
+    s.synchronize()
+    O_eager, idx_eager = O.clone(), kv_idx.clone()
+    O.zero_()
+    kv_idx.zero_()
+    torch.cuda.synchronize()
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g, stream=s):
+        q().quoka_prefill_chunk(Q, K, V, Kc, Vc, x.NQ, x.BSA, O=O, kv_idx=kv_idx, ws=ws, stream=s)
+    for _ in range(3):
+        g.replay()
+    torch.cuda.synchronize()
+    assert q().quoka_get_device_status(ws) == 0
+    assert torch.equal(kv_idx, idx_eager)
+    assert torch.equal(O, O_eager)
