@@ -79,7 +79,11 @@ def test_scoring_timeout_unwinds_and_next_call_is_exact():
     run_prefill_and_check(x, ref, gi, rows=[(0, h, t) for h in (0, 13, 31) for t in range(0, 256, 5)])
 
 
-def test_attention_timeout_unwinds_and_next_call_is_exact():
+@pytest.mark.parametrize("ws_bytes", [256, 16 << 20], ids=["whole", "split_key_ranges"])
+def test_attention_timeout_unwinds_and_next_call_is_exact(ws_bytes):
+    """With a 256-byte workspace every query tile runs whole; with room for
+    the partials its key tiles are split into ranges (16 query tiles), and
+    the merge kernel runs after the kernel that gave up."""
     x = inputs.make_chunk(1, 8, 2, 128, 3000, 200, 8, 700, dtype="bf16", structure="qwen", seed=82)
     ref = orc.select(x.Q, x.K, x.NQ, x.BSA)
     sel = ref["sel"]
@@ -87,7 +91,7 @@ def test_attention_timeout_unwinds_and_next_call_is_exact():
     kv_idx = torch.from_numpy(sel.astype(np.int32)).cuda()
     kv_count = torch.full((1, 2), sel.shape[2], dtype=torch.int32, device="cuda")
     Ks, Vs = q().quoka_gather_kv(K, V, kv_idx, kv_count)
-    ws = torch.zeros(256, dtype=torch.uint8, device="cuda")
+    ws = torch.zeros(ws_bytes, dtype=torch.uint8, device="cuda")
 
     def call():
         q().quoka_sparse_gqa_attn_gathered(Q, Ks, Vs, kv_count, Kc, Vc, ws=ws)
