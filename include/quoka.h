@@ -81,8 +81,9 @@ typedef struct {
 } quoka_tensor;
 
 /* Bytes of workspace any call below needs for these sizes (the maximum over
- * the calls, so one workspace serves all of them; quoka_prefill_chunk needs
- * exactly this much). Returns 0 only for invalid sizes. */
+ * the calls, so one workspace serves all of them at their fastest, split
+ * key ranges of the attention included; quoka_prefill_chunk needs exactly
+ * this much). Returns 0 only for invalid sizes. */
 size_t quoka_workspace_size(int b, int nq, int nkv, int d, int64_t T, int BCP,
                             int NQ, int BSA, quoka_dtype dtype);
 
@@ -188,7 +189,12 @@ quoka_status quoka_gather_kv(const quoka_tensor* K, const quoka_tensor* V,
  *       (bf16, d = 128) the selected rows are first gathered into ws (step
  *       (f) as its own kernel, the copy staying in L2) and the attention
  *       streams them as dense tiles; with less, the bf16 attention gathers
- *       the rows itself while loading them (slower, same results).
+ *       the rows itself while loading them (slower, same results). When
+ *       the chunk has few 128-row query tiles (b * nq * ceil(BCP / 128) at
+ *       most 74) and ws has room past the gathered copy for their partials
+ *       (quoka_workspace_size() includes it), each tile's key tiles are
+ *       split into 2-4 ranges run side by side and merged by a second
+ *       kernel (same results up to rounding).
  *   O   out (b, nq, BCP, d), contiguous, dtype of Q.
  *   lse out (b, nq, BCP) float or NULL: natural-log partition function
  *       log sum_k exp(scale * q.k).
@@ -230,7 +236,9 @@ quoka_status quoka_sparse_gqa_attn_ex(const quoka_tensor* Q, const quoka_tensor*
  *   strides. Rows from kv_count to BSA_eff are masked out but are read: they
  *   must hold finite values (quoka_gather_kv writes zeros there).
  *   kv_count (b, nkv) int32, values above BSA_eff are clamped to it.
- *   ws at least 256 bytes (the status words). Other arguments as in
+ *   ws at least 256 bytes (the status words); room past them for the
+ *   partials of split key ranges lets a chunk with few query tiles split
+ *   them as quoka_sparse_gqa_attn does. Other arguments as in
  *   quoka_sparse_gqa_attn. */
 quoka_status quoka_sparse_gqa_attn_gathered(const quoka_tensor* Q,
                                             const quoka_tensor* Ksel,
