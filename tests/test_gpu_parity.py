@@ -293,6 +293,27 @@ def test_split_key_ranges(ws_kind):
     assert np.abs(lse.cpu().numpy() - L_ref).max() <= P.O_TOL_BF16
 
 
+@pytest.mark.parametrize("no_chunk", [False, True], ids=["with_chunk_keys", "no_chunk_keys"])
+def test_split_key_ranges_ragged_through_the_indexed_entry(no_chunk):
+    """quoka_sparse_gqa_attn(_ex) with room past the gathered copy: 24 query
+    tiles of a ragged chunk (BCP = 200: a full and a 72-row tile per head,
+    G = 3, two batches) split their key ranges; with the chunk's own keys
+    left out (one rank's partial attention) rows see only selected keys.
+    O and lse against the oracle."""
+    x = inputs.make_chunk(2, 6, 2, 128, 3000, 200, 8, 700, dtype="bf16", structure="llama", seed=21)
+    rng = np.random.default_rng(21)
+    sel = np.stack([[np.sort(rng.choice(3000, 700, replace=False)) for _ in range(2)] for _ in range(2)])
+    Q, K, V, Kc, Vc = (P.to_dev(a, "bf16") for a in (x.Q, x.K, x.V, x.Kc, x.Vc))
+    idx = torch.from_numpy(sel.astype(np.int32)).cuda()
+    cnt = torch.full((2, 2), 700, dtype=torch.int32, device="cuda")
+    ws = torch.full((32 << 20,), 255, dtype=torch.uint8, device="cuda")
+    O, lse = q().quoka_sparse_gqa_attn(Q, K, V, idx, cnt, Kc, Vc, want_lse=True, ws=ws, no_chunk=no_chunk)
+    assert q().quoka_get_device_status(ws) == 0
+    O_ref, L_ref = orc.sparse_attention(x.Q, x.K, x.V, sel, x.Kc, x.Vc, include_chunk=not no_chunk)
+    assert np.abs(O.float().cpu().numpy() - O_ref).max() <= P.O_TOL_BF16
+    assert np.abs(lse.cpu().numpy() - L_ref).max() <= P.O_TOL_BF16
+
+
 def test_gathered_attention_fp32_and_partial_counts():
     """quoka_gather_kv + quoka_sparse_gqa_attn_gathered in fp32 (CUDA-core
     path), with counts below the row length: the gather writes zeros past the
