@@ -293,6 +293,43 @@ def test_split_key_ranges(ws_kind):
     assert np.abs(lse.cpu().numpy() - L_ref).max() <= P.O_TOL_BF16
 
 
+@pytest.mark.parametrize("pos,mag,ws_kind", [(300, 40.0, "whole"), (200, 40.0, "whole"), (300, 40.0, "split"),
+                                             (300, 24.0, "whole")],
+                         ids=["far_later_tile", "far_first_tile_of_warpgroup_1", "far_split", "near"])
+def test_scores_far_above_the_first_tile(pos, mag, ws_kind):
+    """A key whose score is far above the rows' max over their first key
+    tile: selected key `pos` of KV head 0 and every third chunk row of its
+    two query heads are mag * e_0, so those rows' score for that key lies
+    ~190 (mag = 40) or ~65 (mag = 24) log2 units above the first tile's max.
+    The running max of those rows jumps by far more than the lazy-rescale
+    threshold, so the O accumulator of the warpgroup that owns the key's
+    tile is rescaled in TMEM, and the two warpgroups' partials meet with
+    maxima ~190 log2 units apart. Key 200 lies in warpgroup 1's first tile, key 300
+    in warpgroup 0's second; "split" cuts the key tiles into ranges. O and
+    lse against the oracle."""
+    from tests.test_decode import oracle_attention
+    x = inputs.make_chunk(1, 4, 2, 128, 3000, 200, 8, 600, dtype="bf16", structure="llama", seed=25)
+    rng = np.random.default_rng(25)
+    sel = np.stack([[np.sort(rng.choice(3000, 600, replace=False)) for _ in range(2)]])
+    counts = np.array([[600, 600]], dtype=np.int32)
+    e0 = np.zeros(128)
+    e0[0] = mag
+    x.K[0, 0, sel[0, 0, pos]] = e0
+    x.Q[0, 0:2, 0::3] = e0
+    Q, K, V, Kc, Vc = (P.to_dev(a, "bf16") for a in (x.Q, x.K, x.V, x.Kc, x.Vc))
+    idx = torch.from_numpy(sel.astype(np.int32)).cuda()
+    cnt = torch.from_numpy(counts).cuda()
+    Ks, Vs = q().quoka_gather_kv(K, V, idx, cnt)
+    n = (16 << 20) if ws_kind == "split" else 256
+    ws = torch.full((n,), 255, dtype=torch.uint8, device="cuda")
+    O, lse = q().quoka_sparse_gqa_attn_gathered(Q, Ks, Vs, cnt, Kc, Vc, want_lse=True, ws=ws)
+    assert q().quoka_get_device_status(ws) == 0
+    O_ref, L_ref = oracle_attention(x, sel, counts)
+    assert np.isfinite(O.float().cpu().numpy()).all()
+    assert np.abs(O.float().cpu().numpy() - O_ref).max() <= P.O_TOL_BF16
+    assert np.abs(lse.cpu().numpy() - L_ref).max() <= P.O_TOL_BF16
+
+
 @pytest.mark.parametrize("no_chunk", [False, True], ids=["with_chunk_keys", "no_chunk_keys"])
 def test_split_key_ranges_ragged_through_the_indexed_entry(no_chunk):
     """quoka_sparse_gqa_attn(_ex) with room past the gathered copy: 24 query
