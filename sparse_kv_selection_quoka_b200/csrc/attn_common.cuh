@@ -1,9 +1,12 @@
 // Pieces shared by the two tcgen05 attention kernels (the one that streams
 // gathered K/V tiles with TMA and the one that gathers rows while loading).
 //
-// Layout shared by both: a CTA owns two 128-row query tiles of one KV head;
-// TMEM holds S0 | S1 | O0 | O1 (128 fp32 columns each, 512 in all). Thread r
-// of softmax warpgroup w owns query row r of tile w, which is TMEM lane r.
+// Layout shared by both: TMEM holds S0 | S1 | O0 | O1 (128 fp32 columns
+// each, 512 in all), S_w and O_w belonging to softmax warpgroup w, whose
+// thread r owns query row r (TMEM lane r) of its query tile. In the
+// gathering kernel the two warpgroups own two query tiles of one KV head;
+// in the streaming kernel they share one query tile and take alternate key
+// tiles.
 #pragma once
 
 #include "common.cuh"

@@ -13,8 +13,9 @@
 // copy of the selected rows; with one, the gather kernel runs first and the
 // TMA-streaming kernel (attn_tma.cu) does the attention, faster.
 //
-// Work split as in attn_tma.cu: a CTA takes two 128-row query tiles (Q0, Q1)
-// of one KV head; its key tiles are ceil(nsel/128) tiles of selected prior
+// Work split: a CTA takes two 128-row query tiles (Q0, Q1) of one KV head
+// (attn_tma.cu instead gives a CTA one query tile and splits its key tiles
+// between the two softmax warpgroups); its key tiles are ceil(nsel/128) tiles of selected prior
 // rows (read in place through the sorted index list; rows past nsel are
 // zero-filled and masked) followed by ceil(nchunk/128) tiles of the chunk's
 // own keys. When the grid would fill less than half of the GPU, the key
