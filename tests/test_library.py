@@ -200,6 +200,94 @@ def test_decode_attention_rejects_bad_arguments_on_host(lib):
     assert lib.quoka_decode_workspace_size(1, 8, 2, 96, 1, 10, 0) == 0  # d = 96
 
 
+def test_select_variants_reject_bad_arguments_on_host(lib):
+    """quoka_select_ex's unknown flag bits, and quoka_select_static's shapes
+    with no valid workspace or one past its fixed scratch array, are turned
+    away before any device call."""
+    Q = _view((1, 8, 64, 128))
+    K = _view((1, 2, 500, 128))
+    buf = ctypes.c_void_p(0x200000)
+    ws = ctypes.c_void_p(0x100000)
+    B = ctypes.byref
+    for flags in (2, 4, 0x80000000):
+        assert lib.quoka_select_ex(B(Q), B(K), 4, 10, buf, buf, None, None, flags, ws, 1 << 30, None) == 1
+    st = lib.quoka_select_static
+    assert st(None, B(K), 4, 10, buf, buf, None, None, None) == 1
+    assert st(B(Q), B(K), 0, 10, buf, buf, None, None, None) == 1                    # NQ < 1
+    assert st(B(Q), B(_view((1, 3, 500, 128))), 4, 10, buf, buf, None, None, None) == 1  # nq % nkv
+    # S_agg alone of (1, 8, 2^20) keys is 32 MiB: past the 8 MiB array
+    Kbig = _view((1, 8, 1 << 20, 128))
+    need = lib.quoka_select_workspace_size(1, 32, 8, 128, 1 << 20, 512, 32, 4096, 1)
+    assert need > (8 << 20)
+    assert st(B(_view((1, 32, 512, 128))), B(Kbig), 32, 4096, buf, buf, None, None, None) == 3
+
+
+def test_gather_and_gathered_attention_reject_bad_arguments_on_host(lib):
+    K = _view((1, 2, 500, 128))
+    buf = ctypes.c_void_p(0x200000)
+    ws = ctypes.c_void_p(0x100000)
+    B = ctypes.byref
+    g = lib.quoka_gather_kv
+    assert g(None, B(K), buf, buf, 10, buf, buf, None, 0, None) == 1
+    assert g(B(K), B(K), None, None, 10, buf, buf, None, 0, None) == 1              # no kv_count
+    assert g(B(K), B(K), buf, buf, -1, buf, buf, None, 0, None) == 1                # BSA_eff < 0
+    assert g(B(K), B(_view((1, 2, 500, 128), dtype=0)), buf, buf, 10, buf, buf, None, 0, None) == 1  # V dtype
+    assert g(B(K), B(K), buf, buf, 10, None, buf, None, 0, None) == 1               # no Ksel
+    assert g(B(K), B(K), buf, buf, 10, ctypes.c_void_p(0x200008), buf, None, 0, None) == 1  # Ksel misaligned
+    assert g(B(_view((1, 2, 500, 96))), B(_view((1, 2, 500, 96))), buf, buf, 10, buf, buf, None, 0, None) == 2
+    assert g(B(K), B(K), buf, buf, 10, buf, buf, ctypes.c_void_p(0x100010), 256, None) == 3  # ws misaligned
+    assert g(B(K), B(K), buf, buf, 10, buf, buf, ws, 4, None) == 3                  # ws under the status words
+    Q = _view((1, 8, 64, 128))
+    Ks = _view((1, 2, 10, 128))
+    Kc = _view((1, 2, 64, 128))
+    a = lib.quoka_sparse_gqa_attn_gathered
+    assert a(B(Q), B(Ks), B(Ks), None, B(Kc), B(Kc), 0.1, buf, None, ws, 256, None) == 1     # no kv_count
+    assert a(B(Q), B(Ks), B(Ks), buf, B(Kc), B(Kc), 0.1, None, None, ws, 256, None) == 1     # no O
+    assert a(B(Q), B(Ks), B(Ks), buf, B(Kc), B(Kc), 0.1, ctypes.c_void_p(0x200004), None, ws, 256,
+             None) == 1                                                                      # O misaligned
+    assert a(B(Q), B(Ks), B(Ks), buf, B(Kc), B(Kc), 0.0, buf, None, ws, 256, None) == 1      # scale <= 0
+    assert a(B(Q), B(Ks), B(Ks), buf, B(Kc), B(Kc), float("nan"), buf, None, ws, 256, None) == 1
+    assert a(B(Q), B(Ks), B(Ks), buf, B(_view((1, 2, 63, 128))), B(Kc), 0.1, buf, None, ws, 256, None) == 1
+    assert a(B(Q), B(Ks), B(Ks), buf, B(Kc), B(Kc), 0.1, buf, None, None, 256, None) == 3
+    assert a(B(Q), B(Ks), B(Ks), buf, B(Kc), B(Kc), 0.1, buf, None, ctypes.c_void_p(0x100010), 256, None) == 3
+    assert a(B(Q), B(Ks), B(Ks), buf, B(Kc), B(Kc), 0.1, buf, None, ws, 255, None) == 3
+    e = lib.quoka_sparse_gqa_attn_ex
+    for flags in (2, 0x100):
+        assert e(B(Q), B(K), B(K), buf, buf, 10, B(Kc), B(Kc), 0.1, buf, None, flags, ws, 1 << 30, None) == 1
+
+
+def test_context_parallel_calls_reject_bad_arguments_on_host(lib):
+    buf = ctypes.c_void_p(0x200000)
+    odd = ctypes.c_void_p(0x200002)
+    cs = lib.quoka_shard_candidate_scores
+    assert cs(buf, 0, 2, 500, buf, buf, 10, 20, buf, buf, None, 0, None) == 1       # b < 1
+    assert cs(buf, 1, 2, 500, buf, buf, 10, 5, buf, buf, None, 0, None) == 1        # C < Cl
+    assert cs(buf, 1, 2, 500, buf, None, 10, 20, buf, buf, None, 0, None) == 1      # no kv_count
+    assert cs(buf, 1, 2, 500, buf, buf, 10, 20, None, buf, None, 0, None) == 1      # no scores out
+    assert cs(buf, 1, 2, 500, buf, buf, 10, 0, buf, buf, None, 0, None) == 1        # C = 0 < Cl
+    assert cs(None, 1, 2, 500, None, buf, 0, 0, None, None, None, 0, None) == 0     # empty: nothing to do
+    il = lib.quoka_shard_interleave
+    assert il(buf, 0, 4, 4, buf, None) == 1                                          # N < 1
+    assert il(buf, 2, -1, 4, buf, None) == 1
+    assert il(odd, 2, 4, 4, buf, None) == 1                                          # not 4-byte aligned
+    assert il(None, 2, 0, 4, None, None) == 0                                        # empty
+    tk = lib.quoka_topk
+    assert tk(buf, 1, 2, 500, -1, buf, buf, None, 0, None) == 1                      # BSA < 0
+    assert tk(buf, 1, 2, 500, 10, buf, None, None, 0, None) == 1                     # no kv_count
+    assert tk(None, 1, 2, 500, 10, buf, buf, None, 0, None) == 1                     # no scores
+    assert tk(buf, 1, 70000, 500, 10, buf, buf, None, 0, None) == 1                  # nkv past the grid
+    tkn = lib.quoka_shard_take
+    assert tkn(buf, buf, 1, 2, 8, buf, 10, -1, buf, buf, None, 0, None) == 1         # rank < 0
+    assert tkn(buf, None, 1, 2, 8, buf, 10, 0, buf, buf, None, 0, None) == 1         # no sel_count
+    assert tkn(None, buf, 1, 2, 8, buf, 10, 0, buf, buf, None, 0, None) == 1         # S > 0 without sel_pos
+    cp = lib.quoka_combine_partials
+    assert cp(buf, buf, 2, 1, 8, 64, 96, 1, buf, None, None) == 1                    # d not 64 / 128
+    assert cp(buf, buf, 2, 1, 8, 64, 128, 7, buf, None, None) == 1                   # dtype
+    assert cp(buf, buf, 0, 1, 8, 64, 128, 1, buf, None, None) == 1                   # N < 1
+    assert cp(ctypes.c_void_p(0x200008), buf, 2, 1, 8, 64, 128, 1, buf, None, None) == 1  # misaligned
+    assert cp(buf, None, 2, 1, 8, 64, 128, 1, buf, None, None) == 1                  # no lse_parts
+
+
 def test_binding_fails_loudly_without_library(tmp_path, monkeypatch):
     from sparse_kv_selection_quoka_b200 import _lib
     monkeypatch.setattr(_lib, "LIB_PATH", str(tmp_path / "missing.so"))
