@@ -193,3 +193,84 @@ def test_step_replays_from_a_cuda_graph(BCP):
     assert q().quoka_get_device_status(ws) == 0
     assert torch.equal(kv_idx, idx_eager)
     assert torch.equal(O, O_eager)
+
+
+GUARD = 4096  # bytes of sentinel on each side of every output
+
+
+class Guarded:
+    """A tensor of the given shape and dtype between two sentinel bands of
+    GUARD bytes inside one larger byte buffer (the band lengths keep the
+    tensor's 256-byte alignment)."""
+
+    def __init__(self, shape, dtype, fill=0x5A):
+        esize = torch.empty((), dtype=dtype).element_size()
+        self.n = int(np.prod(shape)) * esize
+        self.fill = fill
+        self.buf = torch.full((2 * GUARD + self.n,), fill, dtype=torch.uint8, device="cuda")
+        self.t = self.buf[GUARD:GUARD + self.n].view(dtype).view(*shape)
+
+    def intact(self):
+        return bool((self.buf[:GUARD] == self.fill).all()) and bool((self.buf[GUARD + self.n:] == self.fill).all())
+
+
+@pytest.mark.parametrize("BCP", [1, 160], ids=["decode_token", "chunk"])
+def test_calls_write_only_inside_their_outputs_and_workspace(BCP):
+    """Every output of quoka_select, quoka_gather_kv, quoka_sparse_gqa_attn
+    (gathered copy and split key ranges inside its workspace),
+    quoka_decode_attn and quoka_prefill_chunk, and the workspace itself
+    (exactly quoka_workspace_size bytes), sits between sentinel bands; after
+    each call the bands are unchanged and the outputs equal those of the
+    same call on plainly allocated buffers."""
+    NQ, BSA, T = min(8, BCP), 400, 1500
+    x = inputs.make_chunk(1, 8, 2, 128, T, BCP, NQ, BSA, dtype="bf16", structure="llama", seed=31)
+    Q, K, V, Kc, Vc = (P.to_dev(a, "bf16") for a in (x.Q, x.K, x.V, x.Kc, x.Vc))
+    b, nq, _, d = Q.shape
+    nkv = K.shape[1]
+    bf, f32, i32 = torch.bfloat16, torch.float32, torch.int32
+    n = q().quoka_workspace_size(b, nq, nkv, d, T, BCP, NQ, BSA, bf)
+    ws = Guarded((n,), torch.uint8)
+
+    idx, cnt = Guarded((b, nkv, BSA), i32), Guarded((b, nkv), i32)
+    qi, sg = Guarded((b, nq, NQ), i32), Guarded((b, nkv, T), f32)
+    q().quoka_select(Q, K, NQ, BSA, kv_idx=idx.t, kv_count=cnt.t, q_idx=qi.t, s_agg=sg.t, ws=ws.t)
+    r_idx, r_cnt, r_qi, r_sg = q().quoka_select(Q, K, NQ, BSA, want_q_idx=True, want_s_agg=True)
+    torch.cuda.synchronize()
+    assert q().quoka_get_device_status(ws.t) == 0
+    assert torch.equal(idx.t, r_idx) and torch.equal(cnt.t, r_cnt) and torch.equal(qi.t, r_qi)
+    assert torch.equal(sg.t, r_sg)
+
+    Ks, Vs = Guarded((b, nkv, BSA, d), bf), Guarded((b, nkv, BSA, d), bf)
+    q().quoka_gather_kv(K, V, idx.t, cnt.t, Ksel=Ks.t, Vsel=Vs.t, ws=ws.t)
+    r_Ks, r_Vs = q().quoka_gather_kv(K, V, r_idx, r_cnt)
+    torch.cuda.synchronize()
+    assert torch.equal(Ks.t, r_Ks) and torch.equal(Vs.t, r_Vs)
+
+    O, L = Guarded((b, nq, BCP, d), bf), Guarded((b, nq, BCP), f32)
+    q().quoka_sparse_gqa_attn(Q, K, V, idx.t, cnt.t, Kc, Vc, O=O.t, lse=L.t, ws=ws.t)
+    r_O, r_L = q().quoka_sparse_gqa_attn(Q, K, V, r_idx, r_cnt, Kc, Vc, want_lse=True,
+                                         ws=torch.empty(n, dtype=torch.uint8, device="cuda"))
+    torch.cuda.synchronize()
+    assert q().quoka_get_device_status(ws.t) == 0
+    assert torch.equal(O.t, r_O) and torch.equal(L.t, r_L)
+
+    O2, L2, kvi = Guarded((b, nq, BCP, d), bf), Guarded((b, nq, BCP), f32), Guarded((b, nkv, BSA), i32)
+    q().quoka_prefill_chunk(Q, K, V, Kc, Vc, NQ, BSA, O=O2.t, lse=L2.t, kv_idx=kvi.t, ws=ws.t)
+    r_O2, r_L2, r_kvi = q().quoka_prefill_chunk(Q, K, V, Kc, Vc, NQ, BSA, want_lse=True, want_kv_idx=True)
+    torch.cuda.synchronize()
+    assert q().quoka_get_device_status(ws.t) == 0
+    assert torch.equal(O2.t, r_O2) and torch.equal(L2.t, r_L2) and torch.equal(kvi.t, r_kvi)
+
+    bands = [ws, idx, cnt, qi, sg, Ks, Vs, O, L, O2, L2, kvi]
+    if BCP == 1:
+        nd = q().quoka_decode_workspace_size(b, nq, nkv, d, BCP, BSA, bf)
+        wsd = Guarded((nd,), torch.uint8)
+        O3, L3 = Guarded((b, nq, BCP, d), bf), Guarded((b, nq, BCP), f32)
+        q().quoka_decode_attn(Q, K, V, idx.t, cnt.t, Kc, Vc, O=O3.t, lse=L3.t, ws=wsd.t)
+        r_O3, r_L3 = q().quoka_decode_attn(Q, K, V, r_idx, r_cnt, Kc, Vc, want_lse=True)
+        torch.cuda.synchronize()
+        assert q().quoka_get_device_status(wsd.t) == 0
+        assert torch.equal(O3.t, r_O3) and torch.equal(L3.t, r_L3)
+        bands += [wsd, O3, L3]
+    bad = [i for i, g in enumerate(bands) if not g.intact()]
+    assert not bad, f"sentinel bands overwritten around outputs {bad}"
