@@ -9,6 +9,7 @@
 #include <atomic>
 
 #include "common.cuh"
+#include "nvtx_range.h"
 #include "kernels.h"
 #include "quoka.h"
 
@@ -455,12 +456,14 @@ size_t quoka_attn_workspace_size(int b, int nkv, int d, int BSA_eff, quoka_dtype
 quoka_status quoka_select(const quoka_tensor* Q, const quoka_tensor* K, int NQ, int BSA,
                           int32_t* kv_idx, int32_t* kv_count, int32_t* q_idx, float* s_agg,
                           void* ws, size_t ws_bytes, void* stream) {
+  quoka::NvtxRange nvtx_range("quoka_select");
   return quoka_select_ex(Q, K, NQ, BSA, kv_idx, kv_count, q_idx, s_agg, 0u, ws, ws_bytes, stream);
 }
 
 quoka_status quoka_select_ex(const quoka_tensor* Q, const quoka_tensor* K, int NQ, int BSA,
                              int32_t* kv_idx, int32_t* kv_count, int32_t* q_idx, float* s_agg,
                              uint32_t flags, void* ws, size_t ws_bytes, void* stream) {
+  quoka::NvtxRange nvtx_range("quoka_select_ex");
   if ((flags & ~QUOKA_SCORE_DOT_PRODUCT) != 0u) return QUOKA_ERR_INVALID_ARG;
   SelectShapes s;
   quoka_status st = validate_select(Q, K, NQ, BSA, &s);
@@ -478,6 +481,7 @@ quoka_status quoka_select_ex(const quoka_tensor* Q, const quoka_tensor* K, int N
 quoka_status quoka_gather_kv(const quoka_tensor* K, const quoka_tensor* V, const int32_t* kv_idx,
                              const int32_t* kv_count, int BSA_eff, void* Ksel, void* Vsel,
                              void* ws, size_t ws_bytes, void* stream) {
+  quoka::NvtxRange nvtx_range("quoka_gather_kv");
   if (K == nullptr || V == nullptr || kv_count == nullptr || BSA_eff < 0) return QUOKA_ERR_INVALID_ARG;
   int64_t ks[4] = {-1, -1, -1, -1};
   if (!check_tensor(K, K->dtype, ks)) return QUOKA_ERR_INVALID_ARG;
@@ -507,6 +511,7 @@ quoka_status quoka_sparse_gqa_attn(const quoka_tensor* Q, const quoka_tensor* K,
                                    const int32_t* kv_count, int BSA_eff, const quoka_tensor* Kc,
                                    const quoka_tensor* Vc, float scale, void* O, float* lse,
                                    void* ws, size_t ws_bytes, void* stream) {
+  quoka::NvtxRange nvtx_range("quoka_sparse_gqa_attn");
   return quoka_sparse_gqa_attn_ex(Q, K, V, kv_idx, kv_count, BSA_eff, Kc, Vc, scale, O, lse, 0u, ws, ws_bytes,
                                   stream);
 }
@@ -516,6 +521,7 @@ quoka_status quoka_sparse_gqa_attn_ex(const quoka_tensor* Q, const quoka_tensor*
                                       const int32_t* kv_count, int BSA_eff, const quoka_tensor* Kc,
                                       const quoka_tensor* Vc, float scale, void* O, float* lse,
                                       uint32_t flags, void* ws, size_t ws_bytes, void* stream) {
+  quoka::NvtxRange nvtx_range("quoka_sparse_gqa_attn_ex");
   if ((flags & ~QUOKA_ATTN_NO_CHUNK_KEYS) != 0u) return QUOKA_ERR_INVALID_ARG;
   const bool no_chunk = (flags & QUOKA_ATTN_NO_CHUNK_KEYS) != 0u;
   AttnShapes s;
@@ -552,6 +558,7 @@ quoka_status quoka_sparse_gqa_attn_gathered(const quoka_tensor* Q, const quoka_t
                                             const quoka_tensor* Kc, const quoka_tensor* Vc, float scale,
                                             void* O, float* lse, void* ws, size_t ws_bytes,
                                             void* stream) {
+  quoka::NvtxRange nvtx_range("quoka_sparse_gqa_attn_gathered");
   AttnShapes s;
   quoka_status st = validate_attn(Q, Ksel, Vsel, Kc, Vc, &s);
   if (st != QUOKA_OK) return st;
@@ -580,6 +587,7 @@ quoka_status quoka_decode_attn(const quoka_tensor* Q, const quoka_tensor* K, con
                                const int32_t* kv_idx, const int32_t* kv_count, int BSA_eff,
                                const quoka_tensor* Kc, const quoka_tensor* Vc, float scale, void* O,
                                float* lse, void* ws, size_t ws_bytes, void* stream) {
+  quoka::NvtxRange nvtx_range("quoka_decode_attn");
   AttnShapes s;
   quoka_status st = validate_attn(Q, K, V, Kc, Vc, &s);
   if (st != QUOKA_OK) return st;
@@ -604,6 +612,7 @@ quoka_status quoka_prefill_chunk(const quoka_tensor* Q, const quoka_tensor* K,
                                  const quoka_tensor* Vc, int NQ, int BSA, float scale, void* O,
                                  float* lse, int32_t* kv_idx_out, void* ws, size_t ws_bytes,
                                  void* stream) {
+  quoka::NvtxRange nvtx_range("quoka_prefill_chunk");
   AttnShapes as;
   quoka_status st = validate_attn(Q, K, V, Kc, Vc, &as);
   if (st != QUOKA_OK) return st;
@@ -633,6 +642,7 @@ quoka_status quoka_prefill_chunk(const quoka_tensor* Q, const quoka_tensor* K,
 }
 
 quoka_status quoka_get_device_status(const void* ws, void* stream, int32_t* device_status) {
+  quoka::NvtxRange nvtx_range("quoka_get_device_status");
   if (device_status == nullptr) return QUOKA_ERR_INVALID_ARG;
   if (ws == nullptr) {  // the fixed scratch of quoka_select_static
     void* p = nullptr;
@@ -650,6 +660,7 @@ quoka_status quoka_get_device_status(const void* ws, void* stream, int32_t* devi
 }
 
 quoka_status quoka_get_device_fault_site(const void* ws, void* stream, int32_t* site) {
+  quoka::NvtxRange nvtx_range("quoka_get_device_fault_site");
   if (site == nullptr) return QUOKA_ERR_INVALID_ARG;
   if (ws == nullptr) {  // the fixed scratch of quoka_select_static
     void* p = nullptr;

@@ -15,6 +15,7 @@
 // ordering between them) race on it; callers must order them.
 #include <cuda_runtime.h>
 
+#include "nvtx_range.h"
 #include "quoka.h"
 
 namespace {
@@ -42,6 +43,7 @@ quoka_status static_scratch_address(void** out) {
 extern "C" quoka_status quoka_select_static(const quoka_tensor* Q, const quoka_tensor* K, int NQ,
                                             int BSA, int32_t* kv_idx, int32_t* kv_count,
                                             int32_t* q_idx, float* s_agg, void* stream) {
+  quoka::NvtxRange nvtx_range("quoka_select_static");
   if (Q == nullptr || K == nullptr) return QUOKA_ERR_INVALID_ARG;
   const size_t need = quoka_select_workspace_size((int)Q->shape[0], (int)Q->shape[1], (int)K->shape[1],
                                            (int)Q->shape[3], K->shape[2], (int)Q->shape[2], NQ, BSA,

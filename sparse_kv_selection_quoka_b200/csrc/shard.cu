@@ -17,6 +17,7 @@
 
 #include "common.cuh"
 #include "kernels.h"
+#include "nvtx_range.h"
 #include "quoka.h"
 
 namespace quoka {
@@ -160,6 +161,7 @@ extern "C" {
 quoka_status quoka_shard_candidate_scores(const float* s_agg, int b, int nkv, int64_t T, const int32_t* kv_idx,
                                           const int32_t* kv_count, int Cl, int C, float* scores,
                                           int32_t* cand_idx, void* ws, size_t ws_bytes, void* stream) {
+  quoka::NvtxRange nvtx_range("quoka_shard_candidate_scores");
   if (b < 1 || nkv < 1 || b > 65535 || nkv > 65535 || T < 0 || Cl < 0 || C < Cl || kv_count == nullptr)
     return QUOKA_ERR_INVALID_ARG;
   if (C == 0) return QUOKA_OK;
@@ -176,6 +178,7 @@ quoka_status quoka_shard_candidate_scores(const float* s_agg, int b, int nkv, in
 }
 
 quoka_status quoka_shard_interleave(const void* in, int N, int64_t rows, int64_t C, void* out, void* stream) {
+  quoka::NvtxRange nvtx_range("quoka_shard_interleave");
   if (N < 1 || rows < 0 || C < 0) return QUOKA_ERR_INVALID_ARG;
   const int64_t total = (int64_t)N * rows * C;
   if (total == 0) return QUOKA_OK;
@@ -190,6 +193,7 @@ quoka_status quoka_shard_interleave(const void* in, int N, int64_t rows, int64_t
 
 quoka_status quoka_topk(const float* scores, int b, int nkv, int64_t T, int BSA, int32_t* kv_idx,
                         int32_t* kv_count, void* ws, size_t ws_bytes, void* stream) {
+  quoka::NvtxRange nvtx_range("quoka_topk");
   if (b < 1 || nkv < 1 || b > 65535 || nkv > 65535 || T < 0 || BSA < 0 || kv_count == nullptr)
     return QUOKA_ERR_INVALID_ARG;
   const int64_t bsa_eff = BSA < T ? BSA : T;
@@ -208,6 +212,7 @@ quoka_status quoka_topk(const float* scores, int b, int nkv, int64_t T, int BSA,
 quoka_status quoka_shard_take(const int32_t* sel_pos, const int32_t* sel_count, int b, int nkv, int S,
                               const int32_t* cand_idx, int C, int rank, int32_t* kv_idx, int32_t* kv_count,
                               void* ws, size_t ws_bytes, void* stream) {
+  quoka::NvtxRange nvtx_range("quoka_shard_take");
   if (b < 1 || nkv < 1 || b > 65535 || nkv > 65535 || S < 0 || C < 0 || rank < 0 || sel_count == nullptr ||
       kv_count == nullptr)
     return QUOKA_ERR_INVALID_ARG;
@@ -227,6 +232,7 @@ quoka_status quoka_shard_take(const int32_t* sel_pos, const int32_t* sel_count, 
 
 quoka_status quoka_combine_partials(const void* O_parts, const float* lse_parts, int N, int b, int nq, int BCP,
                                     int d, quoka_dtype dtype, void* O, float* lse, void* stream) {
+  quoka::NvtxRange nvtx_range("quoka_combine_partials");
   if (N < 1 || b < 1 || nq < 1 || BCP < 1 || (d != 64 && d != 128)) return QUOKA_ERR_INVALID_ARG;
   if (dtype != QUOKA_F32 && dtype != QUOKA_BF16) return QUOKA_ERR_INVALID_ARG;
   if (O_parts == nullptr || lse_parts == nullptr || O == nullptr) return QUOKA_ERR_INVALID_ARG;
