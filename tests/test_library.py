@@ -32,6 +32,23 @@ def test_header_declares_the_boundary():
         assert n in names
 
 
+@pytest.mark.parametrize("lang,std", [("c", "c99"), ("c++", "c++11")])
+def test_header_compiles_on_its_own(lang, std, tmp_path):
+    """include/quoka.h is a plain C header (fixed-width integers, opaque
+    stream pointers, no CUDA or torch types): it compiles alone as C99 and
+    as C++, and a C translation unit can take the address of every
+    declared function."""
+    import shutil
+    cc = shutil.which("gcc" if lang == "c" else "g++")
+    if cc is None:
+        pytest.skip("no host compiler")
+    src = tmp_path / ("use." + ("c" if lang == "c" else "cpp"))
+    refs = "\n".join(f"  (void)&{n};" for n in declared_functions())
+    src.write_text(f'#include "quoka.h"\nvoid use(void) {{\n{refs}\n}}\n')
+    subprocess.run([cc, "-std=" + std, "-Wall", "-Werror", "-fsyntax-only", "-I", os.path.dirname(HEADER), str(src)],
+                   check=True, capture_output=True, text=True)
+
+
 def test_every_declared_symbol_is_exported(lib):
     from sparse_kv_selection_quoka_b200 import _lib
     out = subprocess.run(["nm", "-D", "--defined-only", _lib.LIB_PATH], capture_output=True,
