@@ -49,6 +49,42 @@ def test_header_compiles_on_its_own(lang, std, tmp_path):
                    check=True, capture_output=True, text=True)
 
 
+def test_plain_c_program_links_and_calls_the_host_entry_points(lib, tmp_path):
+    """A C program linked against libquoka.so (no Python, no torch) sizes a
+    workspace, names a status, and gets a bad call turned away on the host,
+    through the header alone."""
+    import shutil
+    from sparse_kv_selection_quoka_b200 import _lib
+    cc = shutil.which("gcc")
+    if cc is None:
+        pytest.skip("no host compiler")
+    src = tmp_path / "main.c"
+    src.write_text(r"""
+#include <stdio.h>
+#include <string.h>
+#include "quoka.h"
+int main(void) {
+  size_t n = quoka_workspace_size(1, 32, 8, 128, 32768, 512, 32, 4096, QUOKA_BF16);
+  size_t bad = quoka_workspace_size(1, 32, 7, 128, 32768, 512, 32, 4096, QUOKA_BF16);
+  quoka_tensor q;
+  memset(&q, 0, sizeof q);
+  quoka_status st = quoka_select(&q, NULL, 4, 10, NULL, NULL, NULL, NULL, NULL, 0, NULL);
+  printf("%zu %zu %d %s\n", n, bad, (int)st, quoka_status_string(st));
+  return 0;
+}
+""")
+    libdir = os.path.dirname(_lib.LIB_PATH)
+    exe = tmp_path / "main"
+    subprocess.run([cc, "-std=c99", "-Wall", "-Werror", "-I", os.path.dirname(HEADER), str(src), "-L", libdir,
+                    "-lquoka", "-o", str(exe)], check=True, capture_output=True, text=True)
+    env = dict(os.environ, LD_LIBRARY_PATH=libdir + os.pathsep + os.environ.get("LD_LIBRARY_PATH", ""))
+    out = subprocess.run([str(exe)], check=True, capture_output=True, text=True, env=env).stdout.split(" ", 3)
+    assert int(out[0]) == lib.quoka_workspace_size(1, 32, 8, 128, 32768, 512, 32, 4096, 1) > 0
+    assert int(out[1]) == 0  # nq not a multiple of nkv
+    assert int(out[2]) == 1  # QUOKA_ERR_INVALID_ARG
+    assert out[3].strip() == lib.quoka_status_string(1).decode()
+
+
 def test_every_declared_symbol_is_exported(lib):
     from sparse_kv_selection_quoka_b200 import _lib
     out = subprocess.run(["nm", "-D", "--defined-only", _lib.LIB_PATH], capture_output=True,
